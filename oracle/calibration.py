@@ -1,0 +1,200 @@
+"""Per-head eigenspectral calibration (oracle, float64).
+
+Sources
+-------
+* SpectralQuant README, "Repository Structure": ``calibration.py --
+  Eigenspectral calibration (PCA, d_eff, kappa)``; "Overview": a one-time
+  calibration finds the few signal dimensions of the key vectors.
+* spectralquant tests/conftest.py (v1 branch), fixture
+  ``pre_computed_calibration``: C = X^T X / N (no centring), ``eigh``,
+  reversal to descending order, d_eff = round((sum lambda)^2 / sum lambda^2),
+  gap = lambda[d_eff - 1] / lambda[d_eff] (0-based) or inf when d_eff = d.
+* The title of the method ("Water-Filled Bit Allocation") and the Chinese
+  summary ("water-filling non-uniform bit allocation by spectral structure").
+
+Readings taken where the pages are silent
+-----------------------------------------
+* Eigenvalues below zero (round-off) are clamped to 0.
+* Sign of each eigenvector: its entry of largest magnitude is made positive
+  (ties: the lowest index).
+* d_eff rounds half to even (Python's ``round``) and is clamped to [1, d];
+  an all-zero spectrum gives d_eff = d.
+* Quantizer scale per coordinate. Normalized mode (default): the unit vector
+  x/||x|| is quantized, and sigma_i = sqrt(lambda_i / sum lambda), the
+  first-order second moment of its i-th rotated coordinate. Unnormalized
+  mode: sigma_i = sqrt(lambda_i).
+* Bit budget: B = avg_bits * d bits per vector, an integer. A key with QJL
+  spends m = d_eff of them on sign bits, so the codes get B - m bits;
+  otherwise the codes get all B. No coordinate takes more than 8 bits.
+* Water-filling: greedy, one bit at a time, to the coordinate whose expected
+  distortion drops most, lambda_i * (D(b_i) - D(b_i + 1)), among those below
+  the cap; ties go to the lowest index. D is the Gaussian Lloyd-Max
+  distortion table (D(0) = 1). Because D is convex and decreasing the greedy
+  result minimises sum_i lambda_i D(b_i) over integer allocations.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import codebook, rng
+
+FLAG_IS_KEY = 1
+FLAG_QJL = 2
+FLAG_NORMALIZE = 4
+
+
+def second_moment(x: np.ndarray) -> np.ndarray:
+    """C = X^T X / N of the calibration vectors (rows of ``x``), uncentred."""
+    x = np.asarray(x, dtype=np.float64)
+    return x.T @ x / x.shape[0]
+
+
+def eigenbasis(c: np.ndarray):
+    """Eigenvalues (descending, >= 0) and orthonormal eigenvectors (columns)."""
+    lam, vec = np.linalg.eigh(np.asarray(c, dtype=np.float64))
+    lam = lam[::-1].copy()
+    vec = vec[:, ::-1].copy()
+    lam = np.maximum(lam, 0.0)
+    for i in range(vec.shape[1]):
+        j = int(np.argmax(np.abs(vec[:, i])))
+        if vec[j, i] < 0.0:
+            vec[:, i] = -vec[:, i]
+    return lam, vec
+
+
+def participation_ratio(lam: np.ndarray) -> float:
+    """(sum lambda)^2 / sum lambda^2."""
+    lam = np.asarray(lam, dtype=np.float64)
+    s2 = float(np.sum(lam * lam))
+    if s2 == 0.0:
+        return float(lam.size)
+    return float(np.sum(lam)) ** 2 / s2
+
+
+def effective_dim(lam: np.ndarray) -> int:
+    """d_eff: the participation ratio rounded half to even, within [1, d]."""
+    d = len(lam)
+    return int(min(max(round(participation_ratio(lam)), 1), d))
+
+
+def spectral_gap(lam: np.ndarray, d_eff: int) -> float:
+    """kappa = lambda[d_eff - 1] / lambda[d_eff] (0-based); inf if d_eff == d."""
+    d = len(lam)
+    if d_eff >= d or lam[d_eff] == 0.0:
+        return float("inf")
+    return float(lam[d_eff - 1] / lam[d_eff])
+
+
+def scales(lam: np.ndarray, normalize: bool) -> np.ndarray:
+    """Quantizer scale sigma_i of each rotated coordinate."""
+    lam = np.asarray(lam, dtype=np.float64)
+    if not normalize:
+        return np.sqrt(lam)
+    tr = float(np.sum(lam))
+    if tr == 0.0:
+        return np.zeros_like(lam)
+    return np.sqrt(lam / tr)
+
+
+def water_fill(lam: np.ndarray, n_bits: int, max_bits: int = codebook.MAX_BITS) -> np.ndarray:
+    """Greedy integer allocation of ``n_bits`` bits over the coordinates."""
+    lam = np.asarray(lam, dtype=np.float64)
+    d = lam.size
+    if n_bits < 0 or n_bits > max_bits * d:
+        raise ValueError("bit budget outside [0, max_bits * d]")
+    dist = codebook.distortion_table(max_bits)
+    bits = np.zeros(d, dtype=np.int64)
+    for _ in range(n_bits):
+        gain = np.where(bits < max_bits,
+                        lam * (dist[np.minimum(bits, max_bits - 1)] - dist[np.minimum(bits + 1, max_bits)]),
+                        -np.inf)
+        i = int(np.argmax(gain))          # first maximum = lowest index on ties
+        bits[i] += 1
+    return bits
+
+
+def bit_offsets(bits: np.ndarray) -> np.ndarray:
+    """Bit position of coordinate i's code in the packed record."""
+    return np.concatenate([[0], np.cumsum(bits)[:-1]]).astype(np.int64)
+
+
+@dataclass
+class HeadCalib:
+    """One head's calibration: everything the codec and attention read."""
+
+    d: int
+    d_eff: int            # participation ratio, rounded
+    m: int                # QJL sign dimensions (0 without QJL)
+    total_bits: int       # B: bits of one packed record
+    code_bits: int        # sum of b_i
+    words: int            # 32-bit words of one record, ceil(B / 32)
+    flags: int
+    sweeps: int
+    stream: int           # head index of the QJL stream
+    max_bits: int
+    seed: int
+    trace: float
+    kappa: float
+    avg_bits: float
+    lam: np.ndarray       # [d] descending
+    sigma: np.ndarray     # [d]
+    V: np.ndarray         # [d, d], column i = eigenvector i
+    S: np.ndarray         # [m, m] QJL projection
+    bits: np.ndarray      # [d] int
+    offsets: np.ndarray   # [d] int
+
+    @property
+    def is_key(self) -> bool:
+        return bool(self.flags & FLAG_IS_KEY)
+
+    @property
+    def qjl(self) -> bool:
+        return bool(self.flags & FLAG_QJL)
+
+    @property
+    def normalize(self) -> bool:
+        return bool(self.flags & FLAG_NORMALIZE)
+
+
+def budget(d: int, avg_bits: float) -> int:
+    """B = avg_bits * d, which must be a whole number of bits."""
+    total = avg_bits * d
+    if abs(total - round(total)) > 1e-9 or total <= 0:
+        raise ValueError(f"avg_bits * d = {total} is not a positive integer")
+    return int(round(total))
+
+
+def finalize(lam: np.ndarray, vec: np.ndarray, *, avg_bits: float, is_key: bool,
+             qjl: bool = True, normalize: bool = True, d_eff_override: int = 0,
+             max_bits: int = codebook.MAX_BITS, seed: int = 42, stream: int = 0,
+             sweeps: int = 0) -> HeadCalib:
+    """Everything after the eigendecomposition: d_eff, kappa, scales, bits, QJL matrix."""
+    d = lam.size
+    d_eff = effective_dim(lam)
+    kappa = spectral_gap(lam, d_eff)
+    total = budget(d, avg_bits)
+    use_qjl = bool(is_key and qjl)
+    m = (d_eff_override if d_eff_override > 0 else d_eff) if use_qjl else 0
+    if m > d:
+        raise ValueError("QJL dimension above head_dim")
+    code_bits = total - m
+    if code_bits < 0 or code_bits > max_bits * d:
+        raise ValueError("bit budget cannot hold the QJL bits and the codes")
+    bits = water_fill(lam, code_bits, max_bits)
+    flags = (FLAG_IS_KEY if is_key else 0) | (FLAG_QJL if use_qjl else 0) | (FLAG_NORMALIZE if normalize else 0)
+    return HeadCalib(
+        d=d, d_eff=d_eff, m=m, total_bits=total, code_bits=code_bits,
+        words=(total + 31) // 32, flags=flags, sweeps=sweeps, stream=stream,
+        max_bits=max_bits, seed=seed, trace=float(np.sum(lam)), kappa=kappa,
+        avg_bits=float(avg_bits), lam=lam.copy(), sigma=scales(lam, normalize),
+        V=vec.copy(), S=rng.qjl_matrix(seed, stream, m), bits=bits,
+        offsets=bit_offsets(bits))
+
+
+def calibrate(x: np.ndarray, **kw) -> HeadCalib:
+    """Calibrate one head from its calibration vectors ``x`` [N, d]."""
+    lam, vec = eigenbasis(second_moment(x))
+    return finalize(lam, vec, **kw)

@@ -1,0 +1,67 @@
+"""Pins of the oracle's decode attention over the packed cache."""
+
+import math
+
+import numpy as np
+import torch
+
+from oracle import attention, calibration as cal, codec
+from synthetic import make_workload
+
+
+def _build(cfg_name="tiny", g=1, tokens=256, n_kv=2, bits_k=3.0, bits_v=3.0, seq=None):
+    w = make_workload(cfg_name, tokens=tokens)
+    n_kv = min(n_kv, w.cfg["n_kv"])
+    ck, cv, kw, kn, kr, vw, vn = [], [], [], [], [], [], []
+    for h in range(n_kv):
+        a = cal.calibrate(w.k_cal[h].double().numpy(), avg_bits=bits_k, is_key=True, seed=42, stream=h)
+        b = cal.calibrate(w.v_cal[h].double().numpy(), avg_bits=bits_v, is_key=False, seed=42, stream=100 + h)
+        ok = codec.compress(w.k[0, h].double().numpy(), a)
+        ov = codec.compress(w.v[0, h].double().numpy(), b)
+        ck.append(a); cv.append(b)
+        kw.append(ok["words"]); kn.append(ok["norm"]); kr.append(ok["rnorm"])
+        vw.append(ov["words"]); vn.append(ov["norm"])
+    q = np.random.default_rng(0).standard_normal((1, n_kv * g, w.cfg["d"])) * 0.5
+    st = lambda xs: np.stack(xs)[None]
+    return q, st(kw), st(kn), st(kr), st(vw), st(vn), ck, cv
+
+
+def test_equals_dense_attention_on_decompressed_vectors():
+    for g in (1, 3):
+        q, kw, kn, kr, vw, vn, ck, cv = _build(g=g)
+        scale = 1 / math.sqrt(q.shape[-1])
+        out, scores = attention.attn_decode(q, kw, kn, kr, vw, vn, ck, cv, [kw.shape[2]], scale)
+        for h in range(q.shape[1]):
+            kv = h // g
+            keys = codec.decompress(kw[0, kv], kn[0, kv], kr[0, kv], ck[kv], apply_qjl=True)
+            vals = codec.decompress(vw[0, kv], vn[0, kv], None, cv[kv], apply_qjl=False)
+            o, s = attention.dense_attention(q[0, h], keys, vals, scale)
+            assert np.allclose(scores[0, h], s, rtol=1e-11, atol=1e-11)
+            assert np.allclose(out[0, h], o, rtol=1e-11, atol=1e-13)
+
+
+def test_single_token_returns_its_value():
+    q, kw, kn, kr, vw, vn, ck, cv = _build(tokens=8)
+    out, _ = attention.attn_decode(q, kw, kn, kr, vw, vn, ck, cv, [1], None)
+    v0 = codec.decompress(vw[0, 0, :1], vn[0, 0, :1], None, cv[0], apply_qjl=False)[0]
+    assert np.allclose(out[0, 0], v0, rtol=1e-12, atol=1e-14)
+
+
+def test_ragged_lengths_and_nan_padding():
+    q, kw, kn, kr, vw, vn, ck, cv = _build(tokens=40)
+    q2 = np.concatenate([q, q])
+    kw2, kn2, kr2, vw2, vn2 = (np.concatenate([a, a]) for a in (kw, kn, kr, vw, vn))
+    out, scores = attention.attn_decode(q2, kw2, kn2, kr2, vw2, vn2, ck, cv, [40, 17], None)
+    assert np.all(np.isnan(scores[1, :, 17:])) and not np.any(np.isnan(scores[1, :, :17]))
+    o17, _ = attention.attn_decode(q, kw[:, :, :17], kn[:, :, :17], kr[:, :, :17], vw[:, :, :17],
+                                   vn[:, :, :17], ck, cv, [17], None)
+    assert np.allclose(out[1], o17[0], rtol=1e-12)
+
+
+def test_uniform_scores_average_values():
+    """A zero query gives equal weights: the output is the mean decompressed value."""
+    q, kw, kn, kr, vw, vn, ck, cv = _build(tokens=32)
+    out, scores = attention.attn_decode(np.zeros_like(q), kw, kn, kr, vw, vn, ck, cv, [32], None)
+    assert np.all(scores == 0.0)
+    vals = codec.decompress(vw[0, 0], vn[0, 0], None, cv[0], apply_qjl=False)
+    assert np.allclose(out[0, 0], vals.mean(axis=0), rtol=1e-12, atol=1e-14)
