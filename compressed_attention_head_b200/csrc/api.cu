@@ -1,0 +1,318 @@
+// libsq host entry points: argument checks, per-device table upload, launches.
+// The public contract (arguments, layouts, ownership, errors) is in include/sq.h.
+#include <mutex>
+
+#include "sq_common.cuh"
+
+namespace sq {
+__constant__ double c_lv64[kLevelsTotal];
+__constant__ double c_th64[kThreshTotal];
+__constant__ float c_lv32[kLevelsTotal];
+__constant__ double c_D[SQ_MAX_BITS + 1];
+}  // namespace sq
+
+#include "attention.cuh"
+#include "calibrate.cuh"
+#include "codec.cuh"
+
+namespace sq {
+
+const double* codebook_levels(int b);
+const double* codebook_thresholds(int b);
+double codebook_distortion(int b);
+
+namespace {
+
+std::mutex g_mu;
+bool g_ready[128];
+int g_sms[128];
+
+bool supported_d(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+bool valid_dtype(int t) { return t == SQ_F32 || t == SQ_F16 || t == SQ_BF16; }
+
+sq_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA; }
+
+// Uploads the Lloyd-Max tables to the current device once.
+sq_status ensure_init(int* dev_out = nullptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return SQ_ERR_CUDA;
+  if (dev_out) *dev_out = dev;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_ready[dev]) return SQ_OK;
+  double lv[kLevelsTotal], th[kThreshTotal], dist[SQ_MAX_BITS + 1];
+  float lv32[kLevelsTotal];
+  dist[0] = 1.0;
+  for (int b = 1; b <= SQ_MAX_BITS; ++b) {
+    const double* l = codebook_levels(b);
+    const double* t = codebook_thresholds(b);
+    for (int k = 0; k < (1 << b); ++k) lv[lv_off(b) + k] = l[k];
+    for (int k = 0; k + 1 < (1 << b); ++k) th[th_off(b) + k] = t[k];
+    dist[b] = codebook_distortion(b);
+  }
+  for (int k = 0; k < kLevelsTotal; ++k) lv32[k] = (float)lv[k];
+  if (cudaMemcpyToSymbol(c_lv64, lv, sizeof(lv)) != cudaSuccess) return SQ_ERR_CUDA;
+  if (cudaMemcpyToSymbol(c_th64, th, sizeof(th)) != cudaSuccess) return SQ_ERR_CUDA;
+  if (cudaMemcpyToSymbol(c_lv32, lv32, sizeof(lv32)) != cudaSuccess) return SQ_ERR_CUDA;
+  if (cudaMemcpyToSymbol(c_D, dist, sizeof(dist)) != cudaSuccess) return SQ_ERR_CUDA;
+  // Kernels that take more than 48 KB of dynamic shared memory.
+  const int big = 200 * 1024;
+  cudaFuncSetAttribute(k_jacobi, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  cudaFuncSetAttribute(k_compress_ref<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  cudaFuncSetAttribute(k_compress_ref<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  cudaFuncSetAttribute(k_compress_ref<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  cudaFuncSetAttribute(k_decompress_ref, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  cudaFuncSetAttribute(k_attn_partial<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  cudaFuncSetAttribute(k_attn_partial<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  cudaFuncSetAttribute(k_attn_partial<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  cudaFuncSetAttribute(k_attn_partial<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  cudaFuncSetAttribute(k_attn_partial<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  g_sms[dev] = sms > 0 ? sms : 148;
+  g_ready[dev] = true;
+  return SQ_OK;
+}
+
+// Whole number of bits B = avg_bits * d, or -1.
+int budget_bits(double avg_bits, int d) {
+  double t = avg_bits * d;
+  long r = lround(t);
+  if (!(t > 0.0) || fabs(t - (double)r) > 1e-9 || r > (long)SQ_MAX_BITS * 256 + 256) return -1;
+  return (int)r;
+}
+
+bool cache_ok(const sq_cache* c, int batch, int n_heads) {
+  return c && c->codes && c->norm && aligned16(c->codes) && aligned16(c->norm) &&
+         (!c->rnorm || aligned16(c->rnorm)) && c->batch == batch && c->n_heads == n_heads && c->cap >= 16 &&
+         c->cap % 16 == 0 && c->words >= 1 && c->words <= kMaxWords;
+}
+
+CacheArgs cache_args(const sq_cache* c) { return CacheArgs{c->codes, c->norm, c->rnorm, c->cap, c->words}; }
+
+// Splits of the context per (batch, KV head) so that the partial kernel has
+// about two blocks per SM of a 148-SM B200, each over >= one 128-token tile.
+int attn_splits(int batch, int n_kv, int64_t max_ctx) {
+  int64_t units = (int64_t)batch * n_kv;
+  int64_t want = (2 * 148 + units - 1) / units;
+  int64_t tiles = (max_ctx + kAttnTile - 1) / kAttnTile;
+  if (want > tiles) want = tiles;
+  if (want > 256) want = 256;
+  if (want < 1) want = 1;
+  return (int)want;
+}
+
+template <typename T>
+sq_status launch_compress(const void* recs, const void* x, int batch, int n_heads, int d, int64_t n_tok,
+                          const int32_t* sp, const sq_cache* c, uint32_t* flags, cudaStream_t st) {
+  const int tpb = n_tok >= 1024 ? 256 : 64;
+  const int64_t gx = (n_tok + tpb - 1) / tpb;
+  if (gx > 0x7fffffff) return SQ_ERR_ARG;
+  dim3 grid((unsigned)gx, n_heads, batch);
+  k_compress_ref<T><<<grid, 128, codec_ref_smem(d), st>>>((const uint8_t*)recs, (const T*)x, n_heads, d, n_tok,
+                                                          tpb, sp, cache_args(c), flags);
+  return cuda_ok(cudaGetLastError());
+}
+
+}  // namespace
+}  // namespace sq
+
+using namespace sq;
+
+extern "C" {
+
+int sq_abi_version(void) { return SQ_ABI_VERSION; }
+
+const char* sq_status_str(sq_status s) {
+  switch (s) {
+    case SQ_OK: return "ok";
+    case SQ_ERR_ARG: return "invalid argument";
+    case SQ_ERR_UNSUPPORTED: return "unsupported head_dim or dtype";
+    case SQ_ERR_CUDA: return "CUDA error";
+    case SQ_ERR_NOT_CONVERGED: return "eigensolver did not converge within max_sweeps";
+    case SQ_ERR_CAPACITY: return "cache capacity exceeded";
+    case SQ_ERR_WORKSPACE: return "workspace too small";
+    case SQ_ERR_RECORD: return "malformed calibration record";
+  }
+  return "unknown status";
+}
+
+size_t sq_calib_bytes(int d) { return supported_d(d) ? record_bytes(d) : 0; }
+
+int sq_record_words(const sq_calib_params* p) {
+  if (!p || !supported_d(p->d)) return 0;
+  int bits = budget_bits(p->avg_bits, p->d);
+  return bits < 0 ? 0 : (bits + 31) / 32;
+}
+
+sq_status sq_init(void) { return ensure_init(); }
+
+size_t sq_calibrate_workspace(const sq_calib_params* p, int64_t n_tokens) {
+  (void)n_tokens;
+  if (!p || !supported_d(p->d) || p->n_heads < 1) return 0;
+  return (size_t)p->n_heads * 16u * (size_t)p->d * (size_t)p->d;
+}
+
+sq_status sq_calibrate(const sq_calib_params* p, const void* x, sq_dtype dtype, int64_t n_tokens,
+                       int64_t stride_head, int64_t stride_tok, void* calib_out, void* ws, size_t ws_bytes,
+                       int* d_status, sq_stream stream) {
+  if (!p) return SQ_ERR_ARG;
+  if (!supported_d(p->d)) return SQ_ERR_UNSUPPORTED;
+  if (!valid_dtype(dtype)) return SQ_ERR_UNSUPPORTED;
+  const int d = p->d;
+  const int B = budget_bits(p->avg_bits, d);
+  if (p->n_heads < 1 || B < 1 || p->max_bits < 1 || p->max_bits > SQ_MAX_BITS || p->d_eff_override < 0 ||
+      p->d_eff_override > d || p->max_sweeps < 1 || !(p->tol > 0.0) || n_tokens < 1 || stride_tok < d ||
+      stride_head < 0 || !x || !calib_out || ((uintptr_t)calib_out & 255u) || !ws || !aligned16(ws) ||
+      (p->is_key != 0 && p->is_key != 1) || (p->qjl != 0 && p->qjl != 1) ||
+      (p->normalize != 0 && p->normalize != 1) || (d_status && !aligned16(d_status)) || (B + 31) / 32 > kMaxWords)
+    return SQ_ERR_ARG;
+  if (ws_bytes < sq_calibrate_workspace(p, n_tokens)) return SQ_ERR_WORKSPACE;
+  sq_status s = ensure_init();
+  if (s != SQ_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  double* cov = (double*)ws;
+  double* vt = cov + (size_t)p->n_heads * d * d;
+  dim3 g1(p->n_heads, d / 32, d / 32), b1(32, 8);
+  switch (dtype) {
+    case SQ_F32: k_second_moment<float><<<g1, b1, 0, st>>>((const float*)x, d, n_tokens, stride_head, stride_tok, cov); break;
+    case SQ_F16: k_second_moment<__half><<<g1, b1, 0, st>>>((const __half*)x, d, n_tokens, stride_head, stride_tok, cov); break;
+    default: k_second_moment<__nv_bfloat16><<<g1, b1, 0, st>>>((const __nv_bfloat16*)x, d, n_tokens, stride_head, stride_tok, cov); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  size_t jsm = d <= 128 ? (size_t)8 * d * d : 0;
+  k_jacobi<<<p->n_heads, 256, jsm, st>>>(cov, vt, d, p->max_sweeps, p->tol, calib_out, d_status);
+  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  FinalizeArgs fa{B, p->is_key, p->qjl, p->normalize, p->d_eff_override, p->max_bits, p->seed, p->avg_bits};
+  k_finalize<<<p->n_heads, 256, 0, st>>>(calib_out, d, fa, d_status);
+  return cuda_ok(cudaGetLastError());
+}
+
+sq_status sq_calib_import(void* calib, int n_heads, int d, int* d_status, sq_stream stream) {
+  if (!supported_d(d)) return SQ_ERR_UNSUPPORTED;
+  if (!calib || ((uintptr_t)calib & 255u) || n_heads < 1 || (d_status && !aligned16(d_status))) return SQ_ERR_ARG;
+  sq_status s = ensure_init();
+  if (s != SQ_OK) return s;
+  k_import<<<n_heads, 256, 0, (cudaStream_t)stream>>>(calib, d, d_status);
+  return cuda_ok(cudaGetLastError());
+}
+
+sq_status sq_compress_kv(const void* calib_k, const void* calib_v, const void* k, const void* v, sq_dtype dtype,
+                         int batch, int n_heads, int d, int64_t n_tok, const int32_t* d_start_pos,
+                         const sq_cache* kc, const sq_cache* vc, uint32_t* d_flags, sq_stream stream) {
+  if (!supported_d(d) || !valid_dtype(dtype)) return SQ_ERR_UNSUPPORTED;
+  if (batch < 1 || n_heads < 1 || n_tok < 0 || batch > 65535 || n_heads > 65535) return SQ_ERR_ARG;
+  if (n_tok == 0) return SQ_OK;
+  const bool do_k = k != nullptr, do_v = v != nullptr;
+  if (!do_k && !do_v) return SQ_ERR_ARG;
+  if (do_k && (!calib_k || ((uintptr_t)calib_k & 255u) || !aligned16(k) || !cache_ok(kc, batch, n_heads)))
+    return SQ_ERR_ARG;
+  if (do_v && (!calib_v || ((uintptr_t)calib_v & 255u) || !aligned16(v) || !cache_ok(vc, batch, n_heads)))
+    return SQ_ERR_ARG;
+  if (d_start_pos && !aligned16(d_start_pos)) return SQ_ERR_ARG;
+  sq_status s = ensure_init();
+  if (s != SQ_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  for (int side = 0; side < 2; ++side) {
+    const void* x = side == 0 ? k : v;
+    if (!x) continue;
+    const void* recs = side == 0 ? calib_k : calib_v;
+    const sq_cache* c = side == 0 ? kc : vc;
+    switch (dtype) {
+      case SQ_F32: s = launch_compress<float>(recs, x, batch, n_heads, d, n_tok, d_start_pos, c, d_flags, st); break;
+      case SQ_F16: s = launch_compress<__half>(recs, x, batch, n_heads, d, n_tok, d_start_pos, c, d_flags, st); break;
+      default: s = launch_compress<__nv_bfloat16>(recs, x, batch, n_heads, d, n_tok, d_start_pos, c, d_flags, st); break;
+    }
+    if (s != SQ_OK) return s;
+  }
+  return SQ_OK;
+}
+
+sq_status sq_decompress_kv(const void* calib, const sq_cache* cache, int d, int64_t t0, int64_t n_tok,
+                           int apply_qjl, float* out, uint32_t* d_flags, sq_stream stream) {
+  if (!supported_d(d)) return SQ_ERR_UNSUPPORTED;
+  if (!cache) return SQ_ERR_ARG;
+  if (!calib || ((uintptr_t)calib & 255u) || !out || !aligned16(out) || t0 < 0 || n_tok < 0 ||
+      !cache_ok(cache, cache->batch, cache->n_heads) || cache->batch < 1 || cache->n_heads < 1 ||
+      cache->batch > 65535 || cache->n_heads > 65535)
+    return SQ_ERR_ARG;
+  if (n_tok == 0) return SQ_OK;
+  sq_status s = ensure_init();
+  if (s != SQ_OK) return s;
+  const int tpb = n_tok >= 1024 ? 256 : 64;
+  dim3 grid((unsigned)((n_tok + tpb - 1) / tpb), cache->n_heads, cache->batch);
+  k_decompress_ref<<<grid, 128, codec_ref_smem(d), (cudaStream_t)stream>>>(
+      (const uint8_t*)calib, cache->n_heads, d, cache_args(cache), t0, n_tok, tpb, apply_qjl, out, d_flags);
+  return cuda_ok(cudaGetLastError());
+}
+
+size_t sq_attn_workspace(int batch, int n_q_heads, int n_kv_heads, int d, int64_t max_ctx) {
+  if (batch < 1 || n_q_heads < 1 || n_kv_heads < 1 || !supported_d(d) || max_ctx < 0) return 0;
+  int splits = attn_splits(batch, n_kv_heads, max_ctx);
+  return attn_ws_floats(batch, n_q_heads, d, splits) * sizeof(float);
+}
+
+sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
+                         const int32_t* d_seq_lens, int batch, int n_q_heads, int n_kv_heads, int d,
+                         int64_t max_ctx, const void* q, sq_dtype q_dtype, float scale, void* out,
+                         sq_dtype out_dtype, float* scores_out, void* ws, size_t ws_bytes, uint32_t* d_flags,
+                         sq_stream stream) {
+  if (!supported_d(d) || !valid_dtype(q_dtype) || !valid_dtype(out_dtype)) return SQ_ERR_UNSUPPORTED;
+  if (batch < 1 || batch > 65535 || n_q_heads < 1 || n_kv_heads < 1 || n_kv_heads > 65535 ||
+      n_q_heads % n_kv_heads != 0 || n_q_heads / n_kv_heads > kAttnMaxG || n_q_heads > 65535 || max_ctx < 0 ||
+      !calib_k || !calib_v || ((uintptr_t)calib_k & 255u) || ((uintptr_t)calib_v & 255u) ||
+      !cache_ok(kc, batch, n_kv_heads) || !cache_ok(vc, batch, n_kv_heads) || !d_seq_lens ||
+      !aligned16(d_seq_lens) || !q || !aligned16(q) || !out || !aligned16(out) ||
+      (scores_out && !aligned16(scores_out)) || !ws || !aligned16(ws))
+    return SQ_ERR_ARG;
+  if (ws_bytes < sq_attn_workspace(batch, n_q_heads, n_kv_heads, d, max_ctx)) return SQ_ERR_WORKSPACE;
+  sq_status s = ensure_init();
+  if (s != SQ_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  AttnShape sh;
+  sh.batch = batch;
+  sh.n_q = n_q_heads;
+  sh.n_kv = n_kv_heads;
+  sh.group = n_q_heads / n_kv_heads;
+  sh.d = d;
+  sh.splits = attn_splits(batch, n_kv_heads, max_ctx);
+  sh.max_ctx = max_ctx;
+  int64_t per = (max_ctx + sh.splits - 1) / sh.splits;
+  sh.chunk = ((per + kAttnTile - 1) / kAttnTile) * kAttnTile;
+  if (sh.chunk < kAttnTile) sh.chunk = kAttnTile;
+  const float sc = scale > 0.0f ? scale : 1.0f / sqrtf((float)d);
+  float* w = (float*)ws;
+  dim3 gp(n_kv_heads, batch);
+  switch (q_dtype) {
+    case SQ_F32: k_attn_prepare<float><<<gp, 128, 0, st>>>((const uint8_t*)calib_k, (const float*)q, sh, sc, w, d_flags); break;
+    case SQ_F16: k_attn_prepare<__half><<<gp, 128, 0, st>>>((const uint8_t*)calib_k, (const __half*)q, sh, sc, w, d_flags); break;
+    default: k_attn_prepare<__nv_bfloat16><<<gp, 128, 0, st>>>((const uint8_t*)calib_k, (const __nv_bfloat16*)q, sh, sc, w, d_flags); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  dim3 gpart(sh.splits, n_kv_heads, batch);
+  size_t smem = attn_partial_smem(d, sh.group, kc->words, vc->words);
+  CacheArgs ka = cache_args(kc), va = cache_args(vc);
+  const uint8_t* rk = (const uint8_t*)calib_k;
+  const uint8_t* rv = (const uint8_t*)calib_v;
+  if (sh.group <= 1)
+    k_attn_partial<1><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
+  else if (sh.group <= 2)
+    k_attn_partial<2><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
+  else if (sh.group <= 4)
+    k_attn_partial<4><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
+  else if (sh.group <= 8)
+    k_attn_partial<8><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
+  else
+    k_attn_partial<16><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
+  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  dim3 gc(n_q_heads, batch);
+  switch (out_dtype) {
+    case SQ_F32: k_attn_combine<float><<<gc, 128, 0, st>>>(rv, sh, w, (float*)out); break;
+    case SQ_F16: k_attn_combine<__half><<<gc, 128, 0, st>>>(rv, sh, w, (__half*)out); break;
+    default: k_attn_combine<__nv_bfloat16><<<gc, 128, 0, st>>>(rv, sh, w, (__nv_bfloat16*)out); break;
+  }
+  return cuda_ok(cudaGetLastError());
+}
+
+}  // extern "C"

@@ -1,0 +1,328 @@
+// Decode attention straight from the packed cache.
+//
+// SpectralQuant README, "Headline Results" (decode latency per step over the
+// compressed cache) and "Key Findings" 3; keys carry the QJL sign correction on
+// their signal dims, values do not ("KV spectral asymmetry").
+//
+// For batch row b, query head h, KV head g = h / G and length L:
+//   q' = V_K^T q,  w_i = scale * sigma_i * q'_i,
+//   u_j = scale * sqrt(pi/2) / m * (S q'[0:m])_j,
+//   s_t = ||k_t|| * (sum_i w_i level_t,i + rho_t * sum_j u_j (2 bit_t,j - 1)),
+//   p = softmax(s);  o = V_V (sigma_V * sum_t p_t ||v_t|| level^V_t).
+// Three kernels: prepare (q' -> w, u), split-KV partial (online softmax over a
+// token range, flash-decoding style), combine (merge the splits, rotate back).
+#pragma once
+
+#include "sq_common.cuh"
+
+namespace sq {
+
+constexpr int kAttnTile = 128;     // tokens per tile of the partial kernel
+constexpr int kAttnMaxG = 16;      // query heads per KV head
+
+struct AttnShape {
+  int batch, n_q, n_kv, group, d, splits;
+  int64_t max_ctx, chunk;
+};
+
+// Workspace layout (floats): w[batch][n_q][d], u[batch][n_q][d],
+// acc[batch][n_q][splits][d], ml[batch][n_q][splits][2].
+__host__ __device__ inline size_t attn_ws_floats(int batch, int n_q, int d, int splits) {
+  return (size_t)batch * n_q * (2 * (size_t)d + (size_t)splits * (d + 2));
+}
+
+// ---------------------------------------------------------------------------
+// Prepare: grid (n_kv, batch), d threads; one block rotates the G queries of
+// one KV head with the float32 copy of V_K.
+// ---------------------------------------------------------------------------
+template <typename TQ>
+__global__ void k_attn_prepare(const uint8_t* __restrict__ recs_k, const TQ* __restrict__ q, AttnShape s,
+                               float scale, float* __restrict__ ws, uint32_t* __restrict__ flags) {
+  const int g = blockIdx.x, b = blockIdx.y, d = s.d, G = s.group;
+  Rec rec = rec_at(recs_k, d, g);
+  const RecHeader* hd = rec.hdr();
+  if (!record_ok(hd, d)) {
+    if (threadIdx.x == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
+    return;
+  }
+  __shared__ float qs[kAttnMaxG][kMaxD];
+  __shared__ float qp[kAttnMaxG][kMaxD];
+  for (int e = threadIdx.x; e < G * d; e += blockDim.x) {
+    int hh = e / d, j = e % d;
+    qs[hh][j] = to_float<TQ>(q[((size_t)b * s.n_q + g * G + hh) * d + j]);
+  }
+  __syncthreads();
+  const float* V = rec.V_f();
+  const float* sig = rec.sigma_f();
+  float* w = ws;
+  float* u = ws + (size_t)s.batch * s.n_q * d;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    float acc[kAttnMaxG];
+#pragma unroll
+    for (int hh = 0; hh < kAttnMaxG; ++hh) acc[hh] = 0.0f;
+    for (int j = 0; j < d; ++j) {
+      float v = V[(size_t)j * d + i];
+#pragma unroll
+      for (int hh = 0; hh < kAttnMaxG; ++hh)
+        if (hh < G) acc[hh] = fmaf(v, qs[hh][j], acc[hh]);
+    }
+    for (int hh = 0; hh < G; ++hh) {
+      qp[hh][i] = acc[hh];
+      w[((size_t)b * s.n_q + g * G + hh) * d + i] = scale * sig[i] * acc[hh];
+    }
+  }
+  __syncthreads();
+  const int m = hd->m;
+  const float* S = rec.S_f();
+  const float coef = scale * (float)(kQjlScale / (m > 0 ? m : 1));
+  for (int e = threadIdx.x; e < G * m; e += blockDim.x) {
+    int hh = e / m, j = e % m;
+    float acc = 0.0f;
+    for (int k = 0; k < m; ++k) acc = fmaf(S[j * m + k], qp[hh][k], acc);
+    u[((size_t)b * s.n_q + g * G + hh) * d + j] = coef * acc;
+  }
+}
+
+// Shared-memory bytes of the partial kernel.
+__host__ __device__ inline size_t attn_partial_smem(int d, int G, int wk, int wv) {
+  return (size_t)4 * G * d            // w
+         + (size_t)4 * G * d          // u (m <= d)
+         + (size_t)4 * kLevelsTotal   // levels
+         + (size_t)4 * 4 * d          // bits/offsets of K and V
+         + (size_t)4 * d              // sigma_V (unused here, reserved)
+         + (size_t)4 * kAttnTile * (wk + 1) + (size_t)4 * kAttnTile * (wv + 1)
+         + (size_t)4 * 3 * kAttnTile  // k norm, rho, v norm
+         + (size_t)4 * G * kAttnTile  // scores / probabilities
+         + (size_t)4 * 7 * G + 64;     // running max, sum, rescale; per-warp reductions
+}
+
+// ---------------------------------------------------------------------------
+// Partial: grid (splits, n_kv, batch), 128 threads. Token tiles of 128: thread
+// t scores token t for all G heads; online softmax per head; thread i
+// accumulates coordinate i (and i + 128) of sum_t p_t ||v_t|| level^V_t.
+// ---------------------------------------------------------------------------
+template <int MAXG>
+__global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict__ recs_k,
+                                                      const uint8_t* __restrict__ recs_v, CacheArgs kc,
+                                                      CacheArgs vc, const int32_t* __restrict__ seq_lens,
+                                                      AttnShape s, float* __restrict__ ws,
+                                                      float* __restrict__ scores_out,
+                                                      uint32_t* __restrict__ flags) {
+  extern __shared__ __align__(16) unsigned char sm[];
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int d = s.d, G = s.group;
+  Rec rk = rec_at(recs_k, d, g), rv = rec_at(recs_v, d, g);
+  const RecHeader* hk = rk.hdr();
+  const RecHeader* hv = rv.hdr();
+  float* wq = ws;
+  float* uq = ws + (size_t)s.batch * s.n_q * d;
+  float* acc_out = uq + (size_t)s.batch * s.n_q * d;
+  float* ml_out = acc_out + (size_t)s.batch * s.n_q * s.splits * d;
+  const bool ok = record_ok(hk, d) && record_ok(hv, d) && hk->words == kc.words && hv->words == vc.words &&
+                  (hk->m == 0 || kc.rnorm != nullptr);
+  int64_t L = seq_lens[b];
+  if (L < 0 || L > s.max_ctx || L > kc.cap) {
+    if (tid == 0 && split == 0 && g == 0 && flags) atomicOr(flags, SQ_FLAG_SEQLEN);
+    L = L < 0 ? 0 : (L > s.max_ctx ? s.max_ctx : L);
+    L = L > kc.cap ? kc.cap : L;
+  }
+  if (!ok) {
+    if (tid == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
+    L = 0;
+  }
+  const int64_t t_lo = (int64_t)split * s.chunk;
+  const int64_t t_hi = min(L, t_lo + s.chunk);
+  const int m = ok ? hk->m : 0;
+  const int wk = kc.words, wv = vc.words, kcb = ok ? hk->code_bits : 0;
+
+  unsigned char* p = sm;
+  float* w = (float*)p;        p += (size_t)4 * G * d;
+  float* u = (float*)p;        p += (size_t)4 * G * d;
+  float* lv = (float*)p;       p += (size_t)4 * kLevelsTotal;
+  int* kb = (int*)p;           p += (size_t)4 * d;
+  int* ko = (int*)p;           p += (size_t)4 * d;
+  int* vb = (int*)p;           p += (size_t)4 * d;
+  int* vo = (int*)p;           p += (size_t)4 * d;
+  p += (size_t)4 * d;
+  uint32_t* kw = (uint32_t*)p; p += (size_t)4 * kAttnTile * (wk + 1);
+  uint32_t* vw = (uint32_t*)p; p += (size_t)4 * kAttnTile * (wv + 1);
+  float* kn = (float*)p;       p += (size_t)4 * kAttnTile;
+  float* kr = (float*)p;       p += (size_t)4 * kAttnTile;
+  float* vn = (float*)p;       p += (size_t)4 * kAttnTile;
+  float* sc = (float*)p;       p += (size_t)4 * G * kAttnTile;
+  float* mrun = (float*)p;     p += (size_t)4 * G;
+  float* lrun = (float*)p;     p += (size_t)4 * G;
+  float* alpha = (float*)p;    p += (size_t)4 * G;
+  float* red = (float*)p;
+
+  const size_t qbase = ((size_t)b * s.n_q + (size_t)g * G);
+  for (int e = tid; e < G * d; e += blockDim.x) w[e] = wq[qbase * d + e];
+  for (int e = tid; e < G * m; e += blockDim.x) u[e] = uq[(qbase + e / m) * d + e % m];
+  for (int e = tid; e < kLevelsTotal; e += blockDim.x) lv[e] = c_lv32[e];
+  if (ok)
+    for (int i = tid; i < d; i += blockDim.x) {
+      kb[i] = rk.bits()[i]; ko[i] = rk.offsets()[i];
+      vb[i] = rv.bits()[i]; vo[i] = rv.offsets()[i];
+    }
+  for (int hh = tid; hh < G; hh += blockDim.x) { mrun[hh] = -INFINITY; lrun[hh] = 0.0f; }
+  float oacc[MAXG][2];
+#pragma unroll
+  for (int hh = 0; hh < MAXG; ++hh) oacc[hh][0] = oacc[hh][1] = 0.0f;
+  __syncthreads();
+
+  const size_t row = (size_t)b * s.n_kv + g;
+  const uint32_t* kcodes = kc.codes + row * kc.cap * wk;
+  const uint32_t* vcodes = vc.codes + row * vc.cap * wv;
+  for (int64_t t0 = t_lo; t0 < t_hi; t0 += kAttnTile) {
+    const int nt = (int)min((int64_t)kAttnTile, t_hi - t0);
+    for (int e = tid; e < nt * wk; e += blockDim.x) kw[(e / wk) * (wk + 1) + e % wk] = kcodes[t0 * wk + e];
+    for (int e = tid; e < nt * wv; e += blockDim.x) vw[(e / wv) * (wv + 1) + e % wv] = vcodes[t0 * wv + e];
+    if (tid < nt) {
+      kn[tid] = kc.norm[row * kc.cap + t0 + tid];
+      kr[tid] = m > 0 ? kc.rnorm[row * kc.cap + t0 + tid] : 0.0f;
+      vn[tid] = vc.norm[row * vc.cap + t0 + tid];
+    }
+    __syncthreads();
+    // Scores: thread tid <-> token t0 + tid.
+    {
+      float a[MAXG];
+#pragma unroll
+      for (int hh = 0; hh < MAXG; ++hh) a[hh] = 0.0f;
+      if (tid < nt) {
+        const uint32_t* rw = kw + tid * (wk + 1);
+        for (int i = 0; i < d; ++i) {
+          int bw = kb[i];
+          if (bw == 0) continue;
+          float lvv = lv[lv_off(bw) + (int)field(rw, ko[i], bw)];
+#pragma unroll
+          for (int hh = 0; hh < MAXG; ++hh)
+            if (hh < G) a[hh] = fmaf(w[hh * d + i], lvv, a[hh]);
+        }
+        if (m > 0) {
+          float qa[MAXG];
+#pragma unroll
+          for (int hh = 0; hh < MAXG; ++hh) qa[hh] = 0.0f;
+          for (int j = 0; j < m; ++j) {
+            int o = kcb + j;
+            float sg = ((rw[o >> 5] >> (o & 31)) & 1u) ? 1.0f : -1.0f;
+#pragma unroll
+            for (int hh = 0; hh < MAXG; ++hh)
+              if (hh < G) qa[hh] = fmaf(u[hh * m + j], sg, qa[hh]);
+          }
+#pragma unroll
+          for (int hh = 0; hh < MAXG; ++hh) a[hh] = fmaf(kr[tid], qa[hh], a[hh]);
+        }
+      }
+      for (int hh = 0; hh < G; ++hh) {
+        float sv = tid < nt ? kn[tid] * a[hh] : -INFINITY;
+        sc[hh * kAttnTile + tid] = sv;
+        if (scores_out && tid < nt) scores_out[((size_t)b * s.n_q + g * G + hh) * s.max_ctx + t0 + tid] = sv;
+      }
+    }
+    __syncthreads();
+    // Online softmax: tile max per head, then probabilities and their sum.
+    for (int hh = 0; hh < G; ++hh) {
+      float v = warp_max(sc[hh * kAttnTile + tid]);
+      if ((tid & 31) == 0) red[hh * 4 + (tid >> 5)] = v;
+    }
+    __syncthreads();
+    for (int hh = tid; hh < G; hh += blockDim.x) {
+      float tm = fmaxf(fmaxf(red[hh * 4], red[hh * 4 + 1]), fmaxf(red[hh * 4 + 2], red[hh * 4 + 3]));
+      float mn = fmaxf(mrun[hh], tm);
+      alpha[hh] = (mrun[hh] == -INFINITY) ? 0.0f : __expf(mrun[hh] - mn);
+      mrun[hh] = mn;
+    }
+    __syncthreads();
+    for (int hh = 0; hh < G; ++hh) {
+      float pv = tid < nt ? __expf(sc[hh * kAttnTile + tid] - mrun[hh]) : 0.0f;
+      float ps = warp_sum(pv);
+      sc[hh * kAttnTile + tid] = pv * (tid < nt ? vn[tid] : 0.0f);
+      if ((tid & 31) == 0) red[hh * 4 + (tid >> 5)] = ps;
+    }
+    __syncthreads();
+    for (int hh = tid; hh < G; hh += blockDim.x)
+      lrun[hh] = lrun[hh] * alpha[hh] + (red[hh * 4] + red[hh * 4 + 1] + red[hh * 4 + 2] + red[hh * 4 + 3]);
+    // PV: thread tid <-> coordinates tid and tid + 128.
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+      int i = tid + c2 * kAttnTile;
+      if (i >= d) break;
+#pragma unroll
+      for (int hh = 0; hh < MAXG; ++hh)
+        if (hh < G) oacc[hh][c2] *= alpha[hh];
+      int bw = vb[i];
+      if (bw == 0) continue;
+      int o = vo[i];
+      for (int t = 0; t < nt; ++t) {
+        float lvv = lv[lv_off(bw) + (int)field(vw + t * (wv + 1), o, bw)];
+#pragma unroll
+        for (int hh = 0; hh < MAXG; ++hh)
+          if (hh < G) oacc[hh][c2] = fmaf(sc[hh * kAttnTile + t], lvv, oacc[hh][c2]);
+      }
+    }
+    __syncthreads();
+  }
+  // Partial results of this split.
+  for (int hh = 0; hh < G; ++hh) {
+    size_t base = ((qbase + hh) * s.splits + split);
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+      int i = tid + c2 * kAttnTile;
+      if (i < d) acc_out[base * d + i] = oacc[hh][c2];
+    }
+    if (tid == 0) {
+      ml_out[base * 2] = mrun[hh];
+      ml_out[base * 2 + 1] = lrun[hh];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Combine: grid (n_q, batch), 128 threads. a_i = sigma_V,i * sum_s e^(m_s - M)
+// acc_s,i / sum_s e^(m_s - M) l_s; o = V_V a.
+// ---------------------------------------------------------------------------
+template <typename TO>
+__global__ void __launch_bounds__(128) k_attn_combine(const uint8_t* __restrict__ recs_v, AttnShape s,
+                                                      const float* __restrict__ ws, TO* __restrict__ out) {
+  const int h = blockIdx.x, b = blockIdx.y, d = s.d, tid = threadIdx.x;
+  const int g = h / s.group;
+  Rec rv = rec_at(recs_v, d, g);
+  __shared__ float a[kMaxD];
+  __shared__ float sw[256];
+  __shared__ float s_l;
+  const float* acc = ws + (size_t)s.batch * s.n_q * d * 2;
+  const float* ml = acc + (size_t)s.batch * s.n_q * s.splits * d;
+  const size_t qh = (size_t)b * s.n_q + h;
+  float M = -INFINITY;
+  for (int k = 0; k < s.splits; ++k) M = fmaxf(M, ml[(qh * s.splits + k) * 2]);
+  for (int k = tid; k < s.splits; k += blockDim.x) {
+    float mk = ml[(qh * s.splits + k) * 2];
+    sw[k] = (mk == -INFINITY) ? 0.0f : __expf(mk - M);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float l = 0.0f;
+    for (int k = 0; k < s.splits; ++k) l += sw[k] * ml[(qh * s.splits + k) * 2 + 1];
+    s_l = l;
+  }
+  __syncthreads();
+  const float inv_l = s_l > 0.0f ? 1.0f / s_l : 0.0f;
+  const bool ok = record_ok(rv.hdr(), d);
+  const float* sig = rv.sigma_f();
+  for (int i = tid; i < d; i += blockDim.x) {
+    float v = 0.0f;
+    for (int k = 0; k < s.splits; ++k) v = fmaf(sw[k], acc[(qh * s.splits + k) * d + i], v);
+    a[i] = ok ? v * inv_l * sig[i] : 0.0f;
+  }
+  __syncthreads();
+  const float* V = rv.V_f();
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int j = warp; j < d; j += 4) {
+    float v = 0.0f;
+    for (int i = lane; i < d; i += 32) v = fmaf(ok ? V[(size_t)j * d + i] : 0.0f, a[i], v);
+    v = warp_sum(v);
+    if (lane == 0) out[qh * d + j] = from_float<TO>(v);
+  }
+}
+
+}  // namespace sq

@@ -1,0 +1,231 @@
+// Reference-precision codec kernels: compress (rotate, quantize, QJL signs,
+// pack) and decompress.
+//
+// SpectralQuant README, "Overview" (rotation into the calibrated eigenbasis;
+// error correction kept only on the signal dimensions) and "Repository
+// Structure" (spectral_rotation.py, nonuniform_quantization.py: Lloyd-Max
+// codebooks, selective_qjl.py: QJL on the signal dims only).
+//
+// These kernels compute every coordinate in float64 (one warp per vector), so
+// their codes agree with an exact evaluation except within ~1e-13 of a
+// threshold. They serve float32 inputs, head_dim 256, and the decompress path.
+#pragma once
+
+#include "sq_common.cuh"
+
+namespace sq {
+
+constexpr int kCodecWarps = 4;
+
+// Shared-memory bytes of k_compress_ref / k_decompress_ref for head_dim d.
+__host__ __device__ inline size_t codec_ref_smem(int d) {
+  size_t v = d <= 128 ? (size_t)8 * d * (d + 1) : 0;             // V (padded rows) in float64
+  return v + (size_t)8 * (kThreshTotal + kLevelsTotal)             // tables
+         + (size_t)8 * d * 2                                      // sigma, 1/sigma
+         + (size_t)4 * d * 2                                      // bits, offsets
+         + (size_t)kCodecWarps * (8 * d + 4 * kMaxWords + 8 * d);        // per warp: x row, words, residual
+}
+
+// ---------------------------------------------------------------------------
+// Compress: grid (token blocks, heads, batch), 4 warps, one warp per vector.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict__ recs, const T* __restrict__ x,
+                                                      int n_heads, int d, int64_t n_tok, int tok_per_block,
+                                                      const int32_t* __restrict__ start_pos, CacheArgs c,
+                                                      uint32_t* __restrict__ flags) {
+  extern __shared__ __align__(16) unsigned char sm[];
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  Rec rec = rec_at(recs, d, h);
+  const RecHeader* hd = rec.hdr();
+  if (!record_ok(hd, d) || hd->words != c.words || (hd->m > 0 && c.rnorm == nullptr)) {
+    if (threadIdx.x == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
+    return;
+  }
+  const int64_t sp = start_pos ? (int64_t)start_pos[b] : 0;
+  if (sp < 0 || sp + n_tok > c.cap) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && flags) atomicOr(flags, SQ_FLAG_CAPACITY);
+    return;
+  }
+  const bool vsm = d <= 128;
+  const int ld = d + 1;
+  unsigned char* p = sm;
+  double* Vs = (double*)p;            p += vsm ? (size_t)8 * d * ld : 0;
+  double* th = (double*)p;            p += 8 * kThreshTotal;
+  double* lv = (double*)p;            p += 8 * kLevelsTotal;
+  double* sig = (double*)p;           p += 8 * d;
+  double* isig = (double*)p;          p += 8 * d;
+  int* bits = (int*)p;                p += 4 * d;
+  int* offs = (int*)p;                p += 4 * d;
+  double* xs = (double*)p + warp * d;                      p += (size_t)8 * d * kCodecWarps;
+  uint32_t* wb = (uint32_t*)p + warp * kMaxWords;          p += (size_t)4 * kMaxWords * kCodecWarps;
+  double* rs = (double*)p + warp * d;
+
+  const double* Vg = rec.V();
+  if (vsm)
+    for (int e = threadIdx.x; e < d * d; e += blockDim.x) Vs[(e / d) * ld + e % d] = Vg[e];
+  for (int e = threadIdx.x; e < kThreshTotal; e += blockDim.x) th[e] = c_th64[e];
+  for (int e = threadIdx.x; e < kLevelsTotal; e += blockDim.x) lv[e] = c_lv64[e];
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    double s = rec.sigma()[i];
+    sig[i] = s;
+    isig[i] = s > 0.0 ? 1.0 / s : 0.0;
+    bits[i] = rec.bits()[i];
+    offs[i] = rec.offsets()[i];
+  }
+  __syncthreads();
+  const int m = hd->m, W = hd->words, cbits = hd->code_bits;
+  const bool normalize = (hd->flags & kFlagNormalize) != 0;
+  const double* S = rec.S();
+  const int64_t t_begin = (int64_t)blockIdx.x * tok_per_block;
+  const int64_t t_end = min(n_tok, t_begin + tok_per_block);
+  const size_t row = ((size_t)b * n_heads + h);
+  for (int64_t t = t_begin + warp; t < t_end; t += kCodecWarps) {
+    const T* xt = x + (row * n_tok + t) * d;
+    double ss = 0.0;
+    for (int j = lane; j < d; j += 32) {
+      double v = (double)to_float<T>(xt[j]);
+      xs[j] = v;
+      ss += v * v;
+    }
+    for (int w = lane; w < W; w += 32) wb[w] = 0u;
+    ss = warp_sum(ss);
+    __syncwarp();
+    const double nrm = normalize ? sqrt(ss) : 1.0;
+    const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
+    for (int i = lane; i < d; i += 32) {
+      double y = 0.0;
+      if (vsm) {
+        for (int j = 0; j < d; ++j) y = fma(Vs[j * ld + i], xs[j], y);
+      } else {
+        for (int j = 0; j < d; ++j) y = fma(Vg[(size_t)j * d + i], xs[j], y);
+      }
+      y *= inv;
+      int bw = bits[i];
+      int code = 0;
+      if (bw > 0) {
+        code = code_of(y * isig[i], th + th_off(bw), bw);
+        int o = offs[i], wi = o >> 5, sh = o & 31;
+        atomicOr(&wb[wi], (uint32_t)code << sh);
+        if (sh + bw > 32) atomicOr(&wb[wi + 1], (uint32_t)code >> (32 - sh));
+      }
+      if (i < m) rs[i] = y - sig[i] * (bw > 0 ? lv[lv_off(bw) + code] : 0.0);
+    }
+    __syncwarp();
+    float rho = 0.0f;
+    if (m > 0) {
+      double r2 = 0.0;
+      for (int k = lane; k < m; k += 32) r2 += rs[k] * rs[k];
+      r2 = warp_sum(r2);
+      rho = (float)sqrt(r2);
+      for (int j = 0; j < m; ++j) {
+        double pj = 0.0;
+        for (int k = lane; k < m; k += 32) pj = fma(S[j * m + k], rs[k], pj);
+        pj = warp_sum(pj);
+        if (lane == 0 && pj >= 0.0) {
+          int o = cbits + j;
+          atomicOr(&wb[o >> 5], 1u << (o & 31));
+        }
+      }
+    }
+    __syncwarp();
+    const size_t slot = row * c.cap + sp + t;
+    for (int w = lane; w < W; w += 32) c.codes[slot * W + w] = wb[w];
+    if (lane == 0) {
+      c.norm[slot] = (float)nrm;
+      if (c.rnorm) c.rnorm[slot] = rho;
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Decompress: x_hat = norm * V (sigma * level) [+ QJL term]; float32 output.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) k_decompress_ref(const uint8_t* __restrict__ recs, int n_heads, int d,
+                                                        CacheArgs c, int64_t t0, int64_t n_tok, int tok_per_block,
+                                                        int apply_qjl, float* __restrict__ out,
+                                                        uint32_t* __restrict__ flags) {
+  extern __shared__ __align__(16) unsigned char sm[];
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  Rec rec = rec_at(recs, d, h);
+  const RecHeader* hd = rec.hdr();
+  if (!record_ok(hd, d) || hd->words != c.words) {
+    if (threadIdx.x == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
+    return;
+  }
+  if (t0 < 0 || t0 + n_tok > c.cap) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && flags) atomicOr(flags, SQ_FLAG_CAPACITY);
+    return;
+  }
+  const bool vsm = d <= 128;
+  const int ld = d + 1;
+  unsigned char* p = sm;
+  double* Vs = (double*)p;            p += vsm ? (size_t)8 * d * ld : 0;
+  p += 8 * kThreshTotal;
+  double* lv = (double*)p;            p += 8 * kLevelsTotal;
+  double* sig = (double*)p;           p += 8 * d;
+  p += 8 * d;
+  int* bits = (int*)p;                p += 4 * d;
+  int* offs = (int*)p;                p += 4 * d;
+  double* ws = (double*)p + warp * d; p += (size_t)8 * d * kCodecWarps;
+  uint32_t* wb = (uint32_t*)p + warp * kMaxWords;
+
+  const double* Vg = rec.V();
+  if (vsm)
+    for (int e = threadIdx.x; e < d * d; e += blockDim.x) Vs[(e / d) * ld + e % d] = Vg[e];
+  for (int e = threadIdx.x; e < kLevelsTotal; e += blockDim.x) lv[e] = c_lv64[e];
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    sig[i] = rec.sigma()[i];
+    bits[i] = rec.bits()[i];
+    offs[i] = rec.offsets()[i];
+  }
+  __syncthreads();
+  const int m = hd->m, W = hd->words, cbits = hd->code_bits;
+  const bool normalize = (hd->flags & kFlagNormalize) != 0;
+  const double* S = rec.S();
+  const bool qjl = apply_qjl && m > 0 && c.rnorm != nullptr;
+  const int64_t t_begin = (int64_t)blockIdx.x * tok_per_block;
+  const int64_t t_end = min(n_tok, t_begin + tok_per_block);
+  const size_t row = ((size_t)b * n_heads + h);
+  for (int64_t t = t_begin + warp; t < t_end; t += kCodecWarps) {
+    const size_t slot = row * c.cap + t0 + t;
+    for (int w = lane; w < W; w += 32) wb[w] = c.codes[slot * W + w];
+    __syncwarp();
+    for (int i = lane; i < d; i += 32) {
+      int bw = bits[i];
+      ws[i] = bw > 0 ? sig[i] * lv[lv_off(bw) + (int)field(wb, offs[i], bw)] : 0.0;
+    }
+    __syncwarp();
+    if (qjl) {
+      const double rho = (double)c.rnorm[slot];
+      const double coef = kQjlScale / (double)m * rho;
+      for (int k = lane; k < m; k += 32) {
+        double acc = 0.0;
+        for (int j = 0; j < m; ++j) {
+          int o = cbits + j;
+          double s = ((wb[o >> 5] >> (o & 31)) & 1u) ? 1.0 : -1.0;
+          acc = fma(S[j * m + k], s, acc);
+        }
+        ws[k] += coef * acc;
+      }
+      __syncwarp();
+    }
+    const double nrm = normalize ? (double)c.norm[slot] : 1.0;
+    float* ot = out + (row * n_tok + t) * d;
+    for (int j = lane; j < d; j += 32) {
+      double acc = 0.0;
+      if (vsm) {
+        for (int i = 0; i < d; ++i) acc = fma(Vs[j * ld + i], ws[i], acc);
+      } else {
+        for (int i = 0; i < d; ++i) acc = fma(Vg[(size_t)j * d + i], ws[i], acc);
+      }
+      ot[j] = (float)(nrm * acc);
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace sq

@@ -1,0 +1,299 @@
+/*
+ * sq.h -- C ABI of libsq, a CUDA (sm_100a) implementation of the SpectralQuant
+ * compressed-KV hot path: per-head calibration, compression of keys and values
+ * into packed records, decompression, and decode attention straight from the
+ * packed cache.
+ *
+ * The method is described by the SpectralQuant README (Dynamis-Labs/spectralquant):
+ *   - "Overview": keys concentrate their signal in 3-4 % of head_dim; a one-time
+ *     calibration finds those dimensions and error correction is dropped on the
+ *     remaining noise dimensions;
+ *   - "Repository Structure": calibration.py (eigenspectral calibration: PCA,
+ *     d_eff, kappa), spectral_rotation.py (rotation into the calibrated basis),
+ *     nonuniform_quantization.py (Lloyd-Max codebooks), selective_qjl.py (QJL
+ *     correction on the signal dims only);
+ *   - title: "Calibrated Eigenbasis Rotation and Water-Filled Bit Allocation";
+ *   - "Headline Results": compression ratio by bit accounting, decode latency
+ *     per step over the compressed cache;
+ * and by the v1 tests/conftest.py fixture pre_computed_calibration (uncentred
+ * second moment, eigh, descending order, participation-ratio d_eff, gap).
+ *
+ * Conventions (all entry points)
+ * ------------------------------
+ *  - The caller owns all memory. libsq never allocates device memory; calls
+ *    that need scratch take a workspace pointer and a size, with a matching
+ *    *_workspace() query.
+ *  - Device pointers are plain CUDA device addresses; "host" arguments are
+ *    plain host memory. Every call that launches work is asynchronous on the
+ *    given stream and returns once the work is queued.
+ *  - Argument errors are reported synchronously, before any launch:
+ *    SQ_ERR_ARG (bad value / null / misaligned pointer), SQ_ERR_UNSUPPORTED
+ *    (head_dim not in {32, 64, 128, 256}, or a dtype a call does not take),
+ *    SQ_ERR_WORKSPACE (workspace too small). A failed launch returns SQ_ERR_CUDA.
+ *  - Conditions only the device can see (a capacity overflow, a record that
+ *    does not match the cache, a sequence length past the context bound) are
+ *    OR-ed into the optional device word d_flags (SQ_FLAG_*), and the affected
+ *    rows are skipped; the call still returns SQ_OK. No kernel traps.
+ *  - Pointers to device arrays must be 16-byte aligned. Strides are in elements.
+ *  - The library keeps per-device constant tables (the Lloyd-Max codebooks). The
+ *    first launching call on a device uploads them, so make one call (or
+ *    sq_init) before capturing a stream into a CUDA graph.
+ */
+#ifndef SQ_H
+#define SQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sq_stream; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_ARG = 1,
+  SQ_ERR_UNSUPPORTED = 2,
+  SQ_ERR_CUDA = 3,
+  SQ_ERR_NOT_CONVERGED = 4, /* per-head status of sq_calibrate: eigensolver hit max_sweeps */
+  SQ_ERR_CAPACITY = 5,
+  SQ_ERR_WORKSPACE = 6,
+  SQ_ERR_RECORD = 7          /* per-head status: malformed calibration record */
+} sq_status;
+
+typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2 } sq_dtype;
+
+/* Bits of the device flag word. */
+#define SQ_FLAG_CAPACITY 1u   /* start_pos + n_tok > cap (or start_pos < 0): row skipped */
+#define SQ_FLAG_RECORD 2u     /* record magic/version/d/words do not match the call      */
+#define SQ_FLAG_SEQLEN 4u     /* seq_len > max_ctx or > cap, or < 0: row clamped          */
+
+#define SQ_MAX_BITS 8         /* largest code width of one coordinate                     */
+#define SQ_ABI_VERSION 1
+
+/*
+ * Calibration parameters (host struct).
+ *  d              head_dim: 32, 64, 128 or 256.
+ *  n_heads        heads calibrated by one call (e.g. layers x KV heads).
+ *  avg_bits       bits per coordinate; B = avg_bits * d must be a whole number
+ *                 (the record's total bits, QJL bits included).
+ *  is_key         1 for keys (QJL allowed), 0 for values.
+ *  qjl            1: keys store m = d_eff QJL sign bits inside the B bits.
+ *  normalize      1: quantize x/||x|| and store ||x|| (default reading);
+ *                 0: quantize x itself with sigma_i = sqrt(lambda_i).
+ *  d_eff_override 0: m = the participation-ratio d_eff; > 0: m = this value.
+ *  max_bits       cap on one coordinate's code width (1..8).
+ *  seed           seed of the QJL Gaussian streams; head h of the call uses
+ *                 stream h (SplitMix64 state mix(seed ^ mix(h + 1)), 53-bit
+ *                 uniforms in (0,1], Box-Muller pairs).
+ *  max_sweeps     eigensolver sweep limit (e.g. 30).
+ *  tol            eigensolver stop: off-diagonal Frobenius norm <= tol * ||C||_F.
+ */
+typedef struct {
+  int d;
+  int n_heads;
+  double avg_bits;
+  int is_key;
+  int qjl;
+  int normalize;
+  int d_eff_override;
+  int max_bits;
+  uint64_t seed;
+  int max_sweeps;
+  double tol;
+} sq_calib_params;
+
+/*
+ * One packed cache (keys or values of one layer, or of several layers with the
+ * layers folded into the head index). Device arrays, caller-owned:
+ *  codes  uint32 [batch][n_heads][cap][words]   one packed record per token
+ *  norm   float  [batch][n_heads][cap]          ||x|| (1.0 when not normalized)
+ *  rnorm  float  [batch][n_heads][cap]          QJL residual norm rho; NULL when
+ *                                               the records carry no QJL bits
+ *  cap    tokens per (batch, head); a multiple of 16.
+ *  words  32-bit words per record, ceil(B / 32); must equal the records'.
+ *
+ * Record bit layout (the pages fix none; this is the library's reading): stream
+ * bit k of a record is bit k % 32 of word k / 32 (little-endian words). The codes
+ * of coordinates i = 0..d-1 with b_i > 0 come first, in coordinate order, each
+ * least-significant bit first; then the m QJL bits (1 = projection >= 0); then
+ * zero padding up to words * 32 bits.
+ */
+typedef struct {
+  uint32_t* codes;
+  float* norm;
+  float* rnorm;
+  int batch;
+  int n_heads;
+  int64_t cap;
+  int words;
+} sq_cache;
+
+/*
+ * Calibration record of one head: a plain byte block of sq_calib_bytes(d) bytes,
+ * 256-byte aligned when records are stored back to back. Little-endian. The
+ * canonical part can be written by any program; the library derives the rest.
+ *
+ *  offset               type  field
+ *  0                    u32   magic 0x31435153 ("SQC1")
+ *  4                    u32   version 1
+ *  8                    i32   d
+ *  12                   i32   d_eff (participation ratio (sum l)^2 / sum l^2, rounded half to even)
+ *  16                   i32   m (QJL sign dimensions, 0 without QJL)
+ *  20                   i32   total_bits B
+ *  24                   i32   code_bits = sum of b_i = B - m
+ *  28                   i32   words = ceil(B / 32)
+ *  32                   u32   flags: 1 key, 2 QJL, 4 normalized
+ *  36                   i32   eigensolver sweeps used
+ *  40                   i32   stream (head index of the QJL Gaussian stream)
+ *  44                   i32   max_bits
+ *  48                   u64   seed
+ *  56                   f64   trace (sum of eigenvalues)
+ *  64                   f64   kappa = lambda[d_eff-1] / lambda[d_eff], +inf if d_eff = d
+ *  72                   f64   avg_bits
+ *  80                   u32   library use: nonzero once the derived part is built
+ *  84..127                    zero
+ *  128                  f64   lambda[d], descending, >= 0
+ *  128 + 8d             f64   sigma[d]: normalized sqrt(lambda_i / trace), else sqrt(lambda_i)
+ *  128 + 16d            f64   V[d*d], row-major; V[j*d + i] = component j of eigenvector i,
+ *                             whose largest-magnitude component is positive
+ *  128 + 16d + 8d^2     f64   S[d*d]: the m x m QJL matrix, row-major, in the first m*m slots
+ *  128 + 16d + 16d^2    u8    bits[d]: code width b_i (greedy water-filling)
+ *  128 + 17d + 16d^2    i32   offset[d]: bit position of coordinate i's code
+ *  then, from the next 256-byte boundary: the library's derived part (private).
+ */
+size_t sq_calib_bytes(int d);
+
+/* ABI version (SQ_ABI_VERSION). */
+int sq_abi_version(void);
+
+/* Static string naming a status. Never NULL. */
+const char* sq_status_str(sq_status s);
+
+/* Words of one record for these parameters: ceil(avg_bits * d / 32); 0 if invalid. */
+int sq_record_words(const sq_calib_params* p);
+
+/*
+ * Gaussian N(0,1) Lloyd-Max quantizer of b bits (1..8), computed by the library
+ * on the host (README "Repository Structure": nonuniform_quantization.py,
+ * Lloyd-Max codebooks). levels: host array of 2^b doubles, ascending;
+ * thresholds: host array of 2^b - 1 doubles (midpoints of adjacent levels);
+ * D: host double, E[(Z - Q(Z))^2]. Any output pointer may be NULL.
+ * Returns SQ_ERR_ARG for b outside 1..8. Host-only; touches no GPU.
+ */
+sq_status sq_codebook(int b, double* levels, double* thresholds, double* D);
+
+/*
+ * Uploads the per-device constant tables to the current device (done lazily by
+ * every launching call otherwise). Call once per device before stream capture.
+ */
+sq_status sq_init(void);
+
+/* Workspace bytes sq_calibrate needs for these parameters and n_tokens. */
+size_t sq_calibrate_workspace(const sq_calib_params* p, int64_t n_tokens);
+
+/*
+ * Calibrates p->n_heads heads from their calibration vectors (README "Overview":
+ * one-time calibration; conftest fixture pre_computed_calibration).
+ *  x            device, dtype elements; element j of token t of head h at
+ *               x + h * stride_head + t * stride_tok + j.
+ *  n_tokens     calibration tokens per head (>= 1).
+ *  calib_out    device, n_heads records of sq_calib_bytes(d) bytes back to back.
+ *  ws, ws_bytes device workspace of at least sq_calibrate_workspace() bytes.
+ *  d_status     device int[n_heads] (may be NULL): SQ_OK, SQ_ERR_NOT_CONVERGED
+ *               (the record is still written from the last sweep) or SQ_ERR_ARG
+ *               (the budget cannot hold m QJL bits and the codes).
+ * Steps: C = X^T X / N (uncentred, float64 accumulation); cyclic Jacobi on C;
+ * eigenvalues sorted descending, clamped at 0, eigenvector signs fixed; d_eff,
+ * kappa, sigma; greedy water-filling of B - m code bits by the distortion drop
+ * lambda_i (D(b_i) - D(b_i + 1)), ties to the lowest index; offsets; the QJL
+ * matrix from the seed.
+ */
+sq_status sq_calibrate(const sq_calib_params* p, const void* x, sq_dtype dtype, int64_t n_tokens,
+                       int64_t stride_head, int64_t stride_tok, void* calib_out, void* ws,
+                       size_t ws_bytes, int* d_status, sq_stream stream);
+
+/*
+ * Imports n_heads records whose canonical part was written elsewhere (saved
+ * records, or another implementation): checks each header (magic, version,
+ * d, bit counts, offsets) and builds the library's derived part.
+ *  calib     device, n_heads records of sq_calib_bytes(d) bytes.
+ *  d_status  device int[n_heads] (may be NULL): SQ_OK or SQ_ERR_RECORD.
+ */
+sq_status sq_calib_import(void* calib, int n_heads, int d, int* d_status, sq_stream stream);
+
+/*
+ * Compresses keys and/or values into packed caches (README "Overview" and
+ * "Repository Structure": rotation into the calibrated eigenbasis, Lloyd-Max
+ * codes under the water-filled widths, QJL sign bits of the key residual on
+ * the top-m signal dimensions).
+ *  calib_k, calib_v  device, n_heads records each (either side may be NULL
+ *                    together with its input and cache).
+ *  k, v        device, dtype [batch][n_heads][n_tok][d], contiguous.
+ *  dtype       SQ_F32, SQ_F16 or SQ_BF16 (converted exactly to float).
+ *  d_start_pos device int32[batch]: first cache slot written for each row
+ *              (NULL = 0). Appending one decode token is n_tok = 1 at the
+ *              row's current length.
+ *  kc, vc      host structs describing the caches (device arrays inside).
+ *  d_flags     device uint32 (may be NULL): SQ_FLAG_CAPACITY, SQ_FLAG_RECORD.
+ * Per vector: norm = ||x||; u = x / norm; y = V^T u; z_i = y_i / sigma_i;
+ * code_i = number of b_i-bit thresholds strictly below z_i; keys with QJL:
+ * r = y[0:m] - sigma[0:m] * level(code[0:m]), rnorm = ||r||, bit j = [(S r)_j >= 0].
+ * n_tok = 0 is a no-op.
+ */
+sq_status sq_compress_kv(const void* calib_k, const void* calib_v, const void* k, const void* v,
+                         sq_dtype dtype, int batch, int n_heads, int d, int64_t n_tok,
+                         const int32_t* d_start_pos, const sq_cache* kc, const sq_cache* vc,
+                         uint32_t* d_flags, sq_stream stream);
+
+/*
+ * Reconstructs vectors from a packed cache: x_hat = norm * V (sigma * level(code)),
+ * plus, when apply_qjl and the records carry QJL bits,
+ * norm * V[:, 0:m] (sqrt(pi/2) / m * rnorm * S^T s), s_j = 2 bit_j - 1.
+ *  calib  device, cache->n_heads records of head_dim d.
+ *  t0, n_tok  token window [t0, t0 + n_tok) of every (batch, head); must lie
+ *         inside [0, cap) (else SQ_FLAG_CAPACITY and nothing is written).
+ *  out    device float [batch][n_heads][n_tok][d].
+ *  d_flags device uint32 (may be NULL): SQ_FLAG_CAPACITY, SQ_FLAG_RECORD.
+ */
+sq_status sq_decompress_kv(const void* calib, const sq_cache* cache, int d, int64_t t0, int64_t n_tok,
+                           int apply_qjl, float* out, uint32_t* d_flags, sq_stream stream);
+
+/* Workspace bytes sq_attn_decode needs for this shape. */
+size_t sq_attn_workspace(int batch, int n_q_heads, int n_kv_heads, int d, int64_t max_ctx);
+
+/*
+ * Decode attention over packed caches (README "Headline Results": per-step
+ * decode latency over the compressed cache). For batch row b and query head h,
+ * KV head g = h / (n_q_heads / n_kv_heads), L = seq_lens[b]:
+ *   q' = V_K^T q;
+ *   s_t = scale * ||k_t|| * (sum_i q'_i sigma_i level_t,i
+ *                            + sqrt(pi/2) / m * rho_t * sum_j (S q'[0:m])_j (2 bit_t,j - 1));
+ *   p = softmax_t(s_t), t < L;  o = V_V (sigma_V * sum_t p_t ||v_t|| level^V_t).
+ * This is dense softmax attention over the decompressed keys (with their QJL
+ * term) and values (without one).
+ *  calib_k, calib_v  device, n_kv_heads records each.
+ *  kc, vc       packed caches with n_heads = n_kv_heads.
+ *  d_seq_lens   device int32[batch]; each <= max_ctx and <= cap.
+ *  max_ctx      host bound on the sequence lengths (sizes the split of work).
+ *  q            device, q_dtype [batch][n_q_heads][d].
+ *  scale        > 0, or <= 0 for 1/sqrt(d).
+ *  out          device, out_dtype [batch][n_q_heads][d].
+ *  scores_out   device float [batch][n_q_heads][max_ctx] (may be NULL): s_t for
+ *               t < L; entries past L are left unwritten.
+ *  ws, ws_bytes device workspace of at least sq_attn_workspace() bytes.
+ *  d_flags      device uint32 (may be NULL): SQ_FLAG_SEQLEN, SQ_FLAG_RECORD.
+ * A row with L = 0 produces zeros.
+ */
+sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cache* kc,
+                         const sq_cache* vc, const int32_t* d_seq_lens, int batch, int n_q_heads,
+                         int n_kv_heads, int d, int64_t max_ctx, const void* q, sq_dtype q_dtype,
+                         float scale, void* out, sq_dtype out_dtype, float* scores_out, void* ws,
+                         size_t ws_bytes, uint32_t* d_flags, sq_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H */

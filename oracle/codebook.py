@@ -134,7 +134,7 @@ def _accelerated_positive_half(b: int, tol: float):
 
 
 @functools.lru_cache(maxsize=None)
-def lloyd_max(b: int, tol: float = 1e-13):
+def lloyd_max(b: int, tol: float = 1e-15):
     """Gaussian Lloyd-Max quantizer of ``b`` bits.
 
     Returns ``(levels, thresholds, distortion)``: 2**b ascending levels,

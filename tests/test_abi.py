@@ -1,0 +1,86 @@
+"""The C-ABI library: it loads without a GPU, exports every entry point the
+public header declares, and its host-only calls behave as documented."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from compressed_attention_head_b200 import build as sqbuild
+from compressed_attention_head_b200 import sq
+from oracle import codebook as ocb
+from oracle import record as orec
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(sq_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def libsq():
+    sqbuild.build()
+    return sq.lib()
+
+
+def test_exports_every_declared_symbol(libsq):
+    declared = _declared()
+    assert {"sq_calibrate", "sq_compress_kv", "sq_decompress_kv", "sq_attn_decode"} <= declared
+    for name in declared:
+        assert hasattr(libsq, name), name
+        assert name in sq._SIGNATURES, f"binding misses {name}"
+
+
+def test_status_strings_and_version(libsq):
+    assert sq.sq_abi_version() == 1
+    for s in range(8):
+        assert sq.sq_status_str(s) and "unknown" not in sq.sq_status_str(s)
+    assert "unknown" in sq.sq_status_str(99)
+
+
+def test_record_geometry_matches_the_documented_layout(libsq):
+    for d in (32, 64, 128, 256):
+        n = sq.sq_calib_bytes(d)
+        assert n % 256 == 0 and n >= orec.canonical_bytes(d)
+    assert sq.sq_calib_bytes(48) == 0
+
+
+def test_record_words(libsq):
+    assert sq.sq_record_words(sq.calib_params(128, 1, 2.5, True)) == 10
+    assert sq.sq_record_words(sq.calib_params(128, 1, 3.0, True)) == 12
+    assert sq.sq_record_words(sq.calib_params(256, 1, 3.5, False)) == 28
+    assert sq.sq_record_words(sq.calib_params(32, 1, 3.01, False)) == 0     # not a whole number of bits
+    assert sq.sq_record_words(sq.calib_params(40, 1, 3.0, False)) == 0     # unsupported head_dim
+
+
+def test_library_codebook_matches_oracle(libsq):
+    for b in range(1, 9):
+        lv, th, dist = sq.sq_codebook(b)
+        l2, t2, d2 = ocb.lloyd_max(b)
+        assert np.max(np.abs(lv - l2)) < 1e-10
+        assert np.max(np.abs(th - t2)) < 1e-10
+        assert abs(dist - d2) < 1e-14
+    assert sq.lib().sq_codebook(0, None, None, None) == sq.SQ_ERR_ARG
+    assert sq.lib().sq_codebook(9, None, None, None) == sq.SQ_ERR_ARG
+
+
+def test_argument_errors_need_no_gpu(libsq):
+    L = sq.lib()
+    p = sq.calib_params(48, 1, 3.0, True)
+    assert L.sq_calibrate(ctypes.byref(p), None, 0, 16, 0, 48, None, None, 0, None, None) == sq.SQ_ERR_UNSUPPORTED
+    p = sq.calib_params(32, 1, 3.0, True)
+    assert L.sq_calibrate(ctypes.byref(p), None, 0, 16, 0, 32, None, None, 0, None, None) == sq.SQ_ERR_ARG
+    assert L.sq_calib_import(None, 1, 32, None, None) == sq.SQ_ERR_ARG
+    assert L.sq_compress_kv(None, None, None, None, 1, 1, 1, 32, 0, None, None, None, None, None) == sq.SQ_OK
+    assert L.sq_compress_kv(None, None, None, None, 1, 1, 1, 32, 4, None, None, None, None, None) == sq.SQ_ERR_ARG
+    assert L.sq_attn_workspace(1, 3, 2, 128, 100) > 0
+    assert L.sq_attn_workspace(1, 1, 1, 100, 100) == 0

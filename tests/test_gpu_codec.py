@@ -1,0 +1,164 @@
+"""GPU parity of compress / decompress / append against the oracle.
+
+The oracle's calibration records are imported into the library (the
+eigenvectors of a degenerate noise subspace are not unique, so compression
+parity is checked on one shared calibration; the GPU calibration itself is
+checked separately by invariants). Inputs come from the seeded synthetic
+generators; nothing the oracle reads comes from the CUDA path except the
+packed cache that decompress and attention parity feed it on purpose.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import (TOL_RECON, calibrate_oracle, compare_compressed, records_to_device, rel_l2_rows)
+from oracle import codec as ocodec
+from synthetic import CONFIGS, make_workload
+
+pytestmark = pytest.mark.gpu
+
+cuda = pytest.importorskip("torch").cuda
+if not cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+from compressed_attention_head_b200 import sq  # noqa: E402
+
+
+def _case(name, batch=2, tokens=333, heads=None, bits_k=None, bits_v=None, qjl=True, normalize=True):
+    w = make_workload(name, batch=batch, tokens=tokens)
+    cfg = w.cfg
+    nh = heads or cfg["n_kv"]
+    bk = cfg["bits_k"] if bits_k is None else bits_k
+    bv = cfg["bits_v"] if bits_v is None else bits_v
+    ck = calibrate_oracle(w.k_cal[:nh], bk, True, qjl=qjl, normalize=normalize)
+    cv = calibrate_oracle(w.v_cal[:nh], bv, False, normalize=normalize)
+    k = w.k[:, :nh].contiguous()
+    v = w.v[:, :nh].contiguous()
+    return w, ck, cv, k, v, nh
+
+
+def _compress(ck, cv, k, v, cap=None, start=None, flags=None):
+    batch, nh, t, d = k.shape
+    rk = records_to_device(ck)
+    rv = records_to_device(cv)
+    cap = cap or t
+    kc = sq.alloc_cache(batch, nh, cap, ck[0].words, ck[0].m > 0)
+    vc = sq.alloc_cache(batch, nh, cap, cv[0].words, False)
+    sp = None if start is None else torch.tensor(start, dtype=torch.int32, device="cuda")
+    sq.sq_compress_kv(rk, rv, k.cuda(), v.cuda(), batch, nh, d, t, sp, kc, vc, flags)
+    torch.cuda.synchronize()
+    return rk, rv, kc, vc
+
+
+def _check_side(cache, cals, x, t0=0):
+    words = cache.words_u32()
+    norm = cache.norm.cpu().numpy()
+    rn = cache.rnorm.cpu().numpy() if cache.rnorm is not None else None
+    n_ex = 0
+    t = x.shape[2]
+    for b in range(x.shape[0]):
+        for h in range(x.shape[1]):
+            xs = x[b, h].double().cpu().numpy()
+            e1, e2 = compare_compressed(words[b, h, t0:t0 + t], norm[b, h, t0:t0 + t],
+                                        rn[b, h, t0:t0 + t] if rn is not None else None, xs, cals[h])
+            n_ex += e1 + e2
+    return n_ex
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama8b", "qwen14b", "qwen1_5b_long", "gemma9b_sweep"])
+def test_compress_parity_configs(name):
+    heads = None if name in ("tiny", "llama8b") else 4
+    w, ck, cv, k, v, nh = _case(name, heads=heads, tokens=333 if name != "tiny" else 256,
+                                batch=2 if name != "tiny" else 1)
+    _, _, kc, vc = _compress(ck, cv, k, v)
+    ex = _check_side(kc, ck, k) + _check_side(vc, cv, v)
+    total = k.numel() + v.numel()
+    assert ex < 1e-3 * total
+
+
+@pytest.mark.parametrize("bits", [2.0, 2.5, 3.0, 3.5, 4.0])
+@pytest.mark.parametrize("qjl", [True, False])
+def test_gemma_bit_sweep_parity(bits, qjl):
+    w, ck, cv, k, v, nh = _case("gemma9b_sweep", batch=1, tokens=130, heads=2, bits_k=bits, bits_v=bits, qjl=qjl)
+    _, _, kc, vc = _compress(ck, cv, k, v)
+    _check_side(kc, ck, k)
+    _check_side(vc, cv, v)
+    assert (kc.rnorm is not None) == qjl
+
+
+def test_unnormalized_mode_parity():
+    w, ck, cv, k, v, nh = _case("llama8b", batch=1, tokens=100, heads=2, normalize=False)
+    _, _, kc, vc = _compress(ck, cv, k, v)
+    _check_side(kc, ck, k)
+    _check_side(vc, cv, v)
+    assert torch.all(kc.norm[:, :, :100] == 1.0)
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen14b", "gemma9b_sweep"])
+def test_decompress_parity(name):
+    w, ck, cv, k, v, nh = _case(name, batch=1, tokens=150, heads=2)
+    rk, rv, kc, vc = _compress(ck, cv, k, v)
+    d = k.shape[-1]
+    for cache, cals, recs, qjl in ((kc, ck, rk, True), (kc, ck, rk, False), (vc, cv, rv, False)):
+        out = torch.empty(1, nh, 150, d, device="cuda")
+        sq.sq_decompress_kv(recs, cache, d, 0, 150, qjl, out)
+        torch.cuda.synchronize()
+        words = cache.words_u32()
+        for h in range(nh):
+            ref = ocodec.decompress(words[0, h, :150], cache.norm[0, h, :150].cpu().numpy(),
+                                    cache.rnorm[0, h, :150].cpu().numpy() if cache.rnorm is not None else None,
+                                    cals[h], apply_qjl=qjl)
+            err = rel_l2_rows(out[0, h].cpu().numpy(), ref)
+            assert np.max(err) <= TOL_RECON, (name, h, np.max(err))
+
+
+def test_append_decode_tokens_at_start_pos():
+    """One new token per row written at each row's own position (ragged lengths)."""
+    w, ck, cv, k, v, nh = _case("qwen14b", batch=3, tokens=1, heads=2)
+    start = [5, 0, 47]
+    _, _, kc, vc = _compress(ck, cv, k, v, cap=64, start=start)
+    words = kc.words_u32()
+    for b, s in enumerate(start):
+        for h in range(nh):
+            compare_compressed(words[b, h, s:s + 1], kc.norm[b, h, s:s + 1].cpu().numpy(),
+                               kc.rnorm[b, h, s:s + 1].cpu().numpy(), k[b, h].double().numpy(), ck[h])
+            # untouched slots stay zero
+            others = np.delete(np.arange(64), s)
+            assert np.all(words[b, h, others] == 0)
+
+
+def test_zero_tokens_is_noop_and_capacity_flag():
+    w, ck, cv, k, v, nh = _case("tiny", batch=1, tokens=32, heads=2)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rk, rv, kc, vc = _compress(ck, cv, k[:, :, :0], v[:, :, :0], cap=32, flags=flags)
+    assert flags.item() == 0 and torch.all(kc.codes == 0)
+    # 32 tokens at start 16 into a 32-slot cache overflow: flagged, nothing written
+    _, _, kc2, _ = _compress(ck, cv, k, v, cap=32, start=[16], flags=flags)
+    assert flags.item() & sq.SQ_FLAG_CAPACITY
+    assert torch.all(kc2.codes == 0)
+
+
+def test_record_mismatch_flag():
+    w, ck, cv, k, v, nh = _case("tiny", batch=1, tokens=16, heads=1)
+    rk = records_to_device(ck)
+    kc = sq.alloc_cache(1, 1, 16, ck[0].words + 1, True)       # wrong word count
+    vc = sq.alloc_cache(1, 1, 16, cv[0].words, False)
+    rv = records_to_device(cv)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sq.sq_compress_kv(rk, rv, k.cuda(), v.cuda(), 1, 1, 32, 16, None, kc, vc, flags)
+    torch.cuda.synchronize()
+    assert flags.item() & sq.SQ_FLAG_RECORD
+    assert torch.all(kc.codes == 0)
+
+
+def test_argument_errors():
+    w, ck, cv, k, v, nh = _case("tiny", batch=1, tokens=16, heads=1)
+    rk = records_to_device(ck)
+    kc = sq.alloc_cache(1, 1, 16, ck[0].words, True)
+    with pytest.raises(sq.SqError) as e:
+        sq.sq_compress_kv(rk, None, k.cuda(), None, 1, 1, 48, 16, None, kc, None)
+    assert e.value.status == sq.SQ_ERR_UNSUPPORTED
+    with pytest.raises(sq.SqError) as e:
+        sq.sq_compress_kv(rk, None, k.cuda(), None, 2, 1, 32, 16, None, kc, None)   # batch mismatch
+    assert e.value.status == sq.SQ_ERR_ARG
