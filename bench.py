@@ -47,13 +47,16 @@ def _peaks():
 
 
 # --------------------------------------------------------------------------- workload
-def build_workload(name: str, device: str):
+def build_workload(name: str, device: str, layers: int | None = None):
     """All layers of one replica, layers folded into the head index."""
     import torch
 
     from synthetic import CONFIGS, make_workload
 
-    cfg = CONFIGS[name]
+    cfg = dict(CONFIGS[name])
+    cfg["name"] = name
+    if layers:
+        cfg["layers"] = layers
     L, nkv, nq, d = cfg["layers"], cfg["n_kv"], cfg["n_q"], cfg["d"]
     T = cfg["ctx"]
     ks, vs, kcal, vcal, qs, kn, vn = [], [], [], [], [], [], []
@@ -76,6 +79,18 @@ def record_bytes_per_token(cfg, words_k, words_v, qjl):
     k_out = 4 * words_k + 4 + (4 if qjl else 0)
     v_out = 4 * words_v + 4
     return kin + k_out, kin + v_out, k_out, v_out
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The largest per-rank value (elapsed time) across the process group."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 # --------------------------------------------------------------------------- clocks
@@ -247,6 +262,8 @@ def workload_config(cfg, world):
 
 def cfg_name(cfg):
     from synthetic import CONFIGS
+    if "name" in cfg:
+        return cfg["name"]
     for k, v in CONFIGS.items():
         if v is cfg:
             return k
@@ -263,7 +280,7 @@ def run_gpu(args, rank, world, local_rank):
     dev = f"cuda:{local_rank}"
     torch.cuda.set_device(local_rank)
     sq.sq_init()
-    wl = build_workload(args.config, dev)
+    wl = build_workload(args.config, dev, args.layers)
     cfg, H, HQ, d, T, B = wl["cfg"], wl["H"], wl["HQ"], wl["d"], wl["T"], wl["batch"]
     prefill = cfg["mode"] == "prefill"
     stream = torch.cuda.current_stream()
@@ -331,11 +348,7 @@ def run_gpu(args, rank, world, local_rank):
     t_end.record()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    elapsed = t_start.elapsed_time(t_end) / 1e3
-    if world > 1:
-        tt = torch.tensor([elapsed], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed = tt.item()
+    elapsed = max_over_ranks(t_start.elapsed_time(t_end) / 1e3, dev)
     per_step = elapsed / args.steps
     if prefill:
         ck_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
@@ -397,11 +410,7 @@ def run_gpu(args, rank, world, local_rank):
             e2e_step()
         b.record()
         torch.cuda.synchronize()
-        t_e2e = a.elapsed_time(b) / 1e3
-        if world > 1:
-            tt = torch.tensor([t_e2e], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            t_e2e = tt.item()
+        t_e2e = max_over_ranks(a.elapsed_time(b) / 1e3, dev)
         h2d = (hk.numel() * hk.element_size() + hv.numel() * hv.element_size() if prefill else 0) + \
             hkn.numel() * hkn.element_size() + hvn.numel() * hvn.element_size() + hq.numel() * hq.element_size()
         e2e = {"value": tokens / (t_e2e / args.steps), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -442,6 +451,7 @@ def main():
     ap.add_argument("--impl", default="sq", choices=["sq", "reference"])
     ap.add_argument("--config", default="llama8b")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling captures only)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=4096)
     ap.add_argument("--cpu-ctx", type=int, default=2049)

@@ -11,9 +11,13 @@ __constant__ float c_lv32[kLevelsTotal];
 __constant__ double c_D[SQ_MAX_BITS + 1];
 }  // namespace sq
 
+#include <cudaTypedefs.h>
+
 #include "attention.cuh"
 #include "calibrate.cuh"
 #include "codec.cuh"
+#include "fast_attn.cuh"
+#include "tc_compress.cuh"
 
 namespace sq {
 
@@ -25,6 +29,9 @@ namespace {
 
 std::mutex g_mu;
 bool g_ready[128];
+bool g_force_ref = false;   // route compress to the float64 reference kernel
+bool g_attn_ref = false;    // route attention partials to the SIMT kernel
+int g_eacc_units = 128;     // accumulation bound of the tensor-core compress radius, in 2^-24
 int g_sms[128];
 
 bool supported_d(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
@@ -67,6 +74,10 @@ sq_status ensure_init(int* dev_out = nullptr) {
   cudaFuncSetAttribute(k_attn_partial<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   cudaFuncSetAttribute(k_attn_partial<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   cudaFuncSetAttribute(k_attn_partial<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  cudaFuncSetAttribute(tcc::k_compress_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, tcc::SMEM_BYTES);
+  cudaFuncSetAttribute(fa::k_attn_partial_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::smem_bytes<64>());
+  cudaFuncSetAttribute(fa::k_attn_partial_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::smem_bytes<128>());
+  cudaFuncSetAttribute(fa::k_attn_partial_tc<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::smem_bytes<256>());
   if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
   int sms = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -101,6 +112,54 @@ int attn_splits(int batch, int n_kv, int64_t max_ctx) {
   if (want > 256) want = 256;
   if (want < 1) want = 1;
   return (int)want;
+}
+
+// cuTensorMapEncodeTiled, looked up through the runtime so that libsq does not
+// link libcuda (it must load on machines without a GPU driver).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  });
+  return fn;
+}
+
+// Tensor-core compress of one side (fp16, head_dim 128): X viewed as a 2-D
+// [batch * n_heads * n_tok, 128] fp16 tensor read in 128 x 64 boxes.
+sq_status launch_compress_tc(const void* recs, const void* x, int batch, int n_heads, int64_t n_tok,
+                             const int32_t* sp, const sq_cache* c, uint32_t* flags, cudaStream_t st, int dev) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return SQ_ERR_CUDA;
+  const int64_t rows = (int64_t)batch * n_heads * n_tok;
+  if (rows >= ((int64_t)1 << 31)) return SQ_ERR_ARG;
+  CUtensorMap map;
+  cuuint64_t dims[2] = {(cuuint64_t)tcc::D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)tcc::D * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)tcc::TILE};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return SQ_ERR_CUDA;
+  tcc::Params P;
+  P.recs = (const uint8_t*)recs;
+  P.n_heads = n_heads;
+  P.batch = batch;
+  P.n_tok = n_tok;
+  P.start_pos = sp;
+  P.c = cache_args(c);
+  P.flags = flags;
+  P.tiles_per_row = (int)((n_tok + tcc::TILE - 1) / tcc::TILE);
+  P.eacc = (float)ldexp((double)g_eacc_units, -24);
+  P.n_tiles = (int64_t)batch * n_heads * P.tiles_per_row;
+  int64_t grid = P.n_tiles < g_sms[dev] ? P.n_tiles : g_sms[dev];
+  tcc::k_compress_tc<<<(unsigned)grid, tcc::NUM_THREADS, tcc::SMEM_BYTES, st>>>(map, P);
+  return cuda_ok(cudaGetLastError());
 }
 
 template <typename T>
@@ -147,6 +206,22 @@ int sq_record_words(const sq_calib_params* p) {
 }
 
 sq_status sq_init(void) { return ensure_init(); }
+
+sq_status sq_set_option(int option, int value) {
+  if (option == SQ_OPT_COMPRESS_PATH && (value == 0 || value == 1)) {
+    g_force_ref = value == 1;
+    return SQ_OK;
+  }
+  if (option == SQ_OPT_ATTN_PATH && (value == 0 || value == 1)) {
+    g_attn_ref = value == 1;
+    return SQ_OK;
+  }
+  if (option == SQ_OPT_TC_ERROR_BOUND && value >= 0 && value <= (1 << 20)) {
+    g_eacc_units = value;
+    return SQ_OK;
+  }
+  return SQ_ERR_ARG;
+}
 
 size_t sq_calibrate_workspace(const sq_calib_params* p, int64_t n_tokens) {
   (void)n_tokens;
@@ -211,7 +286,8 @@ sq_status sq_compress_kv(const void* calib_k, const void* calib_v, const void* k
   if (do_v && (!calib_v || ((uintptr_t)calib_v & 255u) || !aligned16(v) || !cache_ok(vc, batch, n_heads)))
     return SQ_ERR_ARG;
   if (d_start_pos && !aligned16(d_start_pos)) return SQ_ERR_ARG;
-  sq_status s = ensure_init();
+  int dev = 0;
+  sq_status s = ensure_init(&dev);
   if (s != SQ_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   for (int side = 0; side < 2; ++side) {
@@ -219,6 +295,12 @@ sq_status sq_compress_kv(const void* calib_k, const void* calib_v, const void* k
     if (!x) continue;
     const void* recs = side == 0 ? calib_k : calib_v;
     const sq_cache* c = side == 0 ? kc : vc;
+    // Tensor-core path: fp16 head_dim 128 prompts (records of at most 16 words).
+    if (dtype == SQ_F16 && d == tcc::D && c->words <= tcc::MAX_W && n_tok >= 64 && !g_force_ref) {
+      s = launch_compress_tc(recs, x, batch, n_heads, n_tok, d_start_pos, c, d_flags, st, dev);
+      if (s != SQ_OK) return s;
+      continue;
+    }
     switch (dtype) {
       case SQ_F32: s = launch_compress<float>(recs, x, batch, n_heads, d, n_tok, d_start_pos, c, d_flags, st); break;
       case SQ_F16: s = launch_compress<__half>(recs, x, batch, n_heads, d, n_tok, d_start_pos, c, d_flags, st); break;
@@ -295,7 +377,19 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
   CacheArgs ka = cache_args(kc), va = cache_args(vc);
   const uint8_t* rk = (const uint8_t*)calib_k;
   const uint8_t* rv = (const uint8_t*)calib_v;
-  if (sh.group <= 1)
+  const bool fast = !g_attn_ref && sh.group <= 8 && (d == 64 || d == 128 || d == 256) && kc->words <= fa::MAXW &&
+                    vc->words <= fa::MAXW;
+  if (fast) {
+    if (d == 64)
+      fa::k_attn_partial_tc<64><<<gpart, fa::NTH, fa::smem_bytes<64>(), st>>>(rk, rv, ka, va, d_seq_lens, sh, w,
+                                                                            scores_out, d_flags);
+    else if (d == 128)
+      fa::k_attn_partial_tc<128><<<gpart, fa::NTH, fa::smem_bytes<128>(), st>>>(rk, rv, ka, va, d_seq_lens, sh, w,
+                                                                              scores_out, d_flags);
+    else
+      fa::k_attn_partial_tc<256><<<gpart, fa::NTH, fa::smem_bytes<256>(), st>>>(rk, rv, ka, va, d_seq_lens, sh, w,
+                                                                              scores_out, d_flags);
+  } else if (sh.group <= 1)
     k_attn_partial<1><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
   else if (sh.group <= 2)
     k_attn_partial<2><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);

@@ -8,6 +8,7 @@
 #pragma once
 
 #include "sq_common.cuh"
+#include "tc_compress.cuh"
 
 namespace sq {
 
@@ -222,6 +223,7 @@ __device__ void build_derived(Rec rec, int tid, int nth) {
   }
   for (int e = tid; e < d * d; e += nth) rec.V_f()[e] = (float)rec.V()[e];
   for (int e = tid; e < d * d; e += nth) rec.S_f()[e] = e < m * m ? (float)rec.S()[e] : 0.0f;
+  if (d == tcc::D) tcc::build_tc(rec, tid, nth);
 }
 
 // ---------------------------------------------------------------------------

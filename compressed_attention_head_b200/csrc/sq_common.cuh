@@ -44,11 +44,17 @@ __host__ __device__ inline size_t canon_bytes(int d) {
   return (size_t)kHeader + 21u * (size_t)d + 16u * (size_t)d * (size_t)d;
 }
 __host__ __device__ inline size_t derived_off(int d) { return (canon_bytes(d) + 255u) & ~(size_t)255u; }
-// Derived part: float32 copies used by the kernels.
-//   sigma_f[d], inv_sigma_f[d], pad to 256 B, V_f[d*d] (same layout as V), S_f[d*d]
-__host__ __device__ inline size_t derived_bytes(int d) {
-  return 256u + 8u * (size_t)d + 8u * (size_t)d * (size_t)d + 256u;
+// Derived part: float32 copies used by the kernels,
+//   sigma_f[d], inv_sigma_f[d], pad to 256 B, V_f[d*d] (same layout as V), S_f[d*d],
+// and, for head_dim 128, the tensor-core block of the fast compress kernel
+// (from the next 1024-byte boundary; see tc_compress.cuh).
+__host__ __device__ inline size_t derived_tc_off(int d) {
+  return ((size_t)(256 + 8 * d) + 8 * (size_t)d * d + 1023) & ~(size_t)1023;
 }
+__host__ __device__ inline size_t derived_tc_bytes(int d) {
+  return d == 128 ? 4 * (size_t)d * d + 16 * (size_t)d + 8 * (size_t)d * d : 0;
+}
+__host__ __device__ inline size_t derived_bytes(int d) { return derived_tc_off(d) + derived_tc_bytes(d); }
 __host__ __device__ inline size_t record_bytes(int d) {
   return (derived_off(d) + derived_bytes(d) + 255u) & ~(size_t)255u;
 }

@@ -52,6 +52,7 @@ _SIGNATURES = {
     "sq_record_words": (ctypes.c_int, [ctypes.POINTER(sq_calib_params)]),
     "sq_codebook": (ctypes.c_int, [ctypes.c_int, _P, _P, _P]),
     "sq_init": (ctypes.c_int, []),
+    "sq_set_option": (ctypes.c_int, [ctypes.c_int, ctypes.c_int]),
     "sq_calibrate_workspace": (ctypes.c_size_t, [ctypes.POINTER(sq_calib_params), ctypes.c_int64]),
     "sq_calibrate": (ctypes.c_int, [ctypes.POINTER(sq_calib_params), _P, ctypes.c_int, ctypes.c_int64,
                                     ctypes.c_int64, ctypes.c_int64, _P, _P, ctypes.c_size_t, _P, _P]),
@@ -180,6 +181,15 @@ def alloc_records(n_heads: int, d: int, device="cuda") -> torch.Tensor:
 # --------------------------------------------------------------------------- launching calls
 def sq_init() -> None:
     _check(lib().sq_init(), "sq_init")
+
+
+SQ_OPT_COMPRESS_PATH = 1
+SQ_OPT_ATTN_PATH = 2
+SQ_OPT_TC_ERROR_BOUND = 3
+
+
+def sq_set_option(option: int, value: int) -> None:
+    _check(lib().sq_set_option(option, value), "sq_set_option")
 
 
 def sq_calibrate(params, x, n_tokens, stride_head, stride_tok, calib_out, ws, status=None, stream=None):

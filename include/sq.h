@@ -190,6 +190,26 @@ sq_status sq_codebook(int b, double* levels, double* thresholds, double* D);
  */
 sq_status sq_init(void);
 
+/*
+ * Process-wide options (host-only; no GPU work).
+ *  SQ_OPT_COMPRESS_PATH: 0 = automatic (tensor-core kernel for fp16 head_dim-128
+ *  prompts of >= 64 tokens, float64 reference kernel otherwise), 1 = always the
+ *  float64 reference kernel. Both produce identical codes (see sq_compress_kv).
+ *  SQ_OPT_ATTN_PATH: 0 = automatic (tensor-core partials for head_dim 64/128/256,
+ *  up to 8 query heads per KV head and records of up to 32 words; SIMT partials
+ *  otherwise), 1 = always the SIMT partials.
+ *  SQ_OPT_TC_ERROR_BOUND: the fp32-accumulation term of the tensor-core compress
+ *  error radius, in units of 2^-24 per unit of ||V_i / sigma_i|| (default 128).
+ *  A code whose z lies within the radius of a threshold is recomputed in
+ *  float64; a radius below the hardware's accumulation error can change codes,
+ *  so values under the default exist only to measure that error.
+ * Returns SQ_ERR_ARG for an unknown option or value.
+ */
+#define SQ_OPT_COMPRESS_PATH 1
+#define SQ_OPT_ATTN_PATH 2
+#define SQ_OPT_TC_ERROR_BOUND 3
+sq_status sq_set_option(int option, int value);
+
 /* Workspace bytes sq_calibrate needs for these parameters and n_tokens. */
 size_t sq_calibrate_workspace(const sq_calib_params* p, int64_t n_tokens);
 

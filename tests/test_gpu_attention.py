@@ -113,3 +113,26 @@ def test_attention_seq_len_past_bound_is_flagged():
     with pytest.raises(sq.SqError) as e:
         sq.sq_attn_decode(rk, rv, kc, vc, lens, 1, 1, 1, 32, 32, q, 0.0, out, None, ws[:16], flags)
     assert e.value.status == sq.SQ_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("name,ctx,heads", [("llama8b", 700, 2), ("gemma9b_sweep", 300, 2)])
+def test_tensor_core_partials_match_simt_partials(name, ctx, heads):
+    """Both attention paths against the oracle on the same packed cache."""
+    try:
+        sq.sq_set_option(sq.SQ_OPT_ATTN_PATH, 1)
+        o1, s1, r_o, r_s, _ = _run(name, 1, ctx, [ctx], heads=heads)
+        sq.sq_set_option(sq.SQ_OPT_ATTN_PATH, 0)
+        o0, s0, _, _, _ = _run(name, 1, ctx, [ctx], heads=heads)
+    finally:
+        sq.sq_set_option(sq.SQ_OPT_ATTN_PATH, 0)
+    _assert_close(o1, s1, r_o, r_s, [ctx])
+    _assert_close(o0, s0, r_o, r_s, [ctx])
+
+
+def test_full_size_decode_sampled_rows():
+    """Qwen2.5-14B-shaped decode step (batch 4 at context 8192, one layer's 8 KV /
+    40 query heads, the launch shape of one layer): every output and score row
+    of two KV heads against the oracle."""
+    out, scores, ref_out, ref_scores, flags = _run("qwen14b", 4, 8192, [8192, 8191, 4097, 8192], heads=2)
+    assert flags == 0
+    _assert_close(out, scores, ref_out, ref_scores, [8192, 8191, 4097, 8192])

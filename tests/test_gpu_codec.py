@@ -162,3 +162,53 @@ def test_argument_errors():
     with pytest.raises(sq.SqError) as e:
         sq.sq_compress_kv(rk, None, k.cuda(), None, 2, 1, 32, 16, None, kc, None)   # batch mismatch
     assert e.value.status == sq.SQ_ERR_ARG
+
+
+@pytest.mark.parametrize("name,tokens", [("llama8b", 1000), ("qwen14b", 777), ("qwen1_5b_long", 129)])
+def test_tensor_core_path_matches_oracle_and_reference_kernel(name, tokens):
+    """The fp16 head_dim-128 tensor-core compress against the oracle and, bit for
+    bit, against the float64 reference kernel (both are exact up to ~1e-13)."""
+    w, ck, cv, k, v, nh = _case(name, batch=2, tokens=tokens, heads=4)
+    try:
+        sq.sq_set_option(sq.SQ_OPT_COMPRESS_PATH, 0)
+        _, _, kc, vc = _compress(ck, cv, k, v)
+        sq.sq_set_option(sq.SQ_OPT_COMPRESS_PATH, 1)
+        _, _, kr, vr = _compress(ck, cv, k, v)
+    finally:
+        sq.sq_set_option(sq.SQ_OPT_COMPRESS_PATH, 0)
+    _check_side(kc, ck, k)
+    _check_side(vc, cv, v)
+    for a, b in ((kc, kr), (vc, vr)):
+        diff = (a.words_u32() != b.words_u32()).any(axis=-1)
+        assert diff.sum() <= 1e-4 * diff.size, diff.sum()
+        assert torch.equal(a.norm, b.norm)
+    assert torch.allclose(kc.rnorm, kr.rnorm, rtol=1e-6, atol=0)
+
+
+def test_full_size_prefill_in_bench_launch_configuration():
+    """Llama-shaped prompt: all 32 layers x 8 KV heads (2048 tokens) compressed in one
+    call, as the benchmark times it; sampled (head, token) records against the oracle."""
+    cfg = CONFIGS["llama8b"]
+    L, nkv, d, T = cfg["layers"], cfg["n_kv"], cfg["d"], cfg["ctx"]
+    ks, vs, cks, cvs = [], [], [], []
+    for layer in range(L):
+        w = make_workload("llama8b", layer, batch=1, tokens=T)
+        ks.append(w.k)
+        vs.append(w.v)
+        cks += calibrate_oracle(w.k_cal, cfg["bits_k"], True)
+        cvs += calibrate_oracle(w.v_cal, cfg["bits_v"], False)
+    k = torch.cat(ks, 1).contiguous()
+    v = torch.cat(vs, 1).contiguous()
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _, _, kc, vc = _compress(cks, cvs, k, v, flags=flags)
+    assert flags.item() == 0
+    rng = np.random.default_rng(7)
+    kw, vw = kc.words_u32(), vc.words_u32()
+    for _ in range(48):
+        h = int(rng.integers(0, L * nkv))
+        ts = np.sort(rng.choice(T, size=16, replace=False))
+        xk = k[0, h, ts].double().numpy()
+        xv = v[0, h, ts].double().numpy()
+        compare_compressed(kw[0, h, ts], kc.norm[0, h, ts].cpu().numpy(), kc.rnorm[0, h, ts].cpu().numpy(), xk,
+                           cks[h])
+        compare_compressed(vw[0, h, ts], vc.norm[0, h, ts].cpu().numpy(), None, xv, cvs[h])
