@@ -165,6 +165,12 @@ sq_status launch_compress_tc(const void* recs, const void* x, int batch, int n_h
 template <typename T>
 sq_status launch_compress(const void* recs, const void* x, int batch, int n_heads, int d, int64_t n_tok,
                           const int32_t* sp, const sq_cache* c, uint32_t* flags, cudaStream_t st) {
+  if (n_tok < 16) {      // appends: a warp per (batch, head), nothing staged
+    const int64_t pairs = (int64_t)batch * n_heads;
+    k_append_ref<T><<<(unsigned)((pairs + kCodecWarps - 1) / kCodecWarps), 32 * kCodecWarps, 0, st>>>(
+        (const uint8_t*)recs, (const T*)x, batch, n_heads, d, n_tok, sp, cache_args(c), flags);
+    return cuda_ok(cudaGetLastError());
+  }
   const int tpb = n_tok >= 1024 ? 256 : 64;
   const int64_t gx = (n_tok + tpb - 1) / tpb;
   if (gx > 0x7fffffff) return SQ_ERR_ARG;
@@ -366,10 +372,21 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
   const float sc = scale > 0.0f ? scale : 1.0f / sqrtf((float)d);
   float* w = (float*)ws;
   dim3 gp(n_kv_heads, batch);
-  switch (q_dtype) {
-    case SQ_F32: k_attn_prepare<float><<<gp, 128, 0, st>>>((const uint8_t*)calib_k, (const float*)q, sh, sc, w, d_flags); break;
-    case SQ_F16: k_attn_prepare<__half><<<gp, 128, 0, st>>>((const uint8_t*)calib_k, (const __half*)q, sh, sc, w, d_flags); break;
-    default: k_attn_prepare<__nv_bfloat16><<<gp, 128, 0, st>>>((const uint8_t*)calib_k, (const __nv_bfloat16*)q, sh, sc, w, d_flags); break;
+  {
+    const uint8_t* rk8 = (const uint8_t*)calib_k;
+    const int G = sh.group;
+#define SQ_PREP(MG, T)                                                                          \
+  k_attn_prepare<MG, T><<<gp, 128, 0, st>>>(rk8, (const T*)q, sh, sc, w, d_flags)
+#define SQ_PREP_G(T)                                                                            \
+  if (G <= 1) SQ_PREP(1, T); else if (G <= 2) SQ_PREP(2, T); else if (G <= 4) SQ_PREP(4, T);   \
+  else if (G <= 8) SQ_PREP(8, T); else SQ_PREP(16, T)
+    switch (q_dtype) {
+      case SQ_F32: SQ_PREP_G(float); break;
+      case SQ_F16: SQ_PREP_G(__half); break;
+      default: SQ_PREP_G(__nv_bfloat16); break;
+    }
+#undef SQ_PREP_G
+#undef SQ_PREP
   }
   if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
   dim3 gpart(sh.splits, n_kv_heads, batch);

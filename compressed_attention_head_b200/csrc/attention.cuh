@@ -35,7 +35,7 @@ __host__ __device__ inline size_t attn_ws_floats(int batch, int n_q, int d, int 
 // Prepare: grid (n_kv, batch), d threads; one block rotates the G queries of
 // one KV head with the float32 copy of V_K.
 // ---------------------------------------------------------------------------
-template <typename TQ>
+template <int MAXG, typename TQ>
 __global__ void k_attn_prepare(const uint8_t* __restrict__ recs_k, const TQ* __restrict__ q, AttnShape s,
                                float scale, float* __restrict__ ws, uint32_t* __restrict__ flags) {
   const int g = blockIdx.x, b = blockIdx.y, d = s.d, G = s.group;
@@ -47,9 +47,9 @@ __global__ void k_attn_prepare(const uint8_t* __restrict__ recs_k, const TQ* __r
   }
   __shared__ float qs[kAttnMaxG][kMaxD];
   __shared__ float qp[kAttnMaxG][kMaxD];
-  for (int e = threadIdx.x; e < G * d; e += blockDim.x) {
+  for (int e = threadIdx.x; e < MAXG * d; e += blockDim.x) {
     int hh = e / d, j = e % d;
-    qs[hh][j] = to_float<TQ>(q[((size_t)b * s.n_q + g * G + hh) * d + j]);
+    qs[hh][j] = hh < G ? to_float<TQ>(q[((size_t)b * s.n_q + g * G + hh) * d + j]) : 0.0f;
   }
   __syncthreads();
   const float* V = rec.V_f();
@@ -57,18 +57,20 @@ __global__ void k_attn_prepare(const uint8_t* __restrict__ recs_k, const TQ* __r
   float* w = ws;
   float* u = ws + (size_t)s.batch * s.n_q * d;
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float acc[kAttnMaxG];
+    float acc[MAXG];
 #pragma unroll
-    for (int hh = 0; hh < kAttnMaxG; ++hh) acc[hh] = 0.0f;
+    for (int hh = 0; hh < MAXG; ++hh) acc[hh] = 0.0f;
     for (int j = 0; j < d; ++j) {
-      float v = V[(size_t)j * d + i];
+      const float v = V[(size_t)j * d + i];
 #pragma unroll
-      for (int hh = 0; hh < kAttnMaxG; ++hh)
-        if (hh < G) acc[hh] = fmaf(v, qs[hh][j], acc[hh]);
+      for (int hh = 0; hh < MAXG; ++hh) acc[hh] = fmaf(v, qs[hh][j], acc[hh]);
     }
-    for (int hh = 0; hh < G; ++hh) {
-      qp[hh][i] = acc[hh];
-      w[((size_t)b * s.n_q + g * G + hh) * d + i] = scale * sig[i] * acc[hh];
+#pragma unroll
+    for (int hh = 0; hh < MAXG; ++hh) {
+      if (hh < G) {
+        qp[hh][i] = acc[hh];
+        w[((size_t)b * s.n_q + g * G + hh) * d + i] = scale * sig[i] * acc[hh];
+      }
     }
   }
   __syncthreads();

@@ -141,6 +141,103 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
 }
 
 // ---------------------------------------------------------------------------
+// Append (few tokens per row, e.g. one decode token): one warp per (batch,
+// head), all of that row's n_tok tokens in turn. Nothing is staged: V, the
+// per-coordinate widths and the codebooks are read through the caches, so a
+// block costs no more than its own tokens. Same float64 arithmetic as
+// k_compress_ref.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) k_append_ref(const uint8_t* __restrict__ recs, const T* __restrict__ x,
+                                                    int batch, int n_heads, int d, int64_t n_tok,
+                                                    const int32_t* __restrict__ start_pos, CacheArgs c,
+                                                    uint32_t* __restrict__ flags) {
+  __shared__ double xs_all[kCodecWarps][kMaxD];
+  __shared__ double rs_all[kCodecWarps][kMaxD];
+  __shared__ uint32_t wb_all[kCodecWarps][kMaxWords];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t pair = (int64_t)blockIdx.x * kCodecWarps + warp;
+  if (pair >= (int64_t)batch * n_heads) return;
+  const int b = (int)(pair / n_heads), h = (int)(pair % n_heads);
+  double* xs = xs_all[warp];
+  double* rs = rs_all[warp];
+  uint32_t* wb = wb_all[warp];
+  Rec rec = rec_at(recs, d, h);
+  const RecHeader* hd = rec.hdr();
+  if (!record_ok(hd, d) || hd->words != c.words || (hd->m > 0 && c.rnorm == nullptr)) {
+    if (lane == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
+    return;
+  }
+  const int64_t sp = start_pos ? (int64_t)start_pos[b] : 0;
+  if (sp < 0 || sp + n_tok > c.cap) {
+    if (lane == 0 && flags) atomicOr(flags, SQ_FLAG_CAPACITY);
+    return;
+  }
+  const int m = hd->m, W = hd->words, cbits = hd->code_bits;
+  const bool normalize = (hd->flags & kFlagNormalize) != 0;
+  const double* V = rec.V();
+  const double* sig = rec.sigma();
+  const uint8_t* bits = rec.bits();
+  const int32_t* offs = rec.offsets();
+  const double* S = rec.S();
+  const size_t row = (size_t)b * n_heads + h;
+  for (int64_t t = 0; t < n_tok; ++t) {
+    const T* xt = x + (row * n_tok + t) * d;
+    double ss = 0.0;
+    for (int j = lane; j < d; j += 32) {
+      const double v = (double)to_float<T>(xt[j]);
+      xs[j] = v;
+      ss += v * v;
+    }
+    for (int w = lane; w < W; w += 32) wb[w] = 0u;
+    ss = warp_sum(ss);
+    __syncwarp();
+    const double nrm = normalize ? sqrt(ss) : 1.0;
+    const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
+    for (int i = lane; i < d; i += 32) {
+      double y = 0.0;
+      for (int j = 0; j < d; ++j) y = fma(V[(size_t)j * d + i], xs[j], y);
+      y *= inv;
+      const int bw = bits[i];
+      const double s = sig[i];
+      int code = 0;
+      if (bw > 0) {
+        code = code_of(s > 0.0 ? y * (1.0 / s) : 0.0, c_th64 + th_off(bw), bw);
+        const int o = offs[i], wi = o >> 5, sh = o & 31;
+        atomicOr(&wb[wi], (uint32_t)code << sh);
+        if (sh + bw > 32) atomicOr(&wb[wi + 1], (uint32_t)code >> (32 - sh));
+      }
+      if (i < m) rs[i] = y - s * (bw > 0 ? c_lv64[lv_off(bw) + code] : 0.0);
+    }
+    __syncwarp();
+    float rho = 0.0f;
+    if (m > 0) {
+      double r2 = 0.0;
+      for (int k = lane; k < m; k += 32) r2 += rs[k] * rs[k];
+      r2 = warp_sum(r2);
+      rho = (float)sqrt(r2);
+      for (int j = 0; j < m; ++j) {
+        double pj = 0.0;
+        for (int k = lane; k < m; k += 32) pj = fma(S[j * m + k], rs[k], pj);
+        pj = warp_sum(pj);
+        if (lane == 0 && pj >= 0.0) {
+          const int o = cbits + j;
+          atomicOr(&wb[o >> 5], 1u << (o & 31));
+        }
+      }
+    }
+    __syncwarp();
+    const size_t slot = row * c.cap + sp + t;
+    for (int w = lane; w < W; w += 32) c.codes[slot * W + w] = wb[w];
+    if (lane == 0) {
+      c.norm[slot] = (float)nrm;
+      if (c.rnorm) c.rnorm[slot] = rho;
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Decompress: x_hat = norm * V (sigma * level) [+ QJL term]; float32 output.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) k_decompress_ref(const uint8_t* __restrict__ recs, int n_heads, int d,

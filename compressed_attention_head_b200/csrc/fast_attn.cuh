@@ -41,7 +41,10 @@ struct Geo {
   static constexpr int QROW = QJL_COLS * 2;           // bytes per QJL row (unswizzled)
   static constexpr int KSTEPS = D / 16;               // k-steps of the key tile (+1 for QJL)
   static constexpr int MBLK = D / 16;                 // m16 blocks of coordinates in PV
+  static constexpr bool SPLITW = D <= 128;            // query weights as fp16 hi + lo
 };
+constexpr int LOCOLS = 64;       // key coordinates whose wide (>= 4-bit) levels get an fp16 lo part
+constexpr int LOROW = LOCOLS * 2;
 
 // Shared-memory plan (bytes): pair LUTs 10.5 KB, single-level table, per-pair
 // parameters for K and V, transposed record tiles, fp16 tiles, norms, merge.
@@ -50,23 +53,33 @@ struct Smem {
   static constexpr int LUT2 = LUT1 + 4 * 32 * 4;   // [16][32] u32
   static constexpr int LUT3 = LUT2 + 16 * 32 * 4;  // [64][32] u32
   static constexpr int LV16 = LUT3 + 64 * 32 * 4;  // [kLevelsTotal] half
-  static constexpr int PAR = (LV16 + kLevelsTotal * 2 + 15) & ~15;   // uint2 [2][kMaxD/2]
-  static constexpr int REC = PAR + 2 * (kMaxD / 2) * 8;              // u32 [2 sides][MAXW][TOK + 1]
+  static constexpr int LVLO = LV16 + kLevelsTotal * 2;   // [kLevelsTotal] half: level - fp16(level)
+  static constexpr int PAR = (LVLO + kLevelsTotal * 2 + 15) & ~15;   // uint2 [2][kMaxD/2]
+  static constexpr int REC = PAR + 2 * (kMaxD / 2) * 8;              // u32 [2 bufs][2 sides][MAXW][TOK + 1]
   static constexpr int REC_PITCH = TOK + 1;
-  static constexpr int KT = (REC + 2 * MAXW * REC_PITCH * 4 + 127) & ~127;
+  static constexpr int REC_SIDE = MAXW * REC_PITCH;                   // words per side
+  static constexpr int NRM = REC + 4 * REC_SIDE * 4;                  // float [2 bufs][3][TOK]
+  static constexpr int KT = (NRM + 2 * 3 * TOK * 4 + 127) & ~127;
 };
 
 // Tiles (key, value, QJL), then norms; the four warps' merge buffer
 // [4][8][D + 2] floats reuses the tiles after the last tile.
 template <int D>
 __host__ __device__ constexpr int tiles_bytes() {
-  return TOK * Geo<D>::KROW + TOK * Geo<D>::VROW + TOK * Geo<D>::QROW;
+  return TOK * Geo<D>::KROW + TOK * Geo<D>::VROW + TOK * Geo<D>::QROW + TOK * LOROW;
 }
 template <int D>
 __host__ __device__ constexpr int smem_bytes() {
-  return Smem::KT + (tiles_bytes<D>() > 4 * 8 * (D + 2) * 4 ? tiles_bytes<D>() : 4 * 8 * (D + 2) * 4) +
-         3 * TOK * 4 + 128;
+  return Smem::KT + (tiles_bytes<D>() > 4 * 8 * (D + 2) * 4 ? tiles_bytes<D>() : 4 * 8 * (D + 2) * 4) + 128;
 }
+
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Byte offset of (row, column) in a tile whose rows are `rowbytes` long and
 // whose 16-byte chunks are XOR-swizzled by (row & 7).
@@ -118,13 +131,14 @@ __device__ void build_pair_params(const uint8_t* bits, const int32_t* offs, int 
 
 // Decodes coordinates [c0, c0 + n) (n a multiple of 8) of token t into the fp16
 // tile row t, reading the transposed records rec[word * REC_PITCH + t].
-template <int ROWBYTES>
+template <int ROWBYTES, bool LO>
 __device__ __forceinline__ void decode_row(const uint32_t* rec, const uint2* par, const uint8_t* sm, int t, int c0,
-                                           int n, uint8_t* tile, int lane) {
+                                           int n, uint8_t* tile, uint8_t* lotile, int lane) {
   const uint32_t* lut1 = (const uint32_t*)(sm + Smem::LUT1) + lane;
   const uint32_t* lut2 = (const uint32_t*)(sm + Smem::LUT2) + lane;
   const uint32_t* lut3 = (const uint32_t*)(sm + Smem::LUT3) + lane;
   const __half* lv16 = (const __half*)(sm + Smem::LV16);
+  const __half* lvlo = (const __half*)(sm + Smem::LVLO);
   for (int c = c0; c < c0 + n; c += 8) {
     uint32_t h[4];
 #pragma unroll
@@ -149,6 +163,12 @@ __device__ __forceinline__ void decode_row(const uint32_t* rec, const uint2* par
           __half l1 = b1 ? lv16[lv_off(b1) + c1v] : __float2half(0.0f);
           __half2 hh = __halves2half2(l0, l1);
           out = *reinterpret_cast<uint32_t*>(&hh);
+          if (LO && c + 2 * k < LOCOLS) {
+            __half m0 = b0 ? lvlo[lv_off(b0) + c0v] : __float2half(0.0f);
+            __half m1 = b1 ? lvlo[lv_off(b1) + c1v] : __float2half(0.0f);
+            __half2 mm = __halves2half2(m0, m1);
+            *(uint32_t*)(lotile + swz(t, c + 2 * k, LOROW)) = *reinterpret_cast<uint32_t*>(&mm);
+          }
         }
       }
       h[k] = out;
@@ -196,15 +216,13 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
 
   uint2* park = (uint2*)(sm + Smem::PAR);
   uint2* parv = park + kMaxD / 2;
-  uint32_t* reck = (uint32_t*)(sm + Smem::REC);
-  uint32_t* recv = reck + MAXW * Smem::REC_PITCH;
+  uint32_t* recbase = (uint32_t*)(sm + Smem::REC);
+  float* nrmbase = (float*)(sm + Smem::NRM);
   uint8_t* ktile = sm + Smem::KT;
   uint8_t* vtile = ktile + TOK * G_::KROW;
   uint8_t* qtile = vtile + TOK * G_::VROW;
+  uint8_t* lotile = qtile + TOK * G_::QROW;
   float* mrg = (float*)ktile;            // [4 warps][8 heads][D + 2], after the last tile
-  float* kn = (float*)(sm + Smem::KT + smem_bytes<D>() - Smem::KT - 3 * TOK * 4 - 128);
-  float* kr = kn + TOK;
-  float* vn = kr + TOK;
 
   // Tables: lane-replicated pair LUTs for widths 1..3 and the fp16 levels.
   for (int e = tid; e < 4 * 32; e += NTH) {
@@ -219,7 +237,16 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
     int f = e >> 5;
     ((uint32_t*)(sm + Smem::LUT3))[e] = pack_h2(c_lv32[lv_off(3) + (f & 7)], c_lv32[lv_off(3) + (f >> 3)]);
   }
-  for (int e = tid; e < kLevelsTotal; e += NTH) ((__half*)(sm + Smem::LV16))[e] = __float2half(c_lv32[e]);
+  for (int e = tid; e < kLevelsTotal; e += NTH) {
+    const __half hv = __float2half(c_lv32[e]);
+    ((__half*)(sm + Smem::LV16))[e] = hv;
+    ((__half*)(sm + Smem::LVLO))[e] = __float2half(c_lv32[e] - __half2float(hv));
+  }
+  // Wide key codes among the first LOCOLS coordinates get an fp16 lo part.
+  bool has_lo = false;
+  if (ok)
+    for (int i = 0; i < LOCOLS && i < D; ++i) has_lo |= rk.bits()[i] >= 4;
+  for (int e = tid; e < TOK * LOCOLS / 2; e += NTH) ((uint32_t*)lotile)[e] = 0u;
   if (ok) {
     build_pair_params(rk.bits(), rk.offsets(), D, park, tid, NTH);
     build_pair_params(rv.bits(), rv.offsets(), D, parv, tid, NTH);
@@ -237,6 +264,7 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
   const float wsc = wmax > 0.0f ? exp2f(-ceilf(log2f(wmax))) : 1.0f;
   const int qg = lane >> 2, qq = lane & 3;
   uint32_t afrag[G_::KSTEPS + 1][2];
+  uint32_t afrag_lo[G_::SPLITW ? G_::KSTEPS : 1][2];
 #pragma unroll
   for (int ks = 0; ks <= G_::KSTEPS; ++ks) {
 #pragma unroll
@@ -249,7 +277,12 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
         v0 = col < D ? wrow[col] : ((col - D) < m ? urow[col - D] : 0.0f);
         v1 = col + 1 < D ? wrow[col + 1] : ((col + 1 - D) < m ? urow[col + 1 - D] : 0.0f);
       }
-      afrag[ks][half] = pack_h2(v0 * wsc, v1 * wsc);
+      const __half2 hv = __floats2half2_rn(v0 * wsc, v1 * wsc);
+      afrag[ks][half] = *reinterpret_cast<const uint32_t*>(&hv);
+      if (G_::SPLITW && ks < G_::KSTEPS) {
+        const float2 back = __half22float2(hv);
+        afrag_lo[G_::SPLITW ? ks : 0][half] = pack_h2(v0 * wsc - back.x, v1 * wsc - back.y);
+      }
     }
   }
   const float inv_wsc = 1.0f / wsc;
@@ -264,26 +297,55 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
   const size_t row = (size_t)b * s.n_kv + g;
   const uint32_t* kcodes = kc.codes + row * kc.cap * wk;
   const uint32_t* vcodes = vc.codes + row * vc.cap * wv;
-  for (int64_t t0 = t_lo; t0 < t_hi; t0 += TOK) {
-    const int nt = (int)min((int64_t)TOK, t_hi - t0);
-    // Stage the records transposed: rec[word][token].
-    for (int e = tid; e < nt * wk; e += NTH) reck[(e % wk) * Smem::REC_PITCH + e / wk] = kcodes[t0 * wk + e];
-    for (int e = tid; e < nt * wv; e += NTH) recv[(e % wv) * Smem::REC_PITCH + e / wv] = vcodes[t0 * wv + e];
-    for (int e = nt * wk + tid; e < TOK * wk; e += NTH) reck[(e % wk) * Smem::REC_PITCH + e / wk] = 0u;
-    for (int e = nt * wv + tid; e < TOK * wv; e += NTH) recv[(e % wv) * Smem::REC_PITCH + e / wv] = 0u;
+  // Stage one tile's records (transposed: rec[word][token]) and norms with
+  // 4-byte cp.async; tokens past the range read as zeros.
+  auto stage = [&](int64_t t0s, int bi) {
+    const int nts = (int)min((int64_t)TOK, t_hi - t0s);
+    uint32_t* rk_ = recbase + bi * 2 * Smem::REC_SIDE;
+    uint32_t* rv_ = rk_ + Smem::REC_SIDE;
+    float* nb = nrmbase + bi * 3 * TOK;
+    const int tok = tid & (TOK - 1);
+    for (int w = tid >> 6; w < wk; w += NTH / TOK) {
+      uint32_t* dst = rk_ + w * Smem::REC_PITCH + tok;
+      if (tok < nts) cp_async4(dst, kcodes + (t0s + tok) * wk + w); else *dst = 0u;
+    }
+    for (int w = tid >> 6; w < wv; w += NTH / TOK) {
+      uint32_t* dst = rv_ + w * Smem::REC_PITCH + tok;
+      if (tok < nts) cp_async4(dst, vcodes + (t0s + tok) * wv + w); else *dst = 0u;
+    }
     if (tid < TOK) {
-      const bool v_ = tid < nt;
-      kn[tid] = v_ ? kc.norm[row * kc.cap + t0 + tid] : 0.0f;
-      kr[tid] = (v_ && m > 0) ? kc.rnorm[row * kc.cap + t0 + tid] : 0.0f;
-      vn[tid] = v_ ? vc.norm[row * vc.cap + t0 + tid] : 0.0f;
+      if (tid < nts) {
+        cp_async4(nb + tid, kc.norm + row * kc.cap + t0s + tid);
+        cp_async4(nb + 2 * TOK + tid, vc.norm + row * vc.cap + t0s + tid);
+        if (m > 0) cp_async4(nb + TOK + tid, kc.rnorm + row * kc.cap + t0s + tid); else nb[TOK + tid] = 0.0f;
+      } else {
+        nb[tid] = 0.0f; nb[TOK + tid] = 0.0f; nb[2 * TOK + tid] = 0.0f;
+      }
+    }
+    cp_async_commit();
+  };
+  if (t_lo < t_hi) stage(t_lo, 0);
+  int bi = 0;
+  for (int64_t t0 = t_lo; t0 < t_hi; t0 += TOK, bi ^= 1) {
+    const int nt = (int)min((int64_t)TOK, t_hi - t0);
+    if (t0 + TOK < t_hi) {
+      stage(t0 + TOK, bi ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
+    const uint32_t* reck = recbase + bi * 2 * Smem::REC_SIDE;
+    const uint32_t* recv = reck + Smem::REC_SIDE;
+    const float* kn = nrmbase + bi * 3 * TOK;
+    const float* kr = kn + TOK;
+    const float* vn = kr + TOK;
     // Decode: warp w -> tokens 32 (w & 1) + lane, coordinate half (w >> 1).
     {
       const int t = ((warp & 1) << 5) + lane;
       const int c0 = (warp >> 1) * (D / 2);
-      decode_row<G_::KROW>(reck, park, sm, t, c0, D / 2, ktile, lane);
-      decode_row<G_::VROW>(recv, parv, sm, t, c0, D / 2, vtile, lane);
+      decode_row<G_::KROW, true>(reck, park, sm, t, c0, D / 2, ktile, lotile, lane);
+      decode_row<G_::VROW, false>(recv, parv, sm, t, c0, D / 2, vtile, nullptr, lane);
       if ((warp >> 1) == 0 && m > 0) {
         const float rho = kr[t];
         uint32_t hq[8];
@@ -320,6 +382,18 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
           mma16816(sc[j], a, b0, b1);
           uint32_t a2[4] = {afrag[ks + 1][0], 0u, afrag[ks + 1][1], 0u};
           mma16816(sc[j], a2, b2, b3);
+          if (G_::SPLITW) {
+            uint32_t al[4] = {afrag_lo[G_::SPLITW ? ks : 0][0], 0u, afrag_lo[G_::SPLITW ? ks : 0][1], 0u};
+            mma16816(sc[j], al, b0, b1);
+            uint32_t al2[4] = {afrag_lo[G_::SPLITW ? ks + 1 : 0][0], 0u, afrag_lo[G_::SPLITW ? ks + 1 : 0][1], 0u};
+            mma16816(sc[j], al2, b2, b3);
+          }
+          if (has_lo && ks < LOCOLS / 16) {
+            uint32_t l0, l1, l2, l3;
+            ldsm_x4(smem_addr(lotile + swz(rr, col, LOROW)), l0, l1, l2, l3);
+            mma16816(sc[j], a, l0, l1);
+            mma16816(sc[j], a2, l2, l3);
+          }
         }
         if (m > 0) {       // QJL k-step: matrices (k 0-7, k 8-15) of the QJL tile, twice
           uint32_t b0, b1, b2, b3;

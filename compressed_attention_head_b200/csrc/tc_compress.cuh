@@ -40,11 +40,11 @@ constexpr int B_BYTES = D * D * 2;
 constexpr int NUM_WARPS = 14;
 constexpr int NUM_THREADS = NUM_WARPS * 32;
 constexpr int WARP_PROD = 0, WARP_MMA = 1, WARP_SIG0 = 2, WARP_EPI0 = 6;
-constexpr int MAX_W = 16;
+constexpr int MAX_W = 12;
 constexpr int REC_PITCH = MAX_W + 1;
 constexpr uint32_t TMEM_COLS = 2 * D;
-constexpr float E_ACC = 7.62939453125e-06f;   // 32 * 2^-22: default accumulation bound factor
-constexpr int QCAP = 1024;                    // deferred exact recomputations per tile
+constexpr float E_ACC = 4.76837158203125e-07f;   // 8 * 2^-24: default accumulation bound factor
+constexpr int QCAP = 256;                     // deferred exact recomputations per tile
 constexpr int MSIG = 8;                       // signal coordinates staged in shared memory
 
 struct CoordInfo {
@@ -60,31 +60,35 @@ struct CoordInfo {
 constexpr int OFF_X = 0;
 constexpr int OFF_BHI = OFF_X + STAGES * X_BYTES;
 constexpr int OFF_BLO = OFF_BHI + B_BYTES;
-constexpr int OFF_REC = OFF_BLO + B_BYTES;
+constexpr int OFF_BLO2 = OFF_BLO + B_BYTES;                 // third split term (exact recomputation only)
+constexpr int OFF_REC = OFF_BLO2 + B_BYTES;
 constexpr int REC_BYTES = 2 * TILE * REC_PITCH * 4;
 constexpr int OFF_RT = OFF_REC + REC_BYTES;                 // float [2][TILE]
 constexpr int OFF_N64 = OFF_RT + 2 * TILE * 4;              // double [2][TILE]
 constexpr int OFF_CI = OFF_N64 + 2 * TILE * 8;              // CoordInfo [D]
 constexpr int OFF_SIG = OFF_CI + D * 16;                    // double [D]
-constexpr int OFF_TH32 = OFF_SIG + D * 8;                   // float [kThreshTotal]
-constexpr int OFF_TH64 = (OFF_TH32 + kThreshTotal * 4 + 7) & ~7;  // double [kThreshTotal]
-constexpr int OFF_LV64 = OFF_TH64 + kThreshTotal * 8;       // double [kLevelsTotal]
-constexpr int OFF_VSIG = (OFF_LV64 + kLevelsTotal * 8 + 15) & ~15;   // double [MSIG][D]
+constexpr int OFF_TH64 = OFF_SIG + D * 8;                   // double [kThreshTotal]
+constexpr int OFF_VSIG = (OFF_TH64 + kThreshTotal * 8 + 15) & ~15;   // double [MSIG][D]
 constexpr int OFF_Q = OFF_VSIG + MSIG * D * 8;              // u32 [QCAP] (token << 16 | coordinate)
 constexpr int OFF_BAR = (OFF_Q + QCAP * 4 + 7) & ~7;
 constexpr int N_BARS = 2 * STAGES + 1 + 2 + 2 + 2;
-constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;            // + alignment slack
+constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;              // u32 [16]
+constexpr int OFF_CHUNK = OFF_MISC + 64;                    // u32 [8]: per 16-coordinate chunk, width | offset << 8
+constexpr int OFF_DW = OFF_CHUNK + 32;                      // float [9]: per-width radius
+constexpr int SMEM_BYTES = OFF_DW + 48 + 1024;              // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds 227 KB");
 
 // The tensor-core block inside the record's derived part (derived_tc_off):
-// Bhi [d*d fp16], Blo [d*d fp16] (swizzled B operand), CoordInfo [d], Vt64 [d*d f64].
+// Bhi, Blo, Blo2 [d*d fp16 each] (swizzled B operand; B = hi + lo + lo2 to
+// about 2^-33 relative), CoordInfo [d], Vt64 [d*d f64].
 struct TcView {
   uint8_t* base;
   int d;
   __host__ __device__ __half* bhi() const { return (__half*)base; }
   __host__ __device__ __half* blo() const { return (__half*)(base + 2 * (size_t)d * d); }
-  __host__ __device__ CoordInfo* ci() const { return (CoordInfo*)(base + 4 * (size_t)d * d); }
-  __host__ __device__ double* vt64() const { return (double*)(base + 4 * (size_t)d * d + 16 * (size_t)d); }
+  __host__ __device__ __half* blo2() const { return (__half*)(base + 4 * (size_t)d * d); }
+  __host__ __device__ CoordInfo* ci() const { return (CoordInfo*)(base + 6 * (size_t)d * d); }
+  __host__ __device__ double* vt64() const { return (double*)(base + 6 * (size_t)d * d + 16 * (size_t)d); }
 };
 __host__ __device__ inline TcView tc_view(Rec r) { return TcView{r.derived() + derived_tc_off(r.d), r.d}; }
 
@@ -106,36 +110,52 @@ __device__ void build_tc(Rec rec, int tid, int nth) {
     int i = e / D, j = e % D;
     tv.vt64()[e] = V[(size_t)j * D + i];
   }
+  // One power-of-two scale for the whole head: 2^ex * max |V_ji / sigma_i| <= 2^14.
+  __shared__ double s_mx;
+  if (tid == 0) s_mx = 0.0;
+  __syncthreads();
   for (int i = tid; i < D; i += nth) {
     double s = sig[i];
     double inv = s > 0.0 ? 1.0 / s : 0.0;
     double mx = 0.0;
     for (int j = 0; j < D; ++j) mx = fmax(mx, fabs(V[(size_t)j * D + i] * inv));
+    unsigned long long* p = (unsigned long long*)&s_mx;   // max of non-negative doubles by bits
+    atomicMax(p, (unsigned long long)__double_as_longlong(mx));
+  }
+  __syncthreads();
+  const double hmx = s_mx;
+  for (int i = tid; i < D; i += nth) {
+    double s = sig[i];
+    double inv = s > 0.0 ? 1.0 / s : 0.0;
     int ex = 0;
-    if (mx > 0.0) ex = (int)floor(log2(16384.0 / mx));     // 2^ex * max <= 2^14
+    if (hmx > 0.0) ex = (int)floor(log2(16384.0 / hmx));
     ex = ex < -100 ? -100 : (ex > 100 ? 100 : ex);
     double scale = ldexp(1.0, ex);
     double res2 = 0.0;
     uint8_t* hi = (uint8_t*)tv.bhi();
     uint8_t* lo = (uint8_t*)tv.blo();
+    uint8_t* lo2 = (uint8_t*)tv.blo2();
     for (int j = 0; j < D; ++j) {
       double v = V[(size_t)j * D + i] * inv * scale;
       __half h = __double2half(v);
       double r1 = v - (double)__half2float(h);
       __half l = __double2half(r1);
       double r2 = r1 - (double)__half2float(l);
+      __half l2 = __double2half(r2);
       res2 += r2 * r2;
       uint32_t o = sw128_off(i, j, D);
       *(__half*)(hi + o) = h;
       *(__half*)(lo + o) = l;
+      *(__half*)(lo2 + o) = l2;
     }
     CoordInfo c;
     c.bo = (uint32_t)rec.bits()[i] | ((uint32_t)bits_off[i] << 8);
     c.sc = (float)ldexp(1.0, -ex);
-    // Bound on |z_tensor - z_exact|: split residual, fp32 accumulation over
-    // 2 * 128 exact products (<= E_ACC * ||V_i / sigma_i|| = E_ACC / sigma_i),
-    // and the fp32 roundings of z, 1/||x|| and the thresholds (|z| < 8).
-    c.dfix = s > 0.0 ? (float)(sqrt(res2) / scale + 4.0e-6) : 0.0f;
+    // Bound on |z_tensor - z_exact| (the tensor path uses hi + lo): their
+    // split residual, the fp32 accumulation term (E * ||V_i / sigma_i||, E a
+    // kernel argument) and the fp32 roundings of z, 1/||x|| and the thresholds
+    // (|z| < 8).
+    c.dfix = s > 0.0 ? (float)(sqrt(res2) / scale + 2.0e-6) : 0.0f;
     c.dacc = (float)inv;
     tv.ci()[i] = c;
   }
@@ -170,16 +190,44 @@ __device__ __forceinline__ int q3(float z, float t1, float t2, float t3, float d
   dg = (a < dl) | (fabsf(a - t1) < dl) | (fabsf(a - t2) < dl) | (fabsf(a - t3) < dl);
   return z > 0.0f ? 4 + m : 3 - m;
 }
-__device__ __forceinline__ int qn(float z, const float* th, int b, float dl, bool& dg) {
-  int n = (1 << b) - 1, lo = 0, hi = n;
-  while (lo < hi) {
-    int mid = (lo + hi) >> 1;
-    if (z > th[mid]) lo = mid + 1; else hi = mid;
-  }
-  float dlo = lo > 0 ? z - th[lo - 1] : 1e30f;
-  float dhi = lo < n ? th[lo] - z : 1e30f;
-  dg = fminf(fabsf(dlo), fabsf(dhi)) < dl;
+__device__ __forceinline__ int qn(float z, const double* th, int b, float dl, bool& dg) {
+  const int n = (1 << b) - 1;
+  const int lo = code_of((double)z, th, b);
+  const double dlo = lo > 0 ? (double)z - th[lo - 1] : 1e30;
+  const double dhi = lo < n ? th[lo] - (double)z : 1e30;
+  dg = fmin(fabs(dlo), fabs(dhi)) < (double)dl;
   return lo;
+}
+
+// Codes of 16 consecutive coordinates of width B (1..3) from their tensor-core
+// values v (z = v * zr), packed LSB-first (16 * B bits), and the mask of the
+// coordinates whose z lies within dl of a threshold.
+template <int B>
+__device__ __forceinline__ void chunk_codes(const float* v, float zr, float t1, float t2, float t3, float dl,
+                                            uint64_t& cw, uint32_t& dmask) {
+  cw = 0;
+  dmask = 0;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float z = v[k] * zr;
+    bool dg;
+    int code;
+    if (B == 1) code = q1(z, dl, dg);
+    else if (B == 2) code = q2(z, t1, dl, dg);
+    else code = q3(z, t1, t2, t3, dl, dg);
+    cw |= (uint64_t)(uint32_t)code << (B * k);
+    dmask |= (uint32_t)dg << k;
+  }
+}
+
+// ORs the nbits-bit value cw into a record at bit position o (up to 3 words).
+__device__ __forceinline__ void or_bits(uint32_t* rw, int o, uint64_t cw, int nbits) {
+  const int wi = o >> 5, sh = o & 31;
+  const uint64_t a = cw << sh;
+  const uint32_t top = sh ? (uint32_t)(cw >> (64 - sh)) : 0u;
+  if ((uint32_t)a) atomicOr(&rw[wi], (uint32_t)a);
+  if ((uint32_t)(a >> 32)) atomicOr(&rw[wi + 1], (uint32_t)(a >> 32));
+  if (sh + nbits > 64 && top) atomicOr(&rw[wi + 2], top);
 }
 
 // Byte offset of the 16-byte chunk c (elements 8c .. 8c+7) of token row t in an X stage.
@@ -231,6 +279,31 @@ __device__ __forceinline__ double exact_dot(const uint8_t* xs, int t, const doub
   return acc;
 }
 
+// sum_j x[t][j] * (hi + lo + lo2)[i][j] in float64 by one warp (lane l takes
+// j = 4l .. 4l+3); every lane returns the sum. The three fp16 terms represent
+// B to about 2^-33 relative, so z = sum * 2^-s / ||x|| matches exact
+// arithmetic to ~1e-9, far inside the 1e-5 exemption band.
+__device__ __forceinline__ double exact_sum_warp(const uint8_t* xs, const uint8_t* bh, const uint8_t* bl,
+                                                 const uint8_t* bl2, int t, int i, int lane) {
+  const int j = 4 * lane;
+  const uint2 xr = *(const uint2*)(xs + x_chunk(t, j >> 3) + ((j & 7) << 1));
+  const uint32_t bo = sw128_off(i, j, D);
+  const uint2 h = *(const uint2*)(bh + bo), l = *(const uint2*)(bl + bo), l2 = *(const uint2*)(bl2 + bo);
+  const __half2* xh = reinterpret_cast<const __half2*>(&xr);
+  const __half2* hh = reinterpret_cast<const __half2*>(&h);
+  const __half2* lh = reinterpret_cast<const __half2*>(&l);
+  const __half2* l2h = reinterpret_cast<const __half2*>(&l2);
+  double acc = 0.0;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float2 xf = __half22float2(xh[k]), hf = __half22float2(hh[k]);
+    const float2 lf = __half22float2(lh[k]), l2f = __half22float2(l2h[k]);
+    acc = fma((double)xf.x, ((double)hf.x + (double)lf.x) + (double)l2f.x, acc);
+    acc = fma((double)xf.y, ((double)hf.y + (double)lf.y) + (double)l2f.y, acc);
+  }
+  return warp_sum(acc);
+}
+
 // Overwrites the b-bit field at bit o of a record with code.
 __device__ __forceinline__ void patch_field(uint32_t* rw, int o, int b, uint32_t code) {
   const int wi = o >> 5, sh = o & 31;
@@ -250,14 +323,13 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P) {
   uint8_t* sX = sm + OFF_X;
   uint8_t* sBhi = sm + OFF_BHI;
   uint8_t* sBlo = sm + OFF_BLO;
+  uint8_t* sBlo2 = sm + OFF_BLO2;
   uint32_t* sRec = (uint32_t*)(sm + OFF_REC);
   float* sRt = (float*)(sm + OFF_RT);
   double* sN64 = (double*)(sm + OFF_N64);
   CoordInfo* sCI = (CoordInfo*)(sm + OFF_CI);
   double* sSig = (double*)(sm + OFF_SIG);
-  float* sTh32 = (float*)(sm + OFF_TH32);
   double* sTh64 = (double*)(sm + OFF_TH64);
-  double* sLv64 = (double*)(sm + OFF_LV64);
   double* sVsig = (double*)(sm + OFF_VSIG);
   uint32_t* sQ = (uint32_t*)(sm + OFF_Q);
   uint64_t* bars = (uint64_t*)(sm + OFF_BAR);
@@ -273,11 +345,7 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   for (int e = threadIdx.x; e < 2 * TILE * REC_PITCH; e += NUM_THREADS) sRec[e] = 0u;
-  for (int e = threadIdx.x; e < kThreshTotal; e += NUM_THREADS) {
-    sTh64[e] = c_th64[e];
-    sTh32[e] = (float)c_th64[e];
-  }
-  for (int e = threadIdx.x; e < kLevelsTotal; e += NUM_THREADS) sLv64[e] = c_lv64[e];
+  for (int e = threadIdx.x; e < kThreshTotal; e += NUM_THREADS) sTh64[e] = c_th64[e];
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       sm100::mbar_init(&full[s], 1);
@@ -349,10 +417,29 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P) {
     }
     const int msig = m < MSIG ? m : MSIG;
     for (int e = threadIdx.x; e < msig * D; e += NUM_THREADS) sVsig[e] = tv.vt64()[e];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      // Per-width radius: the largest of its coordinates (the signal ones are exact).
+      float* dw = (float*)(sm + OFF_DW);
+      for (int b = 0; b <= SQ_MAX_BITS; ++b) dw[b] = 0.0f;
+      for (int i = m; i < D; ++i) {
+        const int b = (int)(sCI[i].bo & 0xFFu);
+        dw[b] = fmaxf(dw[b], fmaf(P.eacc, sCI[i].dacc, sCI[i].dfix));
+      }
+      // 16-coordinate chunks of one width in 1..3 with no signal coordinate take the fast path.
+      uint32_t* ch = (uint32_t*)(sm + OFF_CHUNK);
+      for (int c = 0; c < D / 16; ++c) {
+        const int b0 = (int)(sCI[16 * c].bo & 0xFFu);
+        bool uni = b0 >= 1 && b0 <= 3 && 16 * c >= m;
+        for (int k = 1; k < 16 && uni; ++k) uni = (int)(sCI[16 * c + k].bo & 0xFFu) == b0;
+        ch[c] = (uni ? (uint32_t)b0 : 0u) | ((sCI[16 * c].bo >> 8) << 8);
+      }
+    }
     if (warp == WARP_PROD && lane == 0) {
-      sm100::mbar_expect_tx(bfull, 2 * B_BYTES);
+      sm100::mbar_expect_tx(bfull, 3 * B_BYTES);
       sm100::bulk_load(sBhi, tv.bhi(), B_BYTES, bfull);
       sm100::bulk_load(sBlo, tv.blo(), B_BYTES, bfull);
+      sm100::bulk_load(sBlo2, tv.blo2(), B_BYTES, bfull);
     }
     __syncthreads();
     const uint32_t bpar = seg & 1u;
@@ -414,8 +501,10 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P) {
       const int t_epi = q * 32 + lane;
       const int worker = threadIdx.x - WARP_SIG0 * 32;       // 0 .. 383
       const int epi_id = threadIdx.x - WARP_EPI0 * 32;       // 0 .. 255 for epilogue threads
-      const float t21 = sTh32[th_off(2) + 2];
-      const float t31 = sTh32[th_off(3) + 4], t32 = sTh32[th_off(3) + 5], t33 = sTh32[th_off(3) + 6];
+      const float t21 = (float)sTh64[th_off(2) + 2];
+      const float t31 = (float)sTh64[th_off(3) + 4], t32 = (float)sTh64[th_off(3) + 5];
+      const float t33 = (float)sTh64[th_off(3) + 6];
+      const int wid = warp - WARP_SIG0;                        // worker warp 0 .. 11
       const double* S = rec.S();
       for (int64_t k = 0; k < nt; ++k) {
         const uint32_t it = iter + (uint32_t)k;
@@ -467,7 +556,7 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P) {
               if (b > 0) {
                 const double z = sSig[i] > 0.0 ? yn / sSig[i] : 0.0;
                 const int code = code_of(z, sTh64 + th_off(b), b);
-                lvv = sLv64[lv_off(b) + code];
+                lvv = c_lv64[lv_off(b) + code];
                 const int o = (int)(sCI[i].bo >> 8), wi = o >> 5, sh = o & 31;
                 atomicOr(&rw[wi], (uint32_t)code << sh);
                 if (sh + b > 32) atomicOr(&rw[wi + 1], (uint32_t)code >> (32 - sh));
@@ -503,57 +592,71 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P) {
           const bool exact_zero = r == 0.0f;
           uint32_t* rw = sRec + (buf * TILE + t) * REC_PITCH;
           const float eacc = P.eacc;
-          uint64_t acc = 0;
-          int wbase = -1;
+          const float zr = sCI[0].sc * r;
+          const float* dw = (const float*)(sm + OFF_DW);
+          const uint32_t* chd = (const uint32_t*)(sm + OFF_CHUNK);
+          const bool enq_ok = valid && !exact_zero;
           if (live) {
             for (int c = 0; c < 4; ++c) {
               float v[16];
               sm100::tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * D + hh * 64 + c * 16), v);
+              const int i0 = hh * 64 + c * 16;
+              const uint32_t cd = chd[i0 >> 4];
+              const int cb = (int)(cd & 0xFFu);
+              uint32_t dmask = 0;
+              if (cb != 0) {
+                // width-uniform chunk: codes packed with compile-time shifts
+                uint64_t cw;
+                if (cb == 1) chunk_codes<1>(v, zr, 0.f, 0.f, 0.f, dw[1], cw, dmask);
+                else if (cb == 2) chunk_codes<2>(v, zr, t21, 0.f, 0.f, dw[2], cw, dmask);
+                else chunk_codes<3>(v, zr, t31, t32, t33, dw[3], cw, dmask);
+                if (valid) or_bits(rw, (int)(cd >> 8), cw, 16 * cb);
+              } else {
 #pragma unroll
-              for (int kk = 0; kk < 16; ++kk) {
-                const int i = hh * 64 + c * 16 + kk;
-                const CoordInfo ci = sCI[i];
-                const int b = (int)(ci.bo & 0xFFu);
-                if (b == 0 || i < m) continue;
-                const float z = v[kk] * (ci.sc * r);
-                const float dl = fmaf(eacc, ci.dacc, ci.dfix);
-                bool dg;
-                int code;
-                if (b == 1) code = q1(z, dl, dg);
-                else if (b == 2) code = q2(z, t21, dl, dg);
-                else if (b == 3) code = q3(z, t31, t32, t33, dl, dg);
-                else code = qn(z, sTh32 + th_off(b), b, dl, dg);
-                dg = dg && valid && !exact_zero;
-                const uint32_t dm = __ballot_sync(0xffffffffu, dg);
-                if (dm) {
+                for (int kk = 0; kk < 16; ++kk) {
+                  const int i = i0 + kk;
+                  const CoordInfo ci = sCI[i];
+                  const int b = (int)(ci.bo & 0xFFu);
+                  if (b == 0 || i < m) continue;
+                  const float z = v[kk] * zr;
+                  const float dl = fmaf(eacc, ci.dacc, ci.dfix);
+                  bool dg;
+                  int code;
+                  if (b == 1) code = q1(z, dl, dg);
+                  else if (b == 2) code = q2(z, t21, dl, dg);
+                  else if (b == 3) code = q3(z, t31, t32, t33, dl, dg);
+                  else code = qn(z, sTh64 + th_off(b), b, dl, dg);
+                  dmask |= (uint32_t)dg << kk;
+                  if (valid) or_bits(rw, (int)(ci.bo >> 8), (uint64_t)(uint32_t)code, b);
+                }
+              }
+              // Queue the codes within their radius for exact recomputation.
+              dmask = enq_ok ? dmask : 0u;
+              if (__any_sync(0xffffffffu, dmask != 0u)) {
+                for (int kk = 0; kk < 16; ++kk) {
+                  const bool dg = (dmask >> kk) & 1u;
+                  const uint32_t dm = __ballot_sync(0xffffffffu, dg);
+                  if (!dm) continue;
                   uint32_t base = 0;
                   if (lane == 0) base = atomicAdd(&misc[9], (uint32_t)__popc(dm));
                   base = __shfl_sync(0xffffffffu, base, 0);
                   const uint32_t pos = base + (uint32_t)__popc(dm & ((1u << lane) - 1u));
-                  if (dg) {
-                    if (pos < (uint32_t)QCAP) {
-                      sQ[pos] = ((uint32_t)t << 16) | (uint32_t)i;
-                    } else {          // queue full: this lane's code is computed right here
-                      const double zz = exact_dot(xs, t, tv.vt64() + (size_t)i * D) /
-                                        (sN64[buf * TILE + t] * sSig[i]);
-                      code = code_of(zz, sTh64 + th_off(b), b);
-                    }
+                  const int i = i0 + kk;
+                  const bool ov = dg && pos >= (uint32_t)QCAP;
+                  if (dg && !ov) sQ[pos] = ((uint32_t)t << 16) | (uint32_t)i;
+                  uint32_t om = __ballot_sync(0xffffffffu, ov);
+                  while (om) {        // queue full: recompute and patch right here
+                    const int src = __ffs(om) - 1;
+                    om &= om - 1;
+                    const int ts = q * 32 + src;
+                    const CoordInfo ci = sCI[i];
+                    const int b = (int)(ci.bo & 0xFFu);
+                    const double zz = exact_sum_warp(xs, sBhi, sBlo, sBlo2, ts, i, lane) * (double)ci.sc /
+                                      sN64[buf * TILE + ts];
+                    if (lane == src) patch_field(rw, (int)(ci.bo >> 8), b, (uint32_t)code_of(zz, sTh64 + th_off(b), b));
                   }
                 }
-                const int o = (int)(ci.bo >> 8);
-                const int w = o >> 5;
-                if (wbase < 0) wbase = w;
-                if (w > wbase) {
-                  if (valid && (uint32_t)acc) atomicOr(&rw[wbase], (uint32_t)acc);
-                  acc >>= 32;
-                  ++wbase;
-                }
-                acc |= (uint64_t)(uint32_t)code << (o - 32 * wbase);
               }
-            }
-            if (wbase >= 0 && valid) {
-              if ((uint32_t)acc) atomicOr(&rw[wbase], (uint32_t)acc);
-              if ((uint32_t)(acc >> 32)) atomicOr(&rw[wbase + 1], (uint32_t)(acc >> 32));
             }
           }
           sm100::tc_fence_before();
@@ -563,14 +666,15 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P) {
         // ---- all 12 worker warps: exact recomputation of the queued codes
         sm100::named_bar(1, 12 * 32);
         const uint32_t qn_ = min(misc[9], (uint32_t)QCAP);
-        for (uint32_t e = (uint32_t)worker; e < qn_; e += 12 * 32) {
+        for (uint32_t e = (uint32_t)wid; e < qn_; e += 12) {
           const uint32_t ent = sQ[e];
           const int t = (int)(ent >> 16), i = (int)(ent & 0xFFFFu);
           const CoordInfo ci = sCI[i];
           const int b = (int)(ci.bo & 0xFFu);
-          const double zz = exact_dot(xs, t, tv.vt64() + (size_t)i * D) / (sN64[buf * TILE + t] * sSig[i]);
-          const int code = code_of(zz, sTh64 + th_off(b), b);
-          patch_field(sRec + (buf * TILE + t) * REC_PITCH, (int)(ci.bo >> 8), b, (uint32_t)code);
+          const double zz = exact_sum_warp(xs, sBhi, sBlo, sBlo2, t, i, lane) * (double)ci.sc / sN64[buf * TILE + t];
+          if (lane == 0)
+            patch_field(sRec + (buf * TILE + t) * REC_PITCH, (int)(ci.bo >> 8), b,
+                        (uint32_t)code_of(zz, sTh64 + th_off(b), b));
         }
         sm100::named_bar(1, 12 * 32);
         if (lane == 0) sm100::mbar_arrive(&empty[st]);    // the X stage is no longer read

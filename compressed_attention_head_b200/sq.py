@@ -228,3 +228,4 @@ def sq_attn_decode(calib_k, calib_v, kc, vc, seq_lens, batch, n_q_heads, n_kv_he
                                 DTYPE_CODE[q.dtype], float(scale), _ptr(out), DTYPE_CODE[out.dtype],
                                 _ptr(scores_out), _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0,
                                 _ptr(flags), _stream(stream)), "sq_attn_decode")
+
