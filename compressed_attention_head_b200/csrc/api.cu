@@ -426,4 +426,43 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
   return cuda_ok(cudaGetLastError());
 }
 
+// ---------------------------------------------------------------------------
+// Decode attention without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they run decode
+// attention: code running under a CUDA-graph capture or inside a serving loop
+// whose memory is reserved up front, plug-ins that have no handle to the
+// application's allocator, and runtimes that forbid allocation after start-up.
+// They use this entry point: its scratch is a fixed array in the library's own
+// device memory (every GPU that loads libsq keeps it until the process exits).
+// ---------------------------------------------------------------------------
+constexpr size_t kStaticScratchBytes = SQ_ATTN_NOALLOC_MAX_BYTES;
+static __device__ __align__(256) unsigned char g_attn_scratch[kStaticScratchBytes];
+static void* g_attn_scratch_addr[128];     // device address of the array, per device
+
+sq_status sq_attn_decode_noalloc(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
+                                 const int32_t* d_seq_lens, int batch, int n_q_heads, int n_kv_heads, int d,
+                                 int64_t max_ctx, const void* q, sq_dtype q_dtype, float scale, void* out,
+                                 sq_dtype out_dtype, float* scores_out, uint32_t* d_flags, sq_stream stream) {
+  const size_t need = sq_attn_workspace(batch, n_q_heads, n_kv_heads, d, max_ctx);
+  if (need == 0) return supported_d(d) ? SQ_ERR_ARG : SQ_ERR_UNSUPPORTED;
+  if (need > kStaticScratchBytes) return SQ_ERR_WORKSPACE;
+  int dev = 0;
+  sq_status s = ensure_init(&dev);
+  if (s != SQ_OK) return s;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_attn_scratch_addr[dev]) {
+      // The symbol's name is a host-side stand-in; the kernels need the device
+      // address of this device's copy, taken with this device current.
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess || !p) return SQ_ERR_CUDA;
+      g_attn_scratch_addr[dev] = p;
+    }
+  }
+  return sq_attn_decode(calib_k, calib_v, kc, vc, d_seq_lens, batch, n_q_heads, n_kv_heads, d, max_ctx, q, q_dtype,
+                        scale, out, out_dtype, scores_out, g_attn_scratch_addr[dev], kStaticScratchBytes, d_flags,
+                        stream);
+}
+
 }  // extern "C"

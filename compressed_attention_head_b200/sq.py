@@ -68,7 +68,13 @@ _SIGNATURES = {
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
                                       _P, ctypes.c_int, ctypes.c_float, _P, ctypes.c_int, _P, _P,
                                       ctypes.c_size_t, _P, _P]),
+    "sq_attn_decode_noalloc": (ctypes.c_int, [_P, _P, ctypes.POINTER(sq_cache), ctypes.POINTER(sq_cache), _P,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int64, _P, ctypes.c_int, ctypes.c_float, _P, ctypes.c_int,
+                                              _P, _P, _P]),
 }
+
+SQ_ATTN_NOALLOC_MAX_BYTES = 8 << 20
 
 
 def lib() -> ctypes.CDLL:
@@ -229,3 +235,13 @@ def sq_attn_decode(calib_k, calib_v, kc, vc, seq_lens, batch, n_q_heads, n_kv_he
                                 _ptr(scores_out), _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0,
                                 _ptr(flags), _stream(stream)), "sq_attn_decode")
 
+
+def sq_attn_decode_noalloc(calib_k, calib_v, kc, vc, seq_lens, batch, n_q_heads, n_kv_heads, d, max_ctx, q, scale,
+                           out, scores_out=None, flags=None, stream=None):
+    """sq_attn_decode with the library's fixed scratch array instead of a workspace
+    (for callers that cannot allocate device memory; see sq.h)."""
+    kcs, vcs = kc.struct(), vc.struct()
+    _check(lib().sq_attn_decode_noalloc(_ptr(calib_k), _ptr(calib_v), ctypes.byref(kcs), ctypes.byref(vcs),
+                                        _ptr(seq_lens), batch, n_q_heads, n_kv_heads, d, max_ctx, _ptr(q),
+                                        DTYPE_CODE[q.dtype], float(scale), _ptr(out), DTYPE_CODE[out.dtype],
+                                        _ptr(scores_out), _ptr(flags), _stream(stream)), "sq_attn_decode_noalloc")

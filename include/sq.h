@@ -312,6 +312,35 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
                          float scale, void* out, sq_dtype out_dtype, float* scores_out, void* ws,
                          size_t ws_bytes, uint32_t* d_flags, sq_stream stream);
 
+/*
+ * sq_attn_decode without a workspace argument, for callers that cannot
+ * allocate device memory where they run decode attention (inside a captured
+ * CUDA graph or a serving loop whose memory is reserved up front, plug-ins
+ * with no access to the application's allocator, runtimes that forbid
+ * allocation after start-up). The pages have no counterpart: this is a
+ * deployment convenience of this library.
+ *
+ * Arguments and results are those of sq_attn_decode minus ws / ws_bytes. The
+ * scratch is one fixed array of SQ_ATTN_NOALLOC_MAX_BYTES in the library's
+ * device memory, present on every GPU that loads libsq until the process
+ * exits. The call allocates nothing (no cudaMalloc, no allocating library
+ * routine). It returns SQ_ERR_WORKSPACE, before any launch, when the shape
+ * needs more than the array (sq_attn_workspace() > SQ_ATTN_NOALLOC_MAX_BYTES).
+ * The first call on a device looks up the array's device address on that
+ * device (cudaGetSymbolAddress) and caches it; make that first call before
+ * any stream capture. Every call on a device shares the one array, so calls
+ * whose executions overlap on the GPU (different streams, or concurrent
+ * graphs) race and corrupt each other's results; serialize them. Nothing in
+ * the array needs to start at zero: each call writes every scratch entry it
+ * later reads.
+ */
+#define SQ_ATTN_NOALLOC_MAX_BYTES (8u << 20)
+sq_status sq_attn_decode_noalloc(const void* calib_k, const void* calib_v, const sq_cache* kc,
+                                 const sq_cache* vc, const int32_t* d_seq_lens, int batch, int n_q_heads,
+                                 int n_kv_heads, int d, int64_t max_ctx, const void* q, sq_dtype q_dtype,
+                                 float scale, void* out, sq_dtype out_dtype, float* scores_out,
+                                 uint32_t* d_flags, sq_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
