@@ -48,28 +48,41 @@ def _peaks():
 
 # --------------------------------------------------------------------------- workload
 def build_workload(name: str, device: str, layers: int | None = None):
-    """All layers of one replica, layers folded into the head index."""
+    """All layers of one replica, layers folded into the head index. Tensors are
+    preallocated and filled layer by layer (the largest shape holds ~90 GB of fp16 KV)."""
     import torch
 
-    from synthetic import CONFIGS, make_workload
+    from synthetic import CONFIGS, TORCH_DTYPE, make_workload
 
     cfg = dict(CONFIGS[name])
     cfg["name"] = name
     if layers:
         cfg["layers"] = layers
     L, nkv, nq, d = cfg["layers"], cfg["n_kv"], cfg["n_q"], cfg["d"]
-    T = cfg["ctx"]
-    ks, vs, kcal, vcal, qs, kn, vn = [], [], [], [], [], [], []
+    T, B, ncal = cfg["ctx"], cfg["batch"], cfg["n_cal"]
+    dt = TORCH_DTYPE[cfg["dtype"]]
+    H, HQ = L * nkv, L * nq
+    k = torch.empty(B, H, T, d, dtype=dt, device=device)
+    v = torch.empty_like(k)
+    k_cal = torch.empty(H, ncal, d, dtype=dt, device=device)
+    v_cal = torch.empty_like(k_cal)
+    q = torch.empty(B, HQ, d, dtype=dt, device=device)
+    k_new = torch.empty(B, H, 1, d, dtype=dt, device=device)
+    v_new = torch.empty_like(k_new)
     for layer in range(L):
-        w = make_workload(cfg, layer, device=device, batch=cfg["batch"], tokens=T)
-        nxt = make_workload(cfg, layer, device=device, batch=cfg["batch"], tokens=1, data_stream=1,
-                            with_calibration=False)
-        ks.append(w.k); vs.append(w.v); kcal.append(w.k_cal); vcal.append(w.v_cal); qs.append(nxt.q)
-        kn.append(nxt.k); vn.append(nxt.v)
-    cat = lambda xs, dim: torch.cat(xs, dim=dim).contiguous()
-    return dict(cfg=cfg, H=L * nkv, HQ=L * nq, d=d, T=T, batch=cfg["batch"],
-                k=cat(ks, 1), v=cat(vs, 1), k_cal=cat(kcal, 0), v_cal=cat(vcal, 0),
-                q=cat(qs, 1), k_new=cat(kn, 1), v_new=cat(vn, 1))
+        w = make_workload(cfg, layer, device=device, batch=B, tokens=T)
+        nxt = make_workload(cfg, layer, device=device, batch=B, tokens=1, data_stream=1, with_calibration=False)
+        hs = slice(layer * nkv, (layer + 1) * nkv)
+        k[:, hs] = w.k
+        v[:, hs] = w.v
+        k_cal[hs] = w.k_cal
+        v_cal[hs] = w.v_cal
+        q[:, layer * nq:(layer + 1) * nq] = nxt.q
+        k_new[:, hs] = nxt.k
+        v_new[:, hs] = nxt.v
+        del w, nxt
+    return dict(cfg=cfg, H=H, HQ=HQ, d=d, T=T, batch=B, k=k, v=v, k_cal=k_cal, v_cal=v_cal, q=q,
+                k_new=k_new, v_new=v_new)
 
 
 def record_bytes_per_token(cfg, words_k, words_v, qjl):
@@ -79,6 +92,32 @@ def record_bytes_per_token(cfg, words_k, words_v, qjl):
     k_out = 4 * words_k + 4 + (4 if qjl else 0)
     v_out = 4 * words_v + 4
     return kin + k_out, kin + v_out, k_out, v_out
+
+
+def kernel_source_hash() -> str:
+    """Hash of the kernel sources (*.cuh); profile counters are reported only for the
+    kernels they were captured from."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "compressed_attention_head_b200", "csrc")
+    for fn in sorted(f for f in os.listdir(csrc) if f.endswith(".cuh")):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, tokens_per_launch: int):
+    """DRAM bytes per launch of `kernel` from profiles/traffic.json (written from an ncu
+    capture of the same sources), scaled to this launch's tokens; None if stale or absent."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)
+        ent = rec["kernels"][kernel]
+        if rec["source_hash"] != kernel_source_hash():
+            return None
+        return ent["dram_bytes"] * tokens_per_launch / ent["tokens"]
+    except Exception:
+        return None
 
 
 def max_over_ranks(value: float, device) -> float:
@@ -315,8 +354,12 @@ def run_gpu(args, rank, world, local_rank):
     out = torch.empty(B, HQ, d, dtype=torch.float32, device=dev)
     flags = torch.zeros(1, dtype=torch.int32, device=dev)
     if not prefill:
-        # decode configs: the cache of ctx tokens is filled once, outside the timed steps
+        # decode configs: the cache of ctx tokens is filled once, outside the timed steps,
+        # and the fp16 prompt is released
         sq.sq_compress_kv(rk, rv, wl["k"], wl["v"], B, H, d, T, pos0, kc, vc, flags)
+        torch.cuda.synchronize()
+        del wl["k"], wl["v"]
+        torch.cuda.empty_cache()
 
     n_ev = 6
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
@@ -350,6 +393,40 @@ def run_gpu(args, rank, world, local_rank):
     clk = clocks.stop()
     elapsed = max_over_ranks(t_start.elapsed_time(t_end) / 1e3, dev)
     per_step = elapsed / args.steps
+    # The same step captured once as a CUDA graph and replayed: the launch gaps of the
+    # eager loop go away (every call is asynchronous, allocates nothing, and the
+    # per-device tables were uploaded by sq_init before capture).
+    graph_step = None
+    if not args.no_graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                step()
+            torch.cuda.current_stream().wait_stream(side)
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g):
+                step()
+            for _ in range(args.warmup):
+                g.replay()
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(args.steps):
+                g.replay()
+            b_.record()
+            torch.cuda.synchronize()
+            graph_step = max_over_ranks(a.elapsed_time(b_) / 1e3, dev) / args.steps
+            del g
+        except Exception as exc:       # report, keep the eager number
+            print(f"graph capture failed: {exc}", file=sys.stderr)
+            graph_step = None
+    eager_step = per_step
+    if graph_step is not None:
+        per_step = graph_step
     if prefill:
         ck_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
         cv_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
@@ -368,12 +445,15 @@ def run_gpu(args, rank, world, local_rank):
     tokens = step_tokens(cfg) * world
     value = tokens / per_step
     if prefill:
-        dom = {"kernel": "k_compress (prefill, K and V launches)", "bytes": (comp_bytes_k + comp_bytes_v) / 2,
-               "ms": (ck_ms + cv_ms) / 2}
+        dom = {"kernel": "k_compress_tc (prompt compress; mean of the K and V launches)",
+               "bytes": (comp_bytes_k + comp_bytes_v) / 2, "ms": (ck_ms + cv_ms) / 2,
+               "ncu_name": "k_compress_tc", "tokens": B * H * T}
     else:
-        dom = {"kernel": "sq_attn_decode (prepare + partial + combine)", "bytes": attn_bytes, "ms": att_ms}
+        dom = {"kernel": "sq_attn_decode (prepare + partial + combine)", "bytes": attn_bytes, "ms": att_ms,
+               "ncu_name": "k_attn_partial_tc", "tokens": B * H * (T + 1)}
     achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
     breakdown = {
+        "step_ms_eager": 1e3 * eager_step, "step_ms_graph": None if graph_step is None else 1e3 * graph_step,
         "compress_k_ms": ck_ms, "compress_v_ms": cv_ms, "append_ms": app_ms, "attention_ms": att_ms,
         "compress_GBps": ((comp_bytes_k + comp_bytes_v) / ((ck_ms + cv_ms) / 1e3) / 1e9) if prefill else None,
         "attention_GBps": attn_bytes / (att_ms / 1e3) / 1e9,
@@ -386,8 +466,8 @@ def run_gpu(args, rank, world, local_rank):
     # ---- end to end through the C ABI with host buffers
     e2e = None
     if not args.no_e2e:
-        hk = wl["k"].cpu().pin_memory()
-        hv = wl["v"].cpu().pin_memory()
+        hk = wl["k"].cpu().pin_memory() if prefill else None
+        hv = wl["v"].cpu().pin_memory() if prefill else None
         hkn, hvn, hq = wl["k_new"].cpu().pin_memory(), wl["v_new"].cpu().pin_memory(), wl["q"].cpu().pin_memory()
         hout = torch.empty_like(out, device="cpu").pin_memory()
 
@@ -429,10 +509,11 @@ def run_gpu(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16 in; f64 rotate/quantize; f32 attention", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f16 in; fp16 tensor-core rotation, f64 exact recomputation near thresholds; fp16 tensor-core attention with f32 accumulate", "data": "synthetic",
         "config": workload_config(cfg, world),
         "roofline": {"bound": "hbm", "kernel": dom["kernel"], "achieved": achieved, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": profiled_traffic(dom["ncu_name"], dom["tokens"]),
                      "bytes_per_launch": dom["bytes"], "launch_ms": dom["ms"]},
         "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": args.steps * ((2 if prefill else 0) + 2 + 3),
@@ -451,6 +532,7 @@ def main():
     ap.add_argument("--impl", default="sq", choices=["sq", "reference"])
     ap.add_argument("--config", default="llama8b")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time the eager launches only")
     ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling captures only)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=4096)
