@@ -52,7 +52,7 @@ def build_workload(name: str, device: str, layers: int | None = None):
     preallocated and filled layer by layer (the largest shape holds ~90 GB of fp16 KV)."""
     import torch
 
-    from synthetic import CONFIGS, TORCH_DTYPE, make_workload
+    from synthetic.workloads import CONFIGS, TORCH_DTYPE, make_workload
 
     cfg = dict(CONFIGS[name])
     cfg["name"] = name
@@ -94,13 +94,21 @@ def record_bytes_per_token(cfg, words_k, words_v, qjl):
     return kin + k_out, kin + v_out, k_out, v_out
 
 
-def kernel_source_hash() -> str:
-    """Hash of the kernel sources (*.cuh); profile counters are reported only for the
-    kernels they were captured from."""
+# Source files each profiled kernel is built from (its DRAM traffic in
+# profiles/traffic.json is used only while these files are unchanged).
+KERNEL_SOURCES = {
+    "k_compress_tc": ["tc_compress.cuh", "sm100.cuh", "sq_common.cuh"],
+    "k_attn_partial_tc": ["fast_attn.cuh", "attention.cuh", "sq_common.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources of `kernel`; profile counters are reported only for the
+    kernel sources they were captured from."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "compressed_attention_head_b200", "csrc")
-    for fn in sorted(f for f in os.listdir(csrc) if f.endswith(".cuh")):
+    for fn in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
@@ -111,9 +119,8 @@ def profiled_traffic(kernel: str, tokens_per_launch: int):
     capture of the same sources), scaled to this launch's tokens; None if stale or absent."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            rec = json.load(f)
-        ent = rec["kernels"][kernel]
-        if rec["source_hash"] != kernel_source_hash():
+            ent = json.load(f)["kernels"][kernel]
+        if ent["source_hash"] != kernel_source_hash(kernel):
             return None
         return ent["dram_bytes"] * tokens_per_launch / ent["tokens"]
     except Exception:
@@ -516,7 +523,9 @@ def run_gpu(args, rank, world, local_rank):
                      "traffic": profiled_traffic(dom["ncu_name"], dom["tokens"]),
                      "bytes_per_launch": dom["bytes"], "launch_ms": dom["ms"]},
         "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": args.steps * ((2 if prefill else 0) + 2 + 3),
+        # per step: prompt compress K and V (tensor-core kernel + the pass for heads with
+        # more than 16 QJL dimensions, each), two appends, prepare + partial + combine
+        "gpu_launches": args.steps * ((4 if prefill else 0) + 2 + 3),
         "clocks": clk, "breakdown": breakdown,
         "calibration": {"ms": calib_ms, "heads": 2 * H, "tokens_per_head": ncal, "status_nonzero": n_bad},
         "device_flags": flag_val,

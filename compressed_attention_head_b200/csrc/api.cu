@@ -9,6 +9,8 @@ __constant__ double c_lv64[kLevelsTotal];
 __constant__ double c_th64[kThreshTotal];
 __constant__ float c_lv32[kLevelsTotal];
 __constant__ double c_D[SQ_MAX_BITS + 1];
+__constant__ float4 c_tcq[248];        // tcc cell tables: thresholds (T_j, T_j+1, T_j+2) per width 4..8
+__constant__ uint8_t c_tccell[560];    // tcc cell tables: positive thresholds below each cell
 }  // namespace sq
 
 #include <cudaTypedefs.h>
@@ -31,7 +33,8 @@ std::mutex g_mu;
 bool g_ready[128];
 bool g_force_ref = false;   // route compress to the float64 reference kernel
 bool g_attn_ref = false;    // route attention partials to the SIMT kernel
-int g_eacc_units = 128;     // accumulation bound of the tensor-core compress radius, in 2^-24
+int g_eacc_units = tcc::EACC_DEFAULT_UNITS;   // accumulation bound of the tensor-core compress radius, in 2^-24
+tcc::QuantConst g_kq;       // register thresholds and cell counts of the tensor-core compress
 int g_sms[128];
 
 bool supported_d(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
@@ -39,6 +42,41 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 bool valid_dtype(int t) { return t == SQ_F32 || t == SQ_F16 || t == SQ_BF16; }
 
 sq_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA; }
+
+// Cell tables of the tensor-core compress for widths 4..8 (see tc_compress.cuh)
+// from the float32 positive thresholds T_1 < ... < T_n of each width; false if
+// some cell would hold two thresholds (cannot happen for the Gaussian codebook).
+bool build_cell_tables(const double* th, float4* q, uint8_t* cell, tcc::QuantConst* kq) {
+  kq->t2 = (float)th[th_off(2) + 2];
+  for (int j = 0; j < 3; ++j) kq->t3[j] = (float)th[th_off(3) + 4 + j];
+  for (int b = 0; b < 12; ++b) kq->ncell[b] = 1;
+  for (int e = 0; e < tcc::kCellBytes; ++e) cell[e] = 0;
+  const float inf = INFINITY;
+  for (int b = 4; b <= 8; ++b) {
+    const int n = (1 << (b - 1)) - 1;
+    float T[130];
+    T[0] = 0.0f;
+    for (int j = 1; j <= n; ++j) T[j] = (float)th[th_off(b) + n + j];   // thresholds n+1 .. 2n are positive
+    T[n + 1] = inf;
+    T[n + 2] = inf;
+    for (int j = 0; j <= n; ++j) q[tcc::q_off(b) + j] = make_float4(T[j], T[j + 1], T[j + 2], 0.0f);
+    const double h = ldexp(1.0, -(b - 2));
+    const int ncell = (int)floor((double)T[n] / h) + 1;
+    if (ncell > tcc::cell_cap(b)) return false;
+    kq->ncell[b] = ncell;
+    for (int g = 0; g < ncell; ++g) {
+      int lo = 0, inside = 0;
+      for (int j = 1; j <= n; ++j) {
+        if ((double)T[j] < g * h) ++lo;
+        else if (g + 1 < ncell ? (double)T[j] < (g + 1) * h : true) ++inside;
+      }
+      if (inside > 1) return false;
+      cell[tcc::cell_off(b) + g] = (uint8_t)lo;
+    }
+    if (th[th_off(b) + n] != 0.0) return false;   // the middle threshold is 0
+  }
+  return true;
+}
 
 // Uploads the Lloyd-Max tables to the current device once.
 sq_status ensure_init(int* dev_out = nullptr) {
@@ -58,6 +96,11 @@ sq_status ensure_init(int* dev_out = nullptr) {
     dist[b] = codebook_distortion(b);
   }
   for (int k = 0; k < kLevelsTotal; ++k) lv32[k] = (float)lv[k];
+  float4 tq[tcc::kQEntries];
+  uint8_t tcell[tcc::kCellBytes];
+  if (!build_cell_tables(th, tq, tcell, &g_kq)) return SQ_ERR_CUDA;
+  if (cudaMemcpyToSymbol(c_tcq, tq, sizeof(tq)) != cudaSuccess) return SQ_ERR_CUDA;
+  if (cudaMemcpyToSymbol(c_tccell, tcell, sizeof(tcell)) != cudaSuccess) return SQ_ERR_CUDA;
   if (cudaMemcpyToSymbol(c_lv64, lv, sizeof(lv)) != cudaSuccess) return SQ_ERR_CUDA;
   if (cudaMemcpyToSymbol(c_th64, th, sizeof(th)) != cudaSuccess) return SQ_ERR_CUDA;
   if (cudaMemcpyToSymbol(c_lv32, lv32, sizeof(lv32)) != cudaSuccess) return SQ_ERR_CUDA;
@@ -103,10 +146,11 @@ bool cache_ok(const sq_cache* c, int batch, int n_heads) {
 CacheArgs cache_args(const sq_cache* c) { return CacheArgs{c->codes, c->norm, c->rnorm, c->cap, c->words}; }
 
 // Splits of the context per (batch, KV head) so that the partial kernel has
-// about two blocks per SM of a 148-SM B200, each over >= one 128-token tile.
+// about six blocks per SM of a 148-SM B200 (two waves of three resident
+// blocks), each over >= one 128-token tile.
 int attn_splits(int batch, int n_kv, int64_t max_ctx) {
   int64_t units = (int64_t)batch * n_kv;
-  int64_t want = (2 * 148 + units - 1) / units;
+  int64_t want = (6 * 148 + units - 1) / units;
   int64_t tiles = (max_ctx + kAttnTile - 1) / kAttnTile;
   if (want > tiles) want = tiles;
   if (want > 256) want = 256;
@@ -148,6 +192,7 @@ sq_status launch_compress_tc(const void* recs, const void* x, int batch, int n_h
   if (r != CUDA_SUCCESS) return SQ_ERR_CUDA;
   tcc::Params P;
   P.recs = (const uint8_t*)recs;
+  P.x = (const __half*)x;
   P.n_heads = n_heads;
   P.batch = batch;
   P.n_tok = n_tok;
@@ -158,17 +203,25 @@ sq_status launch_compress_tc(const void* recs, const void* x, int batch, int n_h
   P.eacc = (float)ldexp((double)g_eacc_units, -24);
   P.n_tiles = (int64_t)batch * n_heads * P.tiles_per_row;
   int64_t grid = P.n_tiles < g_sms[dev] ? P.n_tiles : g_sms[dev];
-  tcc::k_compress_tc<<<(unsigned)grid, tcc::NUM_THREADS, tcc::SMEM_BYTES, st>>>(map, P);
+  tcc::k_compress_tc<<<(unsigned)grid, tcc::NUM_THREADS, tcc::SMEM_BYTES, st>>>(map, P, g_kq);
+  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  // Heads with more than tcc::MSIG QJL dimensions: the reference kernel, one
+  // block per (batch, head); every other block returns at once.
+  dim3 g2(1, n_heads, batch);
+  k_compress_ref<__half><<<g2, 128, codec_ref_smem(tcc::D), st>>>((const uint8_t*)recs, (const __half*)x, n_heads,
+                                                                tcc::D, n_tok, (int)n_tok, sp, cache_args(c), flags,
+                                                                tcc::MSIG + 1);
   return cuda_ok(cudaGetLastError());
 }
 
 template <typename T>
 sq_status launch_compress(const void* recs, const void* x, int batch, int n_heads, int d, int64_t n_tok,
                           const int32_t* sp, const sq_cache* c, uint32_t* flags, cudaStream_t st) {
-  if (n_tok < 16) {      // appends: a warp per (batch, head), nothing staged
-    const int64_t pairs = (int64_t)batch * n_heads;
-    k_append_ref<T><<<(unsigned)((pairs + kCodecWarps - 1) / kCodecWarps), 32 * kCodecWarps, 0, st>>>(
-        (const uint8_t*)recs, (const T*)x, batch, n_heads, d, n_tok, sp, cache_args(c), flags);
+  if (n_tok < 16) {      // appends: a block per (head, group of vectors)
+    const int64_t groups = ((int64_t)batch * n_tok + kAppendNV - 1) / kAppendNV;
+    dim3 grid((unsigned)n_heads, (unsigned)groups);
+    k_append<T><<<grid, 256, 0, st>>>((const uint8_t*)recs, (const T*)x, batch, n_heads, d, n_tok, sp,
+                                      cache_args(c), flags);
     return cuda_ok(cudaGetLastError());
   }
   const int tpb = n_tok >= 1024 ? 256 : 64;
@@ -176,7 +229,7 @@ sq_status launch_compress(const void* recs, const void* x, int batch, int n_head
   if (gx > 0x7fffffff) return SQ_ERR_ARG;
   dim3 grid((unsigned)gx, n_heads, batch);
   k_compress_ref<T><<<grid, 128, codec_ref_smem(d), st>>>((const uint8_t*)recs, (const T*)x, n_heads, d, n_tok,
-                                                          tpb, sp, cache_args(c), flags);
+                                                          tpb, sp, cache_args(c), flags, 0);
   return cuda_ok(cudaGetLastError());
 }
 
@@ -301,8 +354,8 @@ sq_status sq_compress_kv(const void* calib_k, const void* calib_v, const void* k
     if (!x) continue;
     const void* recs = side == 0 ? calib_k : calib_v;
     const sq_cache* c = side == 0 ? kc : vc;
-    // Tensor-core path: fp16 head_dim 128 prompts (records of at most 16 words).
-    if (dtype == SQ_F16 && d == tcc::D && c->words <= tcc::MAX_W && n_tok >= 64 && !g_force_ref) {
+    // Tensor-core path: fp16 head_dim 128 prompts.
+    if (dtype == SQ_F16 && d == tcc::D && n_tok >= 64 && !g_force_ref) {
       s = launch_compress_tc(recs, x, batch, n_heads, n_tok, d_start_pos, c, d_flags, st, dev);
       if (s != SQ_OK) return s;
       continue;
@@ -394,8 +447,8 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
   CacheArgs ka = cache_args(kc), va = cache_args(vc);
   const uint8_t* rk = (const uint8_t*)calib_k;
   const uint8_t* rv = (const uint8_t*)calib_v;
-  const bool fast = !g_attn_ref && sh.group <= 8 && (d == 64 || d == 128 || d == 256) && kc->words <= fa::MAXW &&
-                    vc->words <= fa::MAXW;
+  const bool fast = !g_attn_ref && sh.group <= 8 && (d == 64 || d == 128 || d == 256) && kc->words <= d / 8 &&
+                    vc->words <= d / 8;
   if (fast) {
     if (d == 64)
       fa::k_attn_partial_tc<64><<<gpart, fa::NTH, fa::smem_bytes<64>(), st>>>(rk, rv, ka, va, d_seq_lens, sh, w,
@@ -417,11 +470,20 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
   else
     k_attn_partial<16><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
   if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
-  dim3 gc(n_q_heads, batch);
-  switch (out_dtype) {
-    case SQ_F32: k_attn_combine<float><<<gc, 128, 0, st>>>(rv, sh, w, (float*)out); break;
-    case SQ_F16: k_attn_combine<__half><<<gc, 128, 0, st>>>(rv, sh, w, (__half*)out); break;
-    default: k_attn_combine<__nv_bfloat16><<<gc, 128, 0, st>>>(rv, sh, w, (__nv_bfloat16*)out); break;
+  dim3 gc(n_kv_heads, batch);
+  {
+    const int G = sh.group;
+#define SQ_COMB(MG, T) k_attn_combine<MG, T><<<gc, 256, 0, st>>>(rv, sh, w, (T*)out)
+#define SQ_COMB_G(T)                                                                             \
+  if (G <= 1) SQ_COMB(1, T); else if (G <= 2) SQ_COMB(2, T); else if (G <= 4) SQ_COMB(4, T);    \
+  else if (G <= 8) SQ_COMB(8, T); else SQ_COMB(16, T)
+    switch (out_dtype) {
+      case SQ_F32: SQ_COMB_G(float); break;
+      case SQ_F16: SQ_COMB_G(__half); break;
+      default: SQ_COMB_G(__nv_bfloat16); break;
+    }
+#undef SQ_COMB_G
+#undef SQ_COMB
   }
   return cuda_ok(cudaGetLastError());
 }

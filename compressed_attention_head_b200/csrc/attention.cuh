@@ -280,50 +280,66 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// Combine: grid (n_q, batch), 128 threads. a_i = sigma_V,i * sum_s e^(m_s - M)
-// acc_s,i / sum_s e^(m_s - M) l_s; o = V_V a.
+// Combine: grid (n_kv, batch), 256 threads; one block finishes the G query
+// heads of one KV head, so V_V is read once for all of them.
+// a_h,i = sigma_V,i * sum_s e^(m_s - M) acc_s,i / sum_s e^(m_s - M) l_s;  o_h = V_V a_h.
 // ---------------------------------------------------------------------------
-template <typename TO>
-__global__ void __launch_bounds__(128) k_attn_combine(const uint8_t* __restrict__ recs_v, AttnShape s,
+template <int MAXG, typename TO>
+__global__ void __launch_bounds__(256) k_attn_combine(const uint8_t* __restrict__ recs_v, AttnShape s,
                                                       const float* __restrict__ ws, TO* __restrict__ out) {
-  const int h = blockIdx.x, b = blockIdx.y, d = s.d, tid = threadIdx.x;
-  const int g = h / s.group;
+  const int g = blockIdx.x, b = blockIdx.y, d = s.d, tid = threadIdx.x, G = s.group;
+  const int lane = tid & 31, warp = tid >> 5;
   Rec rv = rec_at(recs_v, d, g);
-  __shared__ float a[kMaxD];
-  __shared__ float sw[256];
-  __shared__ float s_l;
+  __shared__ float a[MAXG][kMaxD];
+  __shared__ float sw[MAXG][256];   // splits <= 256 (attn_splits)
+  __shared__ float s_inv_l[MAXG];
   const float* acc = ws + (size_t)s.batch * s.n_q * d * 2;
   const float* ml = acc + (size_t)s.batch * s.n_q * s.splits * d;
-  const size_t qh = (size_t)b * s.n_q + h;
-  float M = -INFINITY;
-  for (int k = 0; k < s.splits; ++k) M = fmaxf(M, ml[(qh * s.splits + k) * 2]);
-  for (int k = tid; k < s.splits; k += blockDim.x) {
-    float mk = ml[(qh * s.splits + k) * 2];
-    sw[k] = (mk == -INFINITY) ? 0.0f : __expf(mk - M);
-  }
-  __syncthreads();
-  if (tid == 0) {
-    float l = 0.0f;
-    for (int k = 0; k < s.splits; ++k) l += sw[k] * ml[(qh * s.splits + k) * 2 + 1];
-    s_l = l;
-  }
-  __syncthreads();
-  const float inv_l = s_l > 0.0f ? 1.0f / s_l : 0.0f;
+  const size_t qh0 = (size_t)b * s.n_q + (size_t)g * G;
   const bool ok = record_ok(rv.hdr(), d);
   const float* sig = rv.sigma_f();
-  for (int i = tid; i < d; i += blockDim.x) {
+  // per head (one warp each, round robin): split weights e^(m_s - M) and 1 / l
+  for (int hh = warp; hh < G; hh += 8) {
+    const float* mlh = ml + (qh0 + hh) * s.splits * 2;
+    float M = -INFINITY;
+    for (int k = lane; k < s.splits; k += 32) M = fmaxf(M, mlh[2 * k]);
+    M = warp_max(M);
+    float l = 0.0f;
+    for (int k = lane; k < s.splits; k += 32) {
+      const float mk = mlh[2 * k];
+      const float wk = (mk == -INFINITY) ? 0.0f : __expf(mk - M);
+      sw[hh][k] = wk;
+      l += wk * mlh[2 * k + 1];
+    }
+    l = warp_sum(l);
+    if (lane == 0) s_inv_l[hh] = l > 0.0f ? 1.0f / l : 0.0f;
+  }
+  __syncthreads();
+  for (int e = tid; e < G * d; e += 256) {
+    const int hh = e / d, i = e % d;
+    const float* ah = acc + (qh0 + hh) * s.splits * (size_t)d + i;
     float v = 0.0f;
-    for (int k = 0; k < s.splits; ++k) v = fmaf(sw[k], acc[(qh * s.splits + k) * d + i], v);
-    a[i] = ok ? v * inv_l * sig[i] : 0.0f;
+    for (int k = 0; k < s.splits; ++k) v = fmaf(sw[hh][k], ah[(size_t)k * d], v);
+    a[hh][i] = ok ? v * s_inv_l[hh] * sig[i] : 0.0f;
   }
   __syncthreads();
   const float* V = rv.V_f();
-  const int lane = tid & 31, warp = tid >> 5;
-  for (int j = warp; j < d; j += 4) {
-    float v = 0.0f;
-    for (int i = lane; i < d; i += 32) v = fmaf(ok ? V[(size_t)j * d + i] : 0.0f, a[i], v);
-    v = warp_sum(v);
-    if (lane == 0) out[qh * d + j] = from_float<TO>(v);
+  for (int j = warp; j < d; j += 8) {
+    float o[MAXG];
+#pragma unroll
+    for (int hh = 0; hh < MAXG; ++hh) o[hh] = 0.0f;
+    for (int i = lane; i < d; i += 32) {
+      const float vv = ok ? V[(size_t)j * d + i] : 0.0f;
+#pragma unroll
+      for (int hh = 0; hh < MAXG; ++hh) o[hh] = fmaf(vv, a[hh][i], o[hh]);
+    }
+#pragma unroll
+    for (int hh = 0; hh < MAXG; ++hh) {
+      if (hh < G) {
+        const float r = warp_sum(o[hh]);
+        if (lane == 0) out[(qh0 + hh) * d + j] = from_float<TO>(r);
+      }
+    }
   }
 }
 

@@ -33,12 +33,18 @@ template <typename T>
 __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict__ recs, const T* __restrict__ x,
                                                       int n_heads, int d, int64_t n_tok, int tok_per_block,
                                                       const int32_t* __restrict__ start_pos, CacheArgs c,
-                                                      uint32_t* __restrict__ flags) {
+                                                      uint32_t* __restrict__ flags, int min_m) {
   extern __shared__ __align__(16) unsigned char sm[];
   const int h = blockIdx.y, b = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   Rec rec = rec_at(recs, d, h);
   const RecHeader* hd = rec.hdr();
+  if (min_m > 0) {   // second pass after another kernel: only heads with m >= min_m, no flags
+    const int64_t sp0 = start_pos ? (int64_t)start_pos[b] : 0;
+    if (!record_ok(hd, d) || hd->words != c.words || hd->m < min_m || c.rnorm == nullptr || sp0 < 0 ||
+        sp0 + n_tok > c.cap)
+      return;
+  }
   if (!record_ok(hd, d) || hd->words != c.words || (hd->m > 0 && c.rnorm == nullptr)) {
     if (threadIdx.x == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
     return;
@@ -141,36 +147,34 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// Append (few tokens per row, e.g. one decode token): one warp per (batch,
-// head), all of that row's n_tok tokens in turn. Nothing is staged: V, the
-// per-coordinate widths and the codebooks are read through the caches, so a
-// block costs no more than its own tokens. Same float64 arithmetic as
-// k_compress_ref.
+// Append (decode steps, fewer than 16 tokens per row): grid (n_heads, vector
+// groups), 256 threads. A block compresses up to kAppendNV vectors of one
+// head, the (batch, token) pairs g * kAppendNV ...; every element of V
+// (float64, read straight from the record) is loaded once per block and used
+// for all of them. Same arithmetic as k_compress_ref.
 // ---------------------------------------------------------------------------
+constexpr int kAppendNV = 8;
+
 template <typename T>
-__global__ void __launch_bounds__(128) k_append_ref(const uint8_t* __restrict__ recs, const T* __restrict__ x,
-                                                    int batch, int n_heads, int d, int64_t n_tok,
-                                                    const int32_t* __restrict__ start_pos, CacheArgs c,
-                                                    uint32_t* __restrict__ flags) {
-  __shared__ double xs_all[kCodecWarps][kMaxD];
-  __shared__ double rs_all[kCodecWarps][kMaxD];
-  __shared__ uint32_t wb_all[kCodecWarps][kMaxWords];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t pair = (int64_t)blockIdx.x * kCodecWarps + warp;
-  if (pair >= (int64_t)batch * n_heads) return;
-  const int b = (int)(pair / n_heads), h = (int)(pair % n_heads);
-  double* xs = xs_all[warp];
-  double* rs = rs_all[warp];
-  uint32_t* wb = wb_all[warp];
+__global__ void __launch_bounds__(256) k_append(const uint8_t* __restrict__ recs, const T* __restrict__ x,
+                                                int batch, int n_heads, int d, int64_t n_tok,
+                                                const int32_t* __restrict__ start_pos, CacheArgs c,
+                                                uint32_t* __restrict__ flags) {
+  constexpr int NV = kAppendNV;
+  __shared__ double xs[NV][kMaxD];        // input, then the residual of the signal coordinates
+  __shared__ double ys[NV][256];          // partial sums of V^T x (parts of the j range)
+  __shared__ double th[kThreshTotal];
+  __shared__ double lv[kLevelsTotal];
+  __shared__ uint32_t wb[NV][kMaxWords];
+  __shared__ double s_inv[NV];
+  __shared__ int s_ok[NV];
+  const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t total = (int64_t)batch * n_tok;
+  const int64_t v0 = (int64_t)blockIdx.y * NV;
   Rec rec = rec_at(recs, d, h);
   const RecHeader* hd = rec.hdr();
   if (!record_ok(hd, d) || hd->words != c.words || (hd->m > 0 && c.rnorm == nullptr)) {
-    if (lane == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
-    return;
-  }
-  const int64_t sp = start_pos ? (int64_t)start_pos[b] : 0;
-  if (sp < 0 || sp + n_tok > c.cap) {
-    if (lane == 0 && flags) atomicOr(flags, SQ_FLAG_CAPACITY);
+    if (tid == 0 && blockIdx.y == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
     return;
   }
   const int m = hd->m, W = hd->words, cbits = hd->code_bits;
@@ -180,60 +184,119 @@ __global__ void __launch_bounds__(128) k_append_ref(const uint8_t* __restrict__ 
   const uint8_t* bits = rec.bits();
   const int32_t* offs = rec.offsets();
   const double* S = rec.S();
-  const size_t row = (size_t)b * n_heads + h;
-  for (int64_t t = 0; t < n_tok; ++t) {
-    const T* xt = x + (row * n_tok + t) * d;
+  for (int e = tid; e < kThreshTotal; e += 256) th[e] = c_th64[e];
+  for (int e = tid; e < kLevelsTotal; e += 256) lv[e] = c_lv64[e];
+  for (int e = tid; e < NV * kMaxWords; e += 256) wb[e / kMaxWords][e % kMaxWords] = 0u;
+  // inputs (vectors past the end, or of rows over capacity, are zeros and not stored)
+  if (tid < NV) {
+    const int64_t vi = v0 + tid;
+    bool ok = vi < total;
+    if (ok) {
+      const int b = (int)(vi / n_tok);
+      const int64_t sp = start_pos ? (int64_t)start_pos[b] : 0;
+      if (sp < 0 || sp + n_tok > c.cap) {
+        ok = false;
+        if (flags) atomicOr(flags, SQ_FLAG_CAPACITY);
+      }
+    }
+    s_ok[tid] = ok ? 1 : 0;
+  }
+  for (int e = tid; e < NV * d; e += 256) {
+    const int v = e / d, j = e % d;
+    const int64_t vi = v0 + v;
+    double xv = 0.0;
+    if (vi < total) {
+      const int b = (int)(vi / n_tok);
+      const int64_t t = vi % n_tok;
+      xv = (double)to_float<T>(x[(((size_t)b * n_heads + h) * n_tok + t) * d + j]);
+    }
+    xs[v][j] = xv;
+  }
+  __syncthreads();
+  // norms: warp v
+  {
     double ss = 0.0;
-    for (int j = lane; j < d; j += 32) {
-      const double v = (double)to_float<T>(xt[j]);
-      xs[j] = v;
-      ss += v * v;
-    }
-    for (int w = lane; w < W; w += 32) wb[w] = 0u;
+    for (int j = lane; j < d; j += 32) ss += xs[warp][j] * xs[warp][j];
     ss = warp_sum(ss);
-    __syncwarp();
-    const double nrm = normalize ? sqrt(ss) : 1.0;
-    const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
-    for (int i = lane; i < d; i += 32) {
-      double y = 0.0;
-      for (int j = 0; j < d; ++j) y = fma(V[(size_t)j * d + i], xs[j], y);
-      y *= inv;
-      const int bw = bits[i];
-      const double s = sig[i];
-      int code = 0;
-      if (bw > 0) {
-        code = code_of(s > 0.0 ? y * (1.0 / s) : 0.0, c_th64 + th_off(bw), bw);
-        const int o = offs[i], wi = o >> 5, sh = o & 31;
-        atomicOr(&wb[wi], (uint32_t)code << sh);
-        if (sh + bw > 32) atomicOr(&wb[wi + 1], (uint32_t)code >> (32 - sh));
-      }
-      if (i < m) rs[i] = y - s * (bw > 0 ? c_lv64[lv_off(bw) + code] : 0.0);
-    }
-    __syncwarp();
-    float rho = 0.0f;
-    if (m > 0) {
-      double r2 = 0.0;
-      for (int k = lane; k < m; k += 32) r2 += rs[k] * rs[k];
-      r2 = warp_sum(r2);
-      rho = (float)sqrt(r2);
-      for (int j = 0; j < m; ++j) {
-        double pj = 0.0;
-        for (int k = lane; k < m; k += 32) pj = fma(S[j * m + k], rs[k], pj);
-        pj = warp_sum(pj);
-        if (lane == 0 && pj >= 0.0) {
-          const int o = cbits + j;
-          atomicOr(&wb[o >> 5], 1u << (o & 31));
-        }
-      }
-    }
-    __syncwarp();
-    const size_t slot = row * c.cap + sp + t;
-    for (int w = lane; w < W; w += 32) c.codes[slot * W + w] = wb[w];
     if (lane == 0) {
-      c.norm[slot] = (float)nrm;
-      if (c.rnorm) c.rnorm[slot] = rho;
+      const double nrm = normalize ? sqrt(ss) : 1.0;
+      s_inv[warp] = nrm > 0.0 ? 1.0 / nrm : 0.0;
+      const int64_t vi = v0 + warp;
+      if (s_ok[warp]) {
+        const int b = (int)(vi / n_tok);
+        const int64_t t = vi % n_tok;
+        const int64_t sp = start_pos ? (int64_t)start_pos[b] : 0;
+        c.norm[((size_t)b * n_heads + h) * c.cap + sp + t] = (float)nrm;
+      }
     }
-    __syncwarp();
+  }
+  // y = V^T x: thread (part, i) sums j in its part of [0, d)
+  {
+    const int nparts = 256 / d;
+    const int part = tid / d, i = tid % d;
+    const int jl = d / nparts;
+    double acc[NV];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) acc[v] = 0.0;
+    for (int j = part * jl; j < (part + 1) * jl; ++j) {
+      const double vv = V[(size_t)j * d + i];
+#pragma unroll
+      for (int v = 0; v < NV; ++v) acc[v] = fma(vv, xs[v][j], acc[v]);
+    }
+#pragma unroll
+    for (int v = 0; v < NV; ++v) ys[v][part * d + i] = acc[v];
+  }
+  __syncthreads();
+  // codes, packed into the record words; residual of the signal coordinates
+  for (int e = tid; e < NV * d; e += 256) {
+    const int v = e / d, i = e % d;
+    const int nparts = 256 / d;
+    double y = 0.0;
+    for (int pt = 0; pt < nparts; ++pt) y += ys[v][pt * d + i];
+    y *= s_inv[v];
+    const int bw = bits[i];
+    const double s = sig[i];
+    int code = 0;
+    if (bw > 0) {
+      code = code_of(s > 0.0 ? y * (1.0 / s) : 0.0, th + th_off(bw), bw);
+      const int o = offs[i], wi = o >> 5, sh = o & 31;
+      atomicOr(&wb[v][wi], (uint32_t)code << sh);
+      if (sh + bw > 32) atomicOr(&wb[v][wi + 1], (uint32_t)code >> (32 - sh));
+    }
+    if (i < m) xs[v][i] = y - s * (bw > 0 ? lv[lv_off(bw) + code] : 0.0);
+  }
+  __syncthreads();
+  // rho and the QJL sign bits: warp v
+  if (m > 0) {
+    double r2 = 0.0;
+    for (int k = lane; k < m; k += 32) r2 += xs[warp][k] * xs[warp][k];
+    r2 = warp_sum(r2);
+    for (int j = 0; j < m; ++j) {
+      double pj = 0.0;
+      for (int k = lane; k < m; k += 32) pj = fma(S[j * m + k], xs[warp][k], pj);
+      pj = warp_sum(pj);
+      if (lane == 0 && pj >= 0.0) {
+        const int o = cbits + j;
+        atomicOr(&wb[warp][o >> 5], 1u << (o & 31));
+      }
+    }
+    if (lane == 0 && s_ok[warp]) {
+      const int64_t vi = v0 + warp;
+      const int b = (int)(vi / n_tok);
+      const int64_t t = vi % n_tok;
+      const int64_t sp = start_pos ? (int64_t)start_pos[b] : 0;
+      c.rnorm[((size_t)b * n_heads + h) * c.cap + sp + t] = (float)sqrt(r2);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < NV * W; e += 256) {
+    const int v = e / W, w = e % W;
+    if (!s_ok[v]) continue;
+    const int64_t vi = v0 + v;
+    const int b = (int)(vi / n_tok);
+    const int64_t t = vi % n_tok;
+    const int64_t sp = start_pos ? (int64_t)start_pos[b] : 0;
+    c.codes[(((size_t)b * n_heads + h) * c.cap + sp + t) * W + w] = wb[v][w];
   }
 }
 

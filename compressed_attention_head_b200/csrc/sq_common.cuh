@@ -52,7 +52,7 @@ __host__ __device__ inline size_t derived_tc_off(int d) {
   return ((size_t)(256 + 8 * d) + 8 * (size_t)d * d + 1023) & ~(size_t)1023;
 }
 __host__ __device__ inline size_t derived_tc_bytes(int d) {
-  return d == 128 ? 6 * (size_t)d * d + 16 * (size_t)d + 8 * (size_t)d * d : 0;
+  return d == 128 ? 6 * (size_t)d * d + 16 * (size_t)d + 256 + 8 * (size_t)d * d : 0;
 }
 __host__ __device__ inline size_t derived_bytes(int d) { return derived_tc_off(d) + derived_tc_bytes(d); }
 __host__ __device__ inline size_t record_bytes(int d) {

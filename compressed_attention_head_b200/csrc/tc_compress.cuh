@@ -6,21 +6,25 @@
 // the signal dims), organised for B200:
 //
 //  * TMA streams tiles of 128 tokens x 128 fp16 (two 64-column boxes, 128-byte
-//    swizzle) through a 3-stage shared-memory ring.
-//  * One thread issues tcgen05.mma (M=128 tokens, N=128 coordinates, K=16):
-//    D = X * B with B = 2^s_i V_i / sigma_i split into fp16 hi + lo parts
-//    (about 22 significant bits), accumulated in fp32 in TMEM (two buffers).
-//  * Eight epilogue warps read D from TMEM (thread = token, 64 coordinates
-//    per warp), form z_i = D_i 2^-s_i / ||x||, and pick codes with register
-//    thresholds. Each coordinate carries a rigorous bound delta_i on
-//    |z_tensor - z_exact| (fp16 split residual + fp32 accumulation + rounding);
-//    a z within delta_i of a threshold is recomputed exactly in float64 by the
-//    whole warp, so every code equals the exact-arithmetic code.
-//  * Four signal warps (thread = token) compute ||x|| and the m QJL signal
-//    coordinates y_i exactly in float64, their codes, the residual, rho and
-//    the sign bits.
-//  * Codes are packed LSB-first into a shared-memory record tile and written
-//    back with coalesced stores.
+//    swizzle) into four shared-memory stages.
+//  * One thread issues tcgen05.mma (M = 128 tokens, N = 128 coordinates,
+//    K = 16): D = X * B with B = 2^s V / sigma split into fp16 hi + lo parts
+//    (about 22 significant bits), accumulated in fp32 in one of four TMEM
+//    accumulators.
+//  * Four epilogue groups of four warps each own one stage and one
+//    accumulator (tile k goes to group k mod 4), so no group ever waits for
+//    another. A thread owns one token row: it computes ||x|| (float32, or
+//    float64 with the exact signal coordinates, rho and the QJL signs for
+//    keys) straight from the staged tile, releases the stage, then reads its
+//    row of D from TMEM 16 columns at a time, forms z_i = D_i 2^-s / ||x||,
+//    picks each code (compare chains for widths 1-3, a cell table for 4-8)
+//    and appends it to a register bit stream that goes to global memory one
+//    32-bit word at a time.
+//  * Every z carries a bound on |z_tensor - z_exact| (fp16 split residual,
+//    fp32 accumulation, fp32 roundings). A z within that bound of a threshold
+//    is recomputed exactly in float64 by the whole warp from the input row and
+//    the float64 eigenvectors, so every code equals the exact-arithmetic code.
+// Heads whose QJL dimension m exceeds MSIG are left to the reference kernel.
 // Every mbarrier wait is bounded (see sm100.cuh); a timeout sets a device
 // flag bit and the kernel skips the remaining work without hanging.
 #pragma once
@@ -33,54 +37,72 @@ namespace tcc {
 
 constexpr int D = 128;
 constexpr int TILE = 128;
-constexpr int STAGES = 3;
+constexpr int NGRP = 3;                       // epilogue groups = X stages = TMEM accumulators
 constexpr int KB = D / 64;
 constexpr int X_BYTES = TILE * D * 2;
 constexpr int B_BYTES = D * D * 2;
-constexpr int NUM_WARPS = 14;
+constexpr int NUM_WARPS = 2 + 4 * NGRP;
 constexpr int NUM_THREADS = NUM_WARPS * 32;
-constexpr int WARP_PROD = 0, WARP_MMA = 1, WARP_SIG0 = 2, WARP_EPI0 = 6;
-constexpr int MAX_W = 12;
-constexpr int REC_PITCH = MAX_W + 1;
-constexpr uint32_t TMEM_COLS = 2 * D;
-constexpr float E_ACC = 4.76837158203125e-07f;   // 8 * 2^-24: default accumulation bound factor
-constexpr int QCAP = 256;                     // deferred exact recomputations per tile
-constexpr int MSIG = 8;                       // signal coordinates staged in shared memory
+constexpr int WARP_PROD = 0, WARP_MMA = 1, WARP_EPI0 = 2;
+constexpr uint32_t TMEM_COLS = 512;            // NGRP accumulators of D columns (a power of two)
+constexpr int MSIG = 8;                       // largest QJL dimension handled here
+constexpr int EACC_DEFAULT_UNITS = 32;        // accumulation bound factor, in units of 2^-24
 
 struct CoordInfo {
   uint32_t bo;       // bits (low 8) | bit offset << 8
-  float sc;          // 2^-s_i (column scale of B)
+  float sc;          // 2^-s (column scale of B, one per head)
   float dfix;        // split residual ||e_i|| + fp32 rounding of z, 1/||x||, thresholds
   float dacc;        // ||V_i / sigma_i|| = 1/sigma_i: multiplies the accumulation bound
 };
-// Radius = dfix + E * dacc, with E the fp32 accumulation bound per unit of
-// sum_j |x_j B_ij| / ||x|| <= ||B_i|| (Cauchy-Schwarz); E is a kernel argument.
+// Per-head summary used by the kernel: chunk classes and per-width radii.
+struct TcMeta {
+  uint32_t chunk[D / 16];   // width 0..8 if all 16 coordinates share it (no signal one), else kMixed
+  float dfix_w[12];         // max dfix over the non-signal coordinates of each width
+  float dacc_w[12];         // max dacc over the same
+  uint32_t reserved[32];
+};
+constexpr uint32_t kMixed = 0xFFu;
+static_assert(sizeof(TcMeta) == 256, "meta block is 256 bytes");
+
+// Cell tables of widths 4..8 (built on the host from the library codebook):
+// cell g of width b covers |z| in [g h_b, (g+1) h_b) with h_b = 2^-(b-2),
+// narrower than every gap between consecutive thresholds, so a cell holds at
+// most one threshold. cell[g] = number of positive thresholds below g h_b;
+// q[j] = (T_j, T_j+1, T_j+2) with T_0 = 0 and +inf past the last threshold.
+__host__ __device__ constexpr int cell_off(int b) {
+  return b == 4 ? 0 : b == 5 ? 16 : b == 6 ? 48 : b == 7 ? 112 : 240;
+}
+__host__ __device__ constexpr int cell_cap(int b) {
+  return b == 4 ? 16 : b == 5 ? 32 : b == 6 ? 64 : b == 7 ? 128 : 320;
+}
+constexpr int kCellBytes = 560;
+__host__ __device__ constexpr int q_off(int b) { return (1 << (b - 1)) - 8; }
+constexpr int kQEntries = 248;
+struct QuantConst {
+  float t2;            // positive threshold of width 2
+  float t3[3];         // positive thresholds of width 3
+  int ncell[12];       // cells in use per width (4..8)
+};
 
 // Byte offsets of the dynamic shared memory (base aligned to 1024).
 constexpr int OFF_X = 0;
-constexpr int OFF_BHI = OFF_X + STAGES * X_BYTES;
+constexpr int OFF_BHI = OFF_X + NGRP * X_BYTES;
 constexpr int OFF_BLO = OFF_BHI + B_BYTES;
-constexpr int OFF_BLO2 = OFF_BLO + B_BYTES;                 // third split term (exact recomputation only)
-constexpr int OFF_REC = OFF_BLO2 + B_BYTES;
-constexpr int REC_BYTES = 2 * TILE * REC_PITCH * 4;
-constexpr int OFF_RT = OFF_REC + REC_BYTES;                 // float [2][TILE]
-constexpr int OFF_N64 = OFF_RT + 2 * TILE * 4;              // double [2][TILE]
-constexpr int OFF_CI = OFF_N64 + 2 * TILE * 8;              // CoordInfo [D]
-constexpr int OFF_SIG = OFF_CI + D * 16;                    // double [D]
-constexpr int OFF_TH64 = OFF_SIG + D * 8;                   // double [kThreshTotal]
-constexpr int OFF_VSIG = (OFF_TH64 + kThreshTotal * 8 + 15) & ~15;   // double [MSIG][D]
-constexpr int OFF_Q = OFF_VSIG + MSIG * D * 8;              // u32 [QCAP] (token << 16 | coordinate)
-constexpr int OFF_BAR = (OFF_Q + QCAP * 4 + 7) & ~7;
-constexpr int N_BARS = 2 * STAGES + 1 + 2 + 2 + 2;
-constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;              // u32 [16]
-constexpr int OFF_CHUNK = OFF_MISC + 64;                    // u32 [8]: per 16-coordinate chunk, width | offset << 8
-constexpr int OFF_DW = OFF_CHUNK + 32;                      // float [9]: per-width radius
-constexpr int SMEM_BYTES = OFF_DW + 48 + 1024;              // + alignment slack
+constexpr int OFF_TH64 = OFF_BLO + B_BYTES;                         // double [kThreshTotal]
+constexpr int OFF_LV64 = OFF_TH64 + ((kThreshTotal * 8 + 15) & ~15);   // double [kLevelsTotal]
+constexpr int OFF_Q = OFF_LV64 + ((kLevelsTotal * 8 + 15) & ~15);      // float4 [kQEntries]
+constexpr int OFF_CELL = OFF_Q + kQEntries * 16;                       // u8 [kCellBytes]
+constexpr int OFF_BAR = OFF_CELL + kCellBytes;
+constexpr int N_BARS = 4 * NGRP + 2;
+constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;                         // u32 [16]
+constexpr int OFF_R = OFF_MISC + 64;                                   // float [NUM_WARPS][16]: radius per width
+constexpr int SMEM_BYTES = OFF_R + NUM_WARPS * 64 + 1024;              // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds 227 KB");
+static_assert(OFF_BAR % 8 == 0, "mbarriers need 8-byte alignment");
 
 // The tensor-core block inside the record's derived part (derived_tc_off):
 // Bhi, Blo, Blo2 [d*d fp16 each] (swizzled B operand; B = hi + lo + lo2 to
-// about 2^-33 relative), CoordInfo [d], Vt64 [d*d f64].
+// about 2^-33 relative), CoordInfo [d], TcMeta, Vt64 [d*d f64].
 struct TcView {
   uint8_t* base;
   int d;
@@ -88,7 +110,10 @@ struct TcView {
   __host__ __device__ __half* blo() const { return (__half*)(base + 2 * (size_t)d * d); }
   __host__ __device__ __half* blo2() const { return (__half*)(base + 4 * (size_t)d * d); }
   __host__ __device__ CoordInfo* ci() const { return (CoordInfo*)(base + 6 * (size_t)d * d); }
-  __host__ __device__ double* vt64() const { return (double*)(base + 6 * (size_t)d * d + 16 * (size_t)d); }
+  __host__ __device__ TcMeta* meta() const { return (TcMeta*)(base + 6 * (size_t)d * d + 16 * (size_t)d); }
+  __host__ __device__ double* vt64() const {
+    return (double*)(base + 6 * (size_t)d * d + 16 * (size_t)d + sizeof(TcMeta));
+  }
 };
 __host__ __device__ inline TcView tc_view(Rec r) { return TcView{r.derived() + derived_tc_off(r.d), r.d}; }
 
@@ -99,7 +124,7 @@ __host__ __device__ inline uint32_t sw128_off(int n, int k, int rows) {
   return (uint32_t)(kb * rows * 128 + (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4) + (w << 1));
 }
 
-// Builds the tensor-core block of one record (called with the block's threads).
+// Builds the tensor-core block of one record (called with all of the block's threads).
 __device__ void build_tc(Rec rec, int tid, int nth) {
   if (rec.d != D) return;
   TcView tv = tc_view(rec);
@@ -159,10 +184,31 @@ __device__ void build_tc(Rec rec, int tid, int nth) {
     c.dacc = (float)inv;
     tv.ci()[i] = c;
   }
+  __syncthreads();
+  if (tid == 0) {
+    TcMeta mt;
+    const int m = rec.hdr()->m;
+    for (int b = 0; b < 12; ++b) mt.dfix_w[b] = mt.dacc_w[b] = 0.0f;
+    for (int e = 0; e < 32; ++e) mt.reserved[e] = 0u;
+    for (int i = m; i < D; ++i) {
+      const int b = (int)(tv.ci()[i].bo & 0xFFu);
+      mt.dfix_w[b] = fmaxf(mt.dfix_w[b], tv.ci()[i].dfix);
+      mt.dacc_w[b] = fmaxf(mt.dacc_w[b], tv.ci()[i].dacc);
+    }
+    for (int c = 0; c < D / 16; ++c) {
+      const uint32_t b0 = tv.ci()[16 * c].bo & 0xFFu;
+      bool uni = 16 * c >= m;
+      for (int k = 1; k < 16 && uni; ++k) uni = (tv.ci()[16 * c + k].bo & 0xFFu) == b0;
+      mt.chunk[c] = uni ? b0 : kMixed;
+    }
+    *tv.meta() = mt;
+  }
+  __syncthreads();
 }
 
 struct Params {
   const uint8_t* recs;
+  const __half* x;   // the input rows (exact recomputations reread them)
   int n_heads, batch;
   int64_t n_tok;
   const int32_t* start_pos;
@@ -170,64 +216,96 @@ struct Params {
   uint32_t* flags;
   int64_t n_tiles;
   int tiles_per_row;
-  float eacc;        // accumulation bound factor of the radius (E_ACC by default)
+  float eacc;        // accumulation bound factor of the radius
 };
 
 // ---------------------------------------------------------------- quantizers
-__device__ __forceinline__ int q1(float z, float dl, bool& dg) {
-  dg = fabsf(z) < dl;
-  return z > 0.0f ? 1 : 0;
+// Each returns the code of z under the unit-Gaussian Lloyd-Max thresholds of
+// its width and sets dg when z lies within R of a threshold (including 0).
+// Ties in that band go to the exact recomputation, so the tie rule of the
+// fast path does not matter.
+__device__ __forceinline__ uint32_t qz1(float z, float R, bool& dg) {
+  dg = fabsf(z) < R;
+  return z > 0.0f ? 1u : 0u;
 }
-__device__ __forceinline__ int q2(float z, float t1, float dl, bool& dg) {
-  float a = fabsf(z);
-  int m = a > t1 ? 1 : 0;
-  dg = (a < dl) | (fabsf(a - t1) < dl);
-  return z > 0.0f ? 2 + m : 1 - m;
+__device__ __forceinline__ uint32_t qz2(float z, float t1, float R, bool& dg) {
+  const float a = fabsf(z);
+  dg = fminf(a, fabsf(a - t1)) < R;
+  const uint32_t m = a > t1 ? 1u : 0u;
+  return z > 0.0f ? 2u + m : 1u - m;
 }
-__device__ __forceinline__ int q3(float z, float t1, float t2, float t3, float dl, bool& dg) {
-  float a = fabsf(z);
-  int m = (a > t1 ? 1 : 0) + (a > t2 ? 1 : 0) + (a > t3 ? 1 : 0);
-  dg = (a < dl) | (fabsf(a - t1) < dl) | (fabsf(a - t2) < dl) | (fabsf(a - t3) < dl);
-  return z > 0.0f ? 4 + m : 3 - m;
+__device__ __forceinline__ uint32_t qz3(float z, float t1, float t2, float t3, float R, bool& dg) {
+  const float a = fabsf(z);
+  dg = fminf(fminf(a, fabsf(a - t1)), fminf(fabsf(a - t2), fabsf(a - t3))) < R;
+  const uint32_t m = (a > t1 ? 1u : 0u) + (a > t2 ? 1u : 0u) + (a > t3 ? 1u : 0u);
+  return z > 0.0f ? 4u + m : 3u - m;
 }
-__device__ __forceinline__ int qn(float z, const double* th, int b, float dl, bool& dg) {
-  const int n = (1 << b) - 1;
-  const int lo = code_of((double)z, th, b);
-  const double dlo = lo > 0 ? (double)z - th[lo - 1] : 1e30;
-  const double dhi = lo < n ? th[lo] - (double)z : 1e30;
-  dg = fmin(fabs(dlo), fabs(dhi)) < (double)dl;
-  return lo;
+// Widths 4..8: cell index by the 2^23 rounding trick (floor of |z| / h, or one
+// below it on an exact tie, both of which the table handles), then at most
+// one comparison.
+__device__ __forceinline__ uint32_t qzl(float z, const uint8_t* cell, const float4* q, float invh, int ncell,
+                                        uint32_t half, float R, bool& dg) {
+  const float a = fabsf(z);
+  int g = __float_as_int(fmaf(a, invh, 8388607.5f)) - 0x4B000000;
+  g = min(max(g, 0), ncell - 1);
+  const int lo = cell[g];
+  const float4 e = q[lo];
+  const uint32_t up = a > e.y ? 1u : 0u;
+  dg = fminf(fminf(a - e.x, fabsf(a - e.y)), e.z - a) < R;
+  const uint32_t m = (uint32_t)lo + up;
+  return z > 0.0f ? half + m : half - 1u - m;
 }
 
-// Codes of 16 consecutive coordinates of width B (1..3) from their tensor-core
-// values v (z = v * zr), packed LSB-first (16 * B bits), and the mask of the
-// coordinates whose z lies within dl of a threshold.
+// Per-thread quantization context of one segment (one head).
+struct QCtx {
+  const uint8_t* smb;      // shared-memory base (cell tables, radii)
+  int wr;                  // this warp's radius row: radius of width b at float index wr + b
+  float zr;                // 2^-s / ||x|| of this thread's row
+  __device__ __forceinline__ float R(int b) const { return ((const float*)(smb + OFF_R))[wr + b]; }
+  __device__ __forceinline__ const uint8_t* cell() const { return smb + OFF_CELL; }
+  __device__ __forceinline__ const float4* q() const { return (const float4*)(smb + OFF_Q); }
+};
+
 template <int B>
-__device__ __forceinline__ void chunk_codes(const float* v, float zr, float t1, float t2, float t3, float dl,
-                                            uint64_t& cw, uint32_t& dmask) {
-  cw = 0;
-  dmask = 0;
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const float z = v[k] * zr;
-    bool dg;
-    int code;
-    if (B == 1) code = q1(z, dl, dg);
-    else if (B == 2) code = q2(z, t1, dl, dg);
-    else code = q3(z, t1, t2, t3, dl, dg);
-    cw |= (uint64_t)(uint32_t)code << (B * k);
-    dmask |= (uint32_t)dg << k;
+__device__ __forceinline__ uint32_t quant(float z, const QCtx& c, const QuantConst& k, bool& dg) {
+  if (B == 1) return qz1(z, c.R(1), dg);
+  else if (B == 2) return qz2(z, k.t2, c.R(2), dg);
+  else if (B == 3) return qz3(z, k.t3[0], k.t3[1], k.t3[2], c.R(3), dg);
+  else
+    return qzl(z, c.cell() + cell_off(B), c.q() + q_off(B), (float)(1 << (B - 2)), k.ncell[B], 1u << (B - 1),
+               c.R(B), dg);
+}
+__device__ __forceinline__ uint32_t quant_rt(int b, float z, const QCtx& c, const QuantConst& k, bool& dg) {
+  switch (b) {
+    case 1: return quant<1>(z, c, k, dg);
+    case 2: return quant<2>(z, c, k, dg);
+    case 3: return quant<3>(z, c, k, dg);
+    case 4: return quant<4>(z, c, k, dg);
+    case 5: return quant<5>(z, c, k, dg);
+    case 6: return quant<6>(z, c, k, dg);
+    case 7: return quant<7>(z, c, k, dg);
+    default: return quant<8>(z, c, k, dg);
   }
 }
 
-// ORs the nbits-bit value cw into a record at bit position o (up to 3 words).
-__device__ __forceinline__ void or_bits(uint32_t* rw, int o, uint64_t cw, int nbits) {
-  const int wi = o >> 5, sh = o & 31;
-  const uint64_t a = cw << sh;
-  const uint32_t top = sh ? (uint32_t)(cw >> (64 - sh)) : 0u;
-  if ((uint32_t)a) atomicOr(&rw[wi], (uint32_t)a);
-  if ((uint32_t)(a >> 32)) atomicOr(&rw[wi + 1], (uint32_t)(a >> 32));
-  if (sh + nbits > 64 && top) atomicOr(&rw[wi + 2], top);
+// Little-endian bit stream of one record, written to global memory a word at
+// a time. fill and nw are the same in every lane of a warp (one head).
+struct Stream {
+  uint64_t acc;
+  int fill;
+  int nw;
+  uint32_t* dst;
+  bool st;
+};
+__device__ __forceinline__ void put(Stream& s, uint32_t v, int n) {   // 1 <= n <= 32, v < 2^n
+  s.acc |= (uint64_t)v << s.fill;
+  s.fill += n;
+  if (s.fill >= 32) {
+    if (s.st) s.dst[s.nw] = (uint32_t)s.acc;
+    ++s.nw;
+    s.acc >>= 32;
+    s.fill -= 32;
+  }
 }
 
 // Byte offset of the 16-byte chunk c (elements 8c .. 8c+7) of token row t in an X stage.
@@ -235,130 +313,183 @@ __device__ __forceinline__ uint32_t x_chunk(int t, int c) {
   return (uint32_t)((c >> 3) * (TILE * 128) + (t >> 3) * 1024 + (t & 7) * 128 + (((c & 7) ^ (t & 7)) << 4));
 }
 
-// One pass over token t's row: ||x||^2 and the first MM signal coordinates
-// sum_j x_j V[j][i] (float64), with the V rows staged in shared memory.
+// Exact code of coordinate i of input row xrow (whole warp; every lane returns it):
+// z = (V_i . x) / ||x|| / sigma_i in float64, then the b-bit thresholds.
+__device__ __forceinline__ uint32_t exact_code(const __half* x, int64_t xrow, int i, int b, const double* vt64,
+                                            const double* sig, bool normalize, const double* th64, int lane) {
+  const uint2 raw = *(const uint2*)(x + xrow * D + 4 * lane);
+  const __half2* hh = reinterpret_cast<const __half2*>(&raw);
+  const double2 v01 = *(const double2*)(vt64 + (size_t)i * D + 4 * lane);
+  const double2 v23 = *(const double2*)(vt64 + (size_t)i * D + 4 * lane + 2);
+  const float2 a = __half22float2(hh[0]), c = __half22float2(hh[1]);
+  double dot = (double)a.x * v01.x;
+  dot = fma((double)a.y, v01.y, dot);
+  dot = fma((double)c.x, v23.x, dot);
+  dot = fma((double)c.y, v23.y, dot);
+  double n2 = (double)a.x * a.x;
+  n2 = fma((double)a.y, (double)a.y, n2);
+  n2 = fma((double)c.x, (double)c.x, n2);
+  n2 = fma((double)c.y, (double)c.y, n2);
+  dot = warp_sum(dot);
+  n2 = warp_sum(n2);
+  const double nrm = normalize ? sqrt(n2) : 1.0;
+  const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
+  const double s = sig[i];
+  const double z = s > 0.0 ? dot * inv / s : 0.0;
+  return (uint32_t)code_of(z, th64 + th_off(b), b);
+}
+
+// Norm phase of a key row with QJL (m <= MM signal coordinates): ||x|| and
+// y_i = V_i . x for i < MM in float64 from the staged tile (the rows i >= m
+// are computed and ignored), then the signal codes, the residual
+// r_i = y_i / ||x|| - sigma_i level_i, rho = ||r|| and the m sign bits of S r.
 template <int MM>
-__device__ __forceinline__ void row_pass(const uint8_t* xs, int t, const double* vsig, double& n2, double* ys) {
-#pragma unroll 2
+__device__ __forceinline__ void key_pass(const uint8_t* xs, int t, int m, const double* vt64, const double* sig,
+                                         const uint8_t* bits, const double* S, bool normalize, const double* th64,
+                                         const double* lv64, double& nrm, double& rho2, uint32_t (&sc4)[4],
+                                         uint32_t& qbits) {
+  double n2a = 0.0, n2b = 0.0;
+  double ys[MM];
+#pragma unroll
+  for (int i = 0; i < MM; ++i) ys[i] = 0.0;
+#pragma unroll 1
   for (int c = 0; c < D / 8; ++c) {
     const uint4 raw = *(const uint4*)(xs + x_chunk(t, c));
     const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 f = __half22float2(h2[q]);
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(h2[e]);
       const double x0 = f.x, x1 = f.y;
-      n2 = fma(x0, x0, n2);
-      n2 = fma(x1, x1, n2);
-      const int j = c * 8 + 2 * q;
+      n2a = fma(x0, x0, n2a);
+      n2b = fma(x1, x1, n2b);
+      const int jj = c * 8 + 2 * e;
 #pragma unroll
-      for (int ii = 0; ii < MM; ++ii) {
-        const double2 v = *(const double2*)(vsig + ii * D + j);
-        ys[ii] = fma(x0, v.x, ys[ii]);
-        ys[ii] = fma(x1, v.y, ys[ii]);
+      for (int i = 0; i < MM; ++i) {
+        const double2 vv = __ldg((const double2*)(vt64 + (size_t)i * D + jj));
+        ys[i] = fma(x0, vv.x, ys[i]);
+        ys[i] = fma(x1, vv.y, ys[i]);
+      }
+      asm volatile("" ::: "memory");   // one pair's rows in flight at a time (register budget)
+    }
+  }
+  nrm = normalize ? sqrt(n2a + n2b) : 1.0;
+  const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
+  rho2 = 0.0;
+#pragma unroll
+  for (int i = 0; i < MM; ++i) {
+    if (i < m) {
+      const int b = bits[i];
+      const double yn = ys[i] * inv;
+      double lvv = 0.0;
+      if (b > 0) {
+        const double s = sig[i];
+        const double z = s > 0.0 ? yn / s : 0.0;
+        const int code = code_of(z, th64 + th_off(b), b);
+        lvv = lv64[lv_off(b) + code];
+        sc4[i >> 2] |= (uint32_t)code << ((i & 3) * 8);
+      }
+      ys[i] = yn - sig[i] * lvv;
+      rho2 = fma(ys[i], ys[i], rho2);
+    }
+  }
+  qbits = 0u;
+  for (int j = 0; j < m; ++j) {
+    double pj = 0.0;
+#pragma unroll
+    for (int i = 0; i < MM; ++i)
+      if (i < m) pj = fma(S[j * m + i], ys[i], pj);
+    qbits |= (pj >= 0.0 ? 1u : 0u) << j;
+  }
+}
+
+// Replaces field k (width B) of the 16-code chunk words cw.
+template <int B>
+__device__ __forceinline__ void patch_chunk(uint32_t (&cw)[4], int k, uint32_t code) {
+  const int p = B * k, wi = p >> 5, sh = p & 31;
+  const uint32_t mask = (1u << B) - 1u;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    if (w == wi) cw[w] = (cw[w] & ~(mask << sh)) | (code << sh);
+    if (w == wi + 1 && sh + B > 32) {
+      const int r = 32 - sh;
+      cw[w] = (cw[w] & ~(mask >> r)) | (code >> r);
+    }
+  }
+}
+
+// One width-uniform chunk of 16 coordinates: codes into cw (compile-time
+// positions), exact recomputation of the in-band ones, then the stream.
+template <int B>
+__device__ __forceinline__ void chunk_uniform(const float* v, const QCtx& qc, const QuantConst& kq, bool fix_ok,
+                                              int i0, const __half* x, int64_t xbase, const double* vt64,
+                                              const double* sig, bool normalize, const double* th64, int lane,
+                                              Stream& s) {
+  uint32_t cw[4] = {0u, 0u, 0u, 0u};
+  uint32_t dm = 0u;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    bool dg;
+    const uint32_t code = quant<B>(v[k] * qc.zr, qc, kq, dg);
+    dm |= dg ? (1u << k) : 0u;
+    const int p = B * k;
+    cw[p >> 5] |= code << (p & 31);
+    if ((p & 31) + B > 32) cw[(p >> 5) + 1] |= code >> (32 - (p & 31));
+  }
+  dm = fix_ok ? dm : 0u;
+  if (__any_sync(0xffffffffu, dm != 0u)) {
+    for (;;) {
+      const uint32_t who = __ballot_sync(0xffffffffu, dm != 0u);
+      if (!who) break;
+      const int src = __ffs(who) - 1;
+      const int k = __ffs(__shfl_sync(0xffffffffu, dm, src)) - 1;
+      const uint32_t code = exact_code(x, xbase + src, i0 + k, B, vt64, sig, normalize, th64, lane);
+      if (lane == src) {
+        patch_chunk<B>(cw, k, code);
+        dm &= dm - 1u;
       }
     }
   }
-}
-
-// Exact (float64) dot product of token t's row with a global row of D doubles.
-__device__ __forceinline__ double exact_dot(const uint8_t* xs, int t, const double* vrow) {
-  double acc = 0.0;
-#pragma unroll 2
-  for (int c = 0; c < D / 8; ++c) {
-    const uint4 raw = *(const uint4*)(xs + x_chunk(t, c));
-    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-    const double2* vr = reinterpret_cast<const double2*>(vrow + c * 8);
+  constexpr int NB = 16 * B;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 f = __half22float2(h2[q]);
-      const double2 v = vr[q];
-      acc = fma((double)f.x, v.x, acc);
-      acc = fma((double)f.y, v.y, acc);
-    }
-  }
-  return acc;
-}
-
-// sum_j x[t][j] * (hi + lo + lo2)[i][j] in float64 by one warp (lane l takes
-// j = 4l .. 4l+3); every lane returns the sum. The three fp16 terms represent
-// B to about 2^-33 relative, so z = sum * 2^-s / ||x|| matches exact
-// arithmetic to ~1e-9, far inside the 1e-5 exemption band.
-__device__ __forceinline__ double exact_sum_warp(const uint8_t* xs, const uint8_t* bh, const uint8_t* bl,
-                                                 const uint8_t* bl2, int t, int i, int lane) {
-  const int j = 4 * lane;
-  const uint2 xr = *(const uint2*)(xs + x_chunk(t, j >> 3) + ((j & 7) << 1));
-  const uint32_t bo = sw128_off(i, j, D);
-  const uint2 h = *(const uint2*)(bh + bo), l = *(const uint2*)(bl + bo), l2 = *(const uint2*)(bl2 + bo);
-  const __half2* xh = reinterpret_cast<const __half2*>(&xr);
-  const __half2* hh = reinterpret_cast<const __half2*>(&h);
-  const __half2* lh = reinterpret_cast<const __half2*>(&l);
-  const __half2* l2h = reinterpret_cast<const __half2*>(&l2);
-  double acc = 0.0;
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const float2 xf = __half22float2(xh[k]), hf = __half22float2(hh[k]);
-    const float2 lf = __half22float2(lh[k]), l2f = __half22float2(l2h[k]);
-    acc = fma((double)xf.x, ((double)hf.x + (double)lf.x) + (double)l2f.x, acc);
-    acc = fma((double)xf.y, ((double)hf.y + (double)lf.y) + (double)l2f.y, acc);
-  }
-  return warp_sum(acc);
-}
-
-// Overwrites the b-bit field at bit o of a record with code.
-__device__ __forceinline__ void patch_field(uint32_t* rw, int o, int b, uint32_t code) {
-  const int wi = o >> 5, sh = o & 31;
-  const uint32_t mask = (1u << b) - 1u;
-  atomicAnd(&rw[wi], ~(mask << sh));
-  atomicOr(&rw[wi], code << sh);
-  if (sh + b > 32) {
-    atomicAnd(&rw[wi + 1], ~(mask >> (32 - sh)));
-    atomicOr(&rw[wi + 1], code >> (32 - sh));
-  }
+  for (int w = 0; w < NB / 32; ++w) put(s, cw[w], 32);
+  if (NB % 32) put(s, cw[NB / 32], 16);
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P) {
+k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_constant__ QuantConst KQ) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sX = sm + OFF_X;
   uint8_t* sBhi = sm + OFF_BHI;
   uint8_t* sBlo = sm + OFF_BLO;
-  uint8_t* sBlo2 = sm + OFF_BLO2;
-  uint32_t* sRec = (uint32_t*)(sm + OFF_REC);
-  float* sRt = (float*)(sm + OFF_RT);
-  double* sN64 = (double*)(sm + OFF_N64);
-  CoordInfo* sCI = (CoordInfo*)(sm + OFF_CI);
-  double* sSig = (double*)(sm + OFF_SIG);
   double* sTh64 = (double*)(sm + OFF_TH64);
-  double* sVsig = (double*)(sm + OFF_VSIG);
-  uint32_t* sQ = (uint32_t*)(sm + OFF_Q);
+  double* sLv64 = (double*)(sm + OFF_LV64);
+  float4* sQ = (float4*)(sm + OFF_Q);
+  uint8_t* sCell = sm + OFF_CELL;
   uint64_t* bars = (uint64_t*)(sm + OFF_BAR);
-  uint64_t* full = bars;                    // [STAGES]
-  uint64_t* empty = bars + STAGES;          // [STAGES]
-  uint64_t* bfull = bars + 2 * STAGES;      // 1
-  uint64_t* tfull = bfull + 1;              // [2]
-  uint64_t* tempty = tfull + 2;             // [2]
-  uint64_t* sfull = tempty + 2;             // [2]
-  uint32_t* misc = (uint32_t*)(sm + OFF_MISC);
-  // misc: [0] tmem base, [1] abort, [2] segment ok, [3] m, [4] W, [5] code_bits, [6] flags, [8] start,
-  //       [9] queue length
+  uint64_t* full = bars;                    // [NGRP] X stage landed
+  uint64_t* empty = bars + NGRP;            // [NGRP] X stage free (MMA done + 4 epilogue warps)
+  uint64_t* tfull = bars + 2 * NGRP;        // [NGRP] accumulator ready
+  uint64_t* tempty = bars + 3 * NGRP;       // [NGRP] accumulator drained
+  uint64_t* bfull = bars + 4 * NGRP;        // B operand landed
+  uint64_t* bempty = bfull + 1;             // B operand no longer read
+  uint32_t* misc = (uint32_t*)(sm + OFF_MISC);   // [0] tmem base, [1] abort
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  for (int e = threadIdx.x; e < 2 * TILE * REC_PITCH; e += NUM_THREADS) sRec[e] = 0u;
   for (int e = threadIdx.x; e < kThreshTotal; e += NUM_THREADS) sTh64[e] = c_th64[e];
+  for (int e = threadIdx.x; e < kLevelsTotal; e += NUM_THREADS) sLv64[e] = c_lv64[e];
+  for (int e = threadIdx.x; e < kQEntries; e += NUM_THREADS) sQ[e] = c_tcq[e];
+  for (int e = threadIdx.x; e < kCellBytes; e += NUM_THREADS) sCell[e] = c_tccell[e];
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NGRP; ++s) {
       sm100::mbar_init(&full[s], 1);
-      sm100::mbar_init(&empty[s], 1 + 4 + 8);
+      sm100::mbar_init(&empty[s], 1 + 4);
+      sm100::mbar_init(&tfull[s], 1);
+      sm100::mbar_init(&tempty[s], 4);
     }
     sm100::mbar_init(bfull, 1);
-    for (int b = 0; b < 2; ++b) {
-      sm100::mbar_init(&tfull[b], 1);
-      sm100::mbar_init(&tempty[b], 8);
-      sm100::mbar_init(&sfull[b], 4);
-    }
+    sm100::mbar_init(bempty, 1);
     misc[1] = 0u;
-    misc[9] = 0u;
     sm100::fence_mbar_init();
   }
   if (warp == WARP_MMA) {
@@ -376,8 +507,16 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P) {
   const int64_t per = (P.n_tiles + gridDim.x - 1) / gridDim.x;
   const int64_t tb = (int64_t)blockIdx.x * per;
   const int64_t te = min(P.n_tiles, tb + per);
-  uint32_t iter = 0, seg = 0;   // seg counts the segments that load B
   const uint32_t idesc = sm100::idesc_f16(TILE, D);
+  // Every role walks the same sequence of segments (rows of tiles of one
+  // (batch, head)) and skips the same invalid ones, so k (tiles processed)
+  // and nseg (segments processed) agree across roles.
+  uint32_t k = 0, nseg = 0;
+  uint32_t x_issued = 0, b_issued = 0;   // producer: X tiles and B operands requested (a prefix of each)
+
+  const int grp = (warp - WARP_EPI0) >> 2;             // epilogue group (warps 2..17)
+  const int qtr = warp & 3;                            // TMEM lane quarter of this warp
+  const int t_row = qtr * 32 + lane;                   // token row within the tile
 
   for (int64_t s0 = tb; s0 < te;) {
     const int64_t row = s0 / P.tiles_per_row;
@@ -385,324 +524,234 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P) {
     const int h = (int)(row % P.n_heads);
     const int bidx = (int)(row / P.n_heads);
     Rec rec = rec_at(P.recs, D, h);
-    TcView tv = tc_view(rec);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const RecHeader* hd = rec.hdr();
-      bool ok = record_ok(hd, D) && hd->words == P.c.words && hd->words <= MAX_W &&
-                (hd->m == 0 || P.c.rnorm != nullptr);
-      const int64_t sp = P.start_pos ? (int64_t)P.start_pos[bidx] : 0;
-      bool cap_ok = sp >= 0 && sp + P.n_tok <= P.c.cap;
-      if (!ok && err) atomicOr(err, SQ_FLAG_RECORD);
-      if (ok && !cap_ok && err) atomicOr(err, SQ_FLAG_CAPACITY);
-      misc[2] = (ok && cap_ok) ? 1u : 0u;
-      misc[3] = ok ? hd->m : 0;
-      misc[4] = hd->words;
-      misc[5] = hd->code_bits;
-      misc[6] = hd->flags;
-      misc[8] = (uint32_t)sp;
+    const RecHeader* hd = rec.hdr();
+    const bool rec_ok = record_ok(hd, D) && hd->words == P.c.words && (hd->m == 0 || P.c.rnorm != nullptr);
+    const int64_t sp = P.start_pos ? (int64_t)P.start_pos[bidx] : 0;
+    const bool cap_ok = sp >= 0 && sp + P.n_tok <= P.c.cap;
+    if (threadIdx.x == 0 && err) {
+      if (!rec_ok) atomicOr(err, SQ_FLAG_RECORD);
+      else if (!cap_ok) atomicOr(err, SQ_FLAG_CAPACITY);
     }
-    __syncthreads();
-    const bool seg_ok = misc[2] != 0 && *abort_flag == 0;
-    const int m = (int)misc[3], W = (int)misc[4], cbits = (int)misc[5];
-    const bool normalize = (misc[6] & kFlagNormalize) != 0;
-    const int64_t sp = (int64_t)misc[8];
-    if (!seg_ok) {       // nothing of this segment is touched
+    const int m = rec_ok ? hd->m : 0;
+    if (!rec_ok || !cap_ok || m > MSIG) {   // m > MSIG: the reference kernel takes this head
       s0 = s1;
       continue;
     }
-    for (int i = threadIdx.x; i < D; i += NUM_THREADS) {
-      sCI[i] = tv.ci()[i];
-      sSig[i] = rec.sigma()[i];
-    }
-    const int msig = m < MSIG ? m : MSIG;
-    for (int e = threadIdx.x; e < msig * D; e += NUM_THREADS) sVsig[e] = tv.vt64()[e];
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      // Per-width radius: the largest of its coordinates (the signal ones are exact).
-      float* dw = (float*)(sm + OFF_DW);
-      for (int b = 0; b <= SQ_MAX_BITS; ++b) dw[b] = 0.0f;
-      for (int i = m; i < D; ++i) {
-        const int b = (int)(sCI[i].bo & 0xFFu);
-        dw[b] = fmaxf(dw[b], fmaf(P.eacc, sCI[i].dacc, sCI[i].dfix));
-      }
-      // 16-coordinate chunks of one width in 1..3 with no signal coordinate take the fast path.
-      uint32_t* ch = (uint32_t*)(sm + OFF_CHUNK);
-      for (int c = 0; c < D / 16; ++c) {
-        const int b0 = (int)(sCI[16 * c].bo & 0xFFu);
-        bool uni = b0 >= 1 && b0 <= 3 && 16 * c >= m;
-        for (int k = 1; k < 16 && uni; ++k) uni = (int)(sCI[16 * c + k].bo & 0xFFu) == b0;
-        ch[c] = (uni ? (uint32_t)b0 : 0u) | ((sCI[16 * c].bo >> 8) << 8);
-      }
-    }
-    if (warp == WARP_PROD && lane == 0) {
-      sm100::mbar_expect_tx(bfull, 3 * B_BYTES);
-      sm100::bulk_load(sBhi, tv.bhi(), B_BYTES, bfull);
-      sm100::bulk_load(sBlo, tv.blo(), B_BYTES, bfull);
-      sm100::bulk_load(sBlo2, tv.blo2(), B_BYTES, bfull);
-    }
-    __syncthreads();
-    const uint32_t bpar = seg & 1u;
+    TcView tv = tc_view(rec);
     const int64_t nt = s1 - s0;
 
     if (warp == WARP_PROD) {
       if (lane == 0) {
-        for (int64_t k = 0; k < nt; ++k) {
-          const uint32_t it = iter + (uint32_t)k;
-          const int st = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
+        bool ok = *abort_flag == 0;
+        if (ok && nseg > 0) ok = sm100::mbar_wait(bempty, (nseg - 1) & 1u, err);
+        if (!ok) {
+          *abort_flag = 1;
+        } else {
+          sm100::mbar_expect_tx(bfull, 2 * B_BYTES);
+          sm100::bulk_load(sBhi, tv.bhi(), B_BYTES, bfull);
+          sm100::bulk_load(sBlo, tv.blo(), B_BYTES, bfull);
+          ++b_issued;
+        }
+        for (int64_t j = 0; j < nt; ++j) {
+          const uint32_t kk = k + (uint32_t)j;
+          const int st = (int)(kk % NGRP);
+          const uint32_t ph = (kk / NGRP) & 1u;
           if (*abort_flag || !sm100::mbar_wait(&empty[st], ph ^ 1u, err)) { *abort_flag = 1; continue; }
-          const int64_t tile = s0 + k;
+          const int64_t tile = s0 + j;
           const int t0 = (int)((tile - row * P.tiles_per_row) * TILE);
           const int ycoord = (int)(row * P.n_tok + t0);
           sm100::mbar_expect_tx(&full[st], X_BYTES);
           for (int kb = 0; kb < KB; ++kb)
             sm100::tma_load_2d(sX + st * X_BYTES + kb * (TILE * 128), &tmap, &full[st], kb * 64, ycoord);
+          ++x_issued;
         }
       }
     } else if (warp == WARP_MMA) {
       if (lane == 0) {
-        bool bok = *abort_flag == 0 && sm100::mbar_wait(bfull, bpar, err);
-        if (!bok) *abort_flag = 1;
-        for (int64_t k = 0; k < nt; ++k) {
-          const uint32_t it = iter + (uint32_t)k;
-          const int st = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
-          const int buf = it & 1;
-          const uint32_t bph = (it >> 1) & 1u;
+        if (*abort_flag || !sm100::mbar_wait(bfull, nseg & 1u, err)) *abort_flag = 1;
+        for (int64_t j = 0; j < nt; ++j) {
+          const uint32_t kk = k + (uint32_t)j;
+          const int st = (int)(kk % NGRP);
+          const uint32_t ph = (kk / NGRP) & 1u;
           if (*abort_flag || !sm100::mbar_wait(&full[st], ph, err) ||
-              !sm100::mbar_wait(&tempty[buf], bph ^ 1u, err)) {
+              !sm100::mbar_wait(&tempty[st], ph ^ 1u, err)) {
             *abort_flag = 1;
             continue;
           }
           sm100::tc_fence_after();
-          const uint32_t dt = tmem_base + (uint32_t)(buf * D);
+          const uint32_t dt = tmem_base + (uint32_t)(st * D);
           const uint32_t xa = sm100::smem_u32(sX + st * X_BYTES);
           const uint32_t bh = sm100::smem_u32(sBhi), bl = sm100::smem_u32(sBlo);
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t ao = kb * (TILE * 128) + kk * 32, bo = kb * (D * 128) + kk * 32;
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const uint32_t ao = kb * (TILE * 128) + k4 * 32, bo = kb * (D * 128) + k4 * 32;
               const uint64_t ad = sm100::sw128_desc(xa + ao);
-              sm100::mma_f16(dt, ad, sm100::sw128_desc(bh + bo), idesc, (kb | kk) ? 1u : 0u);
+              sm100::mma_f16(dt, ad, sm100::sw128_desc(bh + bo), idesc, (kb | k4) ? 1u : 0u);
               sm100::mma_f16(dt, ad, sm100::sw128_desc(bl + bo), idesc, 1u);
             }
           }
           sm100::mma_commit(&empty[st]);
-          sm100::mma_commit(&tfull[buf]);
+          sm100::mma_commit(&tfull[st]);
         }
+        sm100::mma_commit(bempty);
       }
     } else {
-      // ---------------- worker warps: signal (2..5) and epilogue (6..13)
-      const bool is_sig = warp < WARP_EPI0;
-      const int q = warp & 3, hh = (warp - WARP_EPI0) >> 2;
-      const int t_sig = (warp - WARP_SIG0) * 32 + lane;
-      const int t_epi = q * 32 + lane;
-      const int worker = threadIdx.x - WARP_SIG0 * 32;       // 0 .. 383
-      const int epi_id = threadIdx.x - WARP_EPI0 * 32;       // 0 .. 255 for epilogue threads
-      const float t21 = (float)sTh64[th_off(2) + 2];
-      const float t31 = (float)sTh64[th_off(3) + 4], t32 = (float)sTh64[th_off(3) + 5];
-      const float t33 = (float)sTh64[th_off(3) + 6];
-      const int wid = warp - WARP_SIG0;                        // worker warp 0 .. 11
+      // ---------------- epilogue group grp: tiles k with k mod NGRP == grp
+      const int W = hd->words;
+      const bool normalize = (hd->flags & kFlagNormalize) != 0;
+      const TcMeta* mt = tv.meta();
+      const double* vt64 = tv.vt64();
+      const double* sig = rec.sigma();
+      const uint8_t* bits = rec.bits();
+      QCtx qc;
+      qc.smb = sm;
+      qc.wr = warp * 16;
+      qc.zr = 0.0f;
+      __syncwarp();
+      if (lane <= 8)
+        ((float*)(sm + OFF_R))[warp * 16 + lane] = fmaf(P.eacc, mt->dacc_w[lane], mt->dfix_w[lane]) + 2.0e-6f;
+      __syncwarp();
+      const float sc = tv.ci()[0].sc;
       const double* S = rec.S();
-      for (int64_t k = 0; k < nt; ++k) {
-        const uint32_t it = iter + (uint32_t)k;
-        const int st = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1u;
-        const int buf = it & 1;
-        const uint32_t bph = (it >> 1) & 1u;
-        const int64_t tile = s0 + k;
+      for (int64_t j = 0; j < nt; ++j) {
+        const uint32_t kk = k + (uint32_t)j;
+        if ((int)(kk % NGRP) != grp) continue;
+        const int st = grp;
+        const uint32_t ph = (kk / NGRP) & 1u;
+        const int64_t tile = s0 + j;
         const int t0 = (int)((tile - row * P.tiles_per_row) * TILE);
         const int n_valid = (int)min((int64_t)TILE, P.n_tok - t0);
+        const bool valid = t_row < n_valid;
         const uint8_t* xs = sX + st * X_BYTES;
-        bool live;
-        if (is_sig) {
-          // ---- norm, exact signal coordinates, their codes, rho, QJL signs
-          live = __all_sync(0xffffffffu, *abort_flag == 0 && sm100::mbar_wait(&full[st], ph, err));
-          if (!live) *abort_flag = 1;
-          const int t = t_sig;
-          const bool valid = live && t < n_valid;
-          uint32_t* rw = sRec + (buf * TILE + t) * REC_PITCH;
-          double n2 = 0.0;
-          double ys[MSIG];
+        const size_t slot = ((size_t)bidx * P.n_heads + h) * P.c.cap + sp + t0 + t_row;
+        const int64_t xbase = row * P.n_tok + t0 + qtr * 32;   // input row of lane 0 of this warp
+
+        bool live = __all_sync(0xffffffffu, *abort_flag == 0 && sm100::mbar_wait(&full[st], ph, err));
+        if (!live) *abort_flag = 1;
+        // ---- norm phase (reads the staged tile)
+        float inv32 = 0.0f;
+        uint32_t sc4[4] = {0u, 0u, 0u, 0u};   // exact codes of the signal coordinates (8 bits each)
+        uint32_t qbits = 0u;
+        if (live) {
+          if (m == 0) {
+            float acc[16];
 #pragma unroll
-          for (int ii = 0; ii < MSIG; ++ii) ys[ii] = 0.0;
-          if (live) {
-            if (msig == 0) row_pass<0>(xs, t, sVsig, n2, ys);
-            else if (msig <= 2) row_pass<2>(xs, t, sVsig, n2, ys);
-            else if (msig <= 4) row_pass<4>(xs, t, sVsig, n2, ys);
-            else row_pass<8>(xs, t, sVsig, n2, ys);
-          }
-          const double nrm = normalize ? sqrt(n2) : 1.0;
-          const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
-          sRt[buf * TILE + t] = (float)inv;
-          sN64[buf * TILE + t] = nrm;
-          double rho2 = 0.0;
-          if (valid && m > 0) {
-            double r[D];     // residual of the signal coordinates (first m used)
-            for (int i = 0; i < m; ++i) {
-              double y;
-              if (i < MSIG) {
-                y = ys[0];
+            for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
 #pragma unroll
-                for (int ii = 1; ii < MSIG; ++ii) if (ii == i) y = ys[ii];
-              } else {
-                y = exact_dot(xs, t, tv.vt64() + (size_t)i * D);
-              }
-              const int b = (int)(sCI[i].bo & 0xFFu);
-              const double yn = y * inv;
-              double lvv = 0.0;
-              if (b > 0) {
-                const double z = sSig[i] > 0.0 ? yn / sSig[i] : 0.0;
-                const int code = code_of(z, sTh64 + th_off(b), b);
-                lvv = c_lv64[lv_off(b) + code];
-                const int o = (int)(sCI[i].bo >> 8), wi = o >> 5, sh = o & 31;
-                atomicOr(&rw[wi], (uint32_t)code << sh);
-                if (sh + b > 32) atomicOr(&rw[wi + 1], (uint32_t)code >> (32 - sh));
-              }
-              r[i] = yn - sSig[i] * lvv;
-              rho2 += r[i] * r[i];
-            }
-            for (int j = 0; j < m; ++j) {
-              double pj = 0.0;
-              for (int i = 0; i < m; ++i) pj = fma(S[j * m + i], r[i], pj);
-              if (pj >= 0.0) {
-                const int o = cbits + j;
-                atomicOr(&rw[o >> 5], 1u << (o & 31));
+            for (int c = 0; c < D / 8; ++c) {
+              const uint4 raw = *(const uint4*)(xs + x_chunk(t_row, c));
+              const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(h2[e]);
+                acc[(c & 1) * 8 + 2 * e] = fmaf(f.x, f.x, acc[(c & 1) * 8 + 2 * e]);
+                acc[(c & 1) * 8 + 2 * e + 1] = fmaf(f.y, f.y, acc[(c & 1) * 8 + 2 * e + 1]);
               }
             }
-          }
-          if (valid) {
-            const size_t slot = ((size_t)bidx * P.n_heads + h) * P.c.cap + sp + t0 + t;
-            P.c.norm[slot] = (float)nrm;
-            if (P.c.rnorm) P.c.rnorm[slot] = (float)sqrt(rho2);
-          }
-          __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(&sfull[buf]);
-        } else {
-          // ---- epilogue: TMEM -> codes -> packed record words
-          live = __all_sync(0xffffffffu, *abort_flag == 0 && sm100::mbar_wait(&tfull[buf], bph, err) &&
-                                             sm100::mbar_wait(&sfull[buf], bph, err));
-          if (!live) *abort_flag = 1;
-          sm100::tc_fence_after();
-          const int t = t_epi;
-          const float r = sRt[buf * TILE + t];
-          const bool valid = live && t < n_valid;
-          const bool exact_zero = r == 0.0f;
-          uint32_t* rw = sRec + (buf * TILE + t) * REC_PITCH;
-          const float eacc = P.eacc;
-          const float zr = sCI[0].sc * r;
-          const float* dw = (const float*)(sm + OFF_DW);
-          const uint32_t* chd = (const uint32_t*)(sm + OFF_CHUNK);
-          const bool enq_ok = valid && !exact_zero;
-          if (live) {
-            for (int c = 0; c < 4; ++c) {
-              float v[16];
-              sm100::tmem_ld16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * D + hh * 64 + c * 16), v);
-              const int i0 = hh * 64 + c * 16;
-              const uint32_t cd = chd[i0 >> 4];
-              const int cb = (int)(cd & 0xFFu);
-              uint32_t dmask = 0;
-              if (cb != 0) {
-                // width-uniform chunk: codes packed with compile-time shifts
-                uint64_t cw;
-                if (cb == 1) chunk_codes<1>(v, zr, 0.f, 0.f, 0.f, dw[1], cw, dmask);
-                else if (cb == 2) chunk_codes<2>(v, zr, t21, 0.f, 0.f, dw[2], cw, dmask);
-                else chunk_codes<3>(v, zr, t31, t32, t33, dw[3], cw, dmask);
-                if (valid) or_bits(rw, (int)(cd >> 8), cw, 16 * cb);
-              } else {
+            double n2 = 0.0;
 #pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
-                  const int i = i0 + kk;
-                  const CoordInfo ci = sCI[i];
-                  const int b = (int)(ci.bo & 0xFFu);
-                  if (b == 0 || i < m) continue;
-                  const float z = v[kk] * zr;
-                  const float dl = fmaf(eacc, ci.dacc, ci.dfix);
+            for (int e = 0; e < 16; ++e) n2 += (double)acc[e];
+            const double nrm = normalize ? sqrt(n2) : 1.0;
+            inv32 = nrm > 0.0 ? (float)(1.0 / nrm) : 0.0f;
+            if (valid) P.c.norm[slot] = (float)nrm;
+          } else {
+            // keys with QJL: ||x||, the m signal coordinates, their codes, the
+            // residual, rho and the sign bits, all in float64
+            double nrm, rho2;
+            if (m <= 2) key_pass<2>(xs, t_row, m, vt64, sig, bits, S, normalize, sTh64, sLv64, nrm, rho2, sc4, qbits);
+            else if (m <= 4) key_pass<4>(xs, t_row, m, vt64, sig, bits, S, normalize, sTh64, sLv64, nrm, rho2, sc4, qbits);
+            else key_pass<8>(xs, t_row, m, vt64, sig, bits, S, normalize, sTh64, sLv64, nrm, rho2, sc4, qbits);
+            inv32 = nrm > 0.0 ? (float)(1.0 / nrm) : 0.0f;
+            if (valid) {
+              P.c.norm[slot] = (float)nrm;
+              P.c.rnorm[slot] = (float)sqrt(rho2);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&empty[st]);   // the stage is no longer read by this warp
+
+        // ---- codes from the accumulator
+        live = __all_sync(0xffffffffu, live && *abort_flag == 0 && sm100::mbar_wait(&tfull[st], ph, err));
+        if (!live) *abort_flag = 1;
+        sm100::tc_fence_after();
+        if (live) {
+          qc.zr = sc * inv32;
+          const bool fix_ok = valid && inv32 != 0.0f;
+          Stream s{0ull, 0, 0, P.c.codes + slot * (size_t)W, valid};
+          const uint32_t taddr = tmem_base + ((uint32_t)(qtr * 32) << 16) + (uint32_t)(st * D);
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            const uint32_t cd = mt->chunk[c];
+            if (cd == 0u) continue;
+            float v[16];
+            sm100::tmem_ld16(taddr + (uint32_t)(c * 16), v);
+            if (cd == kMixed) {
+              // widths vary inside the chunk, or it holds signal coordinates
+#pragma unroll
+              for (int kq = 0; kq < 16; ++kq) {
+                const int i = c * 16 + kq;
+                const int b = bits[i];
+                if (b == 0) continue;
+                uint32_t code;
+                if (i < m) {
+                  code = (i < MSIG) ? (sc4[(kq & 15) >> 2] >> ((kq & 3) * 8)) & 0xFFu : 0u;
+                } else {
                   bool dg;
-                  int code;
-                  if (b == 1) code = q1(z, dl, dg);
-                  else if (b == 2) code = q2(z, t21, dl, dg);
-                  else if (b == 3) code = q3(z, t31, t32, t33, dl, dg);
-                  else code = qn(z, sTh64 + th_off(b), b, dl, dg);
-                  dmask |= (uint32_t)dg << kk;
-                  if (valid) or_bits(rw, (int)(ci.bo >> 8), (uint64_t)(uint32_t)code, b);
-                }
-              }
-              // Queue the codes within their radius for exact recomputation.
-              dmask = enq_ok ? dmask : 0u;
-              if (__any_sync(0xffffffffu, dmask != 0u)) {
-                for (int kk = 0; kk < 16; ++kk) {
-                  const bool dg = (dmask >> kk) & 1u;
-                  const uint32_t dm = __ballot_sync(0xffffffffu, dg);
-                  if (!dm) continue;
-                  uint32_t base = 0;
-                  if (lane == 0) base = atomicAdd(&misc[9], (uint32_t)__popc(dm));
-                  base = __shfl_sync(0xffffffffu, base, 0);
-                  const uint32_t pos = base + (uint32_t)__popc(dm & ((1u << lane) - 1u));
-                  const int i = i0 + kk;
-                  const bool ov = dg && pos >= (uint32_t)QCAP;
-                  if (dg && !ov) sQ[pos] = ((uint32_t)t << 16) | (uint32_t)i;
-                  uint32_t om = __ballot_sync(0xffffffffu, ov);
-                  while (om) {        // queue full: recompute and patch right here
-                    const int src = __ffs(om) - 1;
-                    om &= om - 1;
-                    const int ts = q * 32 + src;
-                    const CoordInfo ci = sCI[i];
-                    const int b = (int)(ci.bo & 0xFFu);
-                    const double zz = exact_sum_warp(xs, sBhi, sBlo, sBlo2, ts, i, lane) * (double)ci.sc /
-                                      sN64[buf * TILE + ts];
-                    if (lane == src) patch_field(rw, (int)(ci.bo >> 8), b, (uint32_t)code_of(zz, sTh64 + th_off(b), b));
+                  code = quant_rt(b, v[kq] * qc.zr, qc, KQ, dg);
+                  dg = dg && fix_ok;
+                  for (;;) {
+                    const uint32_t who = __ballot_sync(0xffffffffu, dg);
+                    if (!who) break;
+                    const int src = __ffs(who) - 1;
+                    const uint32_t ec = exact_code(P.x, xbase + src, i, b, vt64, sig, normalize, sTh64, lane);
+                    if (lane == src) {
+                      code = ec;
+                      dg = false;
+                    }
                   }
                 }
+                put(s, code, b);
+              }
+            } else {
+              switch (cd) {
+                case 1: chunk_uniform<1>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
+                case 2: chunk_uniform<2>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
+                case 3: chunk_uniform<3>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
+                case 4: chunk_uniform<4>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
+                case 5: chunk_uniform<5>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
+                case 6: chunk_uniform<6>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
+                case 7: chunk_uniform<7>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
+                default: chunk_uniform<8>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
               }
             }
           }
-          sm100::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) sm100::mbar_arrive(&tempty[buf]);
+          if (m > 0) put(s, qbits, m);
+          while (s.nw < W) {   // the rest of the record: remaining bits, then zero words
+            if (s.st) s.dst[s.nw] = (uint32_t)s.acc;
+            s.acc >>= 32;
+            ++s.nw;
+          }
         }
-        // ---- all 12 worker warps: exact recomputation of the queued codes
-        sm100::named_bar(1, 12 * 32);
-        const uint32_t qn_ = min(misc[9], (uint32_t)QCAP);
-        for (uint32_t e = (uint32_t)wid; e < qn_; e += 12) {
-          const uint32_t ent = sQ[e];
-          const int t = (int)(ent >> 16), i = (int)(ent & 0xFFFFu);
-          const CoordInfo ci = sCI[i];
-          const int b = (int)(ci.bo & 0xFFu);
-          const double zz = exact_sum_warp(xs, sBhi, sBlo, sBlo2, t, i, lane) * (double)ci.sc / sN64[buf * TILE + t];
-          if (lane == 0)
-            patch_field(sRec + (buf * TILE + t) * REC_PITCH, (int)(ci.bo >> 8), b,
-                        (uint32_t)code_of(zz, sTh64 + th_off(b), b));
-        }
-        sm100::named_bar(1, 12 * 32);
-        if (lane == 0) sm100::mbar_arrive(&empty[st]);    // the X stage is no longer read
-        if (!is_sig) {
-          // ---- store the finished record tile, then clear it for tile + 2
-          const size_t slot0 = ((size_t)bidx * P.n_heads + h) * P.c.cap + sp + t0;
-          uint32_t* gdst = P.c.codes + slot0 * W;
-          uint32_t* rb = sRec + buf * TILE * REC_PITCH;
-          if (live)
-            for (int e = epi_id; e < n_valid * W; e += 256) gdst[e] = rb[(e / W) * REC_PITCH + e % W];
-          if (epi_id == 0) misc[9] = 0u;
-          sm100::named_bar(2, 8 * 32);
-          for (int e = epi_id; e < TILE * REC_PITCH; e += 256) rb[e] = 0u;
-        }
+        sm100::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) sm100::mbar_arrive(&tempty[st]);
       }
     }
-    iter += (uint32_t)nt;
-    ++seg;
+    k += (uint32_t)nt;
+    ++nseg;
     s0 = s1;
   }
   // Every copy this CTA issued has landed before it exits: the last phase of
   // each stage's full barrier and of the B barrier (bounded waits).
   if (warp == WARP_PROD && lane == 0) {
-    for (uint32_t k = 0; k < STAGES && k < iter; ++k) {
-      const uint32_t it = iter - 1 - k;
-      sm100::mbar_wait(&full[it % STAGES], (it / STAGES) & 1u, nullptr);
+    for (uint32_t j = 0; j < NGRP && j < x_issued; ++j) {
+      const uint32_t it = x_issued - 1 - j;
+      sm100::mbar_wait(&full[it % NGRP], (it / NGRP) & 1u, nullptr);
     }
-    if (seg > 0) sm100::mbar_wait(bfull, (seg - 1) & 1u, nullptr);
+    if (b_issued > 0) sm100::mbar_wait(bfull, (b_issued - 1) & 1u, nullptr);
   }
   sm100::tc_fence_before();
   __syncthreads();

@@ -199,7 +199,8 @@ sq_status sq_init(void);
  *  up to 8 query heads per KV head and records of up to 32 words; SIMT partials
  *  otherwise), 1 = always the SIMT partials.
  *  SQ_OPT_TC_ERROR_BOUND: the fp32-accumulation term of the tensor-core compress
- *  error radius, in units of 2^-24 per unit of ||V_i / sigma_i|| (default 128).
+ *  error radius, in units of 2^-24 per unit of ||V_i / sigma_i|| (default 32:
+ *  sixteen accumulation steps of one fp32 rounding each, with truncation).
  *  A code whose z lies within the radius of a threshold is recomputed in
  *  float64; a radius below the hardware's accumulation error can change codes,
  *  so values under the default exist only to measure that error.

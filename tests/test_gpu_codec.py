@@ -181,7 +181,9 @@ def test_tensor_core_path_matches_oracle_and_reference_kernel(name, tokens):
     for a, b in ((kc, kr), (vc, vr)):
         diff = (a.words_u32() != b.words_u32()).any(axis=-1)
         assert diff.sum() <= 1e-4 * diff.size, diff.sum()
-        assert torch.equal(a.norm, b.norm)
+        # value norms are summed in float32 on the tensor-core path: equal up to
+        # the stated norm tolerance (keys are summed in float64 on both)
+        assert torch.allclose(a.norm, b.norm, rtol=1e-6, atol=0)
     assert torch.allclose(kc.rnorm, kr.rnorm, rtol=1e-6, atol=0)
 
 
