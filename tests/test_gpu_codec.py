@@ -214,3 +214,23 @@ def test_full_size_prefill_in_bench_launch_configuration():
         compare_compressed(kw[0, h, ts], kc.norm[0, h, ts].cpu().numpy(), kc.rnorm[0, h, ts].cpu().numpy(), xk,
                            cks[h])
         compare_compressed(vw[0, h, ts], vc.norm[0, h, ts].cpu().numpy(), None, xv, cvs[h])
+
+
+@pytest.mark.parametrize("name,batch,ntok", [("qwen14b", 11, 3), ("tiny", 5, 15), ("gemma9b_sweep", 9, 1)])
+def test_append_groups_of_vectors(name, batch, ntok):
+    """Decode-step compress of several tokens for many rows (vector groups of eight,
+    a ragged last group), each row at its own position, against the oracle."""
+    w, ck, cv, k, v, nh = _case(name, batch=batch, tokens=ntok, heads=2)
+    rng = np.random.default_rng(3)
+    cap = 64
+    start = [int(s) for s in rng.integers(0, cap - ntok + 1, size=batch)]
+    _, _, kc, vc = _compress(ck, cv, k, v, cap=cap, start=start)
+    kw, vw = kc.words_u32(), vc.words_u32()
+    for b, s in enumerate(start):
+        for h in range(nh):
+            compare_compressed(kw[b, h, s:s + ntok], kc.norm[b, h, s:s + ntok].cpu().numpy(),
+                               kc.rnorm[b, h, s:s + ntok].cpu().numpy(), k[b, h].double().numpy(), ck[h])
+            compare_compressed(vw[b, h, s:s + ntok], vc.norm[b, h, s:s + ntok].cpu().numpy(), None,
+                               v[b, h].double().numpy(), cv[h])
+            others = np.setdiff1d(np.arange(cap), np.arange(s, s + ntok))
+            assert np.all(kw[b, h, others] == 0) and np.all(vw[b, h, others] == 0)
