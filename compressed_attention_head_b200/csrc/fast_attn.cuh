@@ -84,6 +84,12 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
                : "memory");
 }
+// 4-byte copy that writes zeros instead when `in` is false (nothing is read then).
+__device__ __forceinline__ void cp_async4_z(void* dst, const void* src, bool in) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(in ? 4 : 0)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
@@ -249,7 +255,9 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
   constexpr int NCH = GE::NCH;
   constexpr int ROW = GE::ROW;
   extern __shared__ __align__(128) uint8_t smraw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smraw + 127) & ~(uintptr_t)127);
+  // aligned by pointer arithmetic on the shared array, so that every access
+  // below stays a shared-memory access (an integer round trip would make them generic)
+  uint8_t* sm = smraw + ((128u - (smem_addr(smraw) & 127u)) & 127u);
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int G = s.group;
@@ -380,22 +388,17 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
   auto stage_rec = [&](uint32_t* rec, const uint32_t* src, int wn, int tile_i) {
     const int64_t t0 = t_lo + (int64_t)tile_i * TT;
     const bool in = t0 + lane < t_hi;
-    const uint32_t* sp = src + (t0 + lane) * wn;
-    for (int w = 0; w < wn; ++w) {
-      if (in) cp_async4(rec + w * RP + lane, sp + w); else rec[w * RP + lane] = 0u;
-    }
+    const uint32_t* sp = src + (in ? (t0 + lane) * wn : 0);
+    uint32_t* dp = rec + lane;
+    for (int w = 0; w < wn; ++w) cp_async4_z(dp + w * RP, sp + w, in);
   };
   auto stage_nrm = [&](int tile_i) {
     const int64_t t0 = t_lo + (int64_t)tile_i * TT;
-    if (t0 + lane < t_hi) {
-      cp_async4(nrm + lane, knorm + t0 + lane);
-      cp_async4(nrm + 2 * TT + lane, vnorm + t0 + lane);
-      if (m > 0) cp_async4(nrm + TT + lane, krho + t0 + lane); else nrm[TT + lane] = 0.0f;
-    } else {
-      nrm[lane] = 0.0f;
-      nrm[TT + lane] = 0.0f;
-      nrm[2 * TT + lane] = 0.0f;
-    }
+    const bool in = t0 + lane < t_hi;
+    const int64_t tt = in ? t0 + lane : 0;
+    cp_async4_z(nrm + lane, knorm + tt, in);
+    cp_async4_z(nrm + 2 * TT + lane, vnorm + tt, in);
+    if (m > 0) cp_async4_z(nrm + TT + lane, krho + tt, in); else nrm[TT + lane] = 0.0f;
   };
 
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};   // heads 2tq, 2tq + 1

@@ -95,8 +95,14 @@ constexpr int OFF_CELL = OFF_Q + kQEntries * 16;                       // u8 [kC
 constexpr int OFF_BAR = OFF_CELL + kCellBytes;
 constexpr int N_BARS = 4 * NGRP + 2;
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;                         // u32 [16]
-constexpr int OFF_R = OFF_MISC + 64;                                   // float [NUM_WARPS][16]: radius per width
-constexpr int SMEM_BYTES = OFF_R + NUM_WARPS * 64 + 1024;              // + alignment slack
+constexpr int OFF_R = OFF_MISC + 64;                                   // float [NGRP][16]: radius per width
+constexpr int OFF_CD = OFF_R + NGRP * 64;                              // u32 [NGRP][8]: chunk classes
+constexpr int OFF_RUN = OFF_CD + NGRP * 32;                            // u16 [NGRP][8][16]: runs of mixed chunks
+constexpr int OFF_SC = OFF_RUN + NGRP * 8 * 16 * 2;                    // u8 [NGRP * 4][32][MSIG]: signal codes
+constexpr int OFF_VS = (OFF_SC + NGRP * 4 * 32 * MSIG + 15) & ~15;     // double [NGRP][MSIG][D]: signal rows of V^T
+constexpr int OFF_MX = OFF_VS + NGRP * MSIG * D * 8;                   // float [NGRP * 4][32][16]: mixed-chunk values
+constexpr int SMEM_BYTES = OFF_MX + NGRP * 4 * 32 * 16 * 4 + 1024;     // + alignment slack
+// A run of a mixed chunk (u16): width (bits 0-3), signal flag (bit 4), length - 1 (bits 8-11).
 static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds 227 KB");
 static_assert(OFF_BAR % 8 == 0, "mbarriers need 8-byte alignment");
 
@@ -259,7 +265,7 @@ __device__ __forceinline__ uint32_t qzl(float z, const uint8_t* cell, const floa
 // Per-thread quantization context of one segment (one head).
 struct QCtx {
   const uint8_t* smb;      // shared-memory base (cell tables, radii)
-  int wr;                  // this warp's radius row: radius of width b at float index wr + b
+  int wr;                  // this group's radius row: radius of width b at float index wr + b
   float zr;                // 2^-s / ||x|| of this thread's row
   __device__ __forceinline__ float R(int b) const { return ((const float*)(smb + OFF_R))[wr + b]; }
   __device__ __forceinline__ const uint8_t* cell() const { return smb + OFF_CELL; }
@@ -300,12 +306,11 @@ struct Stream {
 __device__ __forceinline__ void put(Stream& s, uint32_t v, int n) {   // 1 <= n <= 32, v < 2^n
   s.acc |= (uint64_t)v << s.fill;
   s.fill += n;
-  if (s.fill >= 32) {
-    if (s.st) s.dst[s.nw] = (uint32_t)s.acc;
-    ++s.nw;
-    s.acc >>= 32;
-    s.fill -= 32;
-  }
+  const bool full = s.fill >= 32;
+  if (full && s.st) s.dst[s.nw] = (uint32_t)s.acc;
+  s.nw += full ? 1 : 0;
+  s.acc = full ? (s.acc >> 32) : s.acc;
+  s.fill -= full ? 32 : 0;
 }
 
 // Byte offset of the 16-byte chunk c (elements 8c .. 8c+7) of token row t in an X stage.
@@ -315,7 +320,7 @@ __device__ __forceinline__ uint32_t x_chunk(int t, int c) {
 
 // Exact code of coordinate i of input row xrow (whole warp; every lane returns it):
 // z = (V_i . x) / ||x|| / sigma_i in float64, then the b-bit thresholds.
-__device__ __forceinline__ uint32_t exact_code(const __half* x, int64_t xrow, int i, int b, const double* vt64,
+__device__ __noinline__ uint32_t exact_code(const __half* x, int64_t xrow, int i, int b, const double* vt64,
                                             const double* sig, bool normalize, const double* th64, int lane) {
   const uint2 raw = *(const uint2*)(x + xrow * D + 4 * lane);
   const __half2* hh = reinterpret_cast<const __half2*>(&raw);
@@ -344,9 +349,9 @@ __device__ __forceinline__ uint32_t exact_code(const __half* x, int64_t xrow, in
 // are computed and ignored), then the signal codes, the residual
 // r_i = y_i / ||x|| - sigma_i level_i, rho = ||r|| and the m sign bits of S r.
 template <int MM>
-__device__ __forceinline__ void key_pass(const uint8_t* xs, int t, int m, const double* vt64, const double* sig,
+__device__ __forceinline__ void key_pass(const uint8_t* xs, int t, int m, const double* vsig, const double* sig,
                                          const uint8_t* bits, const double* S, bool normalize, const double* th64,
-                                         const double* lv64, double& nrm, double& rho2, uint32_t (&sc4)[4],
+                                         const double* lv64, double& nrm, double& rho2, uint8_t* scode,
                                          uint32_t& qbits) {
   double n2a = 0.0, n2b = 0.0;
   double ys[MM];
@@ -365,11 +370,10 @@ __device__ __forceinline__ void key_pass(const uint8_t* xs, int t, int m, const 
       const int jj = c * 8 + 2 * e;
 #pragma unroll
       for (int i = 0; i < MM; ++i) {
-        const double2 vv = __ldg((const double2*)(vt64 + (size_t)i * D + jj));
+        const double2 vv = *(const double2*)(vsig + i * D + jj);   // same address in every lane
         ys[i] = fma(x0, vv.x, ys[i]);
         ys[i] = fma(x1, vv.y, ys[i]);
       }
-      asm volatile("" ::: "memory");   // one pair's rows in flight at a time (register budget)
     }
   }
   nrm = normalize ? sqrt(n2a + n2b) : 1.0;
@@ -386,7 +390,7 @@ __device__ __forceinline__ void key_pass(const uint8_t* xs, int t, int m, const 
         const double z = s > 0.0 ? yn / s : 0.0;
         const int code = code_of(z, th64 + th_off(b), b);
         lvv = lv64[lv_off(b) + code];
-        sc4[i >> 2] |= (uint32_t)code << ((i & 3) * 8);
+        scode[i] = (uint8_t)code;
       }
       ys[i] = yn - sig[i] * lvv;
       rho2 = fma(ys[i], ys[i], rho2);
@@ -455,10 +459,50 @@ __device__ __forceinline__ void chunk_uniform(const float* v, const QCtx& qc, co
   if (NB % 32) put(s, cw[NB / 32], 16);
 }
 
+// One run of a mixed chunk: len coordinates of width B starting at chunk
+// position k0 (values in the lane's swizzled scratch row), each code checked
+// against its band and appended to the stream.
+struct RunArgs {
+  const float* mx;
+  int lane, k0, len, i0;
+  bool fix_ok;
+  const __half* x;
+  int64_t xbase;
+  const double* vt64;
+  const double* sig;
+  bool normalize;
+  const double* th64;
+};
+template <int B>
+__device__ __forceinline__ void run_codes(const RunArgs& a, const QCtx& qc, const QuantConst& kqc, Stream& s) {
+#pragma unroll 1
+  for (int k = a.k0; k < a.k0 + a.len; ++k) {
+    bool dg;
+    uint32_t code = quant<B>(a.mx[k ^ (a.lane & 15)] * qc.zr, qc, kqc, dg);
+    dg = dg && a.fix_ok;
+    if (__any_sync(0xffffffffu, dg)) {
+      for (;;) {
+        const uint32_t who = __ballot_sync(0xffffffffu, dg);
+        if (!who) break;
+        const int src = __ffs(who) - 1;
+        const uint32_t ec =
+            exact_code(a.x, a.xbase + src, a.i0 + k, B, a.vt64, a.sig, a.normalize, a.th64, a.lane);
+        if (a.lane == src) {
+          code = ec;
+          dg = false;
+        }
+      }
+    }
+    put(s, code, B);
+  }
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_constant__ QuantConst KQ) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  // aligned by pointer arithmetic on the shared array, so that every access
+  // below stays a shared-memory access (an integer round trip would make them generic)
+  uint8_t* sm = smem_raw + ((1024u - (sm100::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sX = sm + OFF_X;
   uint8_t* sBhi = sm + OFF_BHI;
   uint8_t* sBlo = sm + OFF_BLO;
@@ -607,12 +651,44 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
       const uint8_t* bits = rec.bits();
       QCtx qc;
       qc.smb = sm;
-      qc.wr = warp * 16;
+      qc.wr = grp * 16;
       qc.zr = 0.0f;
-      __syncwarp();
-      if (lane <= 8)
-        ((float*)(sm + OFF_R))[warp * 16 + lane] = fmaf(P.eacc, mt->dacc_w[lane], mt->dfix_w[lane]) + 2.0e-6f;
-      __syncwarp();
+      // Per-segment constants of this group: wait until its four warps are done
+      // with the previous segment, load, and wait again (named barrier 1 + grp).
+      double* vsig = (double*)(sm + OFF_VS) + grp * MSIG * D;
+      uint32_t* cdw = (uint32_t*)(sm + OFF_CD) + grp * 8;
+      uint16_t* runs = (uint16_t*)(sm + OFF_RUN) + grp * 8 * 16;
+      sm100::named_bar(1 + grp, 128);
+      {
+        const int gt = (warp & 3) * 32 + lane;        // 0..127 within the group
+        const int nrow = m < MSIG ? m : MSIG;
+        for (int e = gt; e < nrow * D / 2; e += 128)
+          ((double2*)vsig)[e] = ((const double2*)vt64)[e];
+        if (gt <= 8)
+          ((float*)(sm + OFF_R))[grp * 16 + gt] = fmaf(P.eacc, mt->dacc_w[gt], mt->dfix_w[gt]) + 2.0e-6f;
+        if (gt >= 32 && gt < 40) {
+          // chunk class; for a mixed chunk, its runs of one width (signal
+          // coordinates in runs of their own)
+          const int c = gt - 32;
+          uint32_t cd = mt->chunk[c];
+          if (cd == kMixed) {
+            int nr = 0, k = 0;
+            while (k < 16) {
+              const int i0 = c * 16 + k;
+              const int b0 = bits[i0];
+              const bool s0 = i0 < m;
+              int len = 1;
+              while (k + len < 16 && bits[i0 + len] == b0 && ((i0 + len) < m) == s0) ++len;
+              runs[c * 16 + nr] = (uint16_t)(b0 | (s0 ? 16 : 0) | ((len - 1) << 8));
+              ++nr;
+              k += len;
+            }
+            cd = kMixed | ((uint32_t)nr << 8);
+          }
+          cdw[c] = cd;
+        }
+      }
+      sm100::named_bar(1 + grp, 128);
       const float sc = tv.ci()[0].sc;
       const double* S = rec.S();
       for (int64_t j = 0; j < nt; ++j) {
@@ -632,7 +708,7 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
         if (!live) *abort_flag = 1;
         // ---- norm phase (reads the staged tile)
         float inv32 = 0.0f;
-        uint32_t sc4[4] = {0u, 0u, 0u, 0u};   // exact codes of the signal coordinates (8 bits each)
+        uint8_t* scode = sm + OFF_SC + ((warp - WARP_EPI0) * 32 + lane) * MSIG;   // this lane's signal codes
         uint32_t qbits = 0u;
         if (live) {
           if (m == 0) {
@@ -660,9 +736,10 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
             // keys with QJL: ||x||, the m signal coordinates, their codes, the
             // residual, rho and the sign bits, all in float64
             double nrm, rho2;
-            if (m <= 2) key_pass<2>(xs, t_row, m, vt64, sig, bits, S, normalize, sTh64, sLv64, nrm, rho2, sc4, qbits);
-            else if (m <= 4) key_pass<4>(xs, t_row, m, vt64, sig, bits, S, normalize, sTh64, sLv64, nrm, rho2, sc4, qbits);
-            else key_pass<8>(xs, t_row, m, vt64, sig, bits, S, normalize, sTh64, sLv64, nrm, rho2, sc4, qbits);
+            if (m <= 2) key_pass<2>(xs, t_row, m, vsig, sig, bits, S, normalize, sTh64, sLv64, nrm, rho2, scode, qbits);
+            else if (m == 3) key_pass<3>(xs, t_row, m, vsig, sig, bits, S, normalize, sTh64, sLv64, nrm, rho2, scode, qbits);
+            else if (m <= 4) key_pass<4>(xs, t_row, m, vsig, sig, bits, S, normalize, sTh64, sLv64, nrm, rho2, scode, qbits);
+            else key_pass<8>(xs, t_row, m, vsig, sig, bits, S, normalize, sTh64, sLv64, nrm, rho2, scode, qbits);
             inv32 = nrm > 0.0 ? (float)(1.0 / nrm) : 0.0f;
             if (valid) {
               P.c.norm[slot] = (float)nrm;
@@ -684,36 +761,42 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
           const uint32_t taddr = tmem_base + ((uint32_t)(qtr * 32) << 16) + (uint32_t)(st * D);
 #pragma unroll 1
           for (int c = 0; c < D / 16; ++c) {
-            const uint32_t cd = mt->chunk[c];
+            const uint32_t cd = cdw[c];
             if (cd == 0u) continue;
             float v[16];
             sm100::tmem_ld16(taddr + (uint32_t)(c * 16), v);
-            if (cd == kMixed) {
-              // widths vary inside the chunk, or it holds signal coordinates
+            if ((cd & 0xFFu) == kMixed) {
+              // widths vary inside the chunk, or it holds signal coordinates: its
+              // runs of one width, each with the quantizer of that width; the
+              // values go through this lane's scratch row (16 floats, XOR-swizzled
+              // so that the 32 lanes hit distinct banks)
+              float* mx = (float*)(sm + OFF_MX) + ((warp - WARP_EPI0) * 32 + lane) * 16;
 #pragma unroll
-              for (int kq = 0; kq < 16; ++kq) {
-                const int i = c * 16 + kq;
-                const int b = bits[i];
-                if (b == 0) continue;
-                uint32_t code;
-                if (i < m) {
-                  code = (i < MSIG) ? (sc4[(kq & 15) >> 2] >> ((kq & 3) * 8)) & 0xFFu : 0u;
-                } else {
-                  bool dg;
-                  code = quant_rt(b, v[kq] * qc.zr, qc, KQ, dg);
-                  dg = dg && fix_ok;
-                  for (;;) {
-                    const uint32_t who = __ballot_sync(0xffffffffu, dg);
-                    if (!who) break;
-                    const int src = __ffs(who) - 1;
-                    const uint32_t ec = exact_code(P.x, xbase + src, i, b, vt64, sig, normalize, sTh64, lane);
-                    if (lane == src) {
-                      code = ec;
-                      dg = false;
+              for (int kq = 0; kq < 16; ++kq) mx[kq ^ (lane & 15)] = v[kq];
+              const int nr = (int)((cd >> 8) & 31u);
+              int k0 = 0;
+#pragma unroll 1
+              for (int r = 0; r < nr; ++r) {
+                const uint32_t rn = runs[c * 16 + r];
+                const int w = (int)(rn & 15u), len = (int)((rn >> 8) & 15u) + 1;
+                if (w > 0) {
+                  if (rn & 16u) {
+                    for (int kq = k0; kq < k0 + len; ++kq) put(s, scode[(c * 16 + kq) & (MSIG - 1)], w);
+                  } else {
+                    RunArgs ra{mx, lane, k0, len, c * 16, fix_ok, P.x, xbase, vt64, sig, normalize, sTh64};
+                    switch (w) {
+                      case 1: run_codes<1>(ra, qc, KQ, s); break;
+                      case 2: run_codes<2>(ra, qc, KQ, s); break;
+                      case 3: run_codes<3>(ra, qc, KQ, s); break;
+                      case 4: run_codes<4>(ra, qc, KQ, s); break;
+                      case 5: run_codes<5>(ra, qc, KQ, s); break;
+                      case 6: run_codes<6>(ra, qc, KQ, s); break;
+                      case 7: run_codes<7>(ra, qc, KQ, s); break;
+                      default: run_codes<8>(ra, qc, KQ, s); break;
                     }
                   }
                 }
-                put(s, code, b);
+                k0 += len;
               }
             } else {
               switch (cd) {
