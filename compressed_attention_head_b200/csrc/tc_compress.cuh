@@ -59,7 +59,9 @@ struct TcMeta {
   uint32_t chunk[D / 16];   // width 0..8 if all 16 coordinates share it (no signal one), else kMixed
   float dfix_w[12];         // max dfix over the non-signal coordinates of each width
   float dacc_w[12];         // max dacc over the same
-  uint32_t reserved[32];
+  float dfix_c[D / 16];     // max dfix over the non-signal coordinates of each chunk
+  float dacc_c[D / 16];     // max dacc over the same
+  uint32_t reserved[16];
 };
 constexpr uint32_t kMixed = 0xFFu;
 static_assert(sizeof(TcMeta) == 256, "meta block is 256 bytes");
@@ -95,8 +97,8 @@ constexpr int OFF_CELL = OFF_Q + kQEntries * 16;                       // u8 [kC
 constexpr int OFF_BAR = OFF_CELL + kCellBytes;
 constexpr int N_BARS = 4 * NGRP + 2;
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;                         // u32 [16]
-constexpr int OFF_R = OFF_MISC + 64;                                   // float [NGRP][16]: radius per width
-constexpr int OFF_CD = OFF_R + NGRP * 64;                              // u32 [NGRP][8]: chunk classes
+constexpr int OFF_R = OFF_MISC + 64;                                   // float [NGRP][32]: radius per width, per chunk
+constexpr int OFF_CD = OFF_R + NGRP * 128;                             // u32 [NGRP][8]: chunk classes
 constexpr int OFF_RUN = OFF_CD + NGRP * 32;                            // u16 [NGRP][8][16]: runs of mixed chunks
 constexpr int OFF_SC = OFF_RUN + NGRP * 8 * 16 * 2;                    // u8 [NGRP * 4][32][MSIG]: signal codes
 constexpr int OFF_VS = (OFF_SC + NGRP * 4 * 32 * MSIG + 15) & ~15;     // double [NGRP][MSIG][D]: signal rows of V^T
@@ -195,11 +197,14 @@ __device__ void build_tc(Rec rec, int tid, int nth) {
     TcMeta mt;
     const int m = rec.hdr()->m;
     for (int b = 0; b < 12; ++b) mt.dfix_w[b] = mt.dacc_w[b] = 0.0f;
-    for (int e = 0; e < 32; ++e) mt.reserved[e] = 0u;
+    for (int e = 0; e < 16; ++e) mt.reserved[e] = 0u;
+    for (int c = 0; c < D / 16; ++c) mt.dfix_c[c] = mt.dacc_c[c] = 0.0f;
     for (int i = m; i < D; ++i) {
       const int b = (int)(tv.ci()[i].bo & 0xFFu);
       mt.dfix_w[b] = fmaxf(mt.dfix_w[b], tv.ci()[i].dfix);
       mt.dacc_w[b] = fmaxf(mt.dacc_w[b], tv.ci()[i].dacc);
+      mt.dfix_c[i / 16] = fmaxf(mt.dfix_c[i / 16], tv.ci()[i].dfix);
+      mt.dacc_c[i / 16] = fmaxf(mt.dacc_c[i / 16], tv.ci()[i].dacc);
     }
     for (int c = 0; c < D / 16; ++c) {
       const uint32_t b0 = tv.ci()[16 * c].bo & 0xFFu;
@@ -265,7 +270,7 @@ __device__ __forceinline__ uint32_t qzl(float z, const uint8_t* cell, const floa
 // Per-thread quantization context of one segment (one head).
 struct QCtx {
   const uint8_t* smb;      // shared-memory base (cell tables, radii)
-  int wr;                  // this group's radius row: radius of width b at float index wr + b
+  int wr;                  // this group's radius row: radius of width b at float index wr + b (chunks from wr + 16)
   float zr;                // 2^-s / ||x|| of this thread's row
   __device__ __forceinline__ float R(int b) const { return ((const float*)(smb + OFF_R))[wr + b]; }
   __device__ __forceinline__ const uint8_t* cell() const { return smb + OFF_CELL; }
@@ -273,44 +278,59 @@ struct QCtx {
 };
 
 template <int B>
-__device__ __forceinline__ uint32_t quant(float z, const QCtx& c, const QuantConst& k, bool& dg) {
-  if (B == 1) return qz1(z, c.R(1), dg);
-  else if (B == 2) return qz2(z, k.t2, c.R(2), dg);
-  else if (B == 3) return qz3(z, k.t3[0], k.t3[1], k.t3[2], c.R(3), dg);
+__device__ __forceinline__ uint32_t quant(float z, float R, const QCtx& c, const QuantConst& k, bool& dg) {
+  if (B == 1) return qz1(z, R, dg);
+  else if (B == 2) return qz2(z, k.t2, R, dg);
+  else if (B == 3) return qz3(z, k.t3[0], k.t3[1], k.t3[2], R, dg);
   else
-    return qzl(z, c.cell() + cell_off(B), c.q() + q_off(B), (float)(1 << (B - 2)), k.ncell[B], 1u << (B - 1),
-               c.R(B), dg);
-}
-__device__ __forceinline__ uint32_t quant_rt(int b, float z, const QCtx& c, const QuantConst& k, bool& dg) {
-  switch (b) {
-    case 1: return quant<1>(z, c, k, dg);
-    case 2: return quant<2>(z, c, k, dg);
-    case 3: return quant<3>(z, c, k, dg);
-    case 4: return quant<4>(z, c, k, dg);
-    case 5: return quant<5>(z, c, k, dg);
-    case 6: return quant<6>(z, c, k, dg);
-    case 7: return quant<7>(z, c, k, dg);
-    default: return quant<8>(z, c, k, dg);
-  }
+    return qzl(z, c.cell() + cell_off(B), c.q() + q_off(B), (float)(1 << (B - 2)), k.ncell[B], 1u << (B - 1), R,
+               dg);
 }
 
 // Little-endian bit stream of one record, written to global memory a word at
 // a time. fill and nw are the same in every lane of a warp (one head).
 struct Stream {
-  uint64_t acc;
+  uint32_t acc;      // the fill (< 32) pending low bits of the next word
   int fill;
-  int nw;
+  int nw;            // words written so far
   uint32_t* dst;
   bool st;
 };
 __device__ __forceinline__ void put(Stream& s, uint32_t v, int n) {   // 1 <= n <= 32, v < 2^n
-  s.acc |= (uint64_t)v << s.fill;
-  s.fill += n;
-  const bool full = s.fill >= 32;
-  if (full && s.st) s.dst[s.nw] = (uint32_t)s.acc;
+  const uint32_t lo = s.acc | (v << s.fill);
+  const uint32_t carry = __funnelshift_l(v, 0u, s.fill);   // bits of v past the word
+  const int nf = s.fill + n;
+  const bool full = nf >= 32;
+  if (full && s.st) s.dst[s.nw] = lo;
   s.nw += full ? 1 : 0;
-  s.acc = full ? (s.acc >> 32) : s.acc;
-  s.fill -= full ? 32 : 0;
+  s.acc = full ? carry : lo;
+  s.fill = nf & 31;
+}
+// Appends the NB bits held in cw[0 .. ceil(NB/32)) (NB a multiple of 16, at
+// most 128) in one step: every word that completes is a funnel shift of two
+// neighbours, so the appends of a chunk do not form a serial chain.
+template <int NB>
+__device__ __forceinline__ void put_bits(Stream& s, const uint32_t* cw) {
+  constexpr int NI = (NB + 31) / 32;          // input words
+  uint32_t w[NI + 1];
+  uint32_t prev = s.acc;
+#pragma unroll
+  for (int j = 0; j <= NI; ++j) {
+    const uint32_t cur = j < NI ? cw[j] : 0u;
+    w[j] = s.fill ? __funnelshift_l(prev, cur, s.fill) | 0u : cur;
+    prev = cur;
+  }
+  // word 0 also carries the pending bits
+  w[0] = s.acc | (cw[0] << s.fill);
+  const int tot = s.fill + NB;
+  const int nfull = tot >> 5;                 // NB/32 or NB/32 + 1 (NB/32 rounded down)
+#pragma unroll
+  for (int j = 0; j <= NI; ++j)
+    if (j < nfull && s.st) s.dst[s.nw + j] = w[j];
+  constexpr int lo = NB / 32;
+  s.acc = (nfull == lo) ? w[lo] : w[lo < NI ? lo + 1 : NI];
+  s.nw += nfull;
+  s.fill = tot & 31;
 }
 
 // Byte offset of the 16-byte chunk c (elements 8c .. 8c+7) of token row t in an X stage.
@@ -318,30 +338,102 @@ __device__ __forceinline__ uint32_t x_chunk(int t, int c) {
   return (uint32_t)((c >> 3) * (TILE * 128) + (t >> 3) * 1024 + (t & 7) * 128 + (((c & 7) ^ (t & 7)) << 4));
 }
 
-// Exact code of coordinate i of input row xrow (whole warp; every lane returns it):
-// z = (V_i . x) / ||x|| / sigma_i in float64, then the b-bit thresholds.
-__device__ __noinline__ uint32_t exact_code(const __half* x, int64_t xrow, int i, int b, const double* vt64,
-                                            const double* sig, bool normalize, const double* th64, int lane) {
-  const uint2 raw = *(const uint2*)(x + xrow * D + 4 * lane);
-  const __half2* hh = reinterpret_cast<const __half2*>(&raw);
-  const double2 v01 = *(const double2*)(vt64 + (size_t)i * D + 4 * lane);
-  const double2 v23 = *(const double2*)(vt64 + (size_t)i * D + 4 * lane + 2);
-  const float2 a = __half22float2(hh[0]), c = __half22float2(hh[1]);
-  double dot = (double)a.x * v01.x;
-  dot = fma((double)a.y, v01.y, dot);
-  dot = fma((double)c.x, v23.x, dot);
-  dot = fma((double)c.y, v23.y, dot);
-  double n2 = (double)a.x * a.x;
-  n2 = fma((double)a.y, (double)a.y, n2);
-  n2 = fma((double)c.x, (double)c.x, n2);
-  n2 = fma((double)c.y, (double)c.y, n2);
-  dot = warp_sum(dot);
-  n2 = warp_sum(n2);
-  const double nrm = normalize ? sqrt(n2) : 1.0;
-  const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
-  const double s = sig[i];
-  const double z = s > 0.0 ? dot * inv / s : 0.0;
-  return (uint32_t)code_of(z, th64 + th_off(b), b);
+// Flag bits of the coordinates whose z fell within the radius of a threshold:
+// 128 bits per lane (fm[q] holds coordinates 32q .. 32q + 31).
+__device__ __forceinline__ void flag_chunk(uint32_t (&fm)[4], int c, uint32_t dm) {
+  const uint32_t sh = dm << ((c & 1) * 16);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) fm[q] |= (c >> 1) == q ? sh : 0u;
+}
+__device__ __forceinline__ void flag_coord(uint32_t (&fm)[4], int i, bool dg) {
+  const uint32_t bit = dg ? 1u << (i & 31) : 0u;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) fm[q] |= (i >> 5) == q ? bit : 0u;
+}
+
+// Exact repair of the flagged codes of a warp's 32 records, after they have
+// been written: rounds of up to RB (lane, coordinate) entries, each
+// recomputed by the whole warp in float64 (lane l takes elements 4l .. 4l+3 of
+// the input row and of the eigenvector; the loads of a round are all issued
+// before any reduction), z = (V_i . x) / ||x|| / sigma_i, and the owner lane
+// overwrites the b_i-bit field of its record.
+constexpr int RB = 2;   // repairs per round (their loads are in flight together)
+__device__ __forceinline__ void repair_warp(uint4 fmv, const __half* x, int64_t xbase, uint32_t* rec,
+                                         const double* vt64, const double* sig, const uint8_t* bits,
+                                         const int32_t* offs, bool normalize, const double* th64, int lane) {
+  uint32_t fm[4] = {fmv.x, fmv.y, fmv.z, fmv.w};
+  for (;;) {
+    const uint32_t fl = fm[0] | fm[1] | fm[2] | fm[3];
+    uint32_t have = __ballot_sync(0xffffffffu, fl != 0u);
+    if (!have) break;
+    // my lowest flagged coordinate
+    int mine = -1;
+#pragma unroll
+    for (int q = 3; q >= 0; --q)
+      if (fm[q]) mine = q * 32 + __ffs(fm[q]) - 1;
+    int src[RB], crd[RB];
+    int n = 0;
+#pragma unroll
+    for (int k = 0; k < RB; ++k) {
+      src[k] = -1;
+      crd[k] = 0;
+      if (have) {
+        src[k] = __ffs(have) - 1;
+        have &= have - 1u;
+        crd[k] = __shfl_sync(0xffffffffu, mine, src[k]);
+        ++n;
+      }
+    }
+    uint2 xr[RB];
+    double2 va[RB], vb[RB];
+#pragma unroll
+    for (int k = 0; k < RB; ++k) {
+      if (src[k] >= 0) {
+        xr[k] = *(const uint2*)(x + (xbase + src[k]) * D + 4 * lane);
+        const double* vr = vt64 + (size_t)crd[k] * D + 4 * lane;
+        va[k] = *(const double2*)vr;
+        vb[k] = *(const double2*)(vr + 2);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < RB; ++k) {
+      if (src[k] < 0) continue;
+      const __half2* hh = reinterpret_cast<const __half2*>(&xr[k]);
+      const float2 a = __half22float2(hh[0]), c = __half22float2(hh[1]);
+      double dot = (double)a.x * va[k].x;
+      dot = fma((double)a.y, va[k].y, dot);
+      dot = fma((double)c.x, vb[k].x, dot);
+      dot = fma((double)c.y, vb[k].y, dot);
+      double n2 = (double)a.x * a.x;
+      n2 = fma((double)a.y, (double)a.y, n2);
+      n2 = fma((double)c.x, (double)c.x, n2);
+      n2 = fma((double)c.y, (double)c.y, n2);
+      dot = warp_sum(dot);
+      n2 = warp_sum(n2);
+      if (lane == src[k]) {
+        const int i = crd[k];
+        const double nrm = normalize ? sqrt(n2) : 1.0;
+        const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
+        const double s = sig[i];
+        const int b = bits[i];
+        const double yn = dot * inv;
+        const uint32_t code = (uint32_t)code_of(s > 0.0 ? yn * (1.0 / s) : 0.0, th64 + th_off(b), b);
+        // patch the field with two reductions (no read back of the word; the
+        // same thread's operations on one address stay in order)
+        const int o = offs[i], wi = o >> 5, sh = o & 31;
+        const uint32_t mask = (1u << b) - 1u;
+        atomicAnd(&rec[wi], ~(mask << sh));
+        atomicOr(&rec[wi], code << sh);
+        if (sh + b > 32) {
+          atomicAnd(&rec[wi + 1], ~(mask >> (32 - sh)));
+          atomicOr(&rec[wi + 1], code >> (32 - sh));
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if ((i >> 5) == q) fm[q] &= ~(1u << (i & 31));
+      }
+    }
+  }
 }
 
 // Norm phase of a key row with QJL (m <= MM signal coordinates): ||x|| and
@@ -353,10 +445,11 @@ __device__ __forceinline__ void key_pass(const uint8_t* xs, int t, int m, const 
                                          const uint8_t* bits, const double* S, bool normalize, const double* th64,
                                          const double* lv64, double& nrm, double& rho2, uint8_t* scode,
                                          uint32_t& qbits) {
+  // two partial sums per quantity (even and odd j; for MM <= 4) halve the dependent chains
   double n2a = 0.0, n2b = 0.0;
-  double ys[MM];
+  double ys[MM], yo[MM];
 #pragma unroll
-  for (int i = 0; i < MM; ++i) ys[i] = 0.0;
+  for (int i = 0; i < MM; ++i) ys[i] = yo[i] = 0.0;
 #pragma unroll 1
   for (int c = 0; c < D / 8; ++c) {
     const uint4 raw = *(const uint4*)(xs + x_chunk(t, c));
@@ -372,10 +465,13 @@ __device__ __forceinline__ void key_pass(const uint8_t* xs, int t, int m, const 
       for (int i = 0; i < MM; ++i) {
         const double2 vv = *(const double2*)(vsig + i * D + jj);   // same address in every lane
         ys[i] = fma(x0, vv.x, ys[i]);
-        ys[i] = fma(x1, vv.y, ys[i]);
+        if (MM <= 4) yo[i] = fma(x1, vv.y, yo[i]);
+        else ys[i] = fma(x1, vv.y, ys[i]);
       }
     }
   }
+#pragma unroll
+  for (int i = 0; i < MM; ++i) ys[i] += yo[i];   // (zero when MM > 4)
   nrm = normalize ? sqrt(n2a + n2b) : 1.0;
   const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
   rho2 = 0.0;
@@ -406,93 +502,37 @@ __device__ __forceinline__ void key_pass(const uint8_t* xs, int t, int m, const 
   }
 }
 
-// Replaces field k (width B) of the 16-code chunk words cw.
-template <int B>
-__device__ __forceinline__ void patch_chunk(uint32_t (&cw)[4], int k, uint32_t code) {
-  const int p = B * k, wi = p >> 5, sh = p & 31;
-  const uint32_t mask = (1u << B) - 1u;
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    if (w == wi) cw[w] = (cw[w] & ~(mask << sh)) | (code << sh);
-    if (w == wi + 1 && sh + B > 32) {
-      const int r = 32 - sh;
-      cw[w] = (cw[w] & ~(mask >> r)) | (code >> r);
-    }
-  }
-}
-
 // One width-uniform chunk of 16 coordinates: codes into cw (compile-time
-// positions), exact recomputation of the in-band ones, then the stream.
+// positions), flags of the in-band ones, then the stream.
 template <int B>
-__device__ __forceinline__ void chunk_uniform(const float* v, const QCtx& qc, const QuantConst& kq, bool fix_ok,
-                                              int i0, const __half* x, int64_t xbase, const double* vt64,
-                                              const double* sig, bool normalize, const double* th64, int lane,
-                                              Stream& s) {
+__device__ __forceinline__ void chunk_uniform(const float* v, float Rc, const QCtx& qc, const QuantConst& kq,
+                                              bool fix_ok, int c, uint32_t (&fm)[4], Stream& s) {
   uint32_t cw[4] = {0u, 0u, 0u, 0u};
   uint32_t dm = 0u;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
     bool dg;
-    const uint32_t code = quant<B>(v[k] * qc.zr, qc, kq, dg);
+    const uint32_t code = quant<B>(v[k] * qc.zr, Rc, qc, kq, dg);
     dm |= dg ? (1u << k) : 0u;
     const int p = B * k;
     cw[p >> 5] |= code << (p & 31);
     if ((p & 31) + B > 32) cw[(p >> 5) + 1] |= code >> (32 - (p & 31));
   }
-  dm = fix_ok ? dm : 0u;
-  if (__any_sync(0xffffffffu, dm != 0u)) {
-    for (;;) {
-      const uint32_t who = __ballot_sync(0xffffffffu, dm != 0u);
-      if (!who) break;
-      const int src = __ffs(who) - 1;
-      const int k = __ffs(__shfl_sync(0xffffffffu, dm, src)) - 1;
-      const uint32_t code = exact_code(x, xbase + src, i0 + k, B, vt64, sig, normalize, th64, lane);
-      if (lane == src) {
-        patch_chunk<B>(cw, k, code);
-        dm &= dm - 1u;
-      }
-    }
-  }
-  constexpr int NB = 16 * B;
-#pragma unroll
-  for (int w = 0; w < NB / 32; ++w) put(s, cw[w], 32);
-  if (NB % 32) put(s, cw[NB / 32], 16);
+  flag_chunk(fm, c, fix_ok ? dm : 0u);
+  put_bits<16 * B>(s, cw);
 }
 
 // One run of a mixed chunk: len coordinates of width B starting at chunk
-// position k0 (values in the lane's swizzled scratch row), each code checked
-// against its band and appended to the stream.
-struct RunArgs {
-  const float* mx;
-  int lane, k0, len, i0;
-  bool fix_ok;
-  const __half* x;
-  int64_t xbase;
-  const double* vt64;
-  const double* sig;
-  bool normalize;
-  const double* th64;
-};
+// position k0 (values in the lane's swizzled scratch row), each code flagged
+// if in band and appended to the stream.
 template <int B>
-__device__ __forceinline__ void run_codes(const RunArgs& a, const QCtx& qc, const QuantConst& kqc, Stream& s) {
+__device__ __forceinline__ void run_codes(const float* mx, int lane, int k0, int len, int i0, bool fix_ok,
+                                          const QCtx& qc, const QuantConst& kqc, uint32_t (&fm)[4], Stream& s) {
 #pragma unroll 1
-  for (int k = a.k0; k < a.k0 + a.len; ++k) {
+  for (int k = k0; k < k0 + len; ++k) {
     bool dg;
-    uint32_t code = quant<B>(a.mx[k ^ (a.lane & 15)] * qc.zr, qc, kqc, dg);
-    dg = dg && a.fix_ok;
-    if (__any_sync(0xffffffffu, dg)) {
-      for (;;) {
-        const uint32_t who = __ballot_sync(0xffffffffu, dg);
-        if (!who) break;
-        const int src = __ffs(who) - 1;
-        const uint32_t ec =
-            exact_code(a.x, a.xbase + src, a.i0 + k, B, a.vt64, a.sig, a.normalize, a.th64, a.lane);
-        if (a.lane == src) {
-          code = ec;
-          dg = false;
-        }
-      }
-    }
+    const uint32_t code = quant<B>(mx[k ^ (lane & 15)] * qc.zr, qc.R(B), qc, kqc, dg);
+    flag_coord(fm, i0 + k, dg && fix_ok);
     put(s, code, B);
   }
 }
@@ -651,7 +691,8 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
       const uint8_t* bits = rec.bits();
       QCtx qc;
       qc.smb = sm;
-      qc.wr = grp * 16;
+      qc.wr = grp * 32;
+      const float* rch = (const float*)(sm + OFF_R) + grp * 32 + 16;   // radius per chunk
       qc.zr = 0.0f;
       // Per-segment constants of this group: wait until its four warps are done
       // with the previous segment, load, and wait again (named barrier 1 + grp).
@@ -665,7 +706,10 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
         for (int e = gt; e < nrow * D / 2; e += 128)
           ((double2*)vsig)[e] = ((const double2*)vt64)[e];
         if (gt <= 8)
-          ((float*)(sm + OFF_R))[grp * 16 + gt] = fmaf(P.eacc, mt->dacc_w[gt], mt->dfix_w[gt]) + 2.0e-6f;
+          ((float*)(sm + OFF_R))[grp * 32 + gt] = fmaf(P.eacc, mt->dacc_w[gt], mt->dfix_w[gt]) + 2.0e-6f;
+        if (gt >= 16 && gt < 16 + D / 16)
+          ((float*)(sm + OFF_R))[grp * 32 + gt] =
+              fmaf(P.eacc, mt->dacc_c[gt - 16], mt->dfix_c[gt - 16]) + 2.0e-6f;
         if (gt >= 32 && gt < 40) {
           // chunk class; for a mixed chunk, its runs of one width (signal
           // coordinates in runs of their own)
@@ -757,7 +801,8 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
         if (live) {
           qc.zr = sc * inv32;
           const bool fix_ok = valid && inv32 != 0.0f;
-          Stream s{0ull, 0, 0, P.c.codes + slot * (size_t)W, valid};
+          Stream s{0u, 0, 0, P.c.codes + slot * (size_t)W, valid};
+          uint32_t fm[4] = {0u, 0u, 0u, 0u};   // coordinates to repair exactly
           const uint32_t taddr = tmem_base + ((uint32_t)(qtr * 32) << 16) + (uint32_t)(st * D);
 #pragma unroll 1
           for (int c = 0; c < D / 16; ++c) {
@@ -783,16 +828,15 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
                   if (rn & 16u) {
                     for (int kq = k0; kq < k0 + len; ++kq) put(s, scode[(c * 16 + kq) & (MSIG - 1)], w);
                   } else {
-                    RunArgs ra{mx, lane, k0, len, c * 16, fix_ok, P.x, xbase, vt64, sig, normalize, sTh64};
                     switch (w) {
-                      case 1: run_codes<1>(ra, qc, KQ, s); break;
-                      case 2: run_codes<2>(ra, qc, KQ, s); break;
-                      case 3: run_codes<3>(ra, qc, KQ, s); break;
-                      case 4: run_codes<4>(ra, qc, KQ, s); break;
-                      case 5: run_codes<5>(ra, qc, KQ, s); break;
-                      case 6: run_codes<6>(ra, qc, KQ, s); break;
-                      case 7: run_codes<7>(ra, qc, KQ, s); break;
-                      default: run_codes<8>(ra, qc, KQ, s); break;
+                      case 1: run_codes<1>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
+                      case 2: run_codes<2>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
+                      case 3: run_codes<3>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
+                      case 4: run_codes<4>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
+                      case 5: run_codes<5>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
+                      case 6: run_codes<6>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
+                      case 7: run_codes<7>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
+                      default: run_codes<8>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
                     }
                   }
                 }
@@ -800,27 +844,37 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
               }
             } else {
               switch (cd) {
-                case 1: chunk_uniform<1>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
-                case 2: chunk_uniform<2>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
-                case 3: chunk_uniform<3>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
-                case 4: chunk_uniform<4>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
-                case 5: chunk_uniform<5>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
-                case 6: chunk_uniform<6>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
-                case 7: chunk_uniform<7>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
-                default: chunk_uniform<8>(v, qc, KQ, fix_ok, c * 16, P.x, xbase, vt64, sig, normalize, sTh64, lane, s); break;
+                case 1: chunk_uniform<1>(v, rch[c], qc, KQ, fix_ok, c, fm, s); break;
+                case 2: chunk_uniform<2>(v, rch[c], qc, KQ, fix_ok, c, fm, s); break;
+                case 3: chunk_uniform<3>(v, rch[c], qc, KQ, fix_ok, c, fm, s); break;
+                case 4: chunk_uniform<4>(v, rch[c], qc, KQ, fix_ok, c, fm, s); break;
+                case 5: chunk_uniform<5>(v, rch[c], qc, KQ, fix_ok, c, fm, s); break;
+                case 6: chunk_uniform<6>(v, rch[c], qc, KQ, fix_ok, c, fm, s); break;
+                case 7: chunk_uniform<7>(v, rch[c], qc, KQ, fix_ok, c, fm, s); break;
+                default: chunk_uniform<8>(v, rch[c], qc, KQ, fix_ok, c, fm, s); break;
               }
             }
           }
           if (m > 0) put(s, qbits, m);
           while (s.nw < W) {   // the rest of the record: remaining bits, then zero words
-            if (s.st) s.dst[s.nw] = (uint32_t)s.acc;
-            s.acc >>= 32;
+            if (s.st) s.dst[s.nw] = s.acc;
+            s.acc = 0u;
             ++s.nw;
           }
+          sm100::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&tempty[st]);   // the accumulator is drained
+          // exact repair of the codes whose z fell within the error radius of a
+          // threshold (a few per warp tile; the flagged lanes work in parallel)
+          if (__any_sync(0xffffffffu, (fm[0] | fm[1] | fm[2] | fm[3]) != 0u))
+            repair_warp(make_uint4(fm[0], fm[1], fm[2], fm[3]), P.x, xbase, s.dst, vt64, sig, bits, rec.offsets(),
+                        normalize, sTh64, lane);
+          __syncwarp();
+        } else {
+          sm100::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&tempty[st]);
         }
-        sm100::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) sm100::mbar_arrive(&tempty[st]);
       }
     }
     k += (uint32_t)nt;
