@@ -156,13 +156,24 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            # the sampler is running before the timed region starts (first line written)
+            t0 = time.time()
+            while time.time() - t0 < 5.0 and os.path.getsize(self.path) == 0:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
 
     def stop(self):
         if self.proc is None:
             return None
+        # one more sample at the end of the timed region (short regions see few)
+        try:
+            with open(self.path, "a") as f:
+                subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                "--format=csv,noheader,nounits"], stdout=f, stderr=subprocess.DEVNULL, timeout=10)
+        except Exception:
+            pass
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)

@@ -145,13 +145,14 @@ bool cache_ok(const sq_cache* c, int batch, int n_heads) {
 
 CacheArgs cache_args(const sq_cache* c) { return CacheArgs{c->codes, c->norm, c->rnorm, c->cap, c->words}; }
 
-// Splits of the context per (batch, KV head) so that the partial kernel has
-// about six blocks per SM of a 148-SM B200 (two waves of three resident
-// blocks), each over >= one 128-token tile.
+// Splits of the context per (batch, KV head): about eight waves of the
+// partial kernel's resident blocks (three per SM of a 148-SM B200), so that the
+// last, partly filled wave costs little, with at least 512 tokens per block so
+// that its setup stays small against its tiles.
 int attn_splits(int batch, int n_kv, int64_t max_ctx) {
   int64_t units = (int64_t)batch * n_kv;
-  int64_t want = (6 * 148 + units - 1) / units;
-  int64_t tiles = (max_ctx + kAttnTile - 1) / kAttnTile;
+  int64_t want = (24 * 148 + units - 1) / units;
+  int64_t tiles = (max_ctx + 511) / 512;
   if (want > tiles) want = tiles;
   if (want > 256) want = 256;
   if (want < 1) want = 1;

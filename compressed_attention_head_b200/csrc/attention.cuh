@@ -60,6 +60,7 @@ __global__ void k_attn_prepare(const uint8_t* __restrict__ recs_k, const TQ* __r
     float acc[MAXG];
 #pragma unroll
     for (int hh = 0; hh < MAXG; ++hh) acc[hh] = 0.0f;
+#pragma unroll 8
     for (int j = 0; j < d; ++j) {
       const float v = V[(size_t)j * d + i];
 #pragma unroll
@@ -324,10 +325,12 @@ __global__ void __launch_bounds__(256) k_attn_combine(const uint8_t* __restrict_
   }
   __syncthreads();
   const float* V = rv.V_f();
+#pragma unroll 2
   for (int j = warp; j < d; j += 8) {
     float o[MAXG];
 #pragma unroll
     for (int hh = 0; hh < MAXG; ++hh) o[hh] = 0.0f;
+#pragma unroll 4
     for (int i = lane; i < d; i += 32) {
       const float vv = ok ? V[(size_t)j * d + i] : 0.0f;
 #pragma unroll

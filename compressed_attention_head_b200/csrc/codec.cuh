@@ -238,6 +238,7 @@ __global__ void __launch_bounds__(256) k_append(const uint8_t* __restrict__ recs
     double acc[NV];
 #pragma unroll
     for (int v = 0; v < NV; ++v) acc[v] = 0.0;
+#pragma unroll 8
     for (int j = part * jl; j < (part + 1) * jl; ++j) {
       const double vv = V[(size_t)j * d + i];
 #pragma unroll
