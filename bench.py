@@ -527,7 +527,9 @@ def run_gpu(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16 in; fp16 tensor-core rotation, f64 exact recomputation near thresholds; fp16 tensor-core attention with f32 accumulate", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f16",
+        "dtype_detail": "fp16 tensor-core rotation and attention with f32 accumulation; f64 for the key signal "
+                        "coordinates and for exact recomputation of codes near a threshold", "data": "synthetic",
         "config": workload_config(cfg, world),
         "roofline": {"bound": "hbm", "kernel": dom["kernel"], "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
