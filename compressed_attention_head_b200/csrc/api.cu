@@ -145,18 +145,33 @@ bool cache_ok(const sq_cache* c, int batch, int n_heads) {
 
 CacheArgs cache_args(const sq_cache* c) { return CacheArgs{c->codes, c->norm, c->rnorm, c->cap, c->words}; }
 
-// Splits of the context per (batch, KV head): about eight waves of the
-// partial kernel's resident blocks (three per SM of a 148-SM B200), so that the
-// last, partly filled wave costs little, with at least 512 tokens per block so
-// that its setup stays small against its tiles.
-int attn_splits(int batch, int n_kv, int64_t max_ctx) {
-  int64_t units = (int64_t)batch * n_kv;
-  int64_t want = (24 * 148 + units - 1) / units;
-  int64_t tiles = (max_ctx + 511) / 512;
-  if (want > tiles) want = tiles;
-  if (want > 256) want = 256;
-  if (want < 1) want = 1;
-  return (int)want;
+// Splits of the context per (batch, KV head). Each block of the partial
+// kernel takes a span of whole 128-token tiles (32 tokens per warp) and pays a
+// fixed setup (tables, query fragments, final merge) of about half a warp tile.
+// With `slots` blocks resident at once (148 SMs of a B200 times the blocks per
+// SM the kernel is built for), equal blocks run in ceil(blocks / slots) waves,
+// so the cost of a split count S is waves(S) x (1/2 + tiles per warp); the
+// cheapest S wins (the smaller on ties, which also keeps the combine short).
+int attn_splits(int batch, int n_kv, int d, int64_t max_ctx) {
+  const int64_t units = (int64_t)batch * n_kv;
+  const int64_t slots = 148 * (int64_t)fa::min_blocks(d);
+  const int64_t ctx = max_ctx > 0 ? max_ctx : 1;
+  int best = 1;
+  int64_t best_cost = INT64_MAX;
+  for (int64_t S = 1; S <= 256; ++S) {
+    const int64_t per = (ctx + S - 1) / S;
+    const int64_t chunk = ((per + kAttnTile - 1) / kAttnTile) * kAttnTile;
+    const int64_t used = (ctx + chunk - 1) / chunk;        // splits that hold tokens
+    if (used != S) continue;
+    const int64_t waves = (units * S + slots - 1) / slots;
+    const int64_t cost = waves * (1 + 2 * (chunk / kAttnTile));
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = (int)S;
+    }
+    if (chunk == kAttnTile) break;
+  }
+  return best;
 }
 
 // cuTensorMapEncodeTiled, looked up through the runtime so that libsq does not
@@ -391,7 +406,7 @@ sq_status sq_decompress_kv(const void* calib, const sq_cache* cache, int d, int6
 
 size_t sq_attn_workspace(int batch, int n_q_heads, int n_kv_heads, int d, int64_t max_ctx) {
   if (batch < 1 || n_q_heads < 1 || n_kv_heads < 1 || !supported_d(d) || max_ctx < 0) return 0;
-  int splits = attn_splits(batch, n_kv_heads, max_ctx);
+  int splits = attn_splits(batch, n_kv_heads, d, max_ctx);
   return attn_ws_floats(batch, n_q_heads, d, splits) * sizeof(float);
 }
 
@@ -418,7 +433,7 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
   sh.n_kv = n_kv_heads;
   sh.group = n_q_heads / n_kv_heads;
   sh.d = d;
-  sh.splits = attn_splits(batch, n_kv_heads, max_ctx);
+  sh.splits = attn_splits(batch, n_kv_heads, d, max_ctx);
   sh.max_ctx = max_ctx;
   int64_t per = (max_ctx + sh.splits - 1) / sh.splits;
   sh.chunk = ((per + kAttnTile - 1) / kAttnTile) * kAttnTile;

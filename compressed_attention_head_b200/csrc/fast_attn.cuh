@@ -60,19 +60,31 @@ struct Tab {
   static constexpr int P2 = P1 + 16;                  // u32 [16]: width-2 level pairs
   static constexpr int QS = P2 + 64;                  // u32 [4]: QJL sign pairs (+-1)
   static constexpr int P3R = 128;                     // u32 [64][32]: width-3 pairs, lane-replicated
-  static constexpr int L16 = P3R + 64 * 32 * 4;       // half [kLevelsTotal]
-  static constexpr int HL = L16 + 1024;               // u32 [kLevelsTotal]: fp16 hi | fp16 lo << 16
+  // 16 zero bytes precede L16 and HL: entry -1 of either table reads as 0 (width-0 coordinates)
+  static constexpr int L16 = P3R + 64 * 32 * 4 + 16;  // half [kLevelsTotal]
+  static constexpr int HL = L16 + 1024 + 16;          // u32 [kLevelsTotal]: fp16 hi | fp16 lo << 16
   static constexpr int CH = HL + 2048;                // u32 [2][16]: chunk descriptors K, V
-  static constexpr int K0 = CH + 128;                 // u32 [16]: first key chunk, width | offset << 8
-  static constexpr int CTR = K0 + 64;                 // u32: next tile
-  static constexpr int END = CTR + 128;
+  static constexpr int CTR = CH + 128;                // u32: next tile
+  static constexpr int CD = CTR + 16;                 // u32 [2][D]: coordinate descriptors K, V
 };
-static_assert(Tab::L16 % 16 == 0 && Tab::HL % 16 == 0, "table alignment");
+static_assert(Tab::L16 % 16 == 0 && Tab::HL % 16 == 0 && Tab::CD % 16 == 0, "table alignment");
+static_assert(kLevelsTotal * 2 <= 1024 && kLevelsTotal * 4 <= 2048, "level tables");
 
 template <int D>
-__host__ __device__ constexpr int smem_bytes() {
-  return Tab::END + NW * Geo<D>::WARP_BYTES + 128;
+__host__ __device__ constexpr int tab_end() {
+  return (Tab::CD + 2 * D * 4 + 127) & ~127;
 }
+template <int D>
+__host__ __device__ constexpr int smem_bytes() {
+  return tab_end<D>() + NW * Geo<D>::WARP_BYTES + 128;
+}
+// Resident blocks per SM the kernel is built for (registers capped to match by
+// __launch_bounds__; shared memory checked below against the 228 KB of an SM,
+// 1 KB of it reserved per block).
+__host__ __device__ constexpr int min_blocks(int d) { return d <= 64 ? 4 : (d <= 128 ? 3 : 1); }
+static_assert(min_blocks(64) * (smem_bytes<64>() + 1024) <= 233472, "d 64 residency");
+static_assert(min_blocks(128) * (smem_bytes<128>() + 1024) <= 233472, "d 128 residency");
+static_assert(min_blocks(256) * (smem_bytes<256>() + 1024) <= 233472, "d 256 residency");
 // The merge at the end reuses the warp regions: [NW][8 heads][D + 2] floats.
 static_assert(NW * 8 * (64 + 2) * 4 <= NW * Geo<64>::WARP_BYTES, "merge buffer (d 64)");
 static_assert(NW * 8 * (128 + 2) * 4 <= NW * Geo<128>::WARP_BYTES, "merge buffer (d 128)");
@@ -153,99 +165,127 @@ __device__ __forceinline__ uint32_t fld(const uint32_t* p, int n, int pos) {
   return v & ((1u << n) - 1u);
 }
 
-// Decodes one width-B chunk (16 coordinates starting at bit o) of lane's
-// record into 16 fp16 levels, written as two 16-byte pieces of tile row lane
-// at columns col and col + 8.
-template <int B>
+// Decodes NC consecutive width-B chunks (16 NC coordinates starting at bit o)
+// of lane's record into fp16 levels, written as 16-byte pieces of tile row
+// lane from column col (two chunks at once give the loads of both to the
+// scheduler together).
+template <int B, int NC>
 __device__ __forceinline__ void decode_chunk(const uint32_t* rec, int o, int lane, const uint8_t* tb,
                                              uint8_t* tile, int rowbytes, int col) {
-  constexpr int NP = (16 * B + 31) / 32;
+  constexpr int NP = (16 * NC * B + 31) / 32;
   uint32_t p[NP];
   pieces<NP>(rec, o, lane, p);
-  uint32_t h[8];
+  uint32_t h[8 * NC];
   if (B == 1) {
     const uint32_t* t = (const uint32_t*)(tb + Tab::P1);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) h[k] = t[fld(p, 2, 2 * k)];
+    for (int k = 0; k < 8 * NC; ++k) h[k] = t[fld(p, 2, 2 * k)];
   } else if (B == 2) {
     const uint32_t* t = (const uint32_t*)(tb + Tab::P2);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) h[k] = t[fld(p, 4, 4 * k)];
+    for (int k = 0; k < 8 * NC; ++k) h[k] = t[fld(p, 4, 4 * k)];
   } else if (B == 3) {
     const uint32_t* t = (const uint32_t*)(tb + Tab::P3R) + lane;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) h[k] = t[fld(p, 6, 6 * k) * 32];
+    for (int k = 0; k < 8 * NC; ++k) h[k] = t[fld(p, 6, 6 * k) * 32];
   } else {
     const unsigned short* t = (const unsigned short*)(tb + Tab::L16) + lv_off(B);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < 8 * NC; ++k) {
       const uint32_t a = t[fld(p, B, B * (2 * k))];
       const uint32_t b = t[fld(p, B, B * (2 * k + 1))];
       h[k] = a | (b << 16);
     }
   }
+#pragma unroll
+  for (int q = 0; q < 2 * NC; ++q)
+    *(uint4*)(tile + swz(lane, col + 8 * q, rowbytes)) = make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+}
+
+// Coordinate descriptor: bit shift within the word (bits 0-4), code mask
+// (bits 8-15), byte offset of the word's row in the transposed record tile
+// (bits 16-31); all zero for a width-0 coordinate.
+__host__ __device__ constexpr uint32_t coord_desc(int width, int offset) {
+  return width == 0 ? 0u
+                    : ((uint32_t)(offset & 31) | (((1u << width) - 1u) << 8) |
+                       ((uint32_t)((offset >> 5) * RP * 4) << 16));
+}
+// Level-table index + 1 of the coordinate described by d in the record of the
+// lane whose column starts at rl: mask + code, i.e. lv_off(width) + code + 1,
+// and 0 for width 0 (entry -1 of the tables is zero).
+__device__ __forceinline__ uint32_t code_index(const uint32_t* rl, uint32_t d) {
+  const uint32_t* w = (const uint32_t*)((const uint8_t*)rl + (d >> 16));
+  const uint32_t v = __funnelshift_r(w[0], w[RP], d);
+  const uint32_t mask = (d >> 8) & 0xFFu;
+  return mask + (v & mask);
+}
+
+// Decodes a chunk of mixed widths coordinate by coordinate (fp16 levels),
+// from the chunk's 16 coordinate descriptors cd.
+__device__ __forceinline__ void decode_mixed(const uint32_t* rl, const uint32_t* cd, const uint8_t* tb, int lane,
+                                             uint8_t* tile, int rowbytes, int col) {
+  const unsigned short* t = (const unsigned short*)(tb + Tab::L16) - 1;
+  uint32_t h[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint2 dd = *(const uint2*)(cd + 2 * k);
+    const uint32_t x0 = t[code_index(rl, dd.x)];
+    const uint32_t x1 = t[code_index(rl, dd.y)];
+    h[k] = x0 | (x1 << 16);
+  }
   *(uint4*)(tile + swz(lane, col, rowbytes)) = make_uint4(h[0], h[1], h[2], h[3]);
   *(uint4*)(tile + swz(lane, col + 8, rowbytes)) = make_uint4(h[4], h[5], h[6], h[7]);
 }
 
-// Decodes a chunk of mixed widths coordinate by coordinate (fp16 levels).
-__device__ __forceinline__ void decode_mixed(const uint32_t* rec, const uint8_t* bits, const int32_t* offs, int c,
-                                             int lane, const uint8_t* tb, uint8_t* tile, int rowbytes) {
-  const unsigned short* l16 = (const unsigned short*)(tb + Tab::L16);
-  uint32_t h[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    uint32_t hv[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int i = 16 * c + 2 * k + e;
-      const int b = bits[i];
-      uint32_t v = 0u;
-      if (b > 0) {
-        uint32_t pc;
-        pieces<1>(rec, offs[i], lane, &pc);
-        v = l16[lv_off(b) + (pc & ((1u << b) - 1u))];
-      }
-      hv[e] = v;
-    }
-    h[k] = hv[0] | (hv[1] << 16);
-  }
-  *(uint4*)(tile + swz(lane, 16 * c, rowbytes)) = make_uint4(h[0], h[1], h[2], h[3]);
-  *(uint4*)(tile + swz(lane, 16 * c + 8, rowbytes)) = make_uint4(h[4], h[5], h[6], h[7]);
-}
-
-// Decodes all chunks of one side (first chunk excluded when skip0).
+// Decodes all chunks of one side (first chunk excluded when skip0); two
+// neighbouring chunks of one width go through one call.
 template <int D>
-__device__ __forceinline__ void decode_side(const uint32_t* rec, const uint32_t* chd, const uint8_t* bits,
-                                            const int32_t* offs, bool skip0, int lane, const uint8_t* tb,
-                                            uint8_t* tile) {
+__device__ __forceinline__ void decode_side(const uint32_t* rec, const uint32_t* chd, const uint32_t* cd, bool skip0,
+                                            int lane, const uint8_t* tb, uint8_t* tile) {
   constexpr int ROW = Geo<D>::ROW;
 #pragma unroll 1
-  for (int c = skip0 ? 1 : 0; c < Geo<D>::NCH; ++c) {
-    const uint32_t cd = chd[c];
-    const int o = (int)(cd >> 8);
-    switch (cd & 0xFFu) {
+  for (int c = skip0 ? 1 : 0; c < Geo<D>::NCH;) {
+    const uint32_t cw = chd[c];
+    const int o = (int)(cw >> 8);
+    const uint32_t w = cw & 0xFFu;
+    const bool pair = c + 1 < Geo<D>::NCH && w >= 1u && w <= 8u && (chd[c + 1] & 0xFFu) == w;
+    if (pair) {
+      switch (w) {
+        case 1: decode_chunk<1, 2>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+        case 2: decode_chunk<2, 2>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+        case 3: decode_chunk<3, 2>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+        case 4: decode_chunk<4, 2>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+        case 5: decode_chunk<5, 2>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+        case 6: decode_chunk<6, 2>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+        case 7: decode_chunk<7, 2>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+        default: decode_chunk<8, 2>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+      }
+      c += 2;
+      continue;
+    }
+    switch (w) {
       case 0: {
         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
         *(uint4*)(tile + swz(lane, 16 * c, ROW)) = z;
         *(uint4*)(tile + swz(lane, 16 * c + 8, ROW)) = z;
         break;
       }
-      case 1: decode_chunk<1>(rec, o, lane, tb, tile, ROW, 16 * c); break;
-      case 2: decode_chunk<2>(rec, o, lane, tb, tile, ROW, 16 * c); break;
-      case 3: decode_chunk<3>(rec, o, lane, tb, tile, ROW, 16 * c); break;
-      case 4: decode_chunk<4>(rec, o, lane, tb, tile, ROW, 16 * c); break;
-      case 5: decode_chunk<5>(rec, o, lane, tb, tile, ROW, 16 * c); break;
-      case 6: decode_chunk<6>(rec, o, lane, tb, tile, ROW, 16 * c); break;
-      case 7: decode_chunk<7>(rec, o, lane, tb, tile, ROW, 16 * c); break;
-      case 8: decode_chunk<8>(rec, o, lane, tb, tile, ROW, 16 * c); break;
-      default: decode_mixed(rec, bits, offs, c, lane, tb, tile, ROW); break;
+      case 1: decode_chunk<1, 1>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+      case 2: decode_chunk<2, 1>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+      case 3: decode_chunk<3, 1>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+      case 4: decode_chunk<4, 1>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+      case 5: decode_chunk<5, 1>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+      case 6: decode_chunk<6, 1>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+      case 7: decode_chunk<7, 1>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+      case 8: decode_chunk<8, 1>(rec, o, lane, tb, tile, ROW, 16 * c); break;
+      default: decode_mixed(rec + lane, cd + 16 * c, tb, lane, tile, ROW, 16 * c); break;
     }
+    ++c;
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restrict__ recs_k,
+__global__ void __launch_bounds__(NTH, min_blocks(D)) k_attn_partial_tc(const uint8_t* __restrict__ recs_k,
                                                          const uint8_t* __restrict__ recs_v, CacheArgs kc,
                                                          CacheArgs vc, const int32_t* __restrict__ seq_lens,
                                                          AttnShape s, float* __restrict__ ws,
@@ -295,7 +335,7 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
   __half* tL16 = (__half*)(sm + Tab::L16);
   uint32_t* tHL = (uint32_t*)(sm + Tab::HL);
   uint32_t* tCH = (uint32_t*)(sm + Tab::CH);
-  uint32_t* tK0 = (uint32_t*)(sm + Tab::K0);
+  uint32_t* tCD = (uint32_t*)(sm + Tab::CD);
   uint32_t* tCtr = (uint32_t*)(sm + Tab::CTR);
   if (tid < 4) tP1[tid] = pack_h2(c_lv32[lv_off(1) + (tid & 1)], c_lv32[lv_off(1) + (tid >> 1)]);
   if (tid < 16) tP2[tid] = pack_h2(c_lv32[lv_off(2) + (tid & 3)], c_lv32[lv_off(2) + (tid >> 2)]);
@@ -321,7 +361,16 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
     for (int k = 1; k < 16; ++k) uni = uni && bt[16 * c + k] == b0;
     tCH[(tid < NCH ? 0 : 16) + c] = (uni ? (uint32_t)b0 : kMixedChunk) | ((uint32_t)r.offsets()[16 * c] << 8);
   }
-  if (tid < 16 && ok) tK0[tid] = (uint32_t)rk.bits()[tid] | ((uint32_t)rk.offsets()[tid] << 8);
+  for (int e = tid; e < 2 * D; e += NTH) {
+    const Rec r = e < D ? rk : rv;
+    const int i = e < D ? e : e - D;
+    tCD[e] = ok ? coord_desc(r.bits()[i], r.offsets()[i]) : 0u;
+  }
+  if (tid < 4) {
+    // zero guards: entry -1 of the level tables
+    ((uint32_t*)(sm + Tab::L16))[-1 - tid] = 0u;
+    ((uint32_t*)(sm + Tab::HL))[-1 - tid] = 0u;
+  }
   if (tid == 0) *tCtr = 0u;
 
   // ---- query fragments (B operands): rows k = coordinates, columns n = heads.
@@ -365,7 +414,7 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
   __syncthreads();
 
   // ---- per-warp state
-  uint8_t* wr = sm + Tab::END + warp * GE::WARP_BYTES;
+  uint8_t* wr = sm + tab_end<D>() + warp * GE::WARP_BYTES;
   uint32_t* recK = (uint32_t*)(wr + GE::OFF_RK);
   uint32_t* recV = (uint32_t*)(wr + GE::OFF_RV);
   float* nrm = (float*)(wr + GE::OFF_NRM);   // [3][TT]: ||k||, rho, ||v||
@@ -390,7 +439,12 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
     const bool in = t0 + lane < t_hi;
     const uint32_t* sp = src + (in ? (t0 + lane) * wn : 0);
     uint32_t* dp = rec + lane;
-    for (int w = 0; w < wn; ++w) cp_async4_z(dp + w * RP, sp + w, in);
+    int w = 0;
+    for (; w + 4 <= wn; w += 4) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) cp_async4_z(dp + (w + j) * RP, sp + w + j, in);
+    }
+    for (; w < wn; ++w) cp_async4_z(dp + w * RP, sp + w, in);
   };
   auto stage_nrm = [&](int tile_i) {
     const int64_t t0 = t_lo + (int64_t)tile_i * TT;
@@ -425,29 +479,22 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
     // ---- decode the keys: first chunk as hi + lo, the rest as fp16, QJL signs
     {
       uint32_t hh[8], ll[8];
+      const uint32_t* thl = (const uint32_t*)(sm + Tab::HL) - 1;
+      const uint32_t* rl = recK + lane;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        uint32_t hi2[2], lo2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const uint32_t kd = tK0[2 * k + e];
-          const int bw = (int)(kd & 0xFFu);
-          uint32_t pc;
-          pieces<1>(recK, (int)(kd >> 8), lane, &pc);
-          const uint32_t code = pc & ((1u << bw) - 1u);
-          const uint32_t hl = bw ? tHL[lv_off(bw) + code] : 0u;
-          hi2[e] = hl & 0xFFFFu;
-          lo2[e] = hl >> 16;
-        }
-        hh[k] = hi2[0] | (hi2[1] << 16);
-        ll[k] = lo2[0] | (lo2[1] << 16);
+        const uint2 dd = *(const uint2*)(tCD + 2 * k);
+        const uint32_t x0 = thl[code_index(rl, dd.x)];
+        const uint32_t x1 = thl[code_index(rl, dd.y)];
+        hh[k] = __byte_perm(x0, x1, 0x5410);
+        ll[k] = __byte_perm(x0, x1, 0x7632);
       }
       *(uint4*)(tile + swz(lane, 0, ROW)) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
       *(uint4*)(tile + swz(lane, 8, ROW)) = make_uint4(hh[4], hh[5], hh[6], hh[7]);
       *(uint4*)(lot + swz32(lane, 0)) = make_uint4(ll[0], ll[1], ll[2], ll[3]);
       *(uint4*)(lot + swz32(lane, 8)) = make_uint4(ll[4], ll[5], ll[6], ll[7]);
     }
-    decode_side<D>(recK, chK, rk.bits(), rk.offsets(), true, lane, sm, tile);
+    decode_side<D>(recK, chK, tCD, true, lane, sm, tile);
     {
       uint32_t qh[8];
       uint32_t pc = 0u;
@@ -542,7 +589,7 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
     if (nxt < ntile) stage_nrm(nxt);
 
     // ---- decode the values into the same tile, then O^T += V^T P^T
-    decode_side<D>(recV, chV, rv.bits(), rv.offsets(), false, lane, sm, tile);
+    decode_side<D>(recV, chV, tCD + D, false, lane, sm, tile);
     __syncwarp();
     if (nxt < ntile) {
       stage_rec(recV, vcodes, wv, nxt);
@@ -583,7 +630,7 @@ __global__ void __launch_bounds__(NTH) k_attn_partial_tc(const uint8_t* __restri
     lh[e] = v;
   }
   __syncthreads();
-  float* mrg = (float*)(sm + Tab::END);     // [NW][8][D + 2]: acc[D], m, l
+  float* mrg = (float*)(sm + tab_end<D>());     // [NW][8][D + 2]: acc[D], m, l
   float* mw = mrg + warp * 8 * (D + 2);
   if (hn == 0) {
 #pragma unroll

@@ -283,7 +283,7 @@ __device__ __forceinline__ uint32_t quant(float z, float R, const QCtx& c, const
   else if (B == 2) return qz2(z, k.t2, R, dg);
   else if (B == 3) return qz3(z, k.t3[0], k.t3[1], k.t3[2], R, dg);
   else
-    return qzl(z, c.cell() + cell_off(B), c.q() + q_off(B), (float)(1 << (B - 2)), k.ncell[B], 1u << (B - 1), R,
+    return qzl(z, c.cell() + cell_off(B), c.q() + q_off(B), (float)(1 << (B >= 2 ? B - 2 : 0)), k.ncell[B], 1u << (B - 1), R,
                dg);
 }
 
