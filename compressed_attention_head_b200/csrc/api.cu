@@ -5,12 +5,15 @@
 #include "sq_common.cuh"
 
 namespace sq {
-__constant__ double c_lv64[kLevelsTotal];
-__constant__ double c_th64[kThreshTotal];
-__constant__ float c_lv32[kLevelsTotal];
+// Tables that kernels stage into shared memory with one element per thread
+// live in global memory (coalesced loads; constant memory would serialise the
+// 32 addresses of a warp); c_D is read with warp-uniform indices.
+__device__ double c_lv64[kLevelsTotal];
+__device__ double c_th64[kThreshTotal];
+__device__ float c_lv32[kLevelsTotal];
 __constant__ double c_D[SQ_MAX_BITS + 1];
-__constant__ float4 c_tcq[248];        // tcc cell tables: thresholds (T_j, T_j+1, T_j+2) per width 4..8
-__constant__ uint8_t c_tccell[560];    // tcc cell tables: positive thresholds below each cell
+__device__ float4 c_tcq[248];          // tcc cell tables: thresholds (T_j, T_j+1, T_j+2) per width 4..8
+__device__ uint8_t c_tccell[560];      // tcc cell tables: positive thresholds below each cell
 }  // namespace sq
 
 #include <cudaTypedefs.h>
@@ -234,10 +237,20 @@ template <typename T>
 sq_status launch_compress(const void* recs, const void* x, int batch, int n_heads, int d, int64_t n_tok,
                           const int32_t* sp, const sq_cache* c, uint32_t* flags, cudaStream_t st) {
   if (n_tok < 16) {      // appends: a block per (head, group of vectors)
-    const int64_t groups = ((int64_t)batch * n_tok + kAppendNV - 1) / kAppendNV;
+    const int64_t nvec = (int64_t)batch * n_tok;
+    const int nv = append_nv(nvec);
+    const int64_t groups = (nvec + nv - 1) / nv;
+    if (groups > 65535) return SQ_ERR_ARG;
     dim3 grid((unsigned)n_heads, (unsigned)groups);
-    k_append<T><<<grid, 256, 0, st>>>((const uint8_t*)recs, (const T*)x, batch, n_heads, d, n_tok, sp,
-                                      cache_args(c), flags);
+    const uint8_t* r8 = (const uint8_t*)recs;
+    const T* xt = (const T*)x;
+    const CacheArgs ca = cache_args(c);
+    switch (nv) {
+      case 1: k_append<T, 1><<<grid, 256, 0, st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
+      case 2: k_append<T, 2><<<grid, 256, 0, st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
+      case 4: k_append<T, 4><<<grid, 256, 0, st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
+      default: k_append<T, 8><<<grid, 256, 0, st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
+    }
     return cuda_ok(cudaGetLastError());
   }
   const int tpb = n_tok >= 1024 ? 256 : 64;

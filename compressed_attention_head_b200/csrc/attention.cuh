@@ -60,11 +60,16 @@ __global__ void k_attn_prepare(const uint8_t* __restrict__ recs_k, const TQ* __r
     float acc[MAXG];
 #pragma unroll
     for (int hh = 0; hh < MAXG; ++hh) acc[hh] = 0.0f;
-#pragma unroll 8
-    for (int j = 0; j < d; ++j) {
-      const float v = V[(size_t)j * d + i];
+    // the column of V in batches of 32 loads issued together (d is a multiple of 32)
+    for (int j0 = 0; j0 < d; j0 += 32) {
+      float vv[32];
 #pragma unroll
-      for (int hh = 0; hh < MAXG; ++hh) acc[hh] = fmaf(v, qs[hh][j], acc[hh]);
+      for (int u = 0; u < 32; ++u) vv[u] = V[(size_t)(j0 + u) * d + i];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+#pragma unroll
+        for (int hh = 0; hh < MAXG; ++hh) acc[hh] = fmaf(vv[u], qs[hh][j0 + u], acc[hh]);
+      }
     }
 #pragma unroll
     for (int hh = 0; hh < MAXG; ++hh) {
@@ -286,12 +291,12 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
 // a_h,i = sigma_V,i * sum_s e^(m_s - M) acc_s,i / sum_s e^(m_s - M) l_s;  o_h = V_V a_h.
 // ---------------------------------------------------------------------------
 template <int MAXG, typename TO>
-__global__ void __launch_bounds__(256) k_attn_combine(const uint8_t* __restrict__ recs_v, AttnShape s,
+__global__ void __launch_bounds__(256, 2) k_attn_combine(const uint8_t* __restrict__ recs_v, AttnShape s,
                                                       const float* __restrict__ ws, TO* __restrict__ out) {
   const int g = blockIdx.x, b = blockIdx.y, d = s.d, tid = threadIdx.x, G = s.group;
   const int lane = tid & 31, warp = tid >> 5;
   Rec rv = rec_at(recs_v, d, g);
-  __shared__ float a[MAXG][kMaxD];
+  __shared__ __align__(16) float a[MAXG][kMaxD];
   __shared__ float sw[MAXG][256];   // splits <= 256 (attn_splits)
   __shared__ float s_inv_l[MAXG];
   const float* acc = ws + (size_t)s.batch * s.n_q * d * 2;
@@ -320,27 +325,61 @@ __global__ void __launch_bounds__(256) k_attn_combine(const uint8_t* __restrict_
     const int hh = e / d, i = e % d;
     const float* ah = acc + (qh0 + hh) * s.splits * (size_t)d + i;
     float v = 0.0f;
-    for (int k = 0; k < s.splits; ++k) v = fmaf(sw[hh][k], ah[(size_t)k * d], v);
+    int k = 0;
+    for (; k + 4 <= s.splits; k += 4) {     // four loads in flight
+      const float a0 = ah[(size_t)k * d], a1 = ah[(size_t)(k + 1) * d];
+      const float a2 = ah[(size_t)(k + 2) * d], a3 = ah[(size_t)(k + 3) * d];
+      v = fmaf(sw[hh][k], a0, v);
+      v = fmaf(sw[hh][k + 1], a1, v);
+      v = fmaf(sw[hh][k + 2], a2, v);
+      v = fmaf(sw[hh][k + 3], a3, v);
+    }
+    for (; k < s.splits; ++k) v = fmaf(sw[hh][k], ah[(size_t)k * d], v);
     a[hh][i] = ok ? v * s_inv_l[hh] * sig[i] : 0.0f;
   }
   __syncthreads();
-  const float* V = rv.V_f();
-#pragma unroll 2
-  for (int j = warp; j < d; j += 8) {
-    float o[MAXG];
+  // o_h = V_V a_h: warp w takes rows w, w + 8, ...; lane reads 16-byte pieces
+  // (columns 4 (lane + 32 c)), RB rows of loads in flight
+  const float4* V4 = (const float4*)rv.V_f();
+  const int q4 = d / 4;
+  constexpr int RB = MAXG >= 8 ? 4 : 8;
+  for (int j0 = warp; j0 < d; j0 += 8 * RB) {
+    float4 vv[RB][2];
 #pragma unroll
-    for (int hh = 0; hh < MAXG; ++hh) o[hh] = 0.0f;
-#pragma unroll 4
-    for (int i = lane; i < d; i += 32) {
-      const float vv = ok ? V[(size_t)j * d + i] : 0.0f;
+    for (int r = 0; r < RB; ++r)
 #pragma unroll
-      for (int hh = 0; hh < MAXG; ++hh) o[hh] = fmaf(vv, a[hh][i], o[hh]);
-    }
+      for (int c = 0; c < 2; ++c) {
+        const int j = j0 + 8 * r, col = lane + 32 * c;
+        vv[r][c] = (ok && j < d && col < q4) ? V4[(size_t)j * q4 + col] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
 #pragma unroll
-    for (int hh = 0; hh < MAXG; ++hh) {
-      if (hh < G) {
-        const float r = warp_sum(o[hh]);
-        if (lane == 0) out[(qh0 + hh) * d + j] = from_float<TO>(r);
+    for (int r = 0; r < RB; ++r) {
+      const int j = j0 + 8 * r;
+      float o[MAXG];
+#pragma unroll
+      for (int hh = 0; hh < MAXG; ++hh) o[hh] = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int col = lane + 32 * c;
+        if (col < q4) {
+#pragma unroll
+          for (int hh = 0; hh < MAXG; ++hh) {
+            if (hh < G) {
+              const float4 av = *(const float4*)&a[hh][4 * col];
+              o[hh] = fmaf(vv[r][c].x, av.x, o[hh]);
+              o[hh] = fmaf(vv[r][c].y, av.y, o[hh]);
+              o[hh] = fmaf(vv[r][c].z, av.z, o[hh]);
+              o[hh] = fmaf(vv[r][c].w, av.w, o[hh]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int hh = 0; hh < MAXG; ++hh) {
+        if (hh < G) {
+          const float rs = warp_sum(o[hh]);
+          if (lane == 0 && j < d) out[(qh0 + hh) * d + j] = from_float<TO>(rs);
+        }
       }
     }
   }

@@ -148,19 +148,22 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
 
 // ---------------------------------------------------------------------------
 // Append (decode steps, fewer than 16 tokens per row): grid (n_heads, vector
-// groups), 256 threads. A block compresses up to kAppendNV vectors of one
-// head, the (batch, token) pairs g * kAppendNV ...; every element of V
-// (float64, read straight from the record) is loaded once per block and used
-// for all of them. Same arithmetic as k_compress_ref.
+// groups), 256 threads. A block compresses NV (1, 2, 4 or 8, the fewest that
+// hold the vectors of a head, at most 8) vectors of one head, the (batch,
+// token) pairs g * NV ...; every element of V (float64, read straight from the
+// record) is loaded once per block and used for all of them. Same arithmetic
+// as k_compress_ref.
 // ---------------------------------------------------------------------------
-constexpr int kAppendNV = 8;
 
-template <typename T>
+// Vectors per block for an append of nvec vectors per head: 1, 2, 4 or 8.
+inline int append_nv(int64_t nvec) { return nvec <= 1 ? 1 : (nvec <= 2 ? 2 : (nvec <= 4 ? 4 : 8)); }
+
+template <typename T, int NV>
 __global__ void __launch_bounds__(256) k_append(const uint8_t* __restrict__ recs, const T* __restrict__ x,
                                                 int batch, int n_heads, int d, int64_t n_tok,
                                                 const int32_t* __restrict__ start_pos, CacheArgs c,
                                                 uint32_t* __restrict__ flags) {
-  constexpr int NV = kAppendNV;
+  static_assert(NV >= 1 && NV <= 8, "one warp per vector in the norm and QJL steps");
   __shared__ double xs[NV][kMaxD];        // input, then the residual of the signal coordinates
   __shared__ double ys[NV][256];          // partial sums of V^T x (parts of the j range)
   __shared__ double th[kThreshTotal];
@@ -184,6 +187,16 @@ __global__ void __launch_bounds__(256) k_append(const uint8_t* __restrict__ recs
   const uint8_t* bits = rec.bits();
   const int32_t* offs = rec.offsets();
   const double* S = rec.S();
+  // y = V^T x below: thread (part, i) sums j in its part of [0, d), reading the
+  // column of V in batches of UB loads issued together; the first batch is
+  // requested here, before the tables and inputs are staged
+  constexpr int UB = NV <= 2 ? 32 : 16;
+  const int nparts = 256 / d;
+  const int part = tid / d, i_col = tid % d;
+  const int jl = d / nparts, j_beg = part * jl, j_end = j_beg + jl;
+  double vv[UB];
+#pragma unroll
+  for (int u = 0; u < UB; ++u) vv[u] = j_beg + u < j_end ? V[(size_t)(j_beg + u) * d + i_col] : 0.0;
   for (int e = tid; e < kThreshTotal; e += 256) th[e] = c_th64[e];
   for (int e = tid; e < kLevelsTotal; e += 256) lv[e] = c_lv64[e];
   for (int e = tid; e < NV * kMaxWords; e += 256) wb[e / kMaxWords][e % kMaxWords] = 0u;
@@ -214,7 +227,7 @@ __global__ void __launch_bounds__(256) k_append(const uint8_t* __restrict__ recs
   }
   __syncthreads();
   // norms: warp v
-  {
+  if (warp < NV) {
     double ss = 0.0;
     for (int j = lane; j < d; j += 32) ss += xs[warp][j] * xs[warp][j];
     ss = warp_sum(ss);
@@ -230,22 +243,26 @@ __global__ void __launch_bounds__(256) k_append(const uint8_t* __restrict__ recs
       }
     }
   }
-  // y = V^T x: thread (part, i) sums j in its part of [0, d)
+  // y = V^T x (first batch of V already in flight)
   {
-    const int nparts = 256 / d;
-    const int part = tid / d, i = tid % d;
-    const int jl = d / nparts;
     double acc[NV];
 #pragma unroll
     for (int v = 0; v < NV; ++v) acc[v] = 0.0;
-#pragma unroll 8
-    for (int j = part * jl; j < (part + 1) * jl; ++j) {
-      const double vv = V[(size_t)j * d + i];
+    for (int j0 = j_beg;;) {
 #pragma unroll
-      for (int v = 0; v < NV; ++v) acc[v] = fma(vv, xs[v][j], acc[v]);
+      for (int u = 0; u < UB; ++u) {
+        if (j0 + u < j_end) {
+#pragma unroll
+          for (int v = 0; v < NV; ++v) acc[v] = fma(vv[u], xs[v][j0 + u], acc[v]);
+        }
+      }
+      j0 += UB;
+      if (j0 >= j_end) break;
+#pragma unroll
+      for (int u = 0; u < UB; ++u) vv[u] = j0 + u < j_end ? V[(size_t)(j0 + u) * d + i_col] : 0.0;
     }
 #pragma unroll
-    for (int v = 0; v < NV; ++v) ys[v][part * d + i] = acc[v];
+    for (int v = 0; v < NV; ++v) ys[v][part * d + i_col] = acc[v];
   }
   __syncthreads();
   // codes, packed into the record words; residual of the signal coordinates
@@ -268,7 +285,7 @@ __global__ void __launch_bounds__(256) k_append(const uint8_t* __restrict__ recs
   }
   __syncthreads();
   // rho and the QJL sign bits: warp v
-  if (m > 0) {
+  if (m > 0 && warp < NV) {
     double r2 = 0.0;
     for (int k = lane; k < m; k += 32) r2 += xs[warp][k] * xs[warp][k];
     r2 = warp_sum(r2);

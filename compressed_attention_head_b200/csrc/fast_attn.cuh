@@ -357,8 +357,10 @@ __global__ void __launch_bounds__(NTH, min_blocks(D)) k_attn_partial_tc(const ui
     const int c = tid % NCH;
     const uint8_t* bt = r.bits();
     const int b0 = bt[16 * c];
-    bool uni = true;
-    for (int k = 1; k < 16; ++k) uni = uni && bt[16 * c + k] == b0;
+    uint32_t diff = 0u;
+#pragma unroll
+    for (int k = 1; k < 16; ++k) diff |= (uint32_t)(bt[16 * c + k] ^ b0);   // loads issued together
+    const bool uni = diff == 0u;
     tCH[(tid < NCH ? 0 : 16) + c] = (uni ? (uint32_t)b0 : kMixedChunk) | ((uint32_t)r.offsets()[16 * c] << 8);
   }
   for (int e = tid; e < 2 * D; e += NTH) {
@@ -376,8 +378,18 @@ __global__ void __launch_bounds__(NTH, min_blocks(D)) k_attn_partial_tc(const ui
   // ---- query fragments (B operands): rows k = coordinates, columns n = heads.
   // fp16 of w * wsc (hi; and lo for the first chunk) and of the QJL weights u.
   const size_t qbase = (size_t)b * s.n_q + (size_t)g * G;
+  // max |w| over the G heads (rows qbase .. qbase + G - 1 are contiguous), four
+  // loads in flight per lane; then max |u| over their first m entries
   float wmax = 0.0f;
-  for (int e = lane; e < G * D; e += 32) wmax = fmaxf(wmax, fabsf(wq[(qbase + e / D) * D + e % D]));
+  {
+    const float* wg = wq + qbase * D;
+    int e = lane;
+    for (; e + 96 < G * D; e += 128) {
+      const float a0 = wg[e], a1 = wg[e + 32], a2 = wg[e + 64], a3 = wg[e + 96];
+      wmax = fmaxf(wmax, fmaxf(fmaxf(fabsf(a0), fabsf(a1)), fmaxf(fabsf(a2), fabsf(a3))));
+    }
+    for (; e < G * D; e += 32) wmax = fmaxf(wmax, fabsf(wg[e]));
+  }
   for (int e = lane; e < G * m; e += 32) wmax = fmaxf(wmax, fabsf(uq[(qbase + e / m) * D + e % m]));
   wmax = warp_max(wmax);
   const float wsc = wmax > 0.0f ? exp2f(-ceilf(log2f(wmax))) : 1.0f;

@@ -216,10 +216,13 @@ def test_full_size_prefill_in_bench_launch_configuration():
         compare_compressed(vw[0, h, ts], vc.norm[0, h, ts].cpu().numpy(), None, xv, cvs[h])
 
 
-@pytest.mark.parametrize("name,batch,ntok", [("qwen14b", 11, 3), ("tiny", 5, 15), ("gemma9b_sweep", 9, 1)])
+@pytest.mark.parametrize("name,batch,ntok", [("qwen14b", 11, 3), ("tiny", 5, 15), ("gemma9b_sweep", 9, 1),
+                                             ("llama8b", 1, 1), ("qwen1_5b_long", 2, 1), ("tiny", 1, 3),
+                                             ("qwen14b", 3, 1), ("llama8b", 2, 3)])
 def test_append_groups_of_vectors(name, batch, ntok):
-    """Decode-step compress of several tokens for many rows (vector groups of eight,
-    a ragged last group), each row at its own position, against the oracle."""
+    """Decode-step compress of several tokens for many rows (blocks of 1, 2, 4 or
+    8 vectors of a head, a ragged last group), each row at its own position,
+    against the oracle."""
     w, ck, cv, k, v, nh = _case(name, batch=batch, tokens=ntok, heads=2)
     rng = np.random.default_rng(3)
     cap = 64
