@@ -345,11 +345,6 @@ __device__ __forceinline__ void flag_chunk(uint32_t (&fm)[4], int c, uint32_t dm
 #pragma unroll
   for (int q = 0; q < 4; ++q) fm[q] |= (c >> 1) == q ? sh : 0u;
 }
-__device__ __forceinline__ void flag_coord(uint32_t (&fm)[4], int i, bool dg) {
-  const uint32_t bit = dg ? 1u << (i & 31) : 0u;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) fm[q] |= (i >> 5) == q ? bit : 0u;
-}
 
 // Exact repair of the flagged codes of a warp's 32 records, after they have
 // been written: rounds of up to RB (lane, coordinate) entries, each
@@ -523,18 +518,21 @@ __device__ __forceinline__ void chunk_uniform(const float* v, float Rc, const QC
 }
 
 // One run of a mixed chunk: len coordinates of width B starting at chunk
-// position k0 (values in the lane's swizzled scratch row), each code flagged
-// if in band and appended to the stream.
+// position k0 (values in the lane's swizzled scratch row), each code appended
+// to the stream; returns the in-band flags of the run (bit k for position k).
 template <int B>
-__device__ __forceinline__ void run_codes(const float* mx, int lane, int k0, int len, int i0, bool fix_ok,
-                                          const QCtx& qc, const QuantConst& kqc, uint32_t (&fm)[4], Stream& s) {
+__device__ __forceinline__ uint32_t run_codes(const float* mx, int lane, int k0, int len, const QCtx& qc,
+                                              const QuantConst& kqc, Stream& s) {
+  const float R = qc.R(B);
+  uint32_t dm = 0u;
 #pragma unroll 1
   for (int k = k0; k < k0 + len; ++k) {
     bool dg;
-    const uint32_t code = quant<B>(mx[k ^ (lane & 15)] * qc.zr, qc.R(B), qc, kqc, dg);
-    flag_coord(fm, i0 + k, dg && fix_ok);
+    const uint32_t code = quant<B>(mx[k ^ (lane & 15)] * qc.zr, R, qc, kqc, dg);
+    dm |= (dg ? 1u : 0u) << k;
     put(s, code, B);
   }
+  return dm;
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -820,6 +818,7 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
               for (int kq = 0; kq < 16; ++kq) mx[kq ^ (lane & 15)] = v[kq];
               const int nr = (int)((cd >> 8) & 31u);
               int k0 = 0;
+              uint32_t dmc = 0u;
 #pragma unroll 1
               for (int r = 0; r < nr; ++r) {
                 const uint32_t rn = runs[c * 16 + r];
@@ -829,19 +828,20 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
                     for (int kq = k0; kq < k0 + len; ++kq) put(s, scode[(c * 16 + kq) & (MSIG - 1)], w);
                   } else {
                     switch (w) {
-                      case 1: run_codes<1>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
-                      case 2: run_codes<2>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
-                      case 3: run_codes<3>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
-                      case 4: run_codes<4>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
-                      case 5: run_codes<5>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
-                      case 6: run_codes<6>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
-                      case 7: run_codes<7>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
-                      default: run_codes<8>(mx, lane, k0, len, c * 16, fix_ok, qc, KQ, fm, s); break;
+                      case 1: dmc |= run_codes<1>(mx, lane, k0, len, qc, KQ, s); break;
+                      case 2: dmc |= run_codes<2>(mx, lane, k0, len, qc, KQ, s); break;
+                      case 3: dmc |= run_codes<3>(mx, lane, k0, len, qc, KQ, s); break;
+                      case 4: dmc |= run_codes<4>(mx, lane, k0, len, qc, KQ, s); break;
+                      case 5: dmc |= run_codes<5>(mx, lane, k0, len, qc, KQ, s); break;
+                      case 6: dmc |= run_codes<6>(mx, lane, k0, len, qc, KQ, s); break;
+                      case 7: dmc |= run_codes<7>(mx, lane, k0, len, qc, KQ, s); break;
+                      default: dmc |= run_codes<8>(mx, lane, k0, len, qc, KQ, s); break;
                     }
                   }
                 }
                 k0 += len;
               }
+              flag_chunk(fm, c, fix_ok ? dmc : 0u);
             } else {
               switch (cd) {
                 case 1: chunk_uniform<1>(v, rch[c], qc, KQ, fix_ok, c, fm, s); break;
