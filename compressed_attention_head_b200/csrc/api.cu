@@ -361,6 +361,20 @@ sq_status sq_calib_import(void* calib, int n_heads, int d, int* d_status, sq_str
   return cuda_ok(cudaGetLastError());
 }
 
+// One side of sq_compress_kv: the tensor-core path for fp16 head_dim-128
+// prompts, the float64 reference kernels otherwise.
+static sq_status compress_side(const void* recs, const void* x, sq_dtype dtype, int batch, int n_heads, int d,
+                               int64_t n_tok, const int32_t* sp, const sq_cache* c, uint32_t* flags,
+                               cudaStream_t st, int dev) {
+  if (dtype == SQ_F16 && d == tcc::D && n_tok >= 64 && !g_force_ref)
+    return launch_compress_tc(recs, x, batch, n_heads, n_tok, sp, c, flags, st, dev);
+  switch (dtype) {
+    case SQ_F32: return launch_compress<float>(recs, x, batch, n_heads, d, n_tok, sp, c, flags, st);
+    case SQ_F16: return launch_compress<__half>(recs, x, batch, n_heads, d, n_tok, sp, c, flags, st);
+    default: return launch_compress<__nv_bfloat16>(recs, x, batch, n_heads, d, n_tok, sp, c, flags, st);
+  }
+}
+
 sq_status sq_compress_kv(const void* calib_k, const void* calib_v, const void* k, const void* v, sq_dtype dtype,
                          int batch, int n_heads, int d, int64_t n_tok, const int32_t* d_start_pos,
                          const sq_cache* kc, const sq_cache* vc, uint32_t* d_flags, sq_stream stream) {
@@ -381,22 +395,112 @@ sq_status sq_compress_kv(const void* calib_k, const void* calib_v, const void* k
   for (int side = 0; side < 2; ++side) {
     const void* x = side == 0 ? k : v;
     if (!x) continue;
-    const void* recs = side == 0 ? calib_k : calib_v;
-    const sq_cache* c = side == 0 ? kc : vc;
-    // Tensor-core path: fp16 head_dim 128 prompts.
-    if (dtype == SQ_F16 && d == tcc::D && n_tok >= 64 && !g_force_ref) {
-      s = launch_compress_tc(recs, x, batch, n_heads, n_tok, d_start_pos, c, d_flags, st, dev);
-      if (s != SQ_OK) return s;
-      continue;
-    }
-    switch (dtype) {
-      case SQ_F32: s = launch_compress<float>(recs, x, batch, n_heads, d, n_tok, d_start_pos, c, d_flags, st); break;
-      case SQ_F16: s = launch_compress<__half>(recs, x, batch, n_heads, d, n_tok, d_start_pos, c, d_flags, st); break;
-      default: s = launch_compress<__nv_bfloat16>(recs, x, batch, n_heads, d, n_tok, d_start_pos, c, d_flags, st); break;
-    }
+    s = compress_side(side == 0 ? calib_k : calib_v, x, dtype, batch, n_heads, d, n_tok, d_start_pos,
+                      side == 0 ? kc : vc, d_flags, st, dev);
     if (s != SQ_OK) return s;
   }
   return SQ_OK;
+}
+
+namespace {
+size_t dtype_bytes(sq_dtype t) { return t == SQ_F32 ? 4 : 2; }
+
+// Bytes of one staging slab holding `heads` heads of one batch row.
+size_t host_slab_bytes(int heads, int d, sq_dtype dtype, int64_t n_tok) {
+  const size_t row = (size_t)n_tok * d * dtype_bytes(dtype);
+  return ((size_t)heads * row + 255) & ~(size_t)255;
+}
+
+// The library's copy stream of each device (created on first use, never destroyed).
+cudaStream_t g_copy_stream[128] = {};
+sq_status copy_stream(int dev, cudaStream_t* out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_copy_stream[dev] && cudaStreamCreateWithFlags(&g_copy_stream[dev], cudaStreamNonBlocking) != cudaSuccess) {
+    g_copy_stream[dev] = nullptr;
+    return SQ_ERR_CUDA;
+  }
+  *out = g_copy_stream[dev];
+  return SQ_OK;
+}
+}  // namespace
+
+size_t sq_compress_host_staging(int batch, int n_heads, int d, sq_dtype dtype, int64_t n_tok) {
+  if (batch < 1 || n_heads < 1 || n_tok < 1 || !supported_d(d) || !valid_dtype(dtype)) return 0;
+  const size_t row = (size_t)n_tok * d * dtype_bytes(dtype);
+  size_t heads = ((size_t)16 << 20) / row + ((((size_t)16 << 20) % row) ? 1 : 0);
+  if (heads < 1) heads = 1;
+  if (heads > (size_t)n_heads) heads = (size_t)n_heads;
+  return 2 * host_slab_bytes((int)heads, d, dtype, n_tok);
+}
+
+sq_status sq_compress_kv_host(const void* calib_k, const void* calib_v, const void* h_k, const void* h_v,
+                              sq_dtype dtype, int batch, int n_heads, int d, int64_t n_tok,
+                              const int32_t* d_start_pos, const sq_cache* kc, const sq_cache* vc,
+                              void* d_staging, size_t staging_bytes, uint32_t* d_flags, sq_stream stream) {
+  if (!supported_d(d) || !valid_dtype(dtype)) return SQ_ERR_UNSUPPORTED;
+  if (batch < 1 || n_heads < 1 || n_tok < 0 || batch > 65535 || n_heads > 65535) return SQ_ERR_ARG;
+  if (n_tok == 0) return SQ_OK;
+  const bool do_k = h_k != nullptr, do_v = h_v != nullptr;
+  if (!do_k && !do_v) return SQ_ERR_ARG;
+  if (do_k && (!calib_k || ((uintptr_t)calib_k & 255u) || !cache_ok(kc, batch, n_heads))) return SQ_ERR_ARG;
+  if (do_v && (!calib_v || ((uintptr_t)calib_v & 255u) || !cache_ok(vc, batch, n_heads))) return SQ_ERR_ARG;
+  if ((d_start_pos && !aligned16(d_start_pos)) || !d_staging || ((uintptr_t)d_staging & 255u)) return SQ_ERR_ARG;
+  // pieces of hc whole heads of one batch row, two slabs
+  const size_t row = (size_t)n_tok * d * dtype_bytes(dtype);
+  const size_t half = (staging_bytes / 2) & ~(size_t)255;
+  size_t hc = half / row;
+  if (hc < 1) return SQ_ERR_WORKSPACE;
+  if (hc > (size_t)n_heads) hc = (size_t)n_heads;
+  const size_t slab = host_slab_bytes((int)hc, d, dtype, n_tok);   // <= half
+  int dev = 0;
+  sq_status s = ensure_init(&dev);
+  if (s != SQ_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream, cs = nullptr;
+  if ((s = copy_stream(dev, &cs)) != SQ_OK) return s;
+  cudaEvent_t ev[5] = {};   // fork, copied[2], free[2]
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      for (auto& f : ev)
+        if (f) cudaEventDestroy(f);
+      return SQ_ERR_CUDA;
+    }
+  cudaEvent_t fork = ev[0], copied[2] = {ev[1], ev[2]}, freed[2] = {ev[3], ev[4]};
+  s = (cudaEventRecord(fork, st) == cudaSuccess && cudaStreamWaitEvent(cs, fork, 0) == cudaSuccess) ? SQ_OK
+                                                                                                       : SQ_ERR_CUDA;
+  int64_t piece = 0;
+  for (int side = 0; side < 2 && s == SQ_OK; ++side) {
+    const uint8_t* hx = (const uint8_t*)(side == 0 ? h_k : h_v);
+    if (!hx) continue;
+    const void* recs = side == 0 ? calib_k : calib_v;
+    const sq_cache* c = side == 0 ? kc : vc;
+    for (int b = 0; b < batch && s == SQ_OK; ++b) {
+      for (int h0 = 0; h0 < n_heads && s == SQ_OK; h0 += (int)hc, ++piece) {
+        const int hn = (int)((size_t)(n_heads - h0) < hc ? (size_t)(n_heads - h0) : hc);
+        const int slot = (int)(piece & 1);
+        uint8_t* dx = (uint8_t*)d_staging + (size_t)slot * slab;
+        const size_t row0 = (size_t)b * n_heads + h0;
+        // the slab is free once the compression of the piece two back has run
+        if (piece >= 2 && cudaStreamWaitEvent(cs, freed[slot], 0) != cudaSuccess) { s = SQ_ERR_CUDA; break; }
+        if (cudaMemcpyAsync(dx, hx + row0 * row, (size_t)hn * row, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+            cudaEventRecord(copied[slot], cs) != cudaSuccess || cudaStreamWaitEvent(st, copied[slot], 0) != cudaSuccess) {
+          s = SQ_ERR_CUDA;
+          break;
+        }
+        sq_cache view = *c;
+        view.codes = c->codes + row0 * (size_t)c->cap * c->words;
+        view.norm = c->norm + row0 * (size_t)c->cap;
+        view.rnorm = c->rnorm ? c->rnorm + row0 * (size_t)c->cap : nullptr;
+        view.batch = 1;
+        view.n_heads = hn;
+        const uint8_t* rh = (const uint8_t*)recs + (size_t)h0 * record_bytes(d);
+        s = compress_side(rh, dx, dtype, 1, hn, d, n_tok, d_start_pos ? d_start_pos + b : nullptr, &view, d_flags,
+                          st, dev);
+        if (s == SQ_OK && cudaEventRecord(freed[slot], st) != cudaSuccess) s = SQ_ERR_CUDA;
+      }
+    }
+  }
+  for (auto& e : ev) cudaEventDestroy(e);   // released once their work has completed
+  return s;
 }
 
 sq_status sq_decompress_kv(const void* calib, const sq_cache* cache, int d, int64_t t0, int64_t n_tok,

@@ -60,6 +60,11 @@ _SIGNATURES = {
     "sq_compress_kv": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int64, _P, ctypes.POINTER(sq_cache), ctypes.POINTER(sq_cache),
                                       _P, _P]),
+    "sq_compress_host_staging": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int64]),
+    "sq_compress_kv_host": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int64, _P, ctypes.POINTER(sq_cache), ctypes.POINTER(sq_cache),
+                                           _P, ctypes.c_size_t, _P, _P]),
     "sq_decompress_kv": (ctypes.c_int, [_P, ctypes.POINTER(sq_cache), ctypes.c_int, ctypes.c_int64,
                                         ctypes.c_int64, ctypes.c_int, _P, _P, _P]),
     "sq_attn_workspace": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -218,6 +223,27 @@ def sq_compress_kv(calib_k, calib_v, k, v, batch, n_heads, d, n_tok, start_pos, 
                                 ctypes.byref(kcs) if kcs is not None else None,
                                 ctypes.byref(vcs) if vcs is not None else None, _ptr(flags),
                                 _stream(stream)), "sq_compress_kv")
+
+
+def sq_compress_host_staging(batch, n_heads, d, dtype, n_tok) -> int:
+    return lib().sq_compress_host_staging(batch, n_heads, d, DTYPE_CODE[dtype], n_tok)
+
+
+def sq_compress_kv_host(calib_k, calib_v, k, v, batch, n_heads, d, n_tok, start_pos, kc, vc, staging, flags=None,
+                        stream=None):
+    """k, v: CPU tensors (pinned for overlapped copies); staging: a device uint8 tensor."""
+    x = k if k is not None else v
+    for t in (k, v):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("sq_compress_kv_host takes contiguous host tensors")
+    kcs = kc.struct() if kc is not None else None
+    vcs = vc.struct() if vc is not None else None
+    _check(lib().sq_compress_kv_host(_ptr(calib_k), _ptr(calib_v), _ptr(k), _ptr(v), DTYPE_CODE[x.dtype], batch,
+                                     n_heads, d, n_tok, _ptr(start_pos),
+                                     ctypes.byref(kcs) if kcs is not None else None,
+                                     ctypes.byref(vcs) if vcs is not None else None, _ptr(staging),
+                                     staging.numel() * staging.element_size() if staging is not None else 0,
+                                     _ptr(flags), _stream(stream)), "sq_compress_kv_host")
 
 
 def sq_decompress_kv(calib, cache, d, t0, n_tok, apply_qjl, out, flags=None, stream=None):

@@ -269,6 +269,44 @@ sq_status sq_compress_kv(const void* calib_k, const void* calib_v, const void* k
                          uint32_t* d_flags, sq_stream stream);
 
 /*
+ * Device bytes of the staging buffer sq_compress_kv_host uses for this shape:
+ * two slabs, each holding the vectors of up to ceil(16 MiB / (n_tok * d *
+ * element size)) heads of one batch row (at least one head, at most n_heads),
+ * each slab rounded up to 256 bytes. 0 for an unsupported shape.
+ */
+size_t sq_compress_host_staging(int batch, int n_heads, int d, sq_dtype dtype, int64_t n_tok);
+
+/*
+ * sq_compress_kv with the keys and values in HOST memory: the same codes,
+ * norms and rho as sq_compress_kv on the same vectors (the same kernels run on
+ * the same data), with the host-to-device transfer overlapped with the
+ * compression. The vectors go through the caller's device staging buffer in
+ * pieces of whole heads of one batch row (keys first, then values); while one
+ * piece is compressed on `stream`, the next is copied on the library's copy
+ * stream for this device, so that the copy engine and the SMs work together.
+ *  h_k, h_v     host, dtype [batch][n_heads][n_tok][d], contiguous; page-locked
+ *               (cudaHostAlloc / cudaHostRegister) for the copies to overlap
+ *               (pageable memory works but each copy then blocks the host).
+ *               Either side may be NULL together with its records and cache.
+ *               They must stay valid and unchanged until `stream` has passed
+ *               the call's work.
+ *  d_staging    device, 256-byte aligned; staging_bytes >= the bytes of two
+ *               slabs of one head (else SQ_ERR_WORKSPACE). The piece size is
+ *               the most whole heads half of staging_bytes holds (rounded
+ *               down to 256 bytes per slab). It is scratch owned by the call
+ *               until `stream` has passed its work.
+ * Other arguments, layouts, results and flags as sq_compress_kv. The copy
+ * stream waits on `stream` before the first copy and `stream` waits on every
+ * copy before compressing its piece, so work enqueued on `stream` after the
+ * call runs after all of it. Returns SQ_ERR_CUDA if a stream, event or copy
+ * cannot be set up (nothing after that point is enqueued).
+ */
+sq_status sq_compress_kv_host(const void* calib_k, const void* calib_v, const void* h_k, const void* h_v,
+                              sq_dtype dtype, int batch, int n_heads, int d, int64_t n_tok,
+                              const int32_t* d_start_pos, const sq_cache* kc, const sq_cache* vc,
+                              void* d_staging, size_t staging_bytes, uint32_t* d_flags, sq_stream stream);
+
+/*
  * Reconstructs vectors from a packed cache: x_hat = norm * V (sigma * level(code)),
  * plus, when apply_qjl and the records carry QJL bits,
  * norm * V[:, 0:m] (sqrt(pi/2) / m * rnorm * S^T s), s_j = 2 bit_j - 1.

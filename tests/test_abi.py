@@ -84,3 +84,29 @@ def test_argument_errors_need_no_gpu(libsq):
     assert L.sq_compress_kv(None, None, None, None, 1, 1, 1, 32, 4, None, None, None, None, None) == sq.SQ_ERR_ARG
     assert L.sq_attn_workspace(1, 3, 2, 128, 100) > 0
     assert L.sq_attn_workspace(1, 1, 1, 100, 100) == 0
+
+
+def test_host_compress_staging_and_argument_errors(libsq):
+    """sq_compress_host_staging sizes (two 256-byte-rounded slabs of whole heads,
+    about 16 MiB each) and the host-input compress's checks, which run before
+    any CUDA call."""
+    L = sq.lib()
+    row = 2048 * 128 * 2                                    # one fp16 head of 2048 tokens
+    assert L.sq_compress_host_staging(1, 256, 128, sq.SQ_F16, 2048) == 2 * 32 * row
+    assert L.sq_compress_host_staging(4, 2, 128, sq.SQ_F16, 2048) == 2 * 2 * row
+    assert L.sq_compress_host_staging(1, 8, 32, sq.SQ_F32, 3) == 2 * 3072         # 8 heads of 384 B per slab
+    assert L.sq_compress_host_staging(1, 3, 32, sq.SQ_F32, 1) == 2 * 512          # 3 heads of 128 B, rounded up
+    assert L.sq_compress_host_staging(1, 8, 48, sq.SQ_F16, 64) == 0
+    assert L.sq_compress_host_staging(1, 8, 128, sq.SQ_F16, 0) == 0
+    fake = 1 << 20                                           # aligned addresses, never dereferenced
+    cache = sq.sq_cache(fake, fake, fake, 1, 2, 64, 12)
+    args = (fake, None, fake, None, sq.SQ_F16, 1, 2, 128, 64, None, ctypes.byref(cache), None)
+    one_head = 64 * 128 * 2
+    assert L.sq_compress_kv_host(*args, None, 1 << 20, None, None) == sq.SQ_ERR_ARG          # no staging
+    assert L.sq_compress_kv_host(*args, fake + 16, 1 << 20, None, None) == sq.SQ_ERR_ARG     # misaligned staging
+    assert L.sq_compress_kv_host(*args, fake, 2 * one_head - 1, None, None) == sq.SQ_ERR_WORKSPACE
+    assert L.sq_compress_kv_host(fake, None, None, None, sq.SQ_F16, 1, 2, 128, 64, None, None, None, fake,
+                                 1 << 20, None, None) == sq.SQ_ERR_ARG                       # nothing to compress
+    assert L.sq_compress_kv_host(*args[:8], 0, *args[9:], None, 0, None, None) == sq.SQ_OK    # n_tok = 0
+    assert L.sq_compress_kv_host(fake, None, fake, None, sq.SQ_F16, 1, 2, 48, 64, None, ctypes.byref(cache),
+                                 None, fake, 1 << 20, None, None) == sq.SQ_ERR_UNSUPPORTED

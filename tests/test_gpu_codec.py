@@ -237,3 +237,43 @@ def test_append_groups_of_vectors(name, batch, ntok):
                                v[b, h].double().numpy(), cv[h])
             others = np.setdiff1d(np.arange(cap), np.arange(s, s + ntok))
             assert np.all(kw[b, h, others] == 0) and np.all(vw[b, h, others] == 0)
+
+
+@pytest.mark.parametrize("name,batch,tokens,heads,slab_heads,dtype", [
+    ("llama8b", 2, 333, 3, 1, torch.float16),        # tensor-core path, one head per piece
+    ("qwen14b", 3, 200, 4, 3, torch.float16),        # pieces of 3 heads and a ragged last piece
+    ("tiny", 2, 100, 4, 2, torch.float32),           # float64 reference path, head_dim 32
+])
+def test_host_input_compress_matches_device_input(name, batch, tokens, heads, slab_heads, dtype):
+    """sq_compress_kv_host (pinned host inputs, copies overlapped through a
+    small staging buffer) writes exactly what sq_compress_kv writes from device
+    inputs, at per-row start positions, and matches the oracle."""
+    w, ck, cv, k, v, nh = _case(name, batch=batch, tokens=tokens, heads=heads)
+    k, v = k.to(dtype), v.to(dtype)
+    d = k.shape[-1]
+    cap = ((tokens + 40 + 15) // 16) * 16
+    start = [int(s) for s in np.random.default_rng(5).integers(0, cap - tokens + 1, size=batch)]
+    rk, rv, kd, vd = _compress(ck, cv, k, v, cap=cap, start=start)
+    kh = sq.alloc_cache(batch, nh, cap, ck[0].words, ck[0].m > 0)
+    vh = sq.alloc_cache(batch, nh, cap, cv[0].words, False)
+    sp = torch.tensor(start, dtype=torch.int32, device="cuda")
+    row = tokens * d * k.element_size()
+    slab = ((slab_heads * row + 255) // 256) * 256
+    staging = torch.empty(2 * slab, dtype=torch.uint8, device="cuda")
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sq.sq_compress_kv_host(rk, rv, k.pin_memory(), v.pin_memory(), batch, nh, d, tokens, sp, kh, vh, staging, flags)
+    torch.cuda.synchronize()
+    assert flags.item() == 0
+    assert np.array_equal(kh.words_u32(), kd.words_u32()) and np.array_equal(vh.words_u32(), vd.words_u32())
+    assert torch.equal(kh.norm, kd.norm) and torch.equal(vh.norm, vd.norm)
+    if kd.rnorm is not None:
+        assert torch.equal(kh.rnorm, kd.rnorm)
+    b, h = batch - 1, nh - 1
+    s0 = start[b]
+    compare_compressed(kh.words_u32()[b, h, s0:s0 + tokens], kh.norm[b, h, s0:s0 + tokens].cpu().numpy(),
+                       kh.rnorm[b, h, s0:s0 + tokens].cpu().numpy() if kh.rnorm is not None else None,
+                       k[b, h].double().numpy(), ck[h])
+    with pytest.raises(sq.SqError) as e:
+        sq.sq_compress_kv_host(rk, rv, k.pin_memory(), v.pin_memory(), batch, nh, d, tokens, sp, kh, vh,
+                               staging[: 2 * row - 1], flags)
+    assert e.value.status == sq.SQ_ERR_WORKSPACE
