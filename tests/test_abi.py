@@ -110,3 +110,38 @@ def test_host_compress_staging_and_argument_errors(libsq):
     assert L.sq_compress_kv_host(*args[:8], 0, *args[9:], None, 0, None, None) == sq.SQ_OK    # n_tok = 0
     assert L.sq_compress_kv_host(fake, None, fake, None, sq.SQ_F16, 1, 2, 48, 64, None, ctypes.byref(cache),
                                  None, fake, 1 << 20, None, None) == sq.SQ_ERR_UNSUPPORTED
+
+
+def _splits_from_workspace(L, batch, n_q, n_kv, d, ctx):
+    floats = L.sq_attn_workspace(batch, n_q, n_kv, d, ctx) // 4
+    per_head = floats // (batch * n_q) - 2 * d
+    assert per_head % (d + 2) == 0
+    return per_head // (d + 2)
+
+
+def test_attention_split_count(libsq):
+    """The context split count behind sq_attn_workspace: every split holds
+    tokens (spans of whole 128-token tiles), and it minimises the documented
+    cost waves x (1/2 + 128-token tiles per block), with 148 SMs x 3 (d 128) or
+    4 (d 64) resident blocks, the smaller count on ties."""
+    L = sq.lib()
+    for (batch, n_kv, g, d, ctx) in [(1, 256, 4, 128, 2049), (4, 384, 5, 128, 8193), (16, 56, 6, 128, 32769),
+                                     (1, 2, 1, 64, 600), (2, 3, 2, 128, 1), (3, 7, 1, 128, 100000),
+                                     (1, 1, 1, 128, 300000)]:
+        s = _splits_from_workspace(L, batch, n_kv * g, n_kv, d, ctx)
+        assert 1 <= s <= 256
+        chunk = -(-(-(-ctx // s)) // 128) * 128
+        assert -(-ctx // chunk) == s                       # no empty split
+        slots = 148 * (4 if d <= 64 else 3)
+        units = batch * n_kv
+
+        def cost(S):
+            ch = -(-(-(-ctx // S)) // 128) * 128
+            return -(-units * S // slots) * (1 + 2 * (ch // 128))
+        valid = [S for S in range(1, 257) if -(-ctx // (-(-(-(-ctx // S)) // 128) * 128)) == S]
+        best = min(valid, key=lambda S: (cost(S), S))
+        assert s == best, (batch, n_kv, d, ctx, s, best)
+    # the three decode shapes of the benchmark
+    assert _splits_from_workspace(L, 1, 1024, 256, 128, 2049) == 3
+    assert _splits_from_workspace(L, 4, 1920, 384, 128, 8193) == 2
+    assert _splits_from_workspace(L, 16, 336, 56, 128, 32769) == 13
