@@ -569,8 +569,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="time the eager launches only")
     ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling captures only)")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--cpu-tokens", type=int, default=4096)
-    ap.add_argument("--cpu-ctx", type=int, default=2049)
+    ap.add_argument("--cpu-tokens", type=int, default=32768)
+    ap.add_argument("--cpu-ctx", type=int, default=8192)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
