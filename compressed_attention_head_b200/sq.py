@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(HERE, "libsq.so")
 SQ_OK, SQ_ERR_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_CUDA = 0, 1, 2, 3
 SQ_ERR_NOT_CONVERGED, SQ_ERR_CAPACITY, SQ_ERR_WORKSPACE, SQ_ERR_RECORD = 4, 5, 6, 7
 SQ_F32, SQ_F16, SQ_BF16 = 0, 1, 2
-SQ_FLAG_CAPACITY, SQ_FLAG_RECORD, SQ_FLAG_SEQLEN = 1, 2, 4
+SQ_FLAG_CAPACITY, SQ_FLAG_RECORD, SQ_FLAG_SEQLEN, SQ_FLAG_TIMEOUT = 1, 2, 4, 0x80000000
 DTYPE_CODE = {torch.float32: SQ_F32, torch.float16: SQ_F16, torch.bfloat16: SQ_BF16}
 
 

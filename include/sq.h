@@ -31,7 +31,8 @@
  *    (head_dim not in {32, 64, 128, 256}, or a dtype a call does not take),
  *    SQ_ERR_WORKSPACE (workspace too small). A failed launch returns SQ_ERR_CUDA.
  *  - Conditions only the device can see (a capacity overflow, a record that
- *    does not match the cache, a sequence length past the context bound) are
+ *    does not match the cache, a sequence length past the context bound, a
+ *    pipeline wait that timed out) are
  *    OR-ed into the optional device word d_flags (SQ_FLAG_*), and the affected
  *    rows are skipped; the call still returns SQ_OK. No kernel traps.
  *  - Pointers to device arrays must be 16-byte aligned. Strides are in elements.
@@ -68,6 +69,11 @@ typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2 } sq_dtype;
 #define SQ_FLAG_CAPACITY 1u   /* start_pos + n_tok > cap (or start_pos < 0): row skipped */
 #define SQ_FLAG_RECORD 2u     /* record magic/version/d/words do not match the call      */
 #define SQ_FLAG_SEQLEN 4u     /* seq_len > max_ctx or > cap, or < 0: row clamped          */
+/* A pipeline wait of the tensor-core compress (an mbarrier phase that did not
+ * complete within 2 s) gave up: the kernel stopped its remaining tiles, drained
+ * the copies it had issued, freed its tensor memory and returned; the records
+ * of those tiles are not written. */
+#define SQ_FLAG_TIMEOUT 0x80000000u
 
 #define SQ_MAX_BITS 8         /* largest code width of one coordinate                     */
 #define SQ_ABI_VERSION 1

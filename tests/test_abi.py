@@ -145,3 +145,21 @@ def test_attention_split_count(libsq):
     assert _splits_from_workspace(L, 1, 1024, 256, 128, 2049) == 3
     assert _splits_from_workspace(L, 4, 1920, 384, 128, 8193) == 2
     assert _splits_from_workspace(L, 16, 336, 56, 128, 32769) == 13
+
+
+def test_header_constants_match_the_binding():
+    """Every #define and enum value of the public header that the binding
+    mirrors has the same value there."""
+    text = open(os.path.join(ROOT, "include", "sq.h")).read()
+    defines = {m.group(1): int(m.group(2).rstrip("u"), 0)     # plain literals only, not expressions
+               for m in re.finditer(r"^#define\s+(SQ_\w+)\s+(0x[0-9a-fA-F]+u?|\d+u?)\s*(?:/\*.*)?$", text, re.M)}
+    enums = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(SQ_[A-Z0-9_]+)\s*=\s*(\d+)", text)}
+    mirrored = 0
+    for name, value in {**defines, **enums}.items():
+        if hasattr(sq, name):
+            assert getattr(sq, name) == value, name
+            mirrored += 1
+    for name in ("SQ_FLAG_CAPACITY", "SQ_FLAG_RECORD", "SQ_FLAG_SEQLEN", "SQ_FLAG_TIMEOUT", "SQ_ERR_WORKSPACE",
+                 "SQ_F16"):
+        assert name in defines or name in enums, name
+    assert mirrored >= 10
