@@ -65,3 +65,20 @@ def test_uniform_scores_average_values():
     assert np.all(scores == 0.0)
     vals = codec.decompress(vw[0, 0], vn[0, 0], None, cv[0], apply_qjl=False)
     assert np.allclose(out[0, 0], vals.mean(axis=0), rtol=1e-12, atol=1e-14)
+
+
+def test_dense_attention_matches_library_softmax_attention():
+    """The oracle's dense reference against PyTorch's scaled_dot_product_attention
+    (float64, CPU) on random keys, values and queries, several lengths and
+    scales, including a query that makes the softmax nearly one-hot."""
+    rng = np.random.default_rng(7)
+    for L, d, scale in [(1, 32, 0.2), (17, 64, 1 / 8), (300, 128, 1 / math.sqrt(128)), (64, 32, 40.0)]:
+        keys = rng.standard_normal((L, d))
+        vals = rng.standard_normal((L, d))
+        q = rng.standard_normal(d)
+        o, s = attention.dense_attention(q, keys, vals, scale)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q)[None, None, None], torch.from_numpy(keys)[None, None],
+            torch.from_numpy(vals)[None, None], scale=scale)[0, 0, 0].numpy()
+        assert np.allclose(o, ref, rtol=1e-12, atol=1e-12)
+        assert np.allclose(s, scale * keys @ q, rtol=1e-13, atol=1e-13)
