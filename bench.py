@@ -1,24 +1,34 @@
 #!/usr/bin/env python
 """Benchmark of the compressed-KV hot path (one JSON line on rank 0).
 
-A step is one pass of the per-batch hot path over one batch of synthetic
-input: compress the prompt's keys and values of every layer into packed
-records (rotation, Lloyd-Max codes, QJL signs, packing), append one decode
-token per layer, and run decode attention of every query head over the
-packed cache. Calibration is per model, not per batch (the SpectralQuant
-README calls it a one-time calibration): it runs once before the timed steps
-and is timed and reported on its own in the same line.
+Default (``--config headline``): the largest decode workload, Gemma-2-9B-shaped
+(42 layers, 16 query / 8 KV heads, head_dim 256, bf16, batch 64 at context
+4096, 3 bits per coordinate for keys and values, QJL on): a step is one decode
+step of every layer -- the new token's keys and values compressed into the
+packed cache (append) and decode attention of every query head over the
+whole packed context. ``value`` is decode tokens per second (batch rows per
+step / step time). In the same run and line, the prompt compress of the
+Llama-3.1-8B-shaped prefill (32 layers x 8 KV heads, head_dim 128, fp16, 2048
+tokens, 3 bits) is measured as the compression half of the metric
+(``compress`` object and ``roofline_compress``).
 
-Default workload: Llama-3.1-8B-shaped (32 layers, 32 query / 8 KV heads,
-head_dim 128, fp16, a 2048-token prompt, batch 1 per GPU, 3 bits per
-coordinate for keys and values). Layers are folded into the head index so
-each kernel covers all layers in one launch.
+``--config NAME`` runs one workload of synthetic/workloads.py instead: a
+prefill workload (tiny, llama8b) times compress-prompt + append + attention
+per step; a decode workload (qwen14b, qwen1_5b_long, gemma9b_sweep, with
+``--bits`` for the Gemma sweep and ``--no-qjl``) times append + attention.
+
+Decode caches: filling a context of millions of tokens through the float64
+compress of a bf16 head_dim-256 cache would take minutes, so the packed
+records of one layer's KV heads for a few batch rows are compressed from
+synthetic draws and repeated over the layers and the batch (distinct buffers:
+every step reads the whole cache from HBM); the calibration records repeat
+with them. Layers are folded into the head index, so each kernel covers all
+layers in one launch.
 
 End to end (the ``e2e`` key): the same step with every input in pinned host
-memory, through the C ABI: the prompt through sq_compress_kv_host (its
-host-to-device copies overlap the compression of the previous piece), the
-decode token and query copied in, the output copied back, all inside the
-timed region.
+memory, through the C ABI: the prompt through sq_compress_kv_host (prefill),
+the decode tokens and queries copied in, the output copied back, all inside
+the timed region.
 
 Multi-GPU: ``torchrun --nproc-per-node N bench.py --gpus N``. Each rank runs
 its own independent replica (weak scaling; the path has no exchange step).
@@ -41,6 +51,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "compressed-KV decode tokens/s & compress GB/s, % of B200 HBM roofline"
 HBM_FALLBACK_GBS = 6650.0
+HEADLINE_DECODE = "gemma9b_sweep"
+HEADLINE_COMPRESS = "llama8b"
 
 
 def _peaks():
@@ -53,17 +65,26 @@ def _peaks():
 
 
 # --------------------------------------------------------------------------- workload
-def build_workload(name: str, device: str, layers: int | None = None):
-    """All layers of one replica, layers folded into the head index. Tensors are
-    preallocated and filled layer by layer (the largest shape holds ~90 GB of fp16 KV)."""
-    import torch
-
-    from synthetic.workloads import CONFIGS, TORCH_DTYPE, make_workload
+def workload_cfg(name: str, layers: int | None = None, bits: float | None = None, qjl: bool = True):
+    from synthetic.workloads import CONFIGS
 
     cfg = dict(CONFIGS[name])
     cfg["name"] = name
     if layers:
         cfg["layers"] = layers
+    if bits is not None:
+        cfg["bits_k"] = cfg["bits_v"] = float(bits)
+    cfg["qjl"] = bool(qjl)
+    return cfg
+
+
+def build_prefill(cfg, device: str):
+    """All layers of one replica, layers folded into the head index, every layer
+    drawn on its own (the prompt is compressed inside the timed step)."""
+    import torch
+
+    from synthetic.workloads import TORCH_DTYPE, make_workload
+
     L, nkv, nq, d = cfg["layers"], cfg["n_kv"], cfg["n_q"], cfg["d"]
     T, B, ncal = cfg["ctx"], cfg["batch"], cfg["n_cal"]
     dt = TORCH_DTYPE[cfg["dtype"]]
@@ -91,13 +112,17 @@ def build_workload(name: str, device: str, layers: int | None = None):
                 k_new=k_new, v_new=v_new)
 
 
-def record_bytes_per_token(cfg, words_k, words_v, qjl):
-    """Algorithmic bytes moved per (token, head) by compress: input + record + side scalars."""
-    esz = 4 if cfg["dtype"] == "f32" else 2
-    kin = cfg["d"] * esz
-    k_out = 4 * words_k + 4 + (4 if qjl else 0)
-    v_out = 4 * words_v + 4
-    return kin + k_out, kin + v_out, k_out, v_out
+def record_bytes(words: int, qjl: bool) -> int:
+    """Bytes of one stored vector in the packed cache: record + norm (+ rho)."""
+    return 4 * words + 4 + (4 if qjl else 0)
+
+
+def rep_divisor(n: int, want: int) -> int:
+    """The largest divisor of n that is at most want."""
+    for k in range(min(n, want), 0, -1):
+        if n % k == 0:
+            return k
+    return 1
 
 
 # Source files each profiled kernel is built from (its DRAM traffic in
@@ -208,50 +233,6 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- CPU oracle
-def oracle_sample(name: str, tokens: int, q_heads: int, ctx: int):
-    """Times the oracle on one layer's KV heads: compress `tokens` tokens (K and V) and
-    decode attention of `q_heads` query heads over `ctx` packed tokens. Returns a dict of
-    rates (head-tokens/s for compress, context head-tokens/s for attention)."""
-    import numpy as np
-
-    from oracle import attention as oattn
-    from oracle import calibration as ocal
-    from oracle import codec as ocodec
-    from synthetic import CONFIGS, make_workload
-
-    cfg = CONFIGS[name]
-    n_kv = cfg["n_kv"]
-    w = make_workload(name, 0, batch=1, tokens=max(tokens, ctx))
-    ck = [ocal.calibrate(w.k_cal[h].double().numpy(), avg_bits=cfg["bits_k"], is_key=True, stream=h)
-          for h in range(n_kv)]
-    cv = [ocal.calibrate(w.v_cal[h].double().numpy(), avg_bits=cfg["bits_v"], is_key=False, stream=h)
-          for h in range(n_kv)]
-    t0 = time.perf_counter()
-    packed = []
-    for h in range(n_kv):
-        ok = ocodec.compress(w.k[0, h, :tokens].double().numpy(), ck[h])
-        ov = ocodec.compress(w.v[0, h, :tokens].double().numpy(), cv[h])
-        packed.append((ok, ov))
-    t_c = time.perf_counter() - t0
-    # attention over ctx tokens (reuse compressed records, tiled to ctx)
-    group = cfg["n_q"] // n_kv
-    reps = max(1, math.ceil(ctx / tokens))
-    kw = np.stack([np.tile(p[0]["words"], (reps, 1))[:ctx] for p in packed])[None]
-    kn = np.stack([np.tile(p[0]["norm"], reps)[:ctx] for p in packed])[None]
-    kr = np.stack([np.tile(p[0]["rnorm"], reps)[:ctx] for p in packed])[None]
-    vw = np.stack([np.tile(p[1]["words"], (reps, 1))[:ctx] for p in packed])[None]
-    vn = np.stack([np.tile(p[1]["norm"], reps)[:ctx] for p in packed])[None]
-    nq = min(q_heads, n_kv * group)
-    nkv_used = max(1, nq // group)
-    q = w.q[:, :nkv_used * group].double().numpy()
-    t0 = time.perf_counter()
-    oattn.attn_decode(q, kw[:, :nkv_used], kn[:, :nkv_used], kr[:, :nkv_used], vw[:, :nkv_used],
-                      vn[:, :nkv_used], ck[:nkv_used], cv[:nkv_used], [ctx], None)
-    t_a = time.perf_counter() - t0
-    return {"compress_rate": n_kv * tokens / t_c, "attn_rate": nkv_used * group * ctx / t_a,
-            "seconds": t_c + t_a, "tokens": tokens, "ctx": ctx, "q_heads": nkv_used * group}
-
-
 def cpu_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -263,49 +244,141 @@ def cpu_threads() -> int:
     return os.cpu_count() or 1
 
 
-def oracle_step_seconds(name: str, s: dict) -> float:
-    """Oracle seconds of one full step, extrapolated linearly from the sample rates."""
-    from synthetic import CONFIGS
+def _oracle_head(cfg, n_heads: int, tokens: int):
+    """Oracle calibrations and a seeded draw of ``tokens`` tokens for the first
+    ``n_heads`` KV heads of layer 0 (CPU, float64)."""
+    from oracle import calibration as ocal
+    from synthetic import make_workload
 
-    cfg = CONFIGS[name]
-    H = cfg["layers"] * cfg["n_kv"]
-    HQ = cfg["layers"] * cfg["n_q"]
-    B = cfg["batch"]
-    if cfg["mode"] == "prefill":
-        compress = B * H * (cfg["ctx"] + 1) / s["compress_rate"]
-        attn = B * HQ * (cfg["ctx"] + 1) / s["attn_rate"]
-    else:
-        compress = B * H * 1 / s["compress_rate"]
-        attn = B * HQ * (cfg["ctx"] + 1) / s["attn_rate"]
-    return compress + attn
+    g = cfg["n_q"] // cfg["n_kv"]
+    w = make_workload(dict(cfg, n_kv=n_heads, n_q=n_heads * g), 0, batch=1, tokens=tokens)
+    ck = [ocal.calibrate(w.k_cal[h].double().numpy(), avg_bits=cfg["bits_k"], is_key=True,
+                         qjl=cfg.get("qjl", True), stream=h) for h in range(n_heads)]
+    cv = [ocal.calibrate(w.v_cal[h].double().numpy(), avg_bits=cfg["bits_v"], is_key=False, stream=h)
+          for h in range(n_heads)]
+    return w, ck, cv
+
+
+def oracle_prefill_sample(cfg, tokens: int, ctx: int):
+    """Oracle seconds of one full prefill step (compress the prompt of every
+    layer, append, attention of every query head over the context), from a
+    timed sample of one layer: compress ``tokens`` tokens of its KV heads (K and
+    V) and decode attention of its query heads over ``ctx`` packed tokens,
+    extrapolated linearly in vectors and in attended token-heads."""
+    import numpy as np
+
+    from oracle import attention as oattn
+    from oracle import codec as ocodec
+
+    n_kv, g = cfg["n_kv"], cfg["n_q"] // cfg["n_kv"]
+    w, ck, cv = _oracle_head(cfg, n_kv, max(tokens, ctx))
+    t0 = time.perf_counter()
+    packed = []
+    for h in range(n_kv):
+        packed.append((ocodec.compress(w.k[0, h, :tokens].double().numpy(), ck[h]),
+                       ocodec.compress(w.v[0, h, :tokens].double().numpy(), cv[h])))
+    t_c = time.perf_counter() - t0
+    reps = max(1, math.ceil(ctx / tokens))
+    tile = lambda a: np.tile(a, (reps,) + (1,) * (a.ndim - 1))[:ctx]      # noqa: E731
+    kw = np.stack([tile(p[0]["words"]) for p in packed])[None]
+    kn = np.stack([tile(p[0]["norm"]) for p in packed])[None]
+    kr = np.stack([tile(p[0]["rnorm"]) for p in packed])[None]
+    vw = np.stack([tile(p[1]["words"]) for p in packed])[None]
+    vn = np.stack([tile(p[1]["norm"]) for p in packed])[None]
+    q = w.q.double().numpy()
+    t0 = time.perf_counter()
+    oattn.attn_decode(q, kw, kn, kr, vw, vn, ck, cv, [ctx], None)
+    t_a = time.perf_counter() - t0
+    H, HQ, B, T = cfg["layers"] * n_kv, cfg["layers"] * cfg["n_q"], cfg["batch"], cfg["ctx"]
+    step = B * H * (T + 1) * t_c / (n_kv * tokens) + B * HQ * (T + 1) * t_a / (n_kv * g * ctx)
+    desc = (f"one layer ({n_kv} KV heads): compress of {tokens} tokens K+V and decode attention of "
+            f"{n_kv * g} query heads over {ctx} tokens, {t_c + t_a:.1f} s of CPU work, extrapolated linearly "
+            f"to the full step")
+    return step, t_c + t_a, desc
+
+
+def oracle_decode_sample(cfg, pairs: int):
+    """Oracle seconds of one full decode step (append one token K+V and attend
+    G query heads over the context + 1 tokens, for every (batch row, KV head)),
+    from a timed sample of ``pairs`` (batch row, KV head) pairs at the full
+    context; the packed context is built outside the timing by compressing
+    4096 tokens and repeating them."""
+    import numpy as np
+
+    from oracle import attention as oattn
+    from oracle import codec as ocodec
+
+    g, T = cfg["n_q"] // cfg["n_kv"], cfg["ctx"]
+    base = min(T, 4096)
+    w, ck, cv = _oracle_head(cfg, 1, base + 1)
+    pk = ocodec.compress(w.k[0, 0, :base].double().numpy(), ck[0])
+    pv = ocodec.compress(w.v[0, 0, :base].double().numpy(), cv[0])
+    reps = math.ceil((T + 1) / base)
+    tile = lambda a: np.tile(a, (reps,) + (1,) * (a.ndim - 1))[:T + 1]    # noqa: E731
+    kw, kn, kr = tile(pk["words"]), tile(pk["norm"]), tile(pk["rnorm"])
+    vw, vn = tile(pv["words"]), tile(pv["norm"])
+    xk = w.k[0, 0, base:base + 1].double().numpy()
+    xv = w.v[0, 0, base:base + 1].double().numpy()
+    q = w.q.double().numpy()
+    t0 = time.perf_counter()
+    for _ in range(pairs):
+        ok_ = ocodec.compress(xk, ck[0])
+        ov_ = ocodec.compress(xv, cv[0])
+        kw[T], kn[T], kr[T] = ok_["words"][0], ok_["norm"][0], ok_["rnorm"][0]
+        vw[T], vn[T] = ov_["words"][0], ov_["norm"][0]
+        oattn.attn_decode(q, kw[None, None], kn[None, None], kr[None, None], vw[None, None], vn[None, None],
+                          ck, cv, [T + 1], None)
+    t = time.perf_counter() - t0
+    B, H = cfg["batch"], cfg["layers"] * cfg["n_kv"]
+    step = B * H * t / pairs
+    desc = (f"{pairs} (batch row, KV head) pairs of one decode step: append of the new token (K and V) and "
+            f"decode attention of {g} query heads over {T + 1} packed tokens, {t:.1f} s of CPU work, "
+            f"extrapolated linearly to the {B} x {H} pairs of the step")
+    return step, t, desc
 
 
 def step_tokens(cfg) -> int:
+    """Tokens one step processes: prompt + decode token for prefill, one decode token per row otherwise."""
     return cfg["batch"] * ((cfg["ctx"] + 1) if cfg["mode"] == "prefill" else 1)
+
+
+def workload_config(cfg, world):
+    qjl = cfg.get("qjl", True)
+    return {"workload": f"{cfg['name']}: {cfg['layers']} layers x {cfg['n_kv']} KV / {cfg['n_q']} query heads, "
+                        f"head_dim {cfg['d']}, {cfg['dtype']} KV, "
+                        + (f"prompt {cfg['ctx']} tokens + 1 decode token" if cfg["mode"] == "prefill"
+                           else f"1 decode token over a {cfg['ctx']}-token packed cache")
+                        + f", batch {cfg['batch']} per GPU, K {cfg['bits_k']} / V {cfg['bits_v']} bits per "
+                        f"coordinate, QJL {'on' if qjl else 'off'}",
+            "global_batch": cfg["batch"] * world, "layers": cfg["layers"], "head_dim": cfg["d"],
+            "context": cfg["ctx"], "l2": "inputs larger than L2 every step (no flush needed)"}
 
 
 # --------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
+    """The oracle (NumPy float64, as it stands) on the host cores, on a bounded
+    sample of the same workload each step, extrapolated to the full step."""
     if rank != 0:
         return
-    from synthetic import CONFIGS
-
-    cfg = CONFIGS[args.config]
-    times = []
-    sample = None
+    name = HEADLINE_DECODE if args.config == "headline" else args.config
+    cfg = workload_cfg(name, args.layers, args.bits, not args.no_qjl)
+    times, samples = [], []
+    desc = ""
     for i in range(args.warmup + args.steps):
-        s = oracle_sample(args.config, tokens=64, q_heads=cfg["n_q"] // cfg["n_kv"], ctx=256)
+        if cfg["mode"] == "decode":
+            t, secs, desc = oracle_decode_sample(cfg, pairs=args.ref_pairs)
+        else:
+            t, secs, desc = oracle_prefill_sample(cfg, tokens=args.ref_tokens, ctx=args.ref_ctx)
         if i >= args.warmup:
-            times.append(oracle_step_seconds(args.config, s))
-            sample = s
+            times.append(t)
+            samples.append(secs)
     t = statistics.mean(times)
     value = step_tokens(cfg) / t
-    desc = (f"oracle (NumPy float64) per step on one layer's {cfg['n_kv']} KV heads: compress of "
-            f"{sample['tokens']} tokens (K and V) and decode attention of {sample['q_heads']} query heads over "
-            f"{sample['ctx']} tokens; extrapolated linearly to the full step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t,
+            "ms_per_step_kind": "extrapolated from the timed sample of each step (see cpu_baseline.sample)",
+            "sample_ms_per_step": 1e3 * statistics.mean(samples),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(cfg, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": desc},
@@ -313,62 +386,107 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(cfg, world):
-    return {"workload": f"{cfg_name(cfg)}: {cfg['layers']} layers x {cfg['n_kv']} KV / {cfg['n_q']} query heads, "
-                        f"head_dim {cfg['d']}, {cfg['dtype']} KV, "
-                        + (f"prompt {cfg['ctx']} tokens + 1 decode token" if cfg["mode"] == "prefill"
-                           else f"1 decode token over a {cfg['ctx']}-token packed cache")
-                        + f", batch {cfg['batch']} per GPU, K {cfg['bits_k']} / V {cfg['bits_v']} bits per coordinate",
-            "global_batch": cfg["batch"] * world, "layers": cfg["layers"], "head_dim": cfg["d"],
-            "context": cfg["ctx"], "l2": "inputs larger than L2 every step (no flush needed)"}
-
-
-def cfg_name(cfg):
-    from synthetic import CONFIGS
-    if "name" in cfg:
-        return cfg["name"]
-    for k, v in CONFIGS.items():
-        if v is cfg:
-            return k
-    return "custom"
-
-
 # --------------------------------------------------------------------------- GPU arm
-def run_gpu(args, rank, world, local_rank):
+def _events(n):
+    import torch
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def _time_loop(step, steps, warmup, world, dev, n_marks):
+    """Eager timing of ``steps`` steps (after ``warmup``), barrier + synchronize on
+    both sides; per-step marks for the per-launch breakdown. Returns
+    (seconds per step, max over ranks; list of per-step mark lists)."""
     import torch
     import torch.distributed as dist
 
-    from compressed_attention_head_b200 import sq
+    for _ in range(warmup):
+        step(None)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    marks = [_events(n_marks) for _ in range(steps)]
+    a, b = _events(2)
+    a.record()
+    for i in range(steps):
+        step(marks[i])
+    b.record()
+    torch.cuda.synchronize()
+    return max_over_ranks(a.elapsed_time(b) / 1e3, dev) / steps, marks
 
-    dev = f"cuda:{local_rank}"
-    torch.cuda.set_device(local_rank)
-    sq.sq_init()
-    wl = build_workload(args.config, dev, args.layers)
-    cfg, H, HQ, d, T, B = wl["cfg"], wl["H"], wl["HQ"], wl["d"], wl["T"], wl["batch"]
-    prefill = cfg["mode"] == "prefill"
-    stream = torch.cuda.current_stream()
 
-    # ---- calibration (once per model; timed on its own)
-    pk = sq.calib_params(d, H, cfg["bits_k"], True)
+def _time_graph(step, steps, warmup, world, dev):
+    """The same step captured once as a CUDA graph and replayed (every call is
+    asynchronous and allocates nothing; the per-device tables were uploaded by
+    sq_init before capture). Seconds per step (max over ranks), or None."""
+    import torch
+    import torch.distributed as dist
+
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step(None)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            step(None)
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = _events(2)
+        a.record()
+        for _ in range(steps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        t = max_over_ranks(a.elapsed_time(b) / 1e3, dev) / steps
+        del g
+        return t
+    except Exception as exc:       # report, keep the eager number
+        print(f"graph capture failed: {exc}", file=sys.stderr)
+        return None
+
+
+def _mean_ms(marks, i, j):
+    return statistics.mean(m[i].elapsed_time(m[j]) for m in marks)
+
+
+def _calibrate(sq, cfg, H, k_cal, v_cal, dev):
+    """Records of H heads (GPU calibration); returns (rk, rv, words_k, words_v, ms, bad)."""
+    import torch
+
+    d, ncal = cfg["d"], k_cal.shape[1]
+    pk = sq.calib_params(d, H, cfg["bits_k"], True, qjl=cfg.get("qjl", True))
     pv = sq.calib_params(d, H, cfg["bits_v"], False)
     rk, rv = sq.alloc_records(H, d, dev), sq.alloc_records(H, d, dev)
-    ncal = wl["k_cal"].shape[1]
-    cws = torch.empty(sq.sq_calibrate_workspace(pk, ncal), dtype=torch.uint8, device=dev)
+    ws = torch.empty(sq.sq_calibrate_workspace(pk, ncal), dtype=torch.uint8, device=dev)
     st = torch.zeros(2 * H, dtype=torch.int32, device=dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a, b = _events(2)
     torch.cuda.synchronize()
-    e0.record()
-    sq.sq_calibrate(pk, wl["k_cal"], ncal, ncal * d, d, rk, cws, st[:H])
-    sq.sq_calibrate(pv, wl["v_cal"], ncal, ncal * d, d, rv, cws, st[H:])
-    e1.record()
+    a.record()
+    sq.sq_calibrate(pk, k_cal, ncal, ncal * d, d, rk, ws, st[:H])
+    sq.sq_calibrate(pv, v_cal, ncal, ncal * d, d, rv, ws, st[H:])
+    b.record()
     torch.cuda.synchronize()
-    calib_ms = e0.elapsed_time(e1)
-    n_bad = int((st != 0).sum().item())
-    words_k, words_v = sq.sq_record_words(pk), sq.sq_record_words(pv)
-    del cws
+    return rk, rv, sq.sq_record_words(pk), sq.sq_record_words(pv), a.elapsed_time(b), int((st != 0).sum().item())
 
-    cap = ((T + 1 + 15) // 16) * 16
-    kc = sq.alloc_cache(B, H, cap, words_k, True, dev)
+
+def measure_prefill(cfg, args, world, dev):
+    """Prompt compress of every layer + append + attention per step."""
+    import torch
+
+    from compressed_attention_head_b200 import sq
+
+    wl = build_prefill(cfg, dev)
+    H, HQ, d, T, B = wl["H"], wl["HQ"], wl["d"], wl["T"], wl["batch"]
+    qjl = cfg.get("qjl", True)
+    rk, rv, words_k, words_v, calib_ms, n_bad = _calibrate(sq, cfg, H, wl["k_cal"], wl["v_cal"], dev)
+    cap = ((T + 1 + 31) // 32) * 32
+    kc = sq.alloc_cache(B, H, cap, words_k, qjl, dev)
     vc = sq.alloc_cache(B, H, cap, words_v, False, dev)
     pos0 = torch.zeros(B, dtype=torch.int32, device=dev)
     posT = torch.full((B,), T, dtype=torch.int32, device=dev)
@@ -377,185 +495,232 @@ def run_gpu(args, rank, world, local_rank):
     aws = torch.empty(sq.sq_attn_workspace(B, HQ, H, d, max_ctx), dtype=torch.uint8, device=dev)
     out = torch.empty(B, HQ, d, dtype=torch.float32, device=dev)
     flags = torch.zeros(1, dtype=torch.int32, device=dev)
-    if not prefill:
-        # decode configs: the cache of ctx tokens is filled once, outside the timed steps,
-        # and the fp16 prompt is released
-        sq.sq_compress_kv(rk, rv, wl["k"], wl["v"], B, H, d, T, pos0, kc, vc, flags)
-        torch.cuda.synchronize()
-        del wl["k"], wl["v"]
-        torch.cuda.empty_cache()
 
-    n_ev = 6
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
-
-    def step(ev=None):
+    def step(ev):
         if ev: ev[0].record()
-        if prefill:
-            sq.sq_compress_kv(rk, None, wl["k"], None, B, H, d, T, pos0, kc, None, flags)
-            if ev: ev[1].record()
-            sq.sq_compress_kv(None, rv, None, wl["v"], B, H, d, T, pos0, None, vc, flags)
+        sq.sq_compress_kv(rk, None, wl["k"], None, B, H, d, T, pos0, kc, None, flags)
+        if ev: ev[1].record()
+        sq.sq_compress_kv(None, rv, None, wl["v"], B, H, d, T, pos0, None, vc, flags)
         if ev: ev[2].record()
         sq.sq_compress_kv(rk, rv, wl["k_new"], wl["v_new"], B, H, d, 1, posT, kc, vc, flags)
         if ev: ev[3].record()
         sq.sq_attn_decode(rk, rv, kc, vc, lens, B, HQ, H, d, max_ctx, wl["q"], 0.0, out, None, aws, flags)
         if ev: ev[4].record()
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = ClockSampler(local_rank)
-    clocks.start()
-    torch.cuda.synchronize()
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_start.record()
-    for i in range(args.steps):
-        step(evs[i])
-    t_end.record()
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    elapsed = max_over_ranks(t_start.elapsed_time(t_end) / 1e3, dev)
-    per_step = elapsed / args.steps
-    # The same step captured once as a CUDA graph and replayed: the launch gaps of the
-    # eager loop go away (every call is asynchronous, allocates nothing, and the
-    # per-device tables were uploaded by sq_init before capture).
-    graph_step = None
-    if not args.no_graph:
-        try:
-            g = torch.cuda.CUDAGraph()
-            side = torch.cuda.Stream()
-            side.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(side):
-                step()
-            torch.cuda.current_stream().wait_stream(side)
-            torch.cuda.synchronize()
-            with torch.cuda.graph(g):
-                step()
-            for _ in range(args.warmup):
-                g.replay()
-            torch.cuda.synchronize()
-            if world > 1:
-                dist.barrier()
-            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            for _ in range(args.steps):
-                g.replay()
-            b_.record()
-            torch.cuda.synchronize()
-            graph_step = max_over_ranks(a.elapsed_time(b_) / 1e3, dev) / args.steps
-            del g
-        except Exception as exc:       # report, keep the eager number
-            print(f"graph capture failed: {exc}", file=sys.stderr)
-            graph_step = None
-    eager_step = per_step
-    if graph_step is not None:
-        per_step = graph_step
-    if prefill:
-        ck_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-        cv_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    else:
-        ck_ms = cv_ms = 0.0
-    app_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    att_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
-    flag_val = int(flags.item())
-
-    # ---- algorithmic bytes
-    kb, vb, k_out, v_out = record_bytes_per_token(cfg, words_k, words_v, True)
-    comp_bytes_k = B * H * T * kb
-    comp_bytes_v = B * H * T * vb
-    attn_bytes = B * H * (T + 1) * (k_out + v_out)
-    peak, peak_kind = _peaks()
-    tokens = step_tokens(cfg) * world
-    value = tokens / per_step
-    if prefill:
-        dom = {"kernel": "k_compress_tc (prompt compress; mean of the K and V launches)",
-               "bytes": (comp_bytes_k + comp_bytes_v) / 2, "ms": (ck_ms + cv_ms) / 2,
-               "ncu_name": "k_compress_tc", "tokens": B * H * T}
-    else:
-        dom = {"kernel": "sq_attn_decode (prepare + partial + combine)", "bytes": attn_bytes, "ms": att_ms,
-               "ncu_name": "k_attn_partial_tc", "tokens": B * H * (T + 1)}
-    achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
-    breakdown = {
-        "step_ms_eager": 1e3 * eager_step, "step_ms_graph": None if graph_step is None else 1e3 * graph_step,
-        "compress_k_ms": ck_ms, "compress_v_ms": cv_ms, "append_ms": app_ms, "attention_ms": att_ms,
-        "compress_GBps": ((comp_bytes_k + comp_bytes_v) / ((ck_ms + cv_ms) / 1e3) / 1e9) if prefill else None,
-        "attention_GBps": attn_bytes / (att_ms / 1e3) / 1e9,
-        "attention_frac_of_hbm": attn_bytes / (att_ms / 1e3) / 1e9 / peak,
-        "decode_tokens_per_s": B * world / ((app_ms + att_ms) / 1e3),
-        "compress_tokens_per_s": (B * T * world / ((ck_ms + cv_ms) / 1e3)) if prefill else None,
-        "compress_bytes_per_token_head": {"k": kb, "v": vb}, "attention_bytes_per_token_head": k_out + v_out,
-    }
-
-    # ---- end to end through the C ABI with host buffers
-    e2e = None
+    eager, marks = _time_loop(step, args.steps, args.warmup, world, dev, 5)
+    graph = None if args.no_graph else _time_graph(step, args.steps, args.warmup, world, dev)
+    ck_ms, cv_ms = _mean_ms(marks, 0, 1), _mean_ms(marks, 1, 2)
+    app_ms, att_ms = _mean_ms(marks, 2, 3), _mean_ms(marks, 3, 4)
+    esz = wl["k"].element_size()
+    rec_k, rec_v = record_bytes(words_k, qjl), record_bytes(words_v, False)
+    comp_k = B * H * T * (d * esz + rec_k)
+    comp_v = B * H * T * (d * esz + rec_v)
+    attn_bytes = B * H * (T + 1) * (rec_k + rec_v)
+    res = dict(cfg=cfg, step_s=graph or eager, eager_s=eager, graph_s=graph, calib_ms=calib_ms, n_bad=n_bad,
+               calib_heads=2 * H, ck_ms=ck_ms, cv_ms=cv_ms, app_ms=app_ms, att_ms=att_ms,
+               comp_bytes=(comp_k + comp_v) / 2, comp_ms=(ck_ms + cv_ms) / 2, comp_k=comp_k, comp_v=comp_v,
+               attn_bytes=attn_bytes, rec_k=rec_k, rec_v=rec_v, tokens=step_tokens(cfg),
+               launches=4 + 2 + 3, flags=flags)
     if not args.no_e2e:
-        hk = wl["k"].cpu().pin_memory() if prefill else None
-        hv = wl["v"].cpu().pin_memory() if prefill else None
+        hk, hv = wl["k"].cpu().pin_memory(), wl["v"].cpu().pin_memory()
         hkn, hvn, hq = wl["k_new"].cpu().pin_memory(), wl["v_new"].cpu().pin_memory(), wl["q"].cpu().pin_memory()
         hout = torch.empty_like(out, device="cpu").pin_memory()
-
-        # the prompt goes through the library's host-input compress (its copies
-        # overlap the compression of the previous piece); the decode inputs are
-        # small and copied directly
         staging = torch.empty(sq.sq_compress_host_staging(B, H, d, wl["k"].dtype, T), dtype=torch.uint8,
-                              device=dev) if prefill else None
+                              device=dev)
 
-        def e2e_step():
+        def e2e_step(ev):
             wl["k_new"].copy_(hkn, non_blocking=True)
             wl["v_new"].copy_(hvn, non_blocking=True)
             wl["q"].copy_(hq, non_blocking=True)
-            if prefill:
-                sq.sq_compress_kv_host(rk, rv, hk, hv, B, H, d, T, pos0, kc, vc, staging, flags)
+            sq.sq_compress_kv_host(rk, rv, hk, hv, B, H, d, T, pos0, kc, vc, staging, flags)
             sq.sq_compress_kv(rk, rv, wl["k_new"], wl["v_new"], B, H, d, 1, posT, kc, vc, flags)
             sq.sq_attn_decode(rk, rv, kc, vc, lens, B, HQ, H, d, max_ctx, wl["q"], 0.0, out, None, aws, flags)
             hout.copy_(out, non_blocking=True)
 
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(args.steps):
-            e2e_step()
-        b.record()
-        torch.cuda.synchronize()
-        t_e2e = max_over_ranks(a.elapsed_time(b) / 1e3, dev)
-        h2d = (hk.numel() * hk.element_size() + hv.numel() * hv.element_size() if prefill else 0) + \
-            hkn.numel() * hkn.element_size() + hvn.numel() * hvn.element_size() + hq.numel() * hq.element_size()
-        e2e = {"value": tokens / (t_e2e / args.steps), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+        t_e2e, _ = _time_loop(e2e_step, args.steps, args.warmup, world, dev, 1)
+        h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hkn, hvn, hq))
+        res["e2e"] = {"value": step_tokens(cfg) * world / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+    return res
 
-    if rank != 0:
-        return
-    cpu = None
-    if world == 1 and not args.no_cpu:
-        s = oracle_sample(args.config, tokens=args.cpu_tokens, q_heads=cfg["n_q"], ctx=args.cpu_ctx)
-        t_oracle = oracle_step_seconds(args.config, s)
-        cpu = {"value": step_tokens(cfg) / t_oracle, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"one layer ({cfg['n_kv']} KV heads): compress of {s['tokens']} tokens K+V and decode "
-                         f"attention of {s['q_heads']} query heads over {s['ctx']} tokens, {s['seconds']:.1f} s of "
-                         f"CPU work, extrapolated linearly to the full step"}
+
+def measure_decode(cfg, args, world, dev):
+    """Append one token per (row, KV head) + attention over the packed context."""
+    import torch
+
+    from compressed_attention_head_b200 import sq
+    from synthetic.workloads import make_workload
+
+    L, nkv, nq, d, T, B = cfg["layers"], cfg["n_kv"], cfg["n_q"], cfg["d"], cfg["ctx"], cfg["batch"]
+    H, HQ = L * nkv, L * nq
+    qjl = cfg.get("qjl", True)
+    b0 = rep_divisor(B, args.base_rows)
+    w = make_workload(cfg, 0, device=dev, batch=b0, tokens=T)
+    nxt = make_workload(cfg, 0, device=dev, batch=b0, tokens=1, data_stream=1, with_calibration=False)
+    rk0, rv0, words_k, words_v, calib_ms, n_bad = _calibrate(sq, cfg, nkv, w.k_cal, w.v_cal, dev)
+    size = sq.sq_calib_bytes(d)
+    rk = rk0.view(nkv, size).repeat(L, 1).reshape(-1).contiguous()
+    rv = rv0.view(nkv, size).repeat(L, 1).reshape(-1).contiguous()
+    cap = ((T + 1 + 31) // 32) * 32
+    k1 = sq.alloc_cache(b0, nkv, cap, words_k, qjl, dev)
+    v1 = sq.alloc_cache(b0, nkv, cap, words_v, False, dev)
+    flags = torch.zeros(1, dtype=torch.int32, device=dev)
+    sq.sq_compress_kv(rk0, rv0, w.k, w.v, b0, nkv, d, T, None, k1, v1, flags)
+    torch.cuda.synchronize()
+    del w
+    rb = B // b0
+
+    def grow(c1, with_rnorm):
+        return sq.PackedCache(c1.codes.repeat(rb, L, 1, 1), c1.norm.repeat(rb, L, 1),
+                              c1.rnorm.repeat(rb, L, 1) if with_rnorm else None, B, H, cap, c1.words)
+
+    kc, vc = grow(k1, qjl), grow(v1, False)
+    del k1, v1
+    q = nxt.q.repeat(rb, L, 1).contiguous()
+    k_new = nxt.k.repeat(rb, L, 1, 1).contiguous()
+    v_new = nxt.v.repeat(rb, L, 1, 1).contiguous()
+    del nxt
+    torch.cuda.empty_cache()
+    posT = torch.full((B,), T, dtype=torch.int32, device=dev)
+    lens = torch.full((B,), T + 1, dtype=torch.int32, device=dev)
+    max_ctx = T + 1
+    aws = torch.empty(sq.sq_attn_workspace(B, HQ, H, d, max_ctx), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, HQ, d, dtype=torch.float32, device=dev)
+
+    def step(ev):
+        if ev: ev[0].record()
+        sq.sq_compress_kv(rk, rv, k_new, v_new, B, H, d, 1, posT, kc, vc, flags)
+        if ev: ev[1].record()
+        sq.sq_attn_decode(rk, rv, kc, vc, lens, B, HQ, H, d, max_ctx, q, 0.0, out, None, aws, flags)
+        if ev: ev[2].record()
+
+    eager, marks = _time_loop(step, args.steps, args.warmup, world, dev, 3)
+    graph = None if args.no_graph else _time_graph(step, args.steps, args.warmup, world, dev)
+    app_ms, att_ms = _mean_ms(marks, 0, 1), _mean_ms(marks, 1, 2)
+    rec_k, rec_v = record_bytes(words_k, qjl), record_bytes(words_v, False)
+    attn_bytes = B * H * (T + 1) * (rec_k + rec_v)
+    res = dict(cfg=cfg, step_s=graph or eager, eager_s=eager, graph_s=graph, calib_ms=calib_ms, n_bad=n_bad,
+               calib_heads=2 * nkv, app_ms=app_ms, att_ms=att_ms, attn_bytes=attn_bytes, rec_k=rec_k,
+               rec_v=rec_v, tokens=step_tokens(cfg), launches=2 + 3, flags=flags, base_rows=b0,
+               cache_bytes=sum(t.numel() * t.element_size() for t in (kc.codes, kc.norm, vc.codes, vc.norm)
+                               + ((kc.rnorm,) if kc.rnorm is not None else ())))
+    if not args.no_e2e:
+        hkn, hvn, hq = k_new.cpu().pin_memory(), v_new.cpu().pin_memory(), q.cpu().pin_memory()
+        hout = torch.empty_like(out, device="cpu").pin_memory()
+
+        def e2e_step(ev):
+            k_new.copy_(hkn, non_blocking=True)
+            v_new.copy_(hvn, non_blocking=True)
+            q.copy_(hq, non_blocking=True)
+            sq.sq_compress_kv(rk, rv, k_new, v_new, B, H, d, 1, posT, kc, vc, flags)
+            sq.sq_attn_decode(rk, rv, kc, vc, lens, B, HQ, H, d, max_ctx, q, 0.0, out, None, aws, flags)
+            hout.copy_(out, non_blocking=True)
+
+        t_e2e, _ = _time_loop(e2e_step, args.steps, args.warmup, world, dev, 1)
+        res["e2e"] = {"value": B * world / t_e2e, "unit": "tokens/s",
+                      "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hkn, hvn, hq)),
+                      "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+    return res
+
+
+def _roofline(kernel, ncu_name, nbytes, ms, tokens, peak, peak_kind):
+    achieved = nbytes / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+            "unit": "GB/s", "frac": achieved / peak, "traffic": profiled_traffic(ncu_name, tokens),
+            "bytes_per_launch": nbytes, "launch_ms": ms}
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+
+    from compressed_attention_head_b200 import sq
+
+    dev = f"cuda:{local_rank}"
+    torch.cuda.set_device(local_rank)
+    sq.sq_init()
+    peak, peak_kind = _peaks()
+    headline = args.config == "headline"
+    dec_name = HEADLINE_DECODE if headline else args.config
+    cfg = workload_cfg(dec_name, args.layers, args.bits, not args.no_qjl)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    if cfg["mode"] == "decode":
+        main = measure_decode(cfg, args, world, dev)
+    else:
+        main = measure_prefill(cfg, args, world, dev)
+    comp = None
+    if headline:
+        ccfg = workload_cfg(HEADLINE_COMPRESS, None, None, True)
+        comp = measure_prefill(ccfg, args, world, dev)
+    clk = clocks.stop()
+    flag_val = int(main["flags"].item()) | (int(comp["flags"].item()) if comp else 0)
+    value = main["tokens"] * world / main["step_s"]
+    B, T = cfg["batch"], cfg["ctx"]
+    att = _roofline("sq_attn_decode (prepare + partials + combine)", "k_attn_partial_tc", main["attn_bytes"],
+                    main["att_ms"], B * cfg["layers"] * cfg["n_kv"] * (T + 1), peak, peak_kind)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1e3 * per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": 1e3 * main["step_s"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16",
-        "dtype_detail": "fp16 tensor-core rotation and attention with f32 accumulation; f64 for the key signal "
-                        "coordinates and for exact recomputation of codes near a threshold", "data": "synthetic",
+        "dtype_detail": "fp16 tensor-core contractions with f32 accumulation (attention scores and PV, the "
+                        "compress rotation); f64 for the key signal coordinates and exact recomputation of codes "
+                        "near a threshold", "data": "synthetic",
         "config": workload_config(cfg, world),
-        "roofline": {"bound": "hbm", "kernel": dom["kernel"], "achieved": achieved, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": profiled_traffic(dom["ncu_name"], dom["tokens"]),
-                     "bytes_per_launch": dom["bytes"], "launch_ms": dom["ms"]},
-        "cpu_baseline": cpu, "e2e": e2e,
-        # per step: prompt compress K and V (tensor-core kernel + the pass for heads with
-        # more than 16 QJL dimensions, each), two appends, prepare + partial + combine
-        "gpu_launches": args.steps * ((4 if prefill else 0) + 2 + 3),
-        "clocks": clk, "breakdown": breakdown,
-        "calibration": {"ms": calib_ms, "heads": 2 * H, "tokens_per_head": ncal, "status_nonzero": n_bad},
-        "device_flags": flag_val,
     }
-    print(json.dumps(line), flush=True)
+    if cfg["mode"] == "decode":
+        line["roofline"] = att
+        line["config"]["cache"] = (f"packed records of layer 0's {cfg['n_kv']} KV heads for {main['base_rows']} "
+                                   f"batch rows, compressed from synthetic draws and repeated over the "
+                                   f"{cfg['layers']} layers and {B} rows ({main['cache_bytes'] / 1e9:.1f} GB "
+                                   f"read per step)")
+    else:
+        line["roofline"] = _roofline("k_compress_tc (prompt compress; mean of the K and V launches)",
+                                     "k_compress_tc", main["comp_bytes"], main["comp_ms"],
+                                     B * cfg["layers"] * cfg["n_kv"] * T, peak, peak_kind)
+        line["roofline_attention"] = att
+    if comp is not None:
+        cc = comp["cfg"]
+        ntok = cc["batch"] * cc["layers"] * cc["n_kv"] * cc["ctx"]
+        line["roofline_compress"] = _roofline("k_compress_tc (prompt compress; mean of the K and V launches)",
+                                              "k_compress_tc", comp["comp_bytes"], comp["comp_ms"], ntok, peak,
+                                              peak_kind)
+        line["compress"] = {
+            "workload": workload_config(cc, world)["workload"],
+            "compress_GBps": (comp["comp_k"] + comp["comp_v"]) / ((comp["ck_ms"] + comp["cv_ms"]) / 1e3) / 1e9,
+            "compress_tokens_per_s": cc["batch"] * cc["ctx"] * world / ((comp["ck_ms"] + comp["cv_ms"]) / 1e3),
+            "compress_k_ms": comp["ck_ms"], "compress_v_ms": comp["cv_ms"],
+            "bytes_per_token_head": {"k": comp["comp_k"] / ntok, "v": comp["comp_v"] / ntok},
+            "step_ms": 1e3 * comp["step_s"], "step_tokens_per_s": comp["tokens"] * world / comp["step_s"],
+            "attention_ms": comp["att_ms"], "append_ms": comp["app_ms"],
+            "e2e": comp.get("e2e"), "gpu_launches_per_step": comp["launches"],
+        }
+    line["cpu_baseline"] = None
+    if world == 1 and not args.no_cpu:
+        if cfg["mode"] == "decode":
+            t_o, secs, desc = oracle_decode_sample(cfg, pairs=args.cpu_pairs)
+        else:
+            t_o, secs, desc = oracle_prefill_sample(cfg, tokens=args.cpu_tokens, ctx=args.cpu_ctx)
+        line["cpu_baseline"] = {"value": main["tokens"] / t_o, "unit": "tokens/s", "cores": cpu_threads(),
+                                "kind": "oracle", "sample": desc}
+    line["e2e"] = main.get("e2e")
+    line["gpu_launches"] = args.steps * main["launches"]
+    line["clocks"] = clk
+    bd = {"step_ms_eager": 1e3 * main["eager_s"],
+          "step_ms_graph": None if main["graph_s"] is None else 1e3 * main["graph_s"],
+          "append_ms": main["app_ms"], "attention_ms": main["att_ms"],
+          "attention_GBps": att["achieved"], "attention_frac_of_hbm": att["frac"],
+          "attention_bytes_per_token_head": main["rec_k"] + main["rec_v"],
+          "decode_tokens_per_s": B * world / ((main["app_ms"] + main["att_ms"]) / 1e3)}
+    if cfg["mode"] == "prefill":
+        bd.update({"compress_k_ms": main["ck_ms"], "compress_v_ms": main["cv_ms"],
+                   "compress_GBps": (main["comp_k"] + main["comp_v"]) / ((main["ck_ms"] + main["cv_ms"]) / 1e3)
+                   / 1e9})
+    line["breakdown"] = bd
+    line["calibration"] = {"ms": main["calib_ms"], "heads": main["calib_heads"],
+                           "tokens_per_head": cfg["n_cal"], "status_nonzero": main["n_bad"]}
+    line["device_flags"] = flag_val
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def main():
@@ -564,13 +729,21 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="sq", choices=["sq", "reference"])
-    ap.add_argument("--config", default="llama8b")
+    ap.add_argument("--config", default="headline",
+                    help="headline (Gemma-shaped decode + Llama-shaped prompt compress) or a workload name")
+    ap.add_argument("--bits", type=float, default=None, help="bits per coordinate for K and V (Gemma sweep)")
+    ap.add_argument("--no-qjl", action="store_true")
+    ap.add_argument("--base-rows", type=int, default=2, help="distinct batch rows of a decode cache")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time the eager launches only")
     ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling captures only)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=32768)
     ap.add_argument("--cpu-ctx", type=int, default=8192)
+    ap.add_argument("--cpu-pairs", type=int, default=96)
+    ap.add_argument("--ref-tokens", type=int, default=8192)
+    ap.add_argument("--ref-ctx", type=int, default=8192)
+    ap.add_argument("--ref-pairs", type=int, default=4)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -151,13 +151,30 @@ CacheArgs cache_args(const sq_cache* c) { return CacheArgs{c->codes, c->norm, c-
 // Splits of the context per (batch, KV head). Each block of the partial
 // kernel takes a span of whole 128-token tiles (32 tokens per warp) and pays a
 // fixed setup (tables, query fragments, final merge) of about half a warp tile.
-// With `slots` blocks resident at once (148 SMs of a B200 times the blocks per
-// SM the kernel is built for), equal blocks run in ceil(blocks / slots) waves,
+// With `slots` blocks resident at once (the device's SMs, 148 on a B200, times
+// the blocks per SM the kernel is built for), equal blocks run in ceil(blocks / slots) waves,
 // so the cost of a split count S is waves(S) x (1/2 + tiles per warp); the
 // cheapest S wins (the smaller on ties, which also keeps the combine short).
+// SMs of the current device (its multiprocessor count; 148 on a B200, also the
+// answer when no device can be queried, e.g. for a workspace query on a host
+// without a GPU).
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (g_ready[dev]) return g_sms[dev];
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return sms;
+}
+
 int attn_splits(int batch, int n_kv, int d, int64_t max_ctx) {
   const int64_t units = (int64_t)batch * n_kv;
-  const int64_t slots = 148 * (int64_t)fa::min_blocks(d);
+  const int64_t slots = (int64_t)device_sms() * fa::min_blocks(d);
   const int64_t ctx = max_ctx > 0 ? max_ctx : 1;
   int best = 1;
   int64_t best_cost = INT64_MAX;
@@ -625,11 +642,11 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
 // Decode attention without a caller-provided workspace.
 //
 // Some callers cannot allocate device memory at the point where they run decode
-// attention: code running under a CUDA-graph capture or inside a serving loop
-// whose memory is reserved up front, plug-ins that have no handle to the
-// application's allocator, and runtimes that forbid allocation after start-up.
-// They use this entry point: its scratch is a fixed array in the library's own
-// device memory (every GPU that loads libsq keeps it until the process exits).
+// attention: a serving loop whose device memory is reserved once at start-up
+// and may not grow, plug-ins that have no handle to the host application's
+// allocator, and runtimes that forbid allocation after initialisation. They use
+// this entry point: its scratch is a fixed array in the library's own device
+// memory (every GPU that loads libsq keeps it until the process exits).
 // ---------------------------------------------------------------------------
 constexpr size_t kStaticScratchBytes = SQ_ATTN_NOALLOC_MAX_BYTES;
 static __device__ __align__(256) unsigned char g_attn_scratch[kStaticScratchBytes];

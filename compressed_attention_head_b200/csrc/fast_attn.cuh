@@ -311,8 +311,7 @@ __global__ void __launch_bounds__(NTH, min_blocks(D)) k_attn_partial_tc(const ui
   float* acc_out = uq + (size_t)s.batch * s.n_q * D;
   float* ml_out = acc_out + (size_t)s.batch * s.n_q * s.splits * D;
   const bool ok = record_ok(hk, D) && record_ok(hv, D) && hk->words == kc.words && hv->words == vc.words &&
-                  (hk->m == 0 || kc.rnorm != nullptr) && hk->m <= 16 && kc.words <= GE::MAXW &&
-                  vc.words <= GE::MAXW;
+                  (hk->m == 0 || kc.rnorm != nullptr) && kc.words <= GE::MAXW && vc.words <= GE::MAXW;
   int64_t L = seq_lens[b];
   if (L < 0 || L > s.max_ctx || L > kc.cap) {
     if (tid == 0 && split == 0 && g == 0 && flags) atomicOr(flags, SQ_FLAG_SEQLEN);
@@ -327,6 +326,7 @@ __global__ void __launch_bounds__(NTH, min_blocks(D)) k_attn_partial_tc(const ui
   const int64_t t_hi = min(L, t_lo + s.chunk);
   const int ntile = t_hi > t_lo ? (int)((t_hi - t_lo + TT - 1) / TT) : 0;
   const int m = ok ? hk->m : 0;
+  const int nqs = (m + 15) >> 4;      // 16-column blocks of QJL signs (one in the common case m <= 16)
   const int wk = kc.words, wv = vc.words, kcb = ok ? hk->code_bits : 0;
 
   // ---- block tables
@@ -519,16 +519,20 @@ __global__ void __launch_bounds__(NTH, min_blocks(D)) k_attn_partial_tc(const ui
       *(uint4*)(qt + swz32(lane, 8)) = make_uint4(qh[4], qh[5], qh[6], qh[7]);
     }
     __syncwarp();
-    if (nxt < ntile) {       // the key records of this tile are consumed
+    if (nqs <= 1 && nxt < ntile) {       // the key records of this tile are consumed
       stage_rec(recK, kcodes, wk, nxt);
       cp_async_commit();
     }
 
     // ---- scores: rows = tokens, columns = heads
     float sv[2][4];
+    float acc2[2][4], qa2[2][4];
 #pragma unroll
     for (int mb = 0; mb < 2; ++mb) {
-      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f}, qa[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      float* acc = acc2[mb];
+      float* qa = qa2[mb];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] = qa[e] = 0.0f;
       const int ar = 16 * mb + (lane & 15), ac = (lane >> 4) * 8;
 #pragma unroll
       for (int ks = 0; ks < NCH; ++ks) {
@@ -547,6 +551,47 @@ __global__ void __launch_bounds__(NTH, min_blocks(D)) k_attn_partial_tc(const ui
         ldsm_x4(smem_addr(qt + swz32(ar, ac)), aq);
         mma16816(qa, aq, uB[0], uB[1]);
       }
+    }
+    if (nqs > 1) {
+      // more than 16 QJL dimensions: the further 16-column blocks of signs, one
+      // at a time through the same tile, with their weights u read from the
+      // workspace; the key records are restaged only after the last block
+      const float* urow = uq + (qbase + hn) * D;
+      for (int qs = 1; qs < nqs; ++qs) {
+        __syncwarp();
+        uint32_t pc = 0u;
+        pieces<1>(recK, kcb + 16 * qs, lane, &pc);
+        uint32_t qh[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) qh[k] = tQS[(pc >> (2 * k)) & 3u];
+        *(uint4*)(qt + swz32(lane, 0)) = make_uint4(qh[0], qh[1], qh[2], qh[3]);
+        *(uint4*)(qt + swz32(lane, 8)) = make_uint4(qh[4], qh[5], qh[6], qh[7]);
+        __syncwarp();
+        uint32_t ub[2];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int j = 16 * qs + hf * 8 + 2 * tq;
+          const float u0 = (hn < G && j < m) ? urow[j] * wsc : 0.0f;
+          const float u1 = (hn < G && j + 1 < m) ? urow[j + 1] * wsc : 0.0f;
+          ub[hf] = pack_h2(u0, u1);
+        }
+#pragma unroll
+        for (int mb = 0; mb < 2; ++mb) {
+          uint32_t aq[4];
+          ldsm_x4(smem_addr(qt + swz32(16 * mb + (lane & 15), (lane >> 4) * 8)), aq);
+          mma16816(qa2[mb], aq, ub[0], ub[1]);
+        }
+      }
+      __syncwarp();
+      if (nxt < ntile) {
+        stage_rec(recK, kcodes, wk, nxt);
+        cp_async_commit();
+      }
+    }
+#pragma unroll
+    for (int mb = 0; mb < 2; ++mb) {
+      const float* acc = acc2[mb];
+      const float* qa = qa2[mb];
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         const int tl = 16 * mb + hn + 8 * hr;

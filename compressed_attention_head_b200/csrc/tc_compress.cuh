@@ -95,7 +95,7 @@ constexpr int OFF_LV64 = OFF_TH64 + ((kThreshTotal * 8 + 15) & ~15);   // double
 constexpr int OFF_Q = OFF_LV64 + ((kLevelsTotal * 8 + 15) & ~15);      // float4 [kQEntries]
 constexpr int OFF_CELL = OFF_Q + kQEntries * 16;                       // u8 [kCellBytes]
 constexpr int OFF_BAR = OFF_CELL + kCellBytes;
-constexpr int N_BARS = 4 * NGRP + 2;
+constexpr int N_BARS = 4 * NGRP + 3;
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;                         // u32 [16]
 constexpr int OFF_R = OFF_MISC + 64;                                   // float [NGRP][32]: radius per width, per chunk
 constexpr int OFF_CD = OFF_R + NGRP * 128;                             // u32 [NGRP][8]: chunk classes
@@ -555,6 +555,7 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
   uint64_t* tempty = bars + 3 * NGRP;       // [NGRP] accumulator drained
   uint64_t* bfull = bars + 4 * NGRP;        // B operand landed
   uint64_t* bempty = bfull + 1;             // B operand no longer read
+  uint64_t* drain = bfull + 2;              // every MMA this CTA issued has completed (before the free)
   uint32_t* misc = (uint32_t*)(sm + OFF_MISC);   // [0] tmem base, [1] abort
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -571,6 +572,7 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
     }
     sm100::mbar_init(bfull, 1);
     sm100::mbar_init(bempty, 1);
+    sm100::mbar_init(drain, 1);
     misc[1] = 0u;
     sm100::fence_mbar_init();
   }
@@ -889,6 +891,17 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
       sm100::mbar_wait(&full[it % NGRP], (it / NGRP) & 1u, nullptr);
     }
     if (b_issued > 0) sm100::mbar_wait(bfull, (b_issued - 1) & 1u, nullptr);
+  }
+  // Every MMA this CTA issued has completed before its tensor memory is freed
+  // (on the normal path they have: the epilogue waited for each accumulator;
+  // after a timeout some may still run). Bounded like every other wait; the
+  // memory is freed either way, so that no later CTA on this SM waits on it.
+  if (warp == WARP_MMA) {
+    if (lane == 0) {
+      sm100::mma_commit(drain);
+      if (!sm100::mbar_wait(drain, 0u, err)) *abort_flag = 1;
+    }
+    __syncwarp();
   }
   sm100::tc_fence_before();
   __syncthreads();

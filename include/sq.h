@@ -244,7 +244,10 @@ sq_status sq_calibrate(const sq_calib_params* p, const void* x, sq_dtype dtype, 
 /*
  * Imports n_heads records whose canonical part was written elsewhere (saved
  * records, or another implementation): checks each header (magic, version,
- * d, bit counts, offsets) and builds the library's derived part.
+ * d, bit counts, offsets) and builds the library's derived part. The record
+ * holds what the README's "Overview" calls the one-time calibration (the
+ * calibrated eigenbasis, d_eff and kappa of calibration.py, the water-filled
+ * widths); importing lets a calibration computed once be reused.
  *  calib     device, n_heads records of sq_calib_bytes(d) bytes.
  *  d_status  device int[n_heads] (may be NULL): SQ_OK or SQ_ERR_RECORD.
  */
@@ -313,7 +316,11 @@ sq_status sq_compress_kv_host(const void* calib_k, const void* calib_v, const vo
                               void* d_staging, size_t staging_bytes, uint32_t* d_flags, sq_stream stream);
 
 /*
- * Reconstructs vectors from a packed cache: x_hat = norm * V (sigma * level(code)),
+ * Reconstructs vectors from a packed cache (the inverse of the README's
+ * "Repository Structure" steps: spectral_rotation.py rotated into the
+ * eigenbasis, nonuniform_quantization.py quantized, selective_qjl.py added the
+ * sign correction on the signal dims; here they are undone):
+ * x_hat = norm * V (sigma * level(code)),
  * plus, when apply_qjl and the records carry QJL bits,
  * norm * V[:, 0:m] (sqrt(pi/2) / m * rnorm * S^T s), s_j = 2 bit_j - 1.
  *  calib  device, cache->n_heads records of head_dim d.
@@ -359,10 +366,10 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
 
 /*
  * sq_attn_decode without a workspace argument, for callers that cannot
- * allocate device memory where they run decode attention (inside a captured
- * CUDA graph or a serving loop whose memory is reserved up front, plug-ins
- * with no access to the application's allocator, runtimes that forbid
- * allocation after start-up). The pages have no counterpart: this is a
+ * allocate device memory where they run decode attention: a serving loop whose
+ * device memory is reserved once at start-up and may not grow, plug-ins with
+ * no access to the host application's allocator, runtimes that forbid
+ * allocation after initialisation. The pages have no counterpart: this is a
  * deployment convenience of this library.
  *
  * Arguments and results are those of sq_attn_decode minus ws / ws_bytes. The
@@ -374,12 +381,12 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
  * The first call on a device looks up the array's device address on that
  * device (cudaGetSymbolAddress) and caches it; make that first call before
  * any stream capture. Every call on a device shares the one array, so calls
- * whose executions overlap on the GPU (different streams, or concurrent
- * graphs) race and corrupt each other's results; serialize them. Nothing in
+ * whose executions overlap on the GPU (on different streams, for instance)
+ * race and corrupt each other's results; serialize them. Nothing in
  * the array needs to start at zero: each call writes every scratch entry it
  * later reads.
  */
-#define SQ_ATTN_NOALLOC_MAX_BYTES (8u << 20)
+#define SQ_ATTN_NOALLOC_MAX_BYTES 0x800000u /* 8 MiB */
 sq_status sq_attn_decode_noalloc(const void* calib_k, const void* calib_v, const sq_cache* kc,
                                  const sq_cache* vc, const int32_t* d_seq_lens, int batch, int n_q_heads,
                                  int n_kv_heads, int d, int64_t max_ctx, const void* q, sq_dtype q_dtype,

@@ -10,7 +10,10 @@ Tolerances (stated once, used by every parity test):
 * rho: relative 1e-5 on non-exempt tokens (float64 residual stored as float32);
 * reconstruction: relative L2 per vector <= 1e-4 (vectors without exempt codes);
 * attention scores: relative L2 per (batch, query head) row <= 1e-3;
-* attention outputs: relative L2 per (batch, query head) <= 2e-3.
+* attention outputs: relative L2 per (batch, query head) <= 2e-3;
+* exempt fields (codes plus QJL bits) of one comparison: at most 1e-3 of the
+  fields compared (rounded down), so that an over-permissive exemption rule
+  cannot hide a mismatch.
 """
 
 from __future__ import annotations
@@ -28,6 +31,7 @@ TOL_RHO = 1e-5
 TOL_RECON = 1e-4
 TOL_SCORES = 1e-3
 TOL_OUT = 2e-3
+MAX_EXEMPT_FRACTION = 1e-3
 
 
 def records_to_device(cals, device="cuda") -> torch.Tensor:
@@ -86,6 +90,9 @@ def compare_compressed(gpu_words: np.ndarray, gpu_norm: np.ndarray, gpu_rnorm, x
     ref_n = out["norm64"]
     assert np.all(np.abs(gpu_norm - ref_n) <= TOL_NORM * np.maximum(ref_n, 1e-30)), "norm mismatch"
     code_ex, q_ex, rho_ex = ocodec.exemptions(out, cal)
+    n_fields = code_ex.shape[0] * (int(np.count_nonzero(cal.bits)) + cal.m)
+    n_ex = int(code_ex.sum()) + int(q_ex.sum())
+    assert n_ex <= int(MAX_EXEMPT_FRACTION * n_fields), f"{n_ex} exempt fields of {n_fields}"
     if cal.m > 0:
         ok = ~rho_ex
         ref_r = out["rho64"][ok]

@@ -160,6 +160,6 @@ def test_header_constants_match_the_binding():
             assert getattr(sq, name) == value, name
             mirrored += 1
     for name in ("SQ_FLAG_CAPACITY", "SQ_FLAG_RECORD", "SQ_FLAG_SEQLEN", "SQ_FLAG_TIMEOUT", "SQ_ERR_WORKSPACE",
-                 "SQ_F16"):
+                 "SQ_F16", "SQ_ATTN_NOALLOC_MAX_BYTES"):
         assert name in defines or name in enums, name
     assert mirrored >= 10

@@ -14,7 +14,7 @@ import torch
 
 from gpu_helpers import TOL_OUT, TOL_SCORES, calibrate_oracle, records_to_device, rel_l2_rows
 from oracle import attention as oattn
-from synthetic import make_workload
+from synthetic import CONFIGS, make_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -25,14 +25,15 @@ from compressed_attention_head_b200 import sq  # noqa: E402
 
 
 def _run(name, batch, ctx, seq_lens, heads=None, bits_k=None, bits_v=None, qjl=True, out_dtype=torch.float32,
-         cap=None):
+         cap=None, d_eff_override=0):
     w = make_workload(name, batch=batch, tokens=ctx)
     cfg = w.cfg
     nkv = heads or cfg["n_kv"]
     group = cfg["n_q"] // cfg["n_kv"]
     nq = nkv * group
     d = cfg["d"]
-    ck = calibrate_oracle(w.k_cal[:nkv], cfg["bits_k"] if bits_k is None else bits_k, True, qjl=qjl)
+    ck = calibrate_oracle(w.k_cal[:nkv], cfg["bits_k"] if bits_k is None else bits_k, True, qjl=qjl,
+                          d_eff_override=d_eff_override)
     cv = calibrate_oracle(w.v_cal[:nkv], cfg["bits_v"] if bits_v is None else bits_v, False)
     rk, rv = records_to_device(ck), records_to_device(cv)
     cap = cap or ((ctx + 15) // 16) * 16
@@ -136,3 +137,95 @@ def test_full_size_decode_sampled_rows():
     out, scores, ref_out, ref_scores, flags = _run("qwen14b", 4, 8192, [8192, 8191, 4097, 8192], heads=2)
     assert flags == 0
     _assert_close(out, scores, ref_out, ref_scores, [8192, 8191, 4097, 8192])
+
+
+def test_attention_more_than_sixteen_qjl_dimensions():
+    """Keys with m = 24 QJL sign dimensions (d_eff_override) through the default
+    (tensor-core) path: the signs take two 16-column blocks."""
+    out, scores, ref_out, ref_scores, flags = _run("llama8b", 2, 300, [300, 257], heads=2, d_eff_override=24)
+    assert flags == 0
+    _assert_close(out, scores, ref_out, ref_scores, [300, 257])
+
+
+def test_attention_head_dim_64():
+    """head_dim 64 (a Llama-shaped head at half the width): G = 4, ragged rows."""
+    cfg = dict(CONFIGS["llama8b"], d=64)
+    out, scores, ref_out, ref_scores, flags = _run(cfg, 2, 500, [500, 77], heads=2)
+    assert flags == 0
+    _assert_close(out, scores, ref_out, ref_scores, [500, 77])
+
+
+def _bench_shape_sampled(name, n_layers, batch, ctx, rows, distinct_heads=2, distinct_rows=None):
+    """Decode attention in the launch configuration of the benchmark step (all
+    layers folded into the KV-head index, batch x context of the workload,
+    max_ctx = context + 1 for the appended token): the packed caches of
+    ``distinct_heads`` KV heads and ``distinct_rows`` batch rows are compressed
+    once and repeated over the layers' heads and the batch, and sampled (batch
+    row, query head) rows are checked against the oracle."""
+    cfg = CONFIGS[name]
+    d, g = cfg["d"], cfg["n_q"] // cfg["n_kv"]
+    # only the distinct heads are drawn (on the device: millions of vectors)
+    nb = distinct_rows or batch
+    w = make_workload(dict(cfg, n_kv=distinct_heads, n_q=distinct_heads * g), batch=nb, tokens=ctx,
+                      device="cuda")
+    ck = calibrate_oracle(w.k_cal[:distinct_heads], cfg["bits_k"], True)
+    cv = calibrate_oracle(w.v_cal[:distinct_heads], cfg["bits_v"], False)
+    nkv = n_layers * cfg["n_kv"]
+    nq = nkv * g
+    rk1, rv1 = records_to_device(ck), records_to_device(cv)
+    size = sq.sq_calib_bytes(d)
+    rep = nkv // distinct_heads
+    rk = rk1.view(distinct_heads, size).repeat(rep, 1).reshape(-1).contiguous()
+    rv = rv1.view(distinct_heads, size).repeat(rep, 1).reshape(-1).contiguous()
+    cap = ((ctx + 1 + 31) // 32) * 32
+    k1 = sq.alloc_cache(nb, distinct_heads, cap, ck[0].words, True)
+    v1 = sq.alloc_cache(nb, distinct_heads, cap, cv[0].words, False)
+    sq.sq_compress_kv(rk1, rv1, w.k.contiguous(), w.v.contiguous(), nb, distinct_heads, d, ctx, None, k1, v1)
+    del w.k, w.v
+    kc = sq.alloc_cache(batch, nkv, cap, ck[0].words, True)
+    vc = sq.alloc_cache(batch, nkv, cap, cv[0].words, False)
+    rb = batch // nb
+    for big, small in ((kc, k1), (vc, v1)):
+        big.codes.copy_(small.codes.repeat(rb, rep, 1, 1))
+        big.norm.copy_(small.norm.repeat(rb, rep, 1))
+        if big.rnorm is not None:
+            big.rnorm.copy_(small.rnorm.repeat(rb, rep, 1))
+    q = w.q.repeat(rb, rep, 1).contiguous()
+    lens_l = [ctx - (7 * b) % 301 for b in range(batch)]
+    lens = torch.tensor(lens_l, dtype=torch.int32, device="cuda")
+    max_ctx = ctx + 1
+    ws = torch.empty(sq.sq_attn_workspace(batch, nq, nkv, d, max_ctx), dtype=torch.uint8, device="cuda")
+    out = torch.empty(batch, nq, d, device="cuda")
+    scores = torch.full((batch, nq, max_ctx), float("nan"), device="cuda")
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sq.sq_attn_decode(rk, rv, kc, vc, lens, batch, nq, nkv, d, max_ctx, q, 0.0, out, scores, ws, flags)
+    torch.cuda.synchronize()
+    assert flags.item() == 0
+    kw, vw = k1.words_u32(), v1.words_u32()
+    kn, kr, vn = k1.norm.cpu().numpy(), k1.rnorm.cpu().numpy(), v1.norm.cpu().numpy()
+    scale = 1.0 / math.sqrt(d)
+    for (b, h) in rows:
+        gh = h // g
+        src, sb = gh % distinct_heads, b % nb
+        n = lens_l[b]
+        ro, rs = oattn.attend_one(q[b, h].double().cpu().numpy(), kw[sb, src, :n], kn[sb, src, :n],
+                                  kr[sb, src, :n], vw[sb, src, :n], vn[sb, src, :n], ck[src], cv[src], scale)
+        got_s = scores[b, h, :n].cpu().numpy()
+        got_o = out[b, h].cpu().numpy()
+        assert rel_l2_rows(got_s[None], rs[None])[0] <= TOL_SCORES, (b, h)
+        assert rel_l2_rows(got_o[None], ro[None])[0] <= TOL_OUT, (b, h)
+    return sq.sq_attn_workspace(batch, nq, nkv, d, max_ctx)
+
+
+def test_decode_qwen1_5b_long_bench_shape_sampled():
+    """Qwen2.5-1.5B-shaped decode as benchmarked: batch 16 at context 32768, 28
+    layers x 2 KV heads folded (56 KV / 336 query heads, head_dim 128)."""
+    _bench_shape_sampled("qwen1_5b_long", 28, 16, 32768,
+                         rows=[(0, 0), (3, 7), (9, 200), (15, 335), (12, 101)])
+
+
+def test_decode_gemma_bench_shape_sampled():
+    """Gemma-2-9B-shaped decode as benchmarked: batch 64 at context 4096, 42
+    layers x 8 KV heads folded (336 KV / 672 query heads, head_dim 256, bf16)."""
+    _bench_shape_sampled("gemma9b_sweep", 42, 64, 4096,
+                         rows=[(0, 0), (63, 671), (17, 300), (40, 5), (33, 450)], distinct_rows=2)

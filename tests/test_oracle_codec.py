@@ -169,3 +169,72 @@ def test_qjl_residual_lives_on_signal_dims():
     b = codec.decompress(out["words"], out["norm"], out["rnorm"], c, apply_qjl=False)
     diff_rot = (a - b) @ c.V
     assert np.max(np.abs(diff_rot[:, c.m:])) < 1e-10 * np.max(np.abs(diff_rot))
+
+
+def _place(proj_target, S, r_other, j_free, iters=60):
+    """A residual r with (S r)_j equal to proj_target(rho) for the free coordinate
+    j_free, the other coordinate fixed: a small fixed-point iteration, since the
+    band itself scales with rho = ||r||."""
+    r = np.zeros(2)
+    r[1 - j_free] = r_other
+    for _ in range(iters):
+        rho = float(np.linalg.norm(r))
+        target = proj_target(rho)
+        # solve row j of S r = target for r[j_free] (the row that carries it)
+        row = 0 if j_free == 0 else 1
+        r[j_free] = (target - S[row, 1 - j_free] * r[1 - j_free]) / S[row, j_free]
+    return r
+
+
+def test_qjl_bit_exemption_band():
+    """A QJL bit is exempt exactly when |(S r)_j| <= 1e-5 * ||row j of S|| * rho,
+    and every bit and rho of a token whose signal-dim code is exempt are exempt.
+
+    S = [[3, 0], [4, 1]] has row norms 3 and sqrt(17) but column norms 5 and 1,
+    so a rule built on column norms decides cases 2 and 3 the other way; rho is
+    far from 1 in every case, so a rule without rho fails cases 1 and 3; the
+    exempt bit is 0 in cases 1 and 4 and bit 1 in case 3, so swapped indices fail.
+    """
+    S = np.array([[3.0, 0.0], [4.0, 1.0]])
+    head = _head([0, 0, 3], m=2, S=S, normalize=False)
+    band = lambda j, rho: 1e-5 * np.linalg.norm(S[j]) * rho       # noqa: E731
+    # (r, expected q_ex): bit 0 is driven by r0 alone (row 0 of S), bit 1 by 4 r0 + r1
+    cases = [
+        (_place(lambda rho: 0.5 * band(0, rho), S, -7.0, 0), [True, False]),     # 1: bit 0 at half the band
+        (_place(lambda rho: 1.5 * band(0, rho), S, -7.0, 0), [False, False]),    # 2: 1.5 bands (column rule: inside)
+        (None, [False, True]),                                                     # 3: bit 1 at 0.9 of its band
+        (_place(lambda rho: 0.99 * band(0, rho), S, 5.0, 0), [True, False]),     # 4: just inside
+        (_place(lambda rho: 1.01 * band(0, rho), S, 5.0, 0), [False, False]),    # 5: just outside
+    ]
+    # case 3: r0 = 2 fixed, r1 chosen so that (S r)_1 = 4 r0 + r1 = 0.9 band(1, rho)
+    r = np.array([2.0, -8.0])
+    for _ in range(60):
+        rho = float(np.linalg.norm(r))
+        r[1] = 0.9 * band(1, rho) - 4.0 * r[0]
+    cases[2] = (r, [False, True])
+    x = np.array([[c[0][0], c[0][1], 0.1] for c in cases])
+    out = codec.compress(x, head)
+    code_ex, q_ex, rho_ex = codec.exemptions(out, head)
+    assert not code_ex.any() and not rho_ex.any()
+    assert q_ex.tolist() == [c[1] for c in cases]
+    # the projections sit where the cases put them (relative to the row band)
+    ratios = np.abs(out["proj"]) / (1e-5 * np.linalg.norm(S, axis=1)[None, :] * out["rho64"][:, None])
+    assert np.allclose([ratios[0, 0], ratios[1, 0], ratios[2, 1], ratios[3, 0], ratios[4, 0]],
+                       [0.5, 1.5, 0.9, 0.99, 1.01], rtol=1e-6)
+    assert np.all(out["rho64"] > 4.9)
+
+
+def test_qjl_bits_of_a_token_with_an_exempt_signal_code():
+    """A signal-dim code on a threshold makes rho and all m QJL bits of that token
+    exempt, whatever the projections; a token without one has none exempt."""
+    S = np.array([[1.0, 2.0], [-3.0, 0.5]])
+    head = _head([2, 0, 1], m=2, S=S, normalize=False)
+    _, t2, _ = cb.lloyd_max(2)
+    x = np.array([[t2[2], 0.7, 0.3],        # coordinate 0 exactly on its threshold
+                  [0.2, 0.7, 0.3]])          # nothing near a threshold or a zero projection
+    out = codec.compress(x, head)
+    code_ex, q_ex, rho_ex = codec.exemptions(out, head)
+    assert code_ex.tolist() == [[True, False, False], [False, False, False]]
+    assert rho_ex.tolist() == [True, False]
+    assert q_ex.tolist() == [[True, True], [False, False]]
+    assert np.min(np.abs(out["proj"][0])) > 1e-2     # exempt through the code, not through the band

@@ -1,8 +1,8 @@
 """The no-allocation decode-attention entry point (collected last on purpose).
 
 Callers that cannot allocate device memory where they run decode attention
-(inside a captured CUDA graph or a serving loop with memory reserved up front,
-plug-ins without the application's allocator) call sq_attn_decode_noalloc,
+(a serving loop whose device memory is reserved once at start-up, plug-ins
+without the host application's allocator) call sq_attn_decode_noalloc,
 whose scratch is a fixed array inside libsq. This checks, through the C ABI,
 that two calls in a row give the same outputs and scores as sq_attn_decode
 with a caller workspace, within the attention tolerances, and that shapes
