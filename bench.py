@@ -570,11 +570,7 @@ def measure_decode(cfg, args, world, dev):
     del w
     rb = B // b0
 
-    def grow(c1, with_rnorm):
-        return sq.PackedCache(c1.codes.repeat(rb, L, 1, 1), c1.norm.repeat(rb, L, 1),
-                              c1.rnorm.repeat(rb, L, 1) if with_rnorm else None, B, H, cap, c1.words)
-
-    kc, vc = grow(k1, qjl), grow(v1, False)
+    kc, vc = k1.tiled(rb, L), v1.tiled(rb, L)
     del k1, v1
     q = nxt.q.repeat(rb, L, 1).contiguous()
     k_new = nxt.k.repeat(rb, L, 1, 1).contiguous()

@@ -23,6 +23,7 @@ __device__ uint8_t c_tccell[560];      // tcc cell tables: positive thresholds b
 #include "codec.cuh"
 #include "fast_attn.cuh"
 #include "tc_compress.cuh"
+#include "tc_decode.cuh"
 
 namespace sq {
 
@@ -35,7 +36,7 @@ namespace {
 std::mutex g_mu;
 bool g_ready[128];
 bool g_force_ref = false;   // route compress to the float64 reference kernel
-bool g_attn_ref = false;    // route attention partials to the SIMT kernel
+int g_attn_path = 0;        // attention partials: 0 tcgen05 kernel (auto), 1 SIMT, 2 mma.sync kernel
 int g_eacc_units = tcc::EACC_DEFAULT_UNITS;   // accumulation bound of the tensor-core compress radius, in 2^-24
 tcc::QuantConst g_kq;       // register thresholds and cell counts of the tensor-core compress
 int g_sms[128];
@@ -81,6 +82,10 @@ bool build_cell_tables(const double* th, float4* q, uint8_t* cell, tcc::QuantCon
   return true;
 }
 
+// Dynamic shared memory the tcgen05 decode kernel may take: 227 KB per block
+// minus its static width-3 table (8 KB).
+constexpr int kTdSmemLimit = 232448 - 8192;
+
 // Uploads the Lloyd-Max tables to the current device once.
 sq_status ensure_init(int* dev_out = nullptr) {
   int dev = 0;
@@ -124,6 +129,15 @@ sq_status ensure_init(int* dev_out = nullptr) {
   cudaFuncSetAttribute(fa::k_attn_partial_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::smem_bytes<64>());
   cudaFuncSetAttribute(fa::k_attn_partial_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::smem_bytes<128>());
   cudaFuncSetAttribute(fa::k_attn_partial_tc<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::smem_bytes<256>());
+  {
+    const int dyn = kTdSmemLimit;
+#define SQ_TD_ATTR(DD, MG) \
+  cudaFuncSetAttribute(td::k_decode_tc<DD, MG>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn)
+    SQ_TD_ATTR(64, 2); SQ_TD_ATTR(64, 4); SQ_TD_ATTR(64, 8); SQ_TD_ATTR(64, 16);
+    SQ_TD_ATTR(128, 2); SQ_TD_ATTR(128, 4); SQ_TD_ATTR(128, 8); SQ_TD_ATTR(128, 16);
+    SQ_TD_ATTR(256, 2); SQ_TD_ATTR(256, 4); SQ_TD_ATTR(256, 8); SQ_TD_ATTR(256, 16);
+#undef SQ_TD_ATTR
+  }
   if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
   int sms = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -142,8 +156,8 @@ int budget_bits(double avg_bits, int d) {
 
 bool cache_ok(const sq_cache* c, int batch, int n_heads) {
   return c && c->codes && c->norm && aligned16(c->codes) && aligned16(c->norm) &&
-         (!c->rnorm || aligned16(c->rnorm)) && c->batch == batch && c->n_heads == n_heads && c->cap >= 16 &&
-         c->cap % 16 == 0 && c->words >= 1 && c->words <= kMaxWords;
+         (!c->rnorm || aligned16(c->rnorm)) && c->batch == batch && c->n_heads == n_heads &&
+         c->cap >= kBlockTok && c->cap % kBlockTok == 0 && c->words >= 1 && c->words <= kMaxWords;
 }
 
 CacheArgs cache_args(const sq_cache* c) { return CacheArgs{c->codes, c->norm, c->rnorm, c->cap, c->words}; }
@@ -170,6 +184,47 @@ int device_sms() {
     return 148;
   }
   return sms;
+}
+
+// tcgen05 decode kernel: record buffers per group that fit (2, else 1), or 0
+// when even one does not (records wider than the kernel's shared memory holds).
+int td_nrec(int d, int wk, int wv) {
+  for (int nrec = 2; nrec >= 1; --nrec) {
+    const size_t need = d == 64 ? td::smem_bytes<64>(wk, wv, nrec)
+                                : (d == 128 ? td::smem_bytes<128>(wk, wv, nrec) : td::smem_bytes<256>(wk, wv, nrec));
+    if (need <= (size_t)kTdSmemLimit) return nrec;
+  }
+  return 0;
+}
+int td_groups(int d) { return d == 64 ? td::Cfg<64>::NG : (d == 128 ? td::Cfg<128>::NG : td::Cfg<256>::NG); }
+
+// Splits of the context for the tcgen05 kernel: one block per SM, whose NG
+// warp groups take its 128-token tiles in turn. With equal blocks in
+// ceil(blocks / SMs) waves, the cost of S splits is waves(S) x (1 + tiles per
+// group), the 1 standing for the block's setup (tables, query operand, merge);
+// the cheapest S wins (the smaller on ties).
+int attn_splits_td(int batch, int n_kv, int d, int64_t max_ctx) {
+  const int64_t units = (int64_t)batch * n_kv;
+  const int64_t slots = (int64_t)device_sms();
+  const int64_t ctx = max_ctx > 0 ? max_ctx : 1;
+  const int64_t ng = td_groups(d);
+  int best = 1;
+  int64_t best_cost = INT64_MAX;
+  for (int64_t S = 1; S <= 256; ++S) {
+    const int64_t per = (ctx + S - 1) / S;
+    const int64_t chunk = ((per + kAttnTile - 1) / kAttnTile) * kAttnTile;
+    const int64_t used = (ctx + chunk - 1) / chunk;
+    if (used != S) continue;
+    const int64_t waves = (units * S + slots - 1) / slots;
+    const int64_t tiles = chunk / kAttnTile;
+    const int64_t cost = waves * (1 + (tiles + ng - 1) / ng);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = (int)S;
+    }
+    if (chunk == kAttnTile) break;
+  }
+  return best;
 }
 
 int attn_splits(int batch, int n_kv, int d, int64_t max_ctx) {
@@ -317,8 +372,8 @@ sq_status sq_set_option(int option, int value) {
     g_force_ref = value == 1;
     return SQ_OK;
   }
-  if (option == SQ_OPT_ATTN_PATH && (value == 0 || value == 1)) {
-    g_attn_ref = value == 1;
+  if (option == SQ_OPT_ATTN_PATH && value >= 0 && value <= 2) {
+    g_attn_path = value;
     return SQ_OK;
   }
   if (option == SQ_OPT_TC_ERROR_BOUND && value >= 0 && value <= (1 << 20)) {
@@ -346,7 +401,8 @@ sq_status sq_calibrate(const sq_calib_params* p, const void* x, sq_dtype dtype, 
       p->d_eff_override > d || p->max_sweeps < 1 || !(p->tol > 0.0) || n_tokens < 1 || stride_tok < d ||
       stride_head < 0 || !x || !calib_out || ((uintptr_t)calib_out & 255u) || !ws || !aligned16(ws) ||
       (p->is_key != 0 && p->is_key != 1) || (p->qjl != 0 && p->qjl != 1) ||
-      (p->normalize != 0 && p->normalize != 1) || (d_status && !aligned16(d_status)) || (B + 31) / 32 > kMaxWords)
+      (p->normalize != 0 && p->normalize != 1) || (d_status && !aligned16(d_status)) || (B + 31) / 32 > kMaxWords ||
+      (p->rotation != 0 && p->rotation != 1) || !(p->cumvar >= 0.0 && p->cumvar <= 1.0))
     return SQ_ERR_ARG;
   if (ws_bytes < sq_calibrate_workspace(p, n_tokens)) return SQ_ERR_WORKSPACE;
   sq_status s = ensure_init();
@@ -361,10 +417,15 @@ sq_status sq_calibrate(const sq_calib_params* p, const void* x, sq_dtype dtype, 
     default: k_second_moment<__nv_bfloat16><<<g1, b1, 0, st>>>((const __nv_bfloat16*)x, d, n_tokens, stride_head, stride_tok, cov); break;
   }
   if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
-  size_t jsm = d <= 128 ? (size_t)8 * d * d : 0;
-  k_jacobi<<<p->n_heads, 256, jsm, st>>>(cov, vt, d, p->max_sweeps, p->tol, calib_out, d_status);
+  if (p->rotation == 1) {
+    k_random_basis<<<p->n_heads, 256, 0, st>>>(cov, vt, d, p->seed, calib_out, d_status);
+  } else {
+    size_t jsm = d <= 128 ? (size_t)8 * d * d : 0;
+    k_jacobi<<<p->n_heads, 256, jsm, st>>>(cov, vt, d, p->max_sweeps, p->tol, calib_out, d_status);
+  }
   if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
-  FinalizeArgs fa{B, p->is_key, p->qjl, p->normalize, p->d_eff_override, p->max_bits, p->seed, p->avg_bits};
+  FinalizeArgs fa{B, p->is_key, p->qjl, p->normalize, p->d_eff_override, p->max_bits, p->seed, p->avg_bits,
+                  p->cumvar, p->rotation};
   k_finalize<<<p->n_heads, 256, 0, st>>>(calib_out, d, fa, d_status);
   return cuda_ok(cudaGetLastError());
 }
@@ -540,8 +601,10 @@ sq_status sq_decompress_kv(const void* calib, const sq_cache* cache, int d, int6
 
 size_t sq_attn_workspace(int batch, int n_q_heads, int n_kv_heads, int d, int64_t max_ctx) {
   if (batch < 1 || n_q_heads < 1 || n_kv_heads < 1 || !supported_d(d) || max_ctx < 0) return 0;
-  int splits = attn_splits(batch, n_kv_heads, d, max_ctx);
-  return attn_ws_floats(batch, n_q_heads, d, splits) * sizeof(float);
+  // enough for whichever partial kernel the call picks (that depends on the records)
+  const int s1 = attn_splits(batch, n_kv_heads, d, max_ctx);
+  const int s2 = attn_splits_td(batch, n_kv_heads, d, max_ctx);
+  return attn_ws_floats(batch, n_q_heads, d, s1 > s2 ? s1 : s2) * sizeof(float);
 }
 
 sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
@@ -561,13 +624,18 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
   sq_status s = ensure_init();
   if (s != SQ_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
+  // partial kernel: the tcgen05 kernel unless the SIMT or the mma.sync one is
+  // asked for, or the records do not fit its shared memory
+  const int group = n_q_heads / n_kv_heads;
+  const int nrec = td_nrec(d, kc->words, vc->words);
+  const bool use_td = g_attn_path == 0 && (d == 64 || d == 128 || d == 256) && group <= 16 && nrec > 0;
   AttnShape sh;
   sh.batch = batch;
   sh.n_q = n_q_heads;
   sh.n_kv = n_kv_heads;
-  sh.group = n_q_heads / n_kv_heads;
+  sh.group = group;
   sh.d = d;
-  sh.splits = attn_splits(batch, n_kv_heads, d, max_ctx);
+  sh.splits = use_td ? attn_splits_td(batch, n_kv_heads, d, max_ctx) : attn_splits(batch, n_kv_heads, d, max_ctx);
   sh.max_ctx = max_ctx;
   int64_t per = (max_ctx + sh.splits - 1) / sh.splits;
   sh.chunk = ((per + kAttnTile - 1) / kAttnTile) * kAttnTile;
@@ -597,9 +665,22 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
   CacheArgs ka = cache_args(kc), va = cache_args(vc);
   const uint8_t* rk = (const uint8_t*)calib_k;
   const uint8_t* rv = (const uint8_t*)calib_v;
-  const bool fast = !g_attn_ref && sh.group <= 8 && (d == 64 || d == 128 || d == 256) && kc->words <= d / 8 &&
+  const bool fast = g_attn_path != 1 && sh.group <= 8 && (d == 64 || d == 128 || d == 256) && kc->words <= d / 8 &&
                     vc->words <= d / 8;
-  if (fast) {
+  if (use_td) {
+    const int MGv = sh.group <= 2 ? 2 : (sh.group <= 4 ? 4 : (sh.group <= 8 ? 8 : 16));
+#define SQ_TD_LAUNCH(DD, MG)                                                                                  \
+  td::k_decode_tc<DD, MG><<<gpart, td::Cfg<DD>::NTH, td::smem_bytes<DD>(kc->words, vc->words, nrec), st>>>( \
+      rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags, nrec)
+#define SQ_TD_G(DD)                                                                                       \
+  if (MGv == 2) SQ_TD_LAUNCH(DD, 2); else if (MGv == 4) SQ_TD_LAUNCH(DD, 4); else if (MGv == 8) SQ_TD_LAUNCH(DD, 8); \
+  else SQ_TD_LAUNCH(DD, 16)
+    if (d == 64) { SQ_TD_G(64); }
+    else if (d == 128) { SQ_TD_G(128); }
+    else { SQ_TD_G(256); }
+#undef SQ_TD_G
+#undef SQ_TD_LAUNCH
+  } else if (fast) {
     if (d == 64)
       fa::k_attn_partial_tc<64><<<gpart, fa::NTH, fa::smem_bytes<64>(), st>>>(rk, rv, ka, va, d_seq_lens, sh, w,
                                                                             scores_out, d_flags);

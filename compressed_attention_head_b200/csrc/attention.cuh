@@ -183,8 +183,15 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
   const uint32_t* vcodes = vc.codes + row * vc.cap * wv;
   for (int64_t t0 = t_lo; t0 < t_hi; t0 += kAttnTile) {
     const int nt = (int)min((int64_t)kAttnTile, t_hi - t0);
-    for (int e = tid; e < nt * wk; e += blockDim.x) kw[(e / wk) * (wk + 1) + e % wk] = kcodes[t0 * wk + e];
-    for (int e = tid; e < nt * wv; e += blockDim.x) vw[(e / wv) * (wv + 1) + e % wv] = vcodes[t0 * wv + e];
+    // word w of token t0 + i (interleaved blocks of 32 tokens; t0 is a multiple of 32)
+    for (int e = tid; e < nt * wk; e += blockDim.x) {
+      const int w = e / nt, i = e % nt;
+      kw[i * (wk + 1) + w] = kcodes[(size_t)((t0 + i) >> 5) * wk * 32 + (size_t)w * 32 + ((t0 + i) & 31)];
+    }
+    for (int e = tid; e < nt * wv; e += blockDim.x) {
+      const int w = e / nt, i = e % nt;
+      vw[i * (wv + 1) + w] = vcodes[(size_t)((t0 + i) >> 5) * wv * 32 + (size_t)w * 32 + ((t0 + i) & 31)];
+    }
     if (tid < nt) {
       kn[tid] = kc.norm[row * kc.cap + t0 + tid];
       kr[tid] = m > 0 ? kc.rnorm[row * kc.cap + t0 + tid] : 0.0f;

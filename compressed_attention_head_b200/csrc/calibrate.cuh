@@ -209,6 +209,8 @@ struct FinalizeArgs {
   int total_bits, is_key, qjl, normalize, d_eff_override, max_bits;
   uint64_t seed;
   double avg_bits;
+  double cumvar;      // 0: participation-ratio d_eff; (0, 1]: cumulative-variance d_eff
+  int rotation;       // 1: the basis is the random rotation (record flag only)
 };
 
 // Writes one derived part (float copies) of a record whose canonical part is complete.
@@ -255,6 +257,17 @@ __global__ void __launch_bounds__(256) k_finalize(void* __restrict__ recs, int d
     double pr = (q == 0.0) ? (double)d : t * t / q;
     int deff = (int)rint(pr);
     deff = deff < 1 ? 1 : (deff > d ? d : deff);
+    if (a.cumvar > 0.0) {
+      // smallest k >= 1 whose top-k eigenvalues hold cumvar of the trace
+      deff = d;
+      if (t > 0.0) {
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k) {
+          acc += lam[k];
+          if (acc >= a.cumvar * t) { deff = k + 1; break; }
+        }
+      }
+    }
     s_deff = deff;
     bool use_qjl = a.is_key && a.qjl;
     int m = use_qjl ? (a.d_eff_override > 0 ? a.d_eff_override : deff) : 0;
@@ -330,7 +343,8 @@ __global__ void __launch_bounds__(256) k_finalize(void* __restrict__ recs, int d
     hd->total_bits = a.total_bits;
     hd->code_bits = s_code_bits;
     hd->words = (a.total_bits + 31) / 32;
-    hd->flags = (a.is_key ? kFlagKey : 0u) | (m > 0 ? kFlagQjl : 0u) | (a.normalize ? kFlagNormalize : 0u);
+    hd->flags = (a.is_key ? kFlagKey : 0u) | (m > 0 ? kFlagQjl : 0u) | (a.normalize ? kFlagNormalize : 0u) |
+                (a.rotation ? kFlagRandomRotation : 0u) | (a.cumvar > 0.0 ? kFlagCumvar : 0u);
     hd->stream = h;
     hd->max_bits = a.max_bits;
     hd->seed = a.seed;
@@ -345,6 +359,100 @@ __global__ void __launch_bounds__(256) k_finalize(void* __restrict__ recs, int d
   build_derived(rec, tid, nth);
   __syncthreads();
   if (tid == 0) rec.hdr()->derived_valid = s_bad ? 0u : 1u;
+}
+
+// ---------------------------------------------------------------------------
+// Random rotation (the A/B baseline of the README's spectral_rotation.py),
+// one head per block, in place of the eigensolver: G = d x d N(0,1) draws
+// (row-major, from the stream of seed ^ kRotationSalt and the head's index),
+// Q of G = Q R by modified Gram-Schmidt over the columns (R_jj = ||a_j|| > 0),
+// the variance q_i^T C q_i of each column, and the columns written to the
+// record in descending order of variance (stable), which takes lambda's place.
+// The columns are kept contiguous in the workspace (Gt[j * d + i] = G[i][j]).
+// ---------------------------------------------------------------------------
+constexpr uint64_t kRotationSalt = 0x524F54ull;
+__global__ void __launch_bounds__(256) k_random_basis(const double* __restrict__ cov, double* __restrict__ vt_ws,
+                                                      int d, uint64_t seed, void* __restrict__ recs,
+                                                      int* __restrict__ status) {
+  const int h = blockIdx.x, tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  double* Gt = vt_ws + (size_t)h * d * d;
+  const double* C = cov + (size_t)h * d * d;
+  __shared__ double red[8];
+  __shared__ double s_nrm;
+  __shared__ double var_s[kMaxD];
+  __shared__ int order[kMaxD];
+  const uint64_t s0 = mix64((seed ^ kRotationSalt) ^ mix64((uint64_t)h + 1ull));
+  for (int pidx = tid; 2 * pidx < d * d; pidx += nth) {
+    const uint64_t r1 = sm64_at(s0, 2ull * pidx), r2 = sm64_at(s0, 2ull * pidx + 1ull);
+    const double u1 = (double)((r1 >> 11) + 1ull) * 0x1.0p-53;
+    const double u2 = (double)((r2 >> 11) + 1ull) * 0x1.0p-53;
+    const double rr = sqrt(-2.0 * log(u1));
+    const double th = 6.283185307179586477 * u2;
+    const int e0 = 2 * pidx, e1 = 2 * pidx + 1;                 // row-major draws G[e / d][e % d]
+    Gt[(size_t)(e0 % d) * d + e0 / d] = rr * cos(th);
+    if (e1 < d * d) Gt[(size_t)(e1 % d) * d + e1 / d] = rr * sin(th);
+  }
+  __syncthreads();
+  for (int j = 0; j < d; ++j) {
+    double* qj = Gt + (size_t)j * d;
+    double ss = 0.0;
+    for (int i = tid; i < d; i += nth) ss += qj[i] * qj[i];
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    if (tid == 0) {
+      double t = 0.0;
+      for (int w = 0; w < nth / 32; ++w) t += red[w];
+      s_nrm = sqrt(t);
+    }
+    __syncthreads();
+    const double inv = s_nrm > 0.0 ? 1.0 / s_nrm : 0.0;
+    for (int i = tid; i < d; i += nth) qj[i] *= inv;
+    __syncthreads();
+    // a_k -= (q_j . a_k) q_j for every later column, one warp per column
+    for (int k = j + 1 + warp; k < d; k += nth / 32) {
+      double* ak = Gt + (size_t)k * d;
+      double dot = 0.0;
+      for (int i = lane; i < d; i += 32) dot += qj[i] * ak[i];
+      dot = warp_sum(dot);
+      for (int i = lane; i < d; i += 32) ak[i] -= dot * qj[i];
+    }
+    __syncthreads();
+  }
+  // variance along each column: q^T C q (a warp per column)
+  for (int c = warp; c < d; c += nth / 32) {
+    const double* qc = Gt + (size_t)c * d;
+    double v = 0.0;
+    for (int a = 0; a < d; ++a) {
+      double t = 0.0;
+      for (int b = lane; b < d; b += 32) t += C[(size_t)a * d + b] * qc[b];
+      v += qc[a] * warp_sum(t);
+    }
+    if (lane == 0) var_s[c] = v;
+  }
+  __syncthreads();
+  for (int i = tid; i < d; i += nth) {
+    const double li = var_s[i];
+    int rank = 0;
+    for (int j = 0; j < d; ++j) {
+      const double lj = var_s[j];
+      rank += (lj > li) || (lj == li && j < i);
+    }
+    order[rank] = i;
+  }
+  __syncthreads();
+  Rec rec = rec_at(recs, d, h);
+  double* lam = rec.lam();
+  double* V = rec.V();
+  for (int c = tid; c < d; c += nth) lam[c] = fmax(var_s[order[c]], 0.0);
+  for (int e = tid; e < d * d; e += nth) {
+    const int i = e / d, c = e % d;
+    V[e] = Gt[(size_t)order[c] * d + i];
+  }
+  if (tid == 0) {
+    rec.hdr()->sweeps = 0;
+    if (status) status[h] = SQ_OK;
+  }
 }
 
 // ---------------------------------------------------------------------------

@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
     }
     __syncwarp();
     const size_t slot = row * c.cap + sp + t;
-    for (int w = lane; w < W; w += 32) c.codes[slot * W + w] = wb[w];
+    const size_t r0 = rec_word0(row, c.cap, W, sp + t);
+    for (int w = lane; w < W; w += 32) c.codes[r0 + (size_t)w * 32] = wb[w];
     if (lane == 0) {
       c.norm[slot] = (float)nrm;
       if (c.rnorm) c.rnorm[slot] = rho;
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(256) k_append(const uint8_t* __restrict__ recs
     const int b = (int)(vi / n_tok);
     const int64_t t = vi % n_tok;
     const int64_t sp = start_pos ? (int64_t)start_pos[b] : 0;
-    c.codes[(((size_t)b * n_heads + h) * c.cap + sp + t) * W + w] = wb[v][w];
+    c.codes[rec_word0((size_t)b * n_heads + h, c.cap, W, sp + t) + (size_t)w * 32] = wb[v][w];
   }
 }
 
@@ -370,7 +371,8 @@ __global__ void __launch_bounds__(128) k_decompress_ref(const uint8_t* __restric
   const size_t row = ((size_t)b * n_heads + h);
   for (int64_t t = t_begin + warp; t < t_end; t += kCodecWarps) {
     const size_t slot = row * c.cap + t0 + t;
-    for (int w = lane; w < W; w += 32) wb[w] = c.codes[slot * W + w];
+    const size_t r0 = rec_word0(row, c.cap, W, t0 + t);
+    for (int w = lane; w < W; w += 32) wb[w] = c.codes[r0 + (size_t)w * 32];
     __syncwarp();
     for (int i = lane; i < d; i += 32) {
       int bw = bits[i];

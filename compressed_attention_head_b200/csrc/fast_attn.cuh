@@ -451,14 +451,15 @@ __global__ void __launch_bounds__(NTH, min_blocks(D)) k_attn_partial_tc(const ui
   auto stage_rec = [&](uint32_t* rec, const uint32_t* src, int wn, int tile_i) {
     const int64_t t0 = t_lo + (int64_t)tile_i * TT;
     const bool in = t0 + lane < t_hi;
-    const uint32_t* sp = src + (in ? (t0 + lane) * wn : 0);
+    // t0 is a multiple of 32: this tile is one interleaved block, word w at + 32 w
+    const uint32_t* sp = src + (in ? (size_t)((t0 + lane) >> 5) * wn * 32 + lane : 0);
     uint32_t* dp = rec + lane;
     int w = 0;
     for (; w + 4 <= wn; w += 4) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) cp_async4_z(dp + (w + j) * RP, sp + w + j, in);
+      for (int j = 0; j < 4; ++j) cp_async4_z(dp + (w + j) * RP, sp + (w + j) * 32, in);
     }
-    for (; w < wn; ++w) cp_async4_z(dp + w * RP, sp + w, in);
+    for (; w < wn; ++w) cp_async4_z(dp + w * RP, sp + w * 32, in);
   };
   auto stage_nrm = [&](int tile_i) {
     const int64_t t0 = t_lo + (int64_t)tile_i * TT;

@@ -19,8 +19,20 @@ constexpr uint32_t kMagic = 0x31435153u;
 constexpr uint32_t kVersion = 1u;
 constexpr int kHeader = 128;
 constexpr int kMaxD = 256;
-constexpr uint32_t kFlagKey = 1u, kFlagQjl = 2u, kFlagNormalize = 4u;
+constexpr uint32_t kFlagKey = 1u, kFlagQjl = 2u, kFlagNormalize = 4u, kFlagRandomRotation = 8u, kFlagCumvar = 16u;
 constexpr int kMaxWords = 64;   // B <= 8 bits x 256 coordinates
+
+// Packed-cache layout: the records of 32 consecutive tokens of one (batch,
+// head) row are stored word-interleaved. Word w of token t of row r is
+//   codes[r * cap * W + ((t / 32) * W + w) * 32 + t % 32]
+// (cap a multiple of 32), so a block of 32 tokens is W * 128 contiguous bytes
+// whose 128-byte piece w holds word w of the 32 records: one bulk copy of a
+// block lands it transposed (word-major, token-minor) in shared memory, and 32
+// lanes that write word w of 32 consecutive tokens write one 128-byte line.
+constexpr int kBlockTok = 32;
+__host__ __device__ inline size_t rec_word0(size_t row, int64_t cap, int W, int64_t t) {
+  return row * (size_t)cap * (size_t)W + (size_t)(t >> 5) * (size_t)W * 32u + (size_t)(t & 31);
+}
 
 // Device arrays of one packed cache, as the kernels take them.
 struct CacheArgs {

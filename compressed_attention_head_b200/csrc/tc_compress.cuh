@@ -288,7 +288,9 @@ __device__ __forceinline__ uint32_t quant(float z, float R, const QCtx& c, const
 }
 
 // Little-endian bit stream of one record, written to global memory a word at
-// a time. fill and nw are the same in every lane of a warp (one head).
+// a time (word w at dst[32 w]: the interleaved cache layout, so the 32 lanes of
+// a warp, 32 consecutive tokens, store one 128-byte line per word). fill and nw
+// are the same in every lane of a warp (one head).
 struct Stream {
   uint32_t acc;      // the fill (< 32) pending low bits of the next word
   int fill;
@@ -301,7 +303,7 @@ __device__ __forceinline__ void put(Stream& s, uint32_t v, int n) {   // 1 <= n 
   const uint32_t carry = __funnelshift_l(v, 0u, s.fill);   // bits of v past the word
   const int nf = s.fill + n;
   const bool full = nf >= 32;
-  if (full && s.st) s.dst[s.nw] = lo;
+  if (full && s.st) s.dst[(size_t)s.nw * 32] = lo;
   s.nw += full ? 1 : 0;
   s.acc = full ? carry : lo;
   s.fill = nf & 31;
@@ -326,7 +328,7 @@ __device__ __forceinline__ void put_bits(Stream& s, const uint32_t* cw) {
   const int nfull = tot >> 5;                 // NB/32 or NB/32 + 1 (NB/32 rounded down)
 #pragma unroll
   for (int j = 0; j <= NI; ++j)
-    if (j < nfull && s.st) s.dst[s.nw + j] = w[j];
+    if (j < nfull && s.st) s.dst[(size_t)(s.nw + j) * 32] = w[j];
   constexpr int lo = NB / 32;
   s.acc = (nfull == lo) ? w[lo] : w[lo < NI ? lo + 1 : NI];
   s.nw += nfull;
@@ -346,8 +348,8 @@ __device__ __forceinline__ void flag_chunk(uint32_t (&fm)[4], int c, uint32_t dm
   for (int q = 0; q < 4; ++q) fm[q] |= (c >> 1) == q ? sh : 0u;
 }
 
-// Exact repair of the flagged codes of a warp's 32 records, after they have
-// been written: rounds of up to RB (lane, coordinate) entries, each
+// Exact repair of the flagged codes of a warp's 32 records (word w of the
+// lane's record at rec[32 w]), after they have been written: rounds of up to RB (lane, coordinate) entries, each
 // recomputed by the whole warp in float64 (lane l takes elements 4l .. 4l+3 of
 // the input row and of the eigenvector; the loads of a round are all issued
 // before any reduction), z = (V_i . x) / ||x|| / sigma_i, and the owner lane
@@ -417,11 +419,11 @@ __device__ __forceinline__ void repair_warp(uint4 fmv, const __half* x, int64_t 
         // same thread's operations on one address stay in order)
         const int o = offs[i], wi = o >> 5, sh = o & 31;
         const uint32_t mask = (1u << b) - 1u;
-        atomicAnd(&rec[wi], ~(mask << sh));
-        atomicOr(&rec[wi], code << sh);
+        atomicAnd(&rec[(size_t)wi * 32], ~(mask << sh));
+        atomicOr(&rec[(size_t)wi * 32], code << sh);
         if (sh + b > 32) {
-          atomicAnd(&rec[wi + 1], ~(mask >> (32 - sh)));
-          atomicOr(&rec[wi + 1], code >> (32 - sh));
+          atomicAnd(&rec[(size_t)(wi + 1) * 32], ~(mask >> (32 - sh)));
+          atomicOr(&rec[(size_t)(wi + 1) * 32], code >> (32 - sh));
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q)
@@ -801,7 +803,8 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
         if (live) {
           qc.zr = sc * inv32;
           const bool fix_ok = valid && inv32 != 0.0f;
-          Stream s{0u, 0, 0, P.c.codes + slot * (size_t)W, valid};
+          Stream s{0u, 0, 0, P.c.codes + rec_word0((size_t)bidx * P.n_heads + h, P.c.cap, W, sp + t0 + t_row),
+                   valid};
           uint32_t fm[4] = {0u, 0u, 0u, 0u};   // coordinates to repair exactly
           const uint32_t taddr = tmem_base + ((uint32_t)(qtr * 32) << 16) + (uint32_t)(st * D);
 #pragma unroll 1
@@ -859,7 +862,7 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
           }
           if (m > 0) put(s, qbits, m);
           while (s.nw < W) {   // the rest of the record: remaining bits, then zero words
-            if (s.st) s.dst[s.nw] = s.acc;
+            if (s.st) s.dst[(size_t)s.nw * 32] = s.acc;
             s.acc = 0u;
             ++s.nw;
           }

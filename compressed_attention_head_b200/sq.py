@@ -34,7 +34,8 @@ class sq_calib_params(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int), ("n_heads", ctypes.c_int), ("avg_bits", ctypes.c_double),
                 ("is_key", ctypes.c_int), ("qjl", ctypes.c_int), ("normalize", ctypes.c_int),
                 ("d_eff_override", ctypes.c_int), ("max_bits", ctypes.c_int), ("seed", ctypes.c_uint64),
-                ("max_sweeps", ctypes.c_int), ("tol", ctypes.c_double)]
+                ("max_sweeps", ctypes.c_int), ("tol", ctypes.c_double), ("rotation", ctypes.c_int),
+                ("cumvar", ctypes.c_double)]
 
 
 class sq_cache(ctypes.Structure):
@@ -127,10 +128,12 @@ def sq_calib_bytes(d: int) -> int:
 
 
 def calib_params(d, n_heads, avg_bits, is_key, qjl=True, normalize=True, d_eff_override=0, max_bits=8,
-                 seed=42, max_sweeps=30, tol=1e-13) -> sq_calib_params:
+                 seed=42, max_sweeps=30, tol=1e-13, rotation=0, cumvar=0.0) -> sq_calib_params:
+    """rotation: 0 calibrated eigenbasis, 1 random rotation (A/B baseline);
+    cumvar: 0 participation-ratio d_eff, else the cumulative-variance fraction."""
     return sq_calib_params(d, n_heads, float(avg_bits), int(bool(is_key)), int(bool(qjl)), int(bool(normalize)),
                            int(d_eff_override), int(max_bits), int(seed) & ((1 << 64) - 1), int(max_sweeps),
-                           float(tol))
+                           float(tol), int(rotation), float(cumvar))
 
 
 def sq_record_words(params: sq_calib_params) -> int:
@@ -159,7 +162,7 @@ def sq_attn_workspace(batch, n_q_heads, n_kv_heads, d, max_ctx) -> int:
 class PackedCache:
     """Caller-owned device arrays of one packed cache (see sq_cache in sq.h)."""
 
-    codes: torch.Tensor          # int32 [batch, n_heads, cap, words], read as uint32
+    codes: torch.Tensor          # int32 [batch, n_heads, cap / 32, words, 32], read as uint32
     norm: torch.Tensor           # float32 [batch, n_heads, cap]
     rnorm: torch.Tensor | None   # float32 [batch, n_heads, cap] or None
     batch: int
@@ -173,12 +176,24 @@ class PackedCache:
                         self.batch, self.n_heads, self.cap, self.words)
 
     def words_u32(self) -> np.ndarray:
-        return self.codes.cpu().numpy().view(np.uint32)
+        """The records as [batch, n_heads, cap, words] uint32 (undoing the 32-token interleave)."""
+        c = self.codes.cpu().numpy().view(np.uint32)
+        return np.ascontiguousarray(c.transpose(0, 1, 2, 4, 3)).reshape(self.batch, self.n_heads, self.cap,
+                                                                        self.words)
+
+    def tiled(self, rep_batch: int, rep_heads: int) -> "PackedCache":
+        """A new cache holding this one repeated rep_batch times over the batch and
+        rep_heads times over the heads (row (b, h) = this row (b % batch, h % n_heads))."""
+        return PackedCache(self.codes.repeat(rep_batch, rep_heads, 1, 1, 1),
+                           self.norm.repeat(rep_batch, rep_heads, 1),
+                           self.rnorm.repeat(rep_batch, rep_heads, 1) if self.rnorm is not None else None,
+                           self.batch * rep_batch, self.n_heads * rep_heads, self.cap, self.words)
 
 
 def alloc_cache(batch, n_heads, cap, words, with_rnorm, device="cuda") -> PackedCache:
-    cap = ((int(cap) + 15) // 16) * 16
-    codes = torch.zeros(batch, n_heads, cap, words, dtype=torch.int32, device=device)
+    """Zeroed packed cache; cap is rounded up to a multiple of 32."""
+    cap = ((int(cap) + 31) // 32) * 32
+    codes = torch.zeros(batch, n_heads, cap // 32, words, 32, dtype=torch.int32, device=device)
     norm = torch.zeros(batch, n_heads, cap, dtype=torch.float32, device=device)
     rnorm = torch.zeros_like(norm) if with_rnorm else None
     return PackedCache(codes, norm, rnorm, batch, n_heads, cap, words)

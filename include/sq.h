@@ -76,7 +76,7 @@ typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2 } sq_dtype;
 #define SQ_FLAG_TIMEOUT 0x80000000u
 
 #define SQ_MAX_BITS 8         /* largest code width of one coordinate                     */
-#define SQ_ABI_VERSION 1
+#define SQ_ABI_VERSION 2   /* 2: word-interleaved 32-token blocks in sq_cache.codes */
 
 /*
  * Calibration parameters (host struct).
@@ -95,6 +95,18 @@ typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2 } sq_dtype;
  *                 uniforms in (0,1], Box-Muller pairs).
  *  max_sweeps     eigensolver sweep limit (e.g. 30).
  *  tol            eigensolver stop: off-diagonal Frobenius norm <= tol * ||C||_F.
+ *  rotation       0: the calibrated eigenbasis (the method); 1: a random
+ *                 rotation, the A/B baseline of the README's
+ *                 spectral_rotation.py ("spectral rotation vs random rotation
+ *                 baseline"): Q of the QR factorisation (diag R > 0) of a d x d
+ *                 matrix of N(0,1) draws, row-major, from the stream of seed
+ *                 seed ^ 0x524F54 and the head's index (SplitMix64 / Box-Muller
+ *                 as for the QJL matrix), its columns ordered by descending
+ *                 variance q^T C q, which takes the place of lambda.
+ *  cumvar         0: d_eff is the participation ratio; in (0, 1]: d_eff is the
+ *                 smallest k >= 1 whose top-k lambda hold at least this fraction
+ *                 of the trace (the README's results/deff_sweep/ compares
+ *                 "participation ratio vs cumvar").
  */
 typedef struct {
   int d;
@@ -108,16 +120,26 @@ typedef struct {
   uint64_t seed;
   int max_sweeps;
   double tol;
+  int rotation;
+  double cumvar;
 } sq_calib_params;
 
 /*
  * One packed cache (keys or values of one layer, or of several layers with the
  * layers folded into the head index). Device arrays, caller-owned:
- *  codes  uint32 [batch][n_heads][cap][words]   one packed record per token
+ *  codes  uint32 [batch][n_heads][cap / 32][words][32]
+ *                 one packed record per token, the records of 32 consecutive
+ *                 tokens word-interleaved: word w of token t of a (batch, head)
+ *                 row is element ((t / 32) * words + w) * 32 + t % 32 of the
+ *                 row's cap * words words. A block of 32 tokens is then
+ *                 words * 128 contiguous bytes, piece w holding word w of all
+ *                 32 records, which is how the kernels want it in shared memory
+ *                 (one bulk copy per tile) and how 32 lanes store it (one
+ *                 128-byte line per word).
  *  norm   float  [batch][n_heads][cap]          ||x|| (1.0 when not normalized)
  *  rnorm  float  [batch][n_heads][cap]          QJL residual norm rho; NULL when
  *                                               the records carry no QJL bits
- *  cap    tokens per (batch, head); a multiple of 16.
+ *  cap    tokens per (batch, head); a multiple of 32.
  *  words  32-bit words per record, ceil(B / 32); must equal the records'.
  *
  * Record bit layout (the pages fix none; this is the library's reading): stream
@@ -150,7 +172,8 @@ typedef struct {
  *  20                   i32   total_bits B
  *  24                   i32   code_bits = sum of b_i = B - m
  *  28                   i32   words = ceil(B / 32)
- *  32                   u32   flags: 1 key, 2 QJL, 4 normalized
+ *  32                   u32   flags: 1 key, 2 QJL, 4 normalized, 8 random rotation,
+ *                             16 cumulative-variance d_eff
  *  36                   i32   eigensolver sweeps used
  *  40                   i32   stream (head index of the QJL Gaussian stream)
  *  44                   i32   max_bits
@@ -201,9 +224,12 @@ sq_status sq_init(void);
  *  SQ_OPT_COMPRESS_PATH: 0 = automatic (tensor-core kernel for fp16 head_dim-128
  *  prompts of >= 64 tokens, float64 reference kernel otherwise), 1 = always the
  *  float64 reference kernel. Both produce identical codes (see sq_compress_kv).
- *  SQ_OPT_ATTN_PATH: 0 = automatic (tensor-core partials for head_dim 64/128/256,
- *  up to 8 query heads per KV head and records of up to 32 words; SIMT partials
- *  otherwise), 1 = always the SIMT partials.
+ *  SQ_OPT_ATTN_PATH: 0 = automatic (the tcgen05 partials for head_dim 64/128/256
+ *  and up to 16 query heads per KV head whose records fit its shared memory;
+ *  SIMT partials otherwise), 1 = always the SIMT partials, 2 = the mma.sync
+ *  tensor-core partials where they apply (up to 8 query heads, records of up to
+ *  4 bits per coordinate), SIMT otherwise. All give the same results within the
+ *  attention tolerances.
  *  SQ_OPT_TC_ERROR_BOUND: the fp32-accumulation term of the tensor-core compress
  *  error radius, in units of 2^-24 per unit of ||V_i / sigma_i|| (default 32:
  *  sixteen accumulation steps of one fp32 rounding each, with truncation).

@@ -31,6 +31,20 @@ Readings taken where the pages are silent
   the cap; ties go to the lowest index. D is the Gaussian Lloyd-Max
   distortion table (D(0) = 1). Because D is convex and decreasing the greedy
   result minimises sum_i lambda_i D(b_i) over integer allocations.
+
+Variants the README names ("Repository Structure": results/deff_sweep/ --
+"participation ratio vs cumvar"; spectral_rotation.py -- "Spectral rotation
+vs random rotation baseline"), with the readings taken:
+* cumulative-variance d_eff: the smallest k >= 1 whose top-k eigenvalues hold
+  at least a fraction ``cumvar`` of the trace (the pages give no fraction; the
+  caller chooses it, 0.9 in the tests);
+* random rotation: the basis is Q of the QR factorisation G = Q R (diag R > 0)
+  of a d x d matrix G of N(0,1) draws, row-major, from the stream of seed
+  ``seed ^ ROTATION_SALT`` and the head's index (the same SplitMix64 /
+  Box-Muller stream as the QJL matrix, another seed), i.e. a Haar-random
+  orthogonal matrix; lambda_i = q_i^T C q_i is the variance along column i,
+  and the columns are ordered by descending variance (stable). Everything
+  after the basis is unchanged.
 """
 
 from __future__ import annotations
@@ -44,6 +58,9 @@ from . import codebook, rng
 FLAG_IS_KEY = 1
 FLAG_QJL = 2
 FLAG_NORMALIZE = 4
+FLAG_RANDOM_ROTATION = 8
+FLAG_CUMVAR = 16
+ROTATION_SALT = 0x524F54       # seed salt of the random-rotation stream ("ROT")
 
 
 def second_moment(x: np.ndarray) -> np.ndarray:
@@ -74,10 +91,37 @@ def participation_ratio(lam: np.ndarray) -> float:
     return float(np.sum(lam)) ** 2 / s2
 
 
-def effective_dim(lam: np.ndarray) -> int:
-    """d_eff: the participation ratio rounded half to even, within [1, d]."""
+def effective_dim(lam: np.ndarray, cumvar: float = 0.0) -> int:
+    """d_eff: the participation ratio rounded half to even, within [1, d]; with
+    0 < cumvar <= 1, the smallest k >= 1 whose top-k eigenvalues (descending)
+    hold at least cumvar of the trace (d for an all-zero spectrum)."""
     d = len(lam)
+    if cumvar > 0.0:
+        lam = np.asarray(lam, dtype=np.float64)
+        tr = float(np.sum(lam))
+        if tr == 0.0:
+            return d
+        acc = 0.0
+        for k in range(d):
+            acc += float(lam[k])
+            if acc >= cumvar * tr:
+                return k + 1
+        return d
     return int(min(max(round(participation_ratio(lam)), 1), d))
+
+
+def random_basis(c: np.ndarray, seed: int, stream: int):
+    """(variances, basis) of the random-rotation variant: Q of the QR
+    factorisation of a seeded Gaussian matrix (diag R > 0), its columns ordered
+    by descending variance q_i^T C q_i (stable)."""
+    c = np.asarray(c, dtype=np.float64)
+    d = c.shape[0]
+    g = rng.gaussians(seed ^ ROTATION_SALT, stream, d * d).reshape(d, d)
+    q, r = np.linalg.qr(g)
+    q = q * np.sign(np.diagonal(r))[None, :]
+    var = np.einsum("ji,jk,ki->i", q, c, q)
+    order = np.argsort(-var, kind="stable")
+    return np.maximum(var[order], 0.0), q[:, order].copy()
 
 
 def spectral_gap(lam: np.ndarray, d_eff: int) -> float:
@@ -170,10 +214,10 @@ def budget(d: int, avg_bits: float) -> int:
 def finalize(lam: np.ndarray, vec: np.ndarray, *, avg_bits: float, is_key: bool,
              qjl: bool = True, normalize: bool = True, d_eff_override: int = 0,
              max_bits: int = codebook.MAX_BITS, seed: int = 42, stream: int = 0,
-             sweeps: int = 0) -> HeadCalib:
-    """Everything after the eigendecomposition: d_eff, kappa, scales, bits, QJL matrix."""
+             sweeps: int = 0, cumvar: float = 0.0, random_rotation: bool = False) -> HeadCalib:
+    """Everything after the basis: d_eff, kappa, scales, bits, QJL matrix."""
     d = lam.size
-    d_eff = effective_dim(lam)
+    d_eff = effective_dim(lam, cumvar)
     kappa = spectral_gap(lam, d_eff)
     total = budget(d, avg_bits)
     use_qjl = bool(is_key and qjl)
@@ -184,7 +228,8 @@ def finalize(lam: np.ndarray, vec: np.ndarray, *, avg_bits: float, is_key: bool,
     if code_bits < 0 or code_bits > max_bits * d:
         raise ValueError("bit budget cannot hold the QJL bits and the codes")
     bits = water_fill(lam, code_bits, max_bits)
-    flags = (FLAG_IS_KEY if is_key else 0) | (FLAG_QJL if use_qjl else 0) | (FLAG_NORMALIZE if normalize else 0)
+    flags = ((FLAG_IS_KEY if is_key else 0) | (FLAG_QJL if use_qjl else 0) | (FLAG_NORMALIZE if normalize else 0)
+             | (FLAG_RANDOM_ROTATION if random_rotation else 0) | (FLAG_CUMVAR if cumvar > 0.0 else 0))
     return HeadCalib(
         d=d, d_eff=d_eff, m=m, total_bits=total, code_bits=code_bits,
         words=(total + 31) // 32, flags=flags, sweeps=sweeps, stream=stream,
@@ -194,7 +239,12 @@ def finalize(lam: np.ndarray, vec: np.ndarray, *, avg_bits: float, is_key: bool,
         offsets=bit_offsets(bits))
 
 
-def calibrate(x: np.ndarray, **kw) -> HeadCalib:
-    """Calibrate one head from its calibration vectors ``x`` [N, d]."""
-    lam, vec = eigenbasis(second_moment(x))
+def calibrate(x: np.ndarray, *, rotation: str = "spectral", **kw) -> HeadCalib:
+    """Calibrate one head from its calibration vectors ``x`` [N, d]; ``rotation``
+    is "spectral" (the calibrated eigenbasis) or "random" (the A/B baseline)."""
+    c = second_moment(x)
+    if rotation == "random":
+        lam, vec = random_basis(c, kw.get("seed", 42), kw.get("stream", 0))
+        return finalize(lam, vec, random_rotation=True, **kw)
+    lam, vec = eigenbasis(c)
     return finalize(lam, vec, **kw)

@@ -116,18 +116,20 @@ def test_attention_seq_len_past_bound_is_flagged():
     assert e.value.status == sq.SQ_ERR_WORKSPACE
 
 
-@pytest.mark.parametrize("name,ctx,heads", [("llama8b", 700, 2), ("gemma9b_sweep", 300, 2)])
-def test_tensor_core_partials_match_simt_partials(name, ctx, heads):
-    """Both attention paths against the oracle on the same packed cache."""
+@pytest.mark.parametrize("name,ctx,heads", [("llama8b", 700, 2), ("gemma9b_sweep", 300, 2), ("qwen14b", 1500, 1)])
+def test_every_partial_kernel_matches_the_oracle(name, ctx, heads):
+    """The three attention partial kernels (tcgen05, SIMT, mma.sync) against the
+    oracle on the same packed cache."""
+    outs = {}
     try:
-        sq.sq_set_option(sq.SQ_OPT_ATTN_PATH, 1)
-        o1, s1, r_o, r_s, _ = _run(name, 1, ctx, [ctx], heads=heads)
-        sq.sq_set_option(sq.SQ_OPT_ATTN_PATH, 0)
-        o0, s0, _, _, _ = _run(name, 1, ctx, [ctx], heads=heads)
+        for path in (0, 1, 2):
+            sq.sq_set_option(sq.SQ_OPT_ATTN_PATH, path)
+            outs[path] = _run(name, 1, ctx, [ctx], heads=heads)
     finally:
         sq.sq_set_option(sq.SQ_OPT_ATTN_PATH, 0)
-    _assert_close(o1, s1, r_o, r_s, [ctx])
-    _assert_close(o0, s0, r_o, r_s, [ctx])
+    for path, (o, sc, r_o, r_s, flags) in outs.items():
+        assert flags == 0, path
+        _assert_close(o, sc, r_o, r_s, [ctx])
 
 
 def test_full_size_decode_sampled_rows():
@@ -182,14 +184,8 @@ def _bench_shape_sampled(name, n_layers, batch, ctx, rows, distinct_heads=2, dis
     v1 = sq.alloc_cache(nb, distinct_heads, cap, cv[0].words, False)
     sq.sq_compress_kv(rk1, rv1, w.k.contiguous(), w.v.contiguous(), nb, distinct_heads, d, ctx, None, k1, v1)
     del w.k, w.v
-    kc = sq.alloc_cache(batch, nkv, cap, ck[0].words, True)
-    vc = sq.alloc_cache(batch, nkv, cap, cv[0].words, False)
     rb = batch // nb
-    for big, small in ((kc, k1), (vc, v1)):
-        big.codes.copy_(small.codes.repeat(rb, rep, 1, 1))
-        big.norm.copy_(small.norm.repeat(rb, rep, 1))
-        if big.rnorm is not None:
-            big.rnorm.copy_(small.rnorm.repeat(rb, rep, 1))
+    kc, vc = k1.tiled(rb, rep), v1.tiled(rb, rep)
     q = w.q.repeat(rb, rep, 1).contiguous()
     lens_l = [ctx - (7 * b) % 301 for b in range(batch)]
     lens = torch.tensor(lens_l, dtype=torch.int32, device="cuda")

@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import calibrate_oracle, read_records
+from gpu_helpers import calibrate_oracle, compare_compressed, read_records, records_to_device
 from oracle import calibration as ocal
 from oracle import codebook as ocb
 from oracle import rng as orng
@@ -27,9 +27,10 @@ if not torch.cuda.is_available():
 from compressed_attention_head_b200 import sq  # noqa: E402
 
 
-def _gpu_calibrate(x_cal, avg_bits, is_key, qjl=True, seed=42, max_sweeps=30):
+def _gpu_calibrate(x_cal, avg_bits, is_key, qjl=True, seed=42, max_sweeps=30, rotation=0, cumvar=0.0):
     nh, n, d = x_cal.shape
-    p = sq.calib_params(d, nh, avg_bits, is_key, qjl=qjl, seed=seed, max_sweeps=max_sweeps)
+    p = sq.calib_params(d, nh, avg_bits, is_key, qjl=qjl, seed=seed, max_sweeps=max_sweeps, rotation=rotation,
+                        cumvar=cumvar)
     recs = sq.alloc_records(nh, d)
     ws = torch.empty(sq.sq_calibrate_workspace(p, n), dtype=torch.uint8, device="cuda")
     status = torch.full((nh,), -1, dtype=torch.int32, device="cuda")
@@ -116,3 +117,59 @@ def test_import_rejects_malformed_record():
     sq.sq_calib_import(dev, 2, 32, status)
     torch.cuda.synchronize()
     assert status.cpu().tolist() == [0, sq.SQ_ERR_RECORD]
+
+
+@pytest.mark.parametrize("name", ["llama8b", "gemma9b_sweep"])
+def test_random_rotation_matches_the_oracle(name):
+    """The random-rotation variant (the A/B baseline): the basis is a
+    deterministic function of the seed and head, so the GPU's basis,
+    variances, widths and d_eff equal the oracle's (to float64 rounding of a
+    Gram-Schmidt against a Householder QR); the spectral basis beats it on the
+    expected distortion of the same budget."""
+    w = make_workload(name, batch=1, tokens=16)
+    cfg = w.cfg
+    nh = 2
+    for xcal, bits, is_key in ((w.k_cal[:nh], cfg["bits_k"], True), (w.v_cal[:nh], cfg["bits_v"], False)):
+        gpu, status = _gpu_calibrate(xcal, bits, is_key, seed=11, rotation=1)
+        assert status == [0] * nh
+        for h, g in enumerate(gpu):
+            r = ocal.calibrate(xcal[h].double().numpy(), avg_bits=bits, is_key=is_key, seed=11, stream=h,
+                               rotation="random")
+            assert g.flags == r.flags and g.flags & ocal.FLAG_RANDOM_ROTATION
+            assert np.max(np.abs(g.V - r.V)) < 1e-10
+            assert np.max(np.abs(g.lam - r.lam)) < 1e-10 * r.lam[0]
+            assert g.d_eff == r.d_eff and g.m == r.m
+            assert np.array_equal(g.bits, r.bits)
+            spec = ocal.calibrate(xcal[h].double().numpy(), avg_bits=bits, is_key=is_key, stream=h)
+            dist = ocb.distortion_table()
+            assert np.sum(spec.sigma ** 2 * dist[spec.bits]) < np.sum(r.sigma ** 2 * dist[r.bits])
+
+
+def test_random_rotation_records_compress_like_the_oracle():
+    """Compression with random-rotation records (imported from the oracle)."""
+    w = make_workload("llama8b", batch=1, tokens=200)
+    cals = [ocal.calibrate(w.k_cal[h].double().numpy(), avg_bits=3.0, is_key=True, seed=5, stream=h,
+                           rotation="random") for h in range(2)]
+    recs = records_to_device(cals)
+    kc = sq.alloc_cache(1, 2, 200, cals[0].words, True)
+    x = w.k[:, :2].contiguous()
+    sq.sq_compress_kv(recs, None, x.cuda(), None, 1, 2, 128, 200, None, kc, None)
+    torch.cuda.synchronize()
+    words = kc.words_u32()
+    for h in range(2):
+        compare_compressed(words[0, h, :200], kc.norm[0, h, :200].cpu().numpy(), kc.rnorm[0, h, :200].cpu().numpy(),
+                           x[0, h].double().numpy(), cals[h])
+
+
+@pytest.mark.parametrize("name", ["llama8b", "qwen1_5b_long"])
+def test_cumulative_variance_d_eff(name):
+    """d_eff by cumulative variance (0.9 of the trace): the GPU's d_eff is the
+    oracle's rule applied to the GPU's eigenvalues and equals the oracle's."""
+    w = make_workload(name, batch=1, tokens=16)
+    for xcal, bits, is_key in ((w.k_cal[:2], 3.0, True), (w.v_cal[:2], 3.0, False)):
+        gpu, status = _gpu_calibrate(xcal, bits, is_key, cumvar=0.9)
+        assert status == [0, 0]
+        for h, g in enumerate(gpu):
+            r = ocal.calibrate(xcal[h].double().numpy(), avg_bits=bits, is_key=is_key, stream=h, cumvar=0.9)
+            assert g.d_eff == ocal.effective_dim(g.lam, cumvar=0.9) == r.d_eff
+            assert g.flags & ocal.FLAG_CUMVAR and g.m == (r.m if is_key else 0)

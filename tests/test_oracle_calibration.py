@@ -172,3 +172,82 @@ def test_finalize_budget_identity():
         cal.calibrate(x, avg_bits=3.01, is_key=False)
     o = cal.calibrate(x, avg_bits=3.0, is_key=True, d_eff_override=4)
     assert o.m == 4 and o.d_eff == c.d_eff
+
+
+# ---------------------------------------------------------------- variants
+def test_cumulative_variance_d_eff_exact_spectra():
+    """Smallest k whose top-k eigenvalues hold the fraction of the trace:
+    flat (0.9 x 32 = 28.8 -> 29), four equal spikes (3.6 -> 4), a spiked
+    spectrum (0.9 x 208 = 187.2 reached at 100+50+20+10+8 ones -> 12), and an
+    exact tie (half of 4 equal values is reached at 2, not 3)."""
+    assert cal.effective_dim(np.ones(32), cumvar=0.9) == 29
+    assert cal.effective_dim(np.array([1.0] * 4 + [0.0] * 28), cumvar=0.9) == 4
+    spiked = np.array([100.0, 50.0, 20.0, 10.0] + [1.0] * 28)
+    assert cal.effective_dim(spiked, cumvar=0.9) == 12
+    assert cal.effective_dim(spiked) == 3            # participation ratio 3.32 for comparison
+    assert cal.effective_dim(np.ones(4), cumvar=0.5) == 2
+    assert cal.effective_dim(np.zeros(8), cumvar=0.9) == 8
+    assert cal.effective_dim(np.ones(8), cumvar=1.0) == 8
+
+
+def test_cumulative_variance_d_eff_in_the_record():
+    x = np.random.default_rng(11).standard_normal((4000, 32)) * np.concatenate([np.full(4, 10.0), np.ones(28)])
+    c = cal.calibrate(x, avg_bits=3.0, is_key=True, cumvar=0.9)
+    want = cal.effective_dim(c.lam, cumvar=0.9)
+    assert c.d_eff == want == c.m and c.flags & cal.FLAG_CUMVAR
+    assert c.code_bits + c.m == c.total_bits == 96
+
+
+def test_random_rotation_is_haar_distributed():
+    """Q of QR with a positive diagonal of R is Haar-distributed: over many seeds
+    a fixed entry has mean 0 and mean square 1/d (with isotropic data the
+    variance ordering keeps the columns in place). A QR without the sign fix
+    gives Q[0, 0] = -|g00| / ||g0|| < 0 every time."""
+    d, n = 6, 3000
+    q00 = np.empty(n)
+    q23 = np.empty(n)
+    for s in range(n):
+        lam, v = cal.random_basis(np.eye(d), seed=1000 + s, stream=0)
+        assert np.allclose(lam, 1.0)
+        q00[s], q23[s] = v[0, 0], v[2, 3]
+    se = math.sqrt(1.0 / d / n)
+    assert abs(q00.mean()) < 5 * se and abs(q23.mean()) < 5 * se
+    assert abs((q00 ** 2).mean() - 1.0 / d) < 0.1 / d
+    assert abs((q23 ** 2).mean() - 1.0 / d) < 0.1 / d
+
+
+def test_random_rotation_basis_properties():
+    """Orthonormal, variances q_i^T C q_i summing to the trace, descending,
+    and a different basis per stream and seed."""
+    r = np.random.default_rng(12)
+    x = r.standard_normal((3000, 16)) * np.linspace(5, 1, 16)
+    c = cal.second_moment(x)
+    lam, v = cal.random_basis(c, seed=7, stream=3)
+    assert np.max(np.abs(v.T @ v - np.eye(16))) < 1e-12
+    assert abs(lam.sum() - np.trace(c)) < 1e-10 * np.trace(c)
+    assert np.all(np.diff(lam) <= 0)
+    assert np.allclose(lam, np.einsum("ji,jk,ki->i", v, c, v))
+    _, v2 = cal.random_basis(c, seed=7, stream=4)
+    _, v3 = cal.random_basis(c, seed=8, stream=3)
+    assert np.max(np.abs(v - v2)) > 0.1 and np.max(np.abs(v - v3)) > 0.1
+
+
+def test_spectral_rotation_beats_random_rotation_on_spiked_data():
+    """The A/B the README's spectral_rotation.py runs: on a spiked spectrum the
+    calibrated eigenbasis concentrates the energy (small d_eff) and its
+    water-filled expected distortion sum_i sigma_i^2 D(b_i) is lower than that
+    of a random rotation at the same budget, whose per-direction variances
+    are nearly flat."""
+    r = np.random.default_rng(13)
+    d = 64
+    q, _ = np.linalg.qr(r.standard_normal((d, d)))
+    lam = np.concatenate([np.full(4, 200.0), np.ones(d - 4)])
+    x = (r.standard_normal((20000, d)) * np.sqrt(lam)) @ q.T
+    spec = cal.calibrate(x, avg_bits=3.0, is_key=False, normalize=False)
+    rand = cal.calibrate(x, avg_bits=3.0, is_key=False, normalize=False, rotation="random", seed=3)
+    dist = cb.distortion_table()
+    e_spec = float(np.sum(spec.sigma ** 2 * dist[spec.bits]))
+    e_rand = float(np.sum(rand.sigma ** 2 * dist[rand.bits]))
+    assert spec.d_eff <= 6 < rand.d_eff
+    assert e_spec < 0.6 * e_rand
+    assert rand.flags & cal.FLAG_RANDOM_ROTATION and not spec.flags & cal.FLAG_RANDOM_ROTATION
