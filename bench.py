@@ -464,15 +464,17 @@ def _calibrate(sq, cfg, H, k_cal, v_cal, dev):
     pv = sq.calib_params(d, H, cfg["bits_v"], False)
     rk, rv = sq.alloc_records(H, d, dev), sq.alloc_records(H, d, dev)
     ws = torch.empty(sq.sq_calibrate_workspace(pk, ncal), dtype=torch.uint8, device=dev)
-    st = torch.zeros(2 * H, dtype=torch.int32, device=dev)
+    st_k = torch.zeros(H, dtype=torch.int32, device=dev)      # separate tensors: 16-byte aligned
+    st_v = torch.zeros(H, dtype=torch.int32, device=dev)
     a, b = _events(2)
     torch.cuda.synchronize()
     a.record()
-    sq.sq_calibrate(pk, k_cal, ncal, ncal * d, d, rk, ws, st[:H])
-    sq.sq_calibrate(pv, v_cal, ncal, ncal * d, d, rv, ws, st[H:])
+    sq.sq_calibrate(pk, k_cal, ncal, ncal * d, d, rk, ws, st_k)
+    sq.sq_calibrate(pv, v_cal, ncal, ncal * d, d, rv, ws, st_v)
     b.record()
     torch.cuda.synchronize()
-    return rk, rv, sq.sq_record_words(pk), sq.sq_record_words(pv), a.elapsed_time(b), int((st != 0).sum().item())
+    n_bad = int((st_k != 0).sum().item()) + int((st_v != 0).sum().item())
+    return rk, rv, sq.sq_record_words(pk), sq.sq_record_words(pv), a.elapsed_time(b), n_bad
 
 
 def measure_prefill(cfg, args, world, dev):
@@ -634,6 +636,7 @@ def run_gpu(args, rank, world, local_rank):
     dev = f"cuda:{local_rank}"
     torch.cuda.set_device(local_rank)
     sq.sq_init()
+    sq.sq_set_option(sq.SQ_OPT_ATTN_PATH, args.attn_path)
     peak, peak_kind = _peaks()
     headline = args.config == "headline"
     dec_name = HEADLINE_DECODE if headline else args.config
@@ -729,6 +732,8 @@ def main():
                     help="headline (Gemma-shaped decode + Llama-shaped prompt compress) or a workload name")
     ap.add_argument("--bits", type=float, default=None, help="bits per coordinate for K and V (Gemma sweep)")
     ap.add_argument("--no-qjl", action="store_true")
+    ap.add_argument("--attn-path", type=int, default=0,
+                    help="attention partial kernel: 0 tcgen05 (default), 1 SIMT, 2 mma.sync (comparison runs)")
     ap.add_argument("--base-rows", type=int, default=2, help="distinct batch rows of a decode cache")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time the eager launches only")

@@ -24,6 +24,7 @@ __device__ uint8_t c_tccell[560];      // tcc cell tables: positive thresholds b
 #include "fast_attn.cuh"
 #include "tc_compress.cuh"
 #include "tc_decode.cuh"
+#include "decode_step.cuh"
 
 namespace sq {
 
@@ -137,6 +138,17 @@ sq_status ensure_init(int* dev_out = nullptr) {
     SQ_TD_ATTR(128, 2); SQ_TD_ATTR(128, 4); SQ_TD_ATTR(128, 8); SQ_TD_ATTR(128, 16);
     SQ_TD_ATTR(256, 2); SQ_TD_ATTR(256, 4); SQ_TD_ATTR(256, 8); SQ_TD_ATTR(256, 16);
 #undef SQ_TD_ATTR
+    const int ps = (int)prep_smem(kMaxD);
+    cudaFuncSetAttribute(k_attn_prepare<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, ps);
+    cudaFuncSetAttribute(k_attn_prepare<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, ps);
+    cudaFuncSetAttribute(k_attn_prepare<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, ps);
+#define SQ_SP_ATTR(T)                                                                          \
+  cudaFuncSetAttribute(k_step_prep<T, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, ps);    \
+  cudaFuncSetAttribute(k_step_prep<T, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, ps);    \
+  cudaFuncSetAttribute(k_step_prep<T, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, ps);    \
+  cudaFuncSetAttribute(k_step_prep<T, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, ps)
+    SQ_SP_ATTR(float); SQ_SP_ATTR(__half); SQ_SP_ATTR(__nv_bfloat16);
+#undef SQ_SP_ATTR
   }
   if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
   int sms = 0;
@@ -318,10 +330,10 @@ sq_status launch_compress(const void* recs, const void* x, int batch, int n_head
     const T* xt = (const T*)x;
     const CacheArgs ca = cache_args(c);
     switch (nv) {
-      case 1: k_append<T, 1><<<grid, 256, 0, st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
-      case 2: k_append<T, 2><<<grid, 256, 0, st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
-      case 4: k_append<T, 4><<<grid, 256, 0, st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
-      default: k_append<T, 8><<<grid, 256, 0, st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
+      case 1: k_append<T, 1><<<grid, 256, append_smem(1), st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
+      case 2: k_append<T, 2><<<grid, 256, append_smem(2), st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
+      case 4: k_append<T, 4><<<grid, 256, append_smem(4), st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
+      default: k_append<T, 8><<<grid, 256, append_smem(8), st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
     }
     return cuda_ok(cudaGetLastError());
   }
@@ -604,28 +616,34 @@ size_t sq_attn_workspace(int batch, int n_q_heads, int n_kv_heads, int d, int64_
   // enough for whichever partial kernel the call picks (that depends on the records)
   const int s1 = attn_splits(batch, n_kv_heads, d, max_ctx);
   const int s2 = attn_splits_td(batch, n_kv_heads, d, max_ctx);
-  return attn_ws_floats(batch, n_q_heads, d, s1 > s2 ? s1 : s2) * sizeof(float);
+  return attn_ws_bytes(batch, n_q_heads, n_kv_heads, d, s1 > s2 ? s1 : s2);
 }
 
-sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
-                         const int32_t* d_seq_lens, int batch, int n_q_heads, int n_kv_heads, int d,
-                         int64_t max_ctx, const void* q, sq_dtype q_dtype, float scale, void* out,
-                         sq_dtype out_dtype, float* scores_out, void* ws, size_t ws_bytes, uint32_t* d_flags,
-                         sq_stream stream) {
-  if (!supported_d(d) || !valid_dtype(q_dtype) || !valid_dtype(out_dtype)) return SQ_ERR_UNSUPPORTED;
-  if (batch < 1 || batch > 65535 || n_q_heads < 1 || n_kv_heads < 1 || n_kv_heads > 65535 ||
-      n_q_heads % n_kv_heads != 0 || n_q_heads / n_kv_heads > kAttnMaxG || n_q_heads > 65535 || max_ctx < 0 ||
-      !calib_k || !calib_v || ((uintptr_t)calib_k & 255u) || ((uintptr_t)calib_v & 255u) ||
-      !cache_ok(kc, batch, n_kv_heads) || !cache_ok(vc, batch, n_kv_heads) || !d_seq_lens ||
-      !aligned16(d_seq_lens) || !q || !aligned16(q) || !out || !aligned16(out) ||
-      (scores_out && !aligned16(scores_out)) || !ws || !aligned16(ws))
-    return SQ_ERR_ARG;
-  if (ws_bytes < sq_attn_workspace(batch, n_q_heads, n_kv_heads, d, max_ctx)) return SQ_ERR_WORKSPACE;
-  sq_status s = ensure_init();
-  if (s != SQ_OK) return s;
-  cudaStream_t st = (cudaStream_t)stream;
-  // partial kernel: the tcgen05 kernel unless the SIMT or the mma.sync one is
-  // asked for, or the records do not fit its shared memory
+}  // extern "C"
+
+namespace {
+
+bool attn_args_ok(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
+                  const int32_t* d_lens, int batch, int n_q_heads, int n_kv_heads, const void* q, const void* out,
+                  const float* scores_out, const void* ws) {
+  return !(batch < 1 || batch > 65535 || n_q_heads < 1 || n_kv_heads < 1 || n_kv_heads > 65535 ||
+           n_q_heads % n_kv_heads != 0 || n_q_heads / n_kv_heads > kAttnMaxG || n_q_heads > 65535 || !calib_k ||
+           !calib_v || ((uintptr_t)calib_k & 255u) || ((uintptr_t)calib_v & 255u) ||
+           !cache_ok(kc, batch, n_kv_heads) || !cache_ok(vc, batch, n_kv_heads) || !d_lens || !aligned16(d_lens) ||
+           !q || !aligned16(q) || !out || !aligned16(out) || (scores_out && !aligned16(scores_out)) || !ws ||
+           !aligned16(ws));
+}
+
+// Every launch of one decode-attention call. With k_new / v_new (a decode
+// step) the new token of each row is first compressed into the caches at
+// d_lens[b] and attended (len_offset 1). The tcgen05 path takes two launches
+// (append + prepare in one; partials with the last-block combine); the
+// others take prepare, partials and combine (and the appends before them).
+template <typename TQ>
+sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
+                      const int32_t* d_lens, int len_offset, int batch, int n_q_heads, int n_kv_heads, int d,
+                      int64_t max_ctx, const void* q, float scale, void* out, sq_dtype out_dtype, float* scores_out,
+                      void* ws, uint32_t* d_flags, cudaStream_t st, const void* k_new, const void* v_new, int dev) {
   const int group = n_q_heads / n_kv_heads;
   const int nrec = td_nrec(d, kc->words, vc->words);
   const bool use_td = g_attn_path == 0 && (d == 64 || d == 128 || d == 256) && group <= 16 && nrec > 0;
@@ -637,41 +655,53 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
   sh.d = d;
   sh.splits = use_td ? attn_splits_td(batch, n_kv_heads, d, max_ctx) : attn_splits(batch, n_kv_heads, d, max_ctx);
   sh.max_ctx = max_ctx;
+  sh.len_offset = len_offset;
   int64_t per = (max_ctx + sh.splits - 1) / sh.splits;
   sh.chunk = ((per + kAttnTile - 1) / kAttnTile) * kAttnTile;
   if (sh.chunk < kAttnTile) sh.chunk = kAttnTile;
   const float sc = scale > 0.0f ? scale : 1.0f / sqrtf((float)d);
   float* w = (float*)ws;
-  dim3 gp(n_kv_heads, batch);
-  {
-    const uint8_t* rk8 = (const uint8_t*)calib_k;
-    const int G = sh.group;
-#define SQ_PREP(MG, T)                                                                          \
-  k_attn_prepare<MG, T><<<gp, 128, 0, st>>>(rk8, (const T*)q, sh, sc, w, d_flags)
-#define SQ_PREP_G(T)                                                                            \
-  if (G <= 1) SQ_PREP(1, T); else if (G <= 2) SQ_PREP(2, T); else if (G <= 4) SQ_PREP(4, T);   \
-  else if (G <= 8) SQ_PREP(8, T); else SQ_PREP(16, T)
-    switch (q_dtype) {
-      case SQ_F32: SQ_PREP_G(float); break;
-      case SQ_F16: SQ_PREP_G(__half); break;
-      default: SQ_PREP_G(__nv_bfloat16); break;
-    }
-#undef SQ_PREP_G
-#undef SQ_PREP
-  }
-  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
-  dim3 gpart(sh.splits, n_kv_heads, batch);
-  size_t smem = attn_partial_smem(d, sh.group, kc->words, vc->words);
-  CacheArgs ka = cache_args(kc), va = cache_args(vc);
   const uint8_t* rk = (const uint8_t*)calib_k;
   const uint8_t* rv = (const uint8_t*)calib_v;
+  CacheArgs ka = cache_args(kc), va = cache_args(vc);
+  const int prow = prep_rows(group);
+  const unsigned n_prep = (unsigned)(n_kv_heads * ((batch + prow - 1) / prow));
+  // ---- launch 1: prepare (with the appends of a decode step)
+  if (k_new && use_td) {
+    const int nv = append_nv(batch);
+    const int64_t n_app = (int64_t)n_kv_heads * ((batch + nv - 1) / nv);
+    const int64_t blocks = 2 * n_app + n_prep;
+    if (blocks > 0x7fffffff) return SQ_ERR_ARG;
+    const size_t ps = prep_smem(kMaxD);
+    const TQ* kn = (const TQ*)k_new;
+    const TQ* vn = (const TQ*)v_new;
+    const TQ* qq = (const TQ*)q;
+    switch (nv) {
+      case 1: k_step_prep<TQ, 1><<<(unsigned)blocks, 256, ps, st>>>(rk, rv, kn, vn, qq, batch, n_kv_heads, d, d_lens, ka, va, sh, sc, w, d_flags, (int)n_app); break;
+      case 2: k_step_prep<TQ, 2><<<(unsigned)blocks, 256, ps, st>>>(rk, rv, kn, vn, qq, batch, n_kv_heads, d, d_lens, ka, va, sh, sc, w, d_flags, (int)n_app); break;
+      case 4: k_step_prep<TQ, 4><<<(unsigned)blocks, 256, ps, st>>>(rk, rv, kn, vn, qq, batch, n_kv_heads, d, d_lens, ka, va, sh, sc, w, d_flags, (int)n_app); break;
+      default: k_step_prep<TQ, 8><<<(unsigned)blocks, 256, ps, st>>>(rk, rv, kn, vn, qq, batch, n_kv_heads, d, d_lens, ka, va, sh, sc, w, d_flags, (int)n_app); break;
+    }
+  } else {
+    if (k_new) {
+      sq_status s = launch_compress<TQ>(calib_k, k_new, batch, n_kv_heads, d, 1, d_lens, kc, d_flags, st);
+      if (s == SQ_OK) s = launch_compress<TQ>(calib_v, v_new, batch, n_kv_heads, d, 1, d_lens, vc, d_flags, st);
+      if (s != SQ_OK) return s;
+    }
+    dim3 gp(n_kv_heads, (unsigned)((batch + prow - 1) / prow));
+    k_attn_prepare<TQ><<<gp, 256, prep_smem(d), st>>>(rk, (const TQ*)q, sh, sc, w, d_flags);
+  }
+  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  // ---- launch 2: partials (the tcgen05 kernel merges the splits itself)
+  dim3 gpart(sh.splits, n_kv_heads, batch);
+  size_t smem = attn_partial_smem(d, sh.group, kc->words, vc->words);
   const bool fast = g_attn_path != 1 && sh.group <= 8 && (d == 64 || d == 128 || d == 256) && kc->words <= d / 8 &&
                     vc->words <= d / 8;
   if (use_td) {
     const int MGv = sh.group <= 2 ? 2 : (sh.group <= 4 ? 4 : (sh.group <= 8 ? 8 : 16));
 #define SQ_TD_LAUNCH(DD, MG)                                                                                  \
   td::k_decode_tc<DD, MG><<<gpart, td::Cfg<DD>::NTH, td::smem_bytes<DD>(kc->words, vc->words, nrec), st>>>( \
-      rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags, nrec)
+      rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags, nrec, out, (int)out_dtype)
 #define SQ_TD_G(DD)                                                                                       \
   if (MGv == 2) SQ_TD_LAUNCH(DD, 2); else if (MGv == 4) SQ_TD_LAUNCH(DD, 4); else if (MGv == 8) SQ_TD_LAUNCH(DD, 8); \
   else SQ_TD_LAUNCH(DD, 16)
@@ -680,43 +710,91 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
     else { SQ_TD_G(256); }
 #undef SQ_TD_G
 #undef SQ_TD_LAUNCH
-  } else if (fast) {
+    return cuda_ok(cudaGetLastError());
+  }
+  if (fast) {
     if (d == 64)
-      fa::k_attn_partial_tc<64><<<gpart, fa::NTH, fa::smem_bytes<64>(), st>>>(rk, rv, ka, va, d_seq_lens, sh, w,
+      fa::k_attn_partial_tc<64><<<gpart, fa::NTH, fa::smem_bytes<64>(), st>>>(rk, rv, ka, va, d_lens, sh, w,
                                                                             scores_out, d_flags);
     else if (d == 128)
-      fa::k_attn_partial_tc<128><<<gpart, fa::NTH, fa::smem_bytes<128>(), st>>>(rk, rv, ka, va, d_seq_lens, sh, w,
+      fa::k_attn_partial_tc<128><<<gpart, fa::NTH, fa::smem_bytes<128>(), st>>>(rk, rv, ka, va, d_lens, sh, w,
                                                                               scores_out, d_flags);
     else
-      fa::k_attn_partial_tc<256><<<gpart, fa::NTH, fa::smem_bytes<256>(), st>>>(rk, rv, ka, va, d_seq_lens, sh, w,
+      fa::k_attn_partial_tc<256><<<gpart, fa::NTH, fa::smem_bytes<256>(), st>>>(rk, rv, ka, va, d_lens, sh, w,
                                                                               scores_out, d_flags);
   } else if (sh.group <= 1)
-    k_attn_partial<1><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
+    k_attn_partial<1><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags);
   else if (sh.group <= 2)
-    k_attn_partial<2><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
+    k_attn_partial<2><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags);
   else if (sh.group <= 4)
-    k_attn_partial<4><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
+    k_attn_partial<4><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags);
   else if (sh.group <= 8)
-    k_attn_partial<8><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
+    k_attn_partial<8><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags);
   else
-    k_attn_partial<16><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_seq_lens, sh, w, scores_out, d_flags);
+    k_attn_partial<16><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags);
   if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  // ---- launch 3: combine
   dim3 gc(n_kv_heads, batch);
-  {
-    const int G = sh.group;
-#define SQ_COMB(MG, T) k_attn_combine<MG, T><<<gc, 256, 0, st>>>(rv, sh, w, (T*)out)
-#define SQ_COMB_G(T)                                                                             \
-  if (G <= 1) SQ_COMB(1, T); else if (G <= 2) SQ_COMB(2, T); else if (G <= 4) SQ_COMB(4, T);    \
-  else if (G <= 8) SQ_COMB(8, T); else SQ_COMB(16, T)
-    switch (out_dtype) {
-      case SQ_F32: SQ_COMB_G(float); break;
-      case SQ_F16: SQ_COMB_G(__half); break;
-      default: SQ_COMB_G(__nv_bfloat16); break;
-    }
-#undef SQ_COMB_G
-#undef SQ_COMB
-  }
+  k_attn_combine<<<gc, 256, combine_scratch_floats(d, sh.splits) * 4, st>>>(rv, sh, w, out, (int)out_dtype);
+  (void)dev;
   return cuda_ok(cudaGetLastError());
+}
+
+sq_status attn_dispatch(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
+                        const int32_t* d_lens, int len_offset, int batch, int n_q_heads, int n_kv_heads, int d,
+                        int64_t max_ctx, const void* q, sq_dtype dtype, float scale, void* out, sq_dtype out_dtype,
+                        float* scores_out, void* ws, uint32_t* d_flags, cudaStream_t st, const void* k_new,
+                        const void* v_new, int dev) {
+  switch (dtype) {
+    case SQ_F32:
+      return attn_launch<float>(calib_k, calib_v, kc, vc, d_lens, len_offset, batch, n_q_heads, n_kv_heads, d,
+                                max_ctx, q, scale, out, out_dtype, scores_out, ws, d_flags, st, k_new, v_new, dev);
+    case SQ_F16:
+      return attn_launch<__half>(calib_k, calib_v, kc, vc, d_lens, len_offset, batch, n_q_heads, n_kv_heads, d,
+                                 max_ctx, q, scale, out, out_dtype, scores_out, ws, d_flags, st, k_new, v_new, dev);
+    default:
+      return attn_launch<__nv_bfloat16>(calib_k, calib_v, kc, vc, d_lens, len_offset, batch, n_q_heads, n_kv_heads,
+                                        d, max_ctx, q, scale, out, out_dtype, scores_out, ws, d_flags, st, k_new,
+                                        v_new, dev);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
+                         const int32_t* d_seq_lens, int batch, int n_q_heads, int n_kv_heads, int d,
+                         int64_t max_ctx, const void* q, sq_dtype q_dtype, float scale, void* out,
+                         sq_dtype out_dtype, float* scores_out, void* ws, size_t ws_bytes, uint32_t* d_flags,
+                         sq_stream stream) {
+  if (!supported_d(d) || !valid_dtype(q_dtype) || !valid_dtype(out_dtype)) return SQ_ERR_UNSUPPORTED;
+  if (max_ctx < 0 ||
+      !attn_args_ok(calib_k, calib_v, kc, vc, d_seq_lens, batch, n_q_heads, n_kv_heads, q, out, scores_out, ws))
+    return SQ_ERR_ARG;
+  if (ws_bytes < sq_attn_workspace(batch, n_q_heads, n_kv_heads, d, max_ctx)) return SQ_ERR_WORKSPACE;
+  int dev = 0;
+  sq_status s = ensure_init(&dev);
+  if (s != SQ_OK) return s;
+  return attn_dispatch(calib_k, calib_v, kc, vc, d_seq_lens, 0, batch, n_q_heads, n_kv_heads, d, max_ctx, q, q_dtype,
+                       scale, out, out_dtype, scores_out, ws, d_flags, (cudaStream_t)stream, nullptr, nullptr, dev);
+}
+
+sq_status sq_decode_step(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
+                         const void* k_new, const void* v_new, const void* q, sq_dtype dtype, const int32_t* d_pos,
+                         int batch, int n_q_heads, int n_kv_heads, int d, int64_t max_ctx, float scale, void* out,
+                         sq_dtype out_dtype, float* scores_out, void* ws, size_t ws_bytes, uint32_t* d_flags,
+                         sq_stream stream) {
+  if (!supported_d(d) || !valid_dtype(dtype) || !valid_dtype(out_dtype)) return SQ_ERR_UNSUPPORTED;
+  if (max_ctx < 1 || !k_new || !v_new || !aligned16(k_new) || !aligned16(v_new) ||
+      !attn_args_ok(calib_k, calib_v, kc, vc, d_pos, batch, n_q_heads, n_kv_heads, q, out, scores_out, ws))
+    return SQ_ERR_ARG;
+  if (ws_bytes < sq_attn_workspace(batch, n_q_heads, n_kv_heads, d, max_ctx)) return SQ_ERR_WORKSPACE;
+  int dev = 0;
+  sq_status s = ensure_init(&dev);
+  if (s != SQ_OK) return s;
+  return attn_dispatch(calib_k, calib_v, kc, vc, d_pos, 1, batch, n_q_heads, n_kv_heads, d, max_ctx, q, dtype, scale,
+                       out, out_dtype, scores_out, ws, d_flags, (cudaStream_t)stream, k_new, v_new, dev);
 }
 
 // ---------------------------------------------------------------------------

@@ -23,59 +23,89 @@ constexpr int kAttnMaxG = 16;      // query heads per KV head
 struct AttnShape {
   int batch, n_q, n_kv, group, d, splits;
   int64_t max_ctx, chunk;
+  int len_offset;     // attended length = seq_lens[b] + len_offset (1 when seq_lens holds the new token's position)
 };
 
 // Workspace layout (floats): w[batch][n_q][d], u[batch][n_q][d],
-// acc[batch][n_q][splits][d], ml[batch][n_q][splits][2].
+// acc[batch][n_q][splits][d], ml[batch][n_q][splits][2], then one uint32
+// arrival counter per (batch, KV head) for the last-block combine.
 __host__ __device__ inline size_t attn_ws_floats(int batch, int n_q, int d, int splits) {
   return (size_t)batch * n_q * (2 * (size_t)d + (size_t)splits * (d + 2));
 }
+__host__ __device__ inline size_t attn_ws_bytes(int batch, int n_q, int n_kv, int d, int splits) {
+  return attn_ws_floats(batch, n_q, d, splits) * 4 + (size_t)batch * n_kv * 4;
+}
+__device__ __forceinline__ uint32_t* attn_counters(float* ws, const AttnShape& s) {
+  return (uint32_t*)(ws + attn_ws_floats(s.batch, s.n_q, s.d, s.splits));
+}
+
+// Attended length of row b (the new token included when len_offset is 1).
+__device__ __forceinline__ int64_t attn_len(const int32_t* seq_lens, const AttnShape& s, int b) {
+  return (int64_t)seq_lens[b] + s.len_offset;
+}
 
 // ---------------------------------------------------------------------------
-// Prepare: grid (n_kv, batch), d threads; one block rotates the G queries of
-// one KV head with the float32 copy of V_K.
+// Prepare: one block rotates the G queries of nb consecutive batch rows
+// b0 .. b0 + nb - 1 for one KV head g with the float32 copy of V_K (read once
+// for all of them, eight query vectors per pass), w = scale sigma q',
+// u = scale sqrt(pi/2) / m S q'[0:m]; it also clears the rows' combine
+// counters. smem: floats [nv][d] (queries) + [nv][d] (q'), nv = nb G <= 32.
 // ---------------------------------------------------------------------------
-template <int MAXG, typename TQ>
-__global__ void k_attn_prepare(const uint8_t* __restrict__ recs_k, const TQ* __restrict__ q, AttnShape s,
-                               float scale, float* __restrict__ ws, uint32_t* __restrict__ flags) {
-  const int g = blockIdx.x, b = blockIdx.y, d = s.d, G = s.group;
+constexpr int kPrepVecs = 32;    // query vectors per prepare block
+__host__ __device__ inline int prep_rows(int G) { return G >= kPrepVecs ? 1 : kPrepVecs / G; }
+__host__ __device__ inline size_t prep_smem(int d) { return (size_t)2 * kPrepVecs * d * 4; }
+
+template <typename TQ>
+__device__ void prepare_body(const uint8_t* __restrict__ recs_k, const TQ* __restrict__ q, const AttnShape& s,
+                             float scale, float* __restrict__ ws, uint32_t* __restrict__ flags, int g, int b0,
+                             float* smem, int tid, int nth) {
+  const int d = s.d, G = s.group;
+  const int nb = min(prep_rows(G), s.batch - b0);
+  if (tid < nb) attn_counters(ws, s)[(size_t)(b0 + tid) * s.n_kv + g] = 0u;   // for the last-block combine
   Rec rec = rec_at(recs_k, d, g);
   const RecHeader* hd = rec.hdr();
   if (!record_ok(hd, d)) {
-    if (threadIdx.x == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
+    if (tid == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
     return;
   }
-  __shared__ float qs[kAttnMaxG][kMaxD];
-  __shared__ float qp[kAttnMaxG][kMaxD];
-  for (int e = threadIdx.x; e < MAXG * d; e += blockDim.x) {
-    int hh = e / d, j = e % d;
-    qs[hh][j] = hh < G ? to_float<TQ>(q[((size_t)b * s.n_q + g * G + hh) * d + j]) : 0.0f;
+  const int nv = nb * G;                 // query vectors: (row r, head hh) -> r * G + hh
+  float* qs = smem;                      // [nv][d]
+  float* qp = smem + (size_t)kPrepVecs * d;
+  for (int e = tid; e < nv * d; e += nth) {
+    const int v = e / d, j = e % d;
+    const int r = v / G, hh = v % G;
+    qs[e] = to_float<TQ>(q[((size_t)(b0 + r) * s.n_q + (size_t)g * G + hh) * d + j]);
   }
   __syncthreads();
   const float* V = rec.V_f();
   const float* sig = rec.sigma_f();
   float* w = ws;
   float* u = ws + (size_t)s.batch * s.n_q * d;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    float acc[MAXG];
+  for (int v0 = 0; v0 < nv; v0 += 8) {
+    for (int i = tid; i < d; i += nth) {
+      float acc[8];
 #pragma unroll
-    for (int hh = 0; hh < MAXG; ++hh) acc[hh] = 0.0f;
-    // the column of V in batches of 32 loads issued together (d is a multiple of 32)
-    for (int j0 = 0; j0 < d; j0 += 32) {
-      float vv[32];
+      for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
+      // the column of V in batches of 32 loads issued together (d is a multiple of 32)
+      for (int j0 = 0; j0 < d; j0 += 32) {
+        float vv[32];
 #pragma unroll
-      for (int u = 0; u < 32; ++u) vv[u] = V[(size_t)(j0 + u) * d + i];
+        for (int t = 0; t < 32; ++t) vv[t] = V[(size_t)(j0 + t) * d + i];
 #pragma unroll
-      for (int u = 0; u < 32; ++u) {
+        for (int t = 0; t < 32; ++t) {
 #pragma unroll
-        for (int hh = 0; hh < MAXG; ++hh) acc[hh] = fmaf(vv[u], qs[hh][j0 + u], acc[hh]);
+          for (int k = 0; k < 8; ++k)
+            if (v0 + k < nv) acc[k] = fmaf(vv[t], qs[(size_t)(v0 + k) * d + j0 + t], acc[k]);
+        }
       }
-    }
 #pragma unroll
-    for (int hh = 0; hh < MAXG; ++hh) {
-      if (hh < G) {
-        qp[hh][i] = acc[hh];
-        w[((size_t)b * s.n_q + g * G + hh) * d + i] = scale * sig[i] * acc[hh];
+      for (int k = 0; k < 8; ++k) {
+        const int v = v0 + k;
+        if (v < nv) {
+          qp[(size_t)v * d + i] = acc[k];
+          const int r = v / G, hh = v % G;
+          w[((size_t)(b0 + r) * s.n_q + (size_t)g * G + hh) * d + i] = scale * sig[i] * acc[k];
+        }
       }
     }
   }
@@ -83,12 +113,23 @@ __global__ void k_attn_prepare(const uint8_t* __restrict__ recs_k, const TQ* __r
   const int m = hd->m;
   const float* S = rec.S_f();
   const float coef = scale * (float)(kQjlScale / (m > 0 ? m : 1));
-  for (int e = threadIdx.x; e < G * m; e += blockDim.x) {
-    int hh = e / m, j = e % m;
+  for (int e = tid; e < nv * m; e += nth) {
+    const int v = e / m, j = e % m;
     float acc = 0.0f;
-    for (int k = 0; k < m; ++k) acc = fmaf(S[j * m + k], qp[hh][k], acc);
-    u[((size_t)b * s.n_q + g * G + hh) * d + j] = coef * acc;
+    for (int k = 0; k < m; ++k) acc = fmaf(S[j * m + k], qp[(size_t)v * d + k], acc);
+    const int r = v / G, hh = v % G;
+    u[((size_t)(b0 + r) * s.n_q + (size_t)g * G + hh) * d + j] = coef * acc;
   }
+}
+
+// Prepare as a kernel of its own: grid (n_kv, row groups of prep_rows(G)), 256 threads.
+template <typename TQ>
+__global__ void __launch_bounds__(256) k_attn_prepare(const uint8_t* __restrict__ recs_k, const TQ* __restrict__ q,
+                                                      AttnShape s, float scale, float* __restrict__ ws,
+                                                      uint32_t* __restrict__ flags) {
+  extern __shared__ __align__(16) float pscr[];
+  prepare_body<TQ>(recs_k, q, s, scale, ws, flags, blockIdx.x, blockIdx.y * prep_rows(s.group), pscr, threadIdx.x,
+                   blockDim.x);
 }
 
 // Shared-memory bytes of the partial kernel.
@@ -128,7 +169,7 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
   float* ml_out = acc_out + (size_t)s.batch * s.n_q * s.splits * d;
   const bool ok = record_ok(hk, d) && record_ok(hv, d) && hk->words == kc.words && hv->words == vc.words &&
                   (hk->m == 0 || kc.rnorm != nullptr);
-  int64_t L = seq_lens[b];
+  int64_t L = attn_len(seq_lens, s, b);
   if (L < 0 || L > s.max_ctx || L > kc.cap) {
     if (tid == 0 && split == 0 && g == 0 && flags) atomicOr(flags, SQ_FLAG_SEQLEN);
     L = L < 0 ? 0 : (L > s.max_ctx ? s.max_ctx : L);
@@ -293,103 +334,105 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// Combine: grid (n_kv, batch), 256 threads; one block finishes the G query
-// heads of one KV head, so V_V is read once for all of them.
+// Combine of one (batch, KV head): merges the splits of its G query heads and
+// rotates back with V_V, which is read once for all of them:
 // a_h,i = sigma_V,i * sum_s e^(m_s - M) acc_s,i / sum_s e^(m_s - M) l_s;  o_h = V_V a_h.
+// scr: [16][d] floats (a), [16][splits] floats (split weights), [16] (1 / l).
 // ---------------------------------------------------------------------------
-template <int MAXG, typename TO>
-__global__ void __launch_bounds__(256, 2) k_attn_combine(const uint8_t* __restrict__ recs_v, AttnShape s,
-                                                      const float* __restrict__ ws, TO* __restrict__ out) {
-  const int g = blockIdx.x, b = blockIdx.y, d = s.d, tid = threadIdx.x, G = s.group;
-  const int lane = tid & 31, warp = tid >> 5;
+__device__ __forceinline__ void store_out(void* out, int dt, size_t idx, float v) {
+  if (dt == SQ_F32) ((float*)out)[idx] = v;
+  else if (dt == SQ_F16) ((__half*)out)[idx] = __float2half_rn(v);
+  else ((__nv_bfloat16*)out)[idx] = __float2bfloat16_rn(v);
+}
+
+__device__ void combine_one(const uint8_t* __restrict__ recs_v, const AttnShape& s, const float* ws, void* out,
+                            int out_dt, int g, int b, float* scr, int tid, int nth) {
+  const int d = s.d, G = s.group;
+  const int lane = tid & 31, warp = tid >> 5, nwarp = nth >> 5;
   Rec rv = rec_at(recs_v, d, g);
-  __shared__ __align__(16) float a[MAXG][kMaxD];
-  __shared__ float sw[MAXG][256];   // splits <= 256 (attn_splits)
-  __shared__ float s_inv_l[MAXG];
+  float* a = scr;                       // [16][d]
+  float* sw = scr + 16 * d;             // [16][splits]
+  float* s_inv_l = sw + 16 * s.splits;  // [16]
   const float* acc = ws + (size_t)s.batch * s.n_q * d * 2;
   const float* ml = acc + (size_t)s.batch * s.n_q * s.splits * d;
   const size_t qh0 = (size_t)b * s.n_q + (size_t)g * G;
   const bool ok = record_ok(rv.hdr(), d);
   const float* sig = rv.sigma_f();
-  // per head (one warp each, round robin): split weights e^(m_s - M) and 1 / l
-  for (int hh = warp; hh < G; hh += 8) {
+  for (int hh = warp; hh < G; hh += nwarp) {
     const float* mlh = ml + (qh0 + hh) * s.splits * 2;
     float M = -INFINITY;
-    for (int k = lane; k < s.splits; k += 32) M = fmaxf(M, mlh[2 * k]);
+    // partials of other blocks of the same launch may be read here: L2 loads (__ldcg)
+    for (int k = lane; k < s.splits; k += 32) M = fmaxf(M, __ldcg(mlh + 2 * k));
     M = warp_max(M);
     float l = 0.0f;
     for (int k = lane; k < s.splits; k += 32) {
-      const float mk = mlh[2 * k];
+      const float mk = __ldcg(mlh + 2 * k);
       const float wk = (mk == -INFINITY) ? 0.0f : __expf(mk - M);
-      sw[hh][k] = wk;
-      l += wk * mlh[2 * k + 1];
+      sw[hh * s.splits + k] = wk;
+      l += wk * __ldcg(mlh + 2 * k + 1);
     }
     l = warp_sum(l);
     if (lane == 0) s_inv_l[hh] = l > 0.0f ? 1.0f / l : 0.0f;
   }
   __syncthreads();
-  for (int e = tid; e < G * d; e += 256) {
+  for (int e = tid; e < G * d; e += nth) {
     const int hh = e / d, i = e % d;
     const float* ah = acc + (qh0 + hh) * s.splits * (size_t)d + i;
+    const float* swh = sw + hh * s.splits;
     float v = 0.0f;
     int k = 0;
     for (; k + 4 <= s.splits; k += 4) {     // four loads in flight
-      const float a0 = ah[(size_t)k * d], a1 = ah[(size_t)(k + 1) * d];
-      const float a2 = ah[(size_t)(k + 2) * d], a3 = ah[(size_t)(k + 3) * d];
-      v = fmaf(sw[hh][k], a0, v);
-      v = fmaf(sw[hh][k + 1], a1, v);
-      v = fmaf(sw[hh][k + 2], a2, v);
-      v = fmaf(sw[hh][k + 3], a3, v);
+      const float a0 = __ldcg(ah + (size_t)k * d), a1 = __ldcg(ah + (size_t)(k + 1) * d);
+      const float a2 = __ldcg(ah + (size_t)(k + 2) * d), a3 = __ldcg(ah + (size_t)(k + 3) * d);
+      v = fmaf(swh[k], a0, v);
+      v = fmaf(swh[k + 1], a1, v);
+      v = fmaf(swh[k + 2], a2, v);
+      v = fmaf(swh[k + 3], a3, v);
     }
-    for (; k < s.splits; ++k) v = fmaf(sw[hh][k], ah[(size_t)k * d], v);
-    a[hh][i] = ok ? v * s_inv_l[hh] * sig[i] : 0.0f;
+    for (; k < s.splits; ++k) v = fmaf(swh[k], __ldcg(ah + (size_t)k * d), v);
+    a[hh * d + i] = ok ? v * s_inv_l[hh] * sig[i] : 0.0f;
   }
   __syncthreads();
-  // o_h = V_V a_h: warp w takes rows w, w + 8, ...; lane reads 16-byte pieces
-  // (columns 4 (lane + 32 c)), RB rows of loads in flight
+  // o_h = V_V a_h: warp w takes rows w, w + nwarp, ...; lane reads 16-byte pieces
   const float4* V4 = (const float4*)rv.V_f();
   const int q4 = d / 4;
-  constexpr int RB = MAXG >= 8 ? 4 : 8;
-  for (int j0 = warp; j0 < d; j0 += 8 * RB) {
-    float4 vv[RB][2];
+  for (int j = warp; j < d; j += nwarp) {
+    float4 vv[2];
 #pragma unroll
-    for (int r = 0; r < RB; ++r)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int j = j0 + 8 * r, col = lane + 32 * c;
-        vv[r][c] = (ok && j < d && col < q4) ? V4[(size_t)j * q4 + col] : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      const int j = j0 + 8 * r;
-      float o[MAXG];
-#pragma unroll
-      for (int hh = 0; hh < MAXG; ++hh) o[hh] = 0.0f;
+    for (int c = 0; c < 2; ++c) {
+      const int col = lane + 32 * c;
+      vv[c] = (ok && col < q4) ? V4[(size_t)j * q4 + col] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int hh = 0; hh < G; ++hh) {
+      float o = 0.0f;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const int col = lane + 32 * c;
         if (col < q4) {
-#pragma unroll
-          for (int hh = 0; hh < MAXG; ++hh) {
-            if (hh < G) {
-              const float4 av = *(const float4*)&a[hh][4 * col];
-              o[hh] = fmaf(vv[r][c].x, av.x, o[hh]);
-              o[hh] = fmaf(vv[r][c].y, av.y, o[hh]);
-              o[hh] = fmaf(vv[r][c].z, av.z, o[hh]);
-              o[hh] = fmaf(vv[r][c].w, av.w, o[hh]);
-            }
-          }
+          const float4 av = *(const float4*)&a[hh * d + 4 * col];
+          o = fmaf(vv[c].x, av.x, o);
+          o = fmaf(vv[c].y, av.y, o);
+          o = fmaf(vv[c].z, av.z, o);
+          o = fmaf(vv[c].w, av.w, o);
         }
       }
-#pragma unroll
-      for (int hh = 0; hh < MAXG; ++hh) {
-        if (hh < G) {
-          const float rs = warp_sum(o[hh]);
-          if (lane == 0 && j < d) out[(qh0 + hh) * d + j] = from_float<TO>(rs);
-        }
-      }
+      o = warp_sum(o);
+      if (lane == 0) store_out(out, out_dt, (qh0 + hh) * d + j, o);
     }
   }
+}
+
+// Combine as a kernel of its own (for the partial kernels that do not merge
+// their splits themselves): grid (n_kv, batch), 256 threads.
+__global__ void __launch_bounds__(256, 2) k_attn_combine(const uint8_t* __restrict__ recs_v, AttnShape s,
+                                                      const float* __restrict__ ws, void* out, int out_dt) {
+  extern __shared__ __align__(16) float cscr[];
+  combine_one(recs_v, s, ws, out, out_dt, blockIdx.x, blockIdx.y, cscr, threadIdx.x, blockDim.x);
+}
+
+// Shared-memory floats combine_one needs.
+__host__ __device__ inline size_t combine_scratch_floats(int d, int splits) {
+  return (size_t)16 * d + (size_t)16 * splits + 16;
 }
 
 }  // namespace sq

@@ -159,26 +159,33 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
 // Vectors per block for an append of nvec vectors per head: 1, 2, 4 or 8.
 inline int append_nv(int64_t nvec) { return nvec <= 1 ? 1 : (nvec <= 2 ? 2 : (nvec <= 4 ? 4 : 8)); }
 
+// Shared-memory bytes of append_body<T, NV>.
+__host__ __device__ constexpr size_t append_smem(int nv) {
+  return (size_t)nv * kMaxD * 8 + (size_t)nv * 256 * 8 + (size_t)kThreshTotal * 8 + (size_t)kLevelsTotal * 8 +
+         (size_t)nv * kMaxWords * 4 + (size_t)nv * 8 + (size_t)nv * 4 + 64;
+}
+
+// One append block: head h, vectors (batch, token) pairs grp * NV ...; sm is
+// append_smem(NV) bytes of shared memory; 256 threads.
 template <typename T, int NV>
-__global__ void __launch_bounds__(256) k_append(const uint8_t* __restrict__ recs, const T* __restrict__ x,
-                                                int batch, int n_heads, int d, int64_t n_tok,
-                                                const int32_t* __restrict__ start_pos, CacheArgs c,
-                                                uint32_t* __restrict__ flags) {
+__device__ void append_body(const uint8_t* __restrict__ recs, const T* __restrict__ x, int batch, int n_heads, int d,
+                            int64_t n_tok, const int32_t* __restrict__ start_pos, const CacheArgs& c,
+                            uint32_t* __restrict__ flags, int h, int64_t grp, uint8_t* sm) {
   static_assert(NV >= 1 && NV <= 8, "one warp per vector in the norm and QJL steps");
-  __shared__ double xs[NV][kMaxD];        // input, then the residual of the signal coordinates
-  __shared__ double ys[NV][256];          // partial sums of V^T x (parts of the j range)
-  __shared__ double th[kThreshTotal];
-  __shared__ double lv[kLevelsTotal];
-  __shared__ uint32_t wb[NV][kMaxWords];
-  __shared__ double s_inv[NV];
-  __shared__ int s_ok[NV];
-  const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  double (*xs)[kMaxD] = (double (*)[kMaxD])sm;                            // input, then the signal residual
+  double (*ys)[256] = (double (*)[256])(sm + (size_t)NV * kMaxD * 8);    // partial sums of V^T x
+  double* th = (double*)(sm + (size_t)NV * kMaxD * 8 + (size_t)NV * 256 * 8);
+  double* lv = th + kThreshTotal;
+  uint32_t (*wb)[kMaxWords] = (uint32_t (*)[kMaxWords])(lv + kLevelsTotal);
+  double* s_inv = (double*)(wb + NV);
+  int* s_ok = (int*)(s_inv + NV);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t total = (int64_t)batch * n_tok;
-  const int64_t v0 = (int64_t)blockIdx.y * NV;
+  const int64_t v0 = grp * NV;
   Rec rec = rec_at(recs, d, h);
   const RecHeader* hd = rec.hdr();
   if (!record_ok(hd, d) || hd->words != c.words || (hd->m > 0 && c.rnorm == nullptr)) {
-    if (tid == 0 && blockIdx.y == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
+    if (tid == 0 && grp == 0 && flags) atomicOr(flags, SQ_FLAG_RECORD);
     return;
   }
   const int m = hd->m, W = hd->words, cbits = hd->code_bits;
@@ -317,6 +324,15 @@ __global__ void __launch_bounds__(256) k_append(const uint8_t* __restrict__ recs
     const int64_t sp = start_pos ? (int64_t)start_pos[b] : 0;
     c.codes[rec_word0((size_t)b * n_heads + h, c.cap, W, sp + t) + (size_t)w * 32] = wb[v][w];
   }
+}
+
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) k_append(const uint8_t* __restrict__ recs, const T* __restrict__ x,
+                                                int batch, int n_heads, int d, int64_t n_tok,
+                                                const int32_t* __restrict__ start_pos, CacheArgs c,
+                                                uint32_t* __restrict__ flags) {
+  extern __shared__ __align__(16) uint8_t asmem[];
+  append_body<T, NV>(recs, x, batch, n_heads, d, n_tok, start_pos, c, flags, blockIdx.x, blockIdx.y, asmem);
 }
 
 // ---------------------------------------------------------------------------

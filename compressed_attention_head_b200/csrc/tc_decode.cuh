@@ -276,7 +276,7 @@ template <int D, int MG>
 __global__ void __launch_bounds__(Cfg<D>::NTH, 1)
 k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs_v, CacheArgs kc, CacheArgs vc,
             const int32_t* __restrict__ seq_lens, AttnShape s, float* __restrict__ ws,
-            float* __restrict__ scores_out, uint32_t* __restrict__ flags, int nrec) {
+            float* __restrict__ scores_out, uint32_t* __restrict__ flags, int nrec, void* out, int out_dt) {
   using C = Cfg<D>;
   using PL = Plan<D>;
   constexpr int NCH = C::NCH;
@@ -297,7 +297,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   float* ml_out = acc_out + (size_t)s.batch * s.n_q * s.splits * D;
   const bool ok = record_ok(hk, D) && record_ok(hv, D) && hk->words == kc.words && hv->words == vc.words &&
                   (hk->m == 0 || kc.rnorm != nullptr);
-  int64_t L = seq_lens[b];
+  int64_t L = attn_len(seq_lens, s, b);
   if (L < 0 || L > s.max_ctx || L > kc.cap) {
     if (tid == 0 && split == 0 && g == 0 && flags) atomicOr(flags, SQ_FLAG_SEQLEN);
     L = L < 0 ? 0 : (L > s.max_ctx ? s.max_ctx : L);
@@ -745,6 +745,22 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
       ml_out[base * 2 + 1] = lt;
     }
   }
+  // ---- the last block of (b, g) to finish merges the splits (every block
+  // publishes its partials, then counts itself; the counter was cleared by
+  // the prepare step of this call)
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    int last = 1;
+    if (s.splits > 1) {
+      uint32_t* cnt = attn_counters(ws, s) + (size_t)b * s.n_kv + g;
+      last = atomicAdd(cnt, 1u) == (uint32_t)(s.splits - 1);
+      if (last) *cnt = 0u;
+    }
+    s_last = last;
+  }
+  __syncthreads();
   // every copy and MMA a group's issuer started has completed before the block
   // frees its tensor memory and exits (on the normal path they have; after a
   // timed-out wait some may still run): bounded waits
@@ -761,6 +777,10 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     sm100::tmem_dealloc(tmem_base, 512);
   }
   if (tid == 0 && *abort_flag && err) atomicOr(err, SQ_FLAG_TIMEOUT);
+  if (s_last) {
+    __threadfence();
+    combine_one(recs_v, s, ws, out, out_dt, g, b, (float*)sm, tid, C::NTH);
+  }
 }
 
 }  // namespace td

@@ -74,6 +74,10 @@ _SIGNATURES = {
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
                                       _P, ctypes.c_int, ctypes.c_float, _P, ctypes.c_int, _P, _P,
                                       ctypes.c_size_t, _P, _P]),
+    "sq_decode_step": (ctypes.c_int, [_P, _P, ctypes.POINTER(sq_cache), ctypes.POINTER(sq_cache), _P, _P, _P,
+                                      ctypes.c_int, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int64, ctypes.c_float, _P, ctypes.c_int, _P, _P, ctypes.c_size_t, _P,
+                                      _P]),
     "sq_attn_decode_noalloc": (ctypes.c_int, [_P, _P, ctypes.POINTER(sq_cache), ctypes.POINTER(sq_cache), _P,
                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_int64, _P, ctypes.c_int, ctypes.c_float, _P, ctypes.c_int,
@@ -275,6 +279,17 @@ def sq_attn_decode(calib_k, calib_v, kc, vc, seq_lens, batch, n_q_heads, n_kv_he
                                 DTYPE_CODE[q.dtype], float(scale), _ptr(out), DTYPE_CODE[out.dtype],
                                 _ptr(scores_out), _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0,
                                 _ptr(flags), _stream(stream)), "sq_attn_decode")
+
+
+def sq_decode_step(calib_k, calib_v, kc, vc, k_new, v_new, q, pos, batch, n_q_heads, n_kv_heads, d, max_ctx, scale,
+                   out, scores_out=None, ws=None, flags=None, stream=None):
+    """Append the new token at pos[b] and attend over pos[b] + 1 tokens (see sq.h)."""
+    kcs, vcs = kc.struct(), vc.struct()
+    _check(lib().sq_decode_step(_ptr(calib_k), _ptr(calib_v), ctypes.byref(kcs), ctypes.byref(vcs), _ptr(k_new),
+                                _ptr(v_new), _ptr(q), DTYPE_CODE[q.dtype], _ptr(pos), batch, n_q_heads, n_kv_heads, d,
+                                max_ctx, float(scale), _ptr(out), DTYPE_CODE[out.dtype], _ptr(scores_out), _ptr(ws),
+                                ws.numel() * ws.element_size() if ws is not None else 0, _ptr(flags),
+                                _stream(stream)), "sq_decode_step")
 
 
 def sq_attn_decode_noalloc(calib_k, calib_v, kc, vc, seq_lens, batch, n_q_heads, n_kv_heads, d, max_ctx, q, scale,

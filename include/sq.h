@@ -391,6 +391,30 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
                          size_t ws_bytes, uint32_t* d_flags, sq_stream stream);
 
 /*
+ * One decode step (README "Headline Results": decode latency per step over the
+ * compressed cache): for every batch row b, the new token's keys k_new and
+ * values v_new of every KV head are compressed into the caches at position
+ * d_pos[b] (as sq_compress_kv with n_tok = 1 and start_pos = d_pos), then
+ * decode attention runs over d_pos[b] + 1 tokens, the new one included (as
+ * sq_attn_decode with seq_lens = d_pos + 1).
+ *  k_new, v_new  device, dtype [batch][n_kv_heads][1][d]; q device, dtype
+ *                [batch][n_q_heads][d] (one dtype for the three).
+ *  d_pos         device int32[batch]; d_pos[b] + 1 <= max_ctx and <= cap.
+ *  Other arguments, workspace (sq_attn_workspace of the same shape), results
+ *  and flags as sq_compress_kv and sq_attn_decode; max_ctx >= 1.
+ * On the tcgen05 path (head_dim 64/128/256, up to 16 query heads per KV head)
+ * the step is two launches: the appends share one with the query preparation,
+ * and the attention partials merge their splits themselves (the last block of
+ * each (row, KV head) to finish combines them); otherwise the step runs the
+ * appends, prepare, partials and combine as separate launches.
+ */
+sq_status sq_decode_step(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
+                         const void* k_new, const void* v_new, const void* q, sq_dtype dtype, const int32_t* d_pos,
+                         int batch, int n_q_heads, int n_kv_heads, int d, int64_t max_ctx, float scale, void* out,
+                         sq_dtype out_dtype, float* scores_out, void* ws, size_t ws_bytes, uint32_t* d_flags,
+                         sq_stream stream);
+
+/*
  * sq_attn_decode without a workspace argument, for callers that cannot
  * allocate device memory where they run decode attention: a serving loop whose
  * device memory is reserved once at start-up and may not grow, plug-ins with

@@ -160,8 +160,10 @@ class Workload:
 
 def make_workload(name_or_cfg, layer: int = 0, *, device="cpu", batch: int | None = None,
                   tokens: int | None = None, n_cal: int | None = None, data_stream: int = 0,
-                  with_calibration: bool = True) -> Workload:
-    """Draw one layer's inputs. ``tokens`` overrides the context length."""
+                  with_calibration: bool = True, calib_draw: int = 0) -> Workload:
+    """Draw one layer's inputs. ``tokens`` overrides the context length;
+    ``calib_draw`` selects an independent draw of the calibration vectors from
+    the same population (same head model, keys, values and queries)."""
     cfg = CONFIGS[name_or_cfg] if isinstance(name_or_cfg, str) else name_or_cfg
     bsz = cfg["batch"] if batch is None else batch
     t = cfg["ctx"] if tokens is None else tokens
@@ -184,8 +186,9 @@ def make_workload(name_or_cfg, layer: int = 0, *, device="cpu", batch: int | Non
         k[:, h] = draw(mk, bsz * t, gk, device, dt).reshape(bsz, t, d)
         v[:, h] = draw(mv, bsz * t, gv, device, dt).reshape(bsz, t, d)
         if with_calibration:
-            gck = _gen(device, cfg["seed"], _STREAMS["calib"], layer, h, 0)
-            gcv = _gen(device, cfg["seed"], _STREAMS["calib"], layer, h, 1)
+            extra = (calib_draw,) if calib_draw else ()
+            gck = _gen(device, cfg["seed"], _STREAMS["calib"], layer, h, 0, *extra)
+            gcv = _gen(device, cfg["seed"], _STREAMS["calib"], layer, h, 1, *extra)
             k_cal[h] = draw(mk, ncal, gck, device, dt)
             v_cal[h] = draw(mv, ncal, gcv, device, dt)
         gq = _gen(device, cfg["seed"], _STREAMS["query"], layer, h, data_stream)

@@ -225,3 +225,64 @@ def test_decode_gemma_bench_shape_sampled():
     layers x 8 KV heads folded (336 KV / 672 query heads, head_dim 256, bf16)."""
     _bench_shape_sampled("gemma9b_sweep", 42, 64, 4096,
                          rows=[(0, 0), (63, 671), (17, 300), (40, 5), (33, 450)], distinct_rows=2)
+
+
+@pytest.mark.parametrize("name,batch,ctx,heads", [("llama8b", 3, 700, 2), ("gemma9b_sweep", 2, 300, 2),
+                                                  ("qwen14b", 2, 1100, 1), ("tiny", 2, 100, 2)])
+def test_decode_step_appends_then_attends(name, batch, ctx, heads):
+    """sq_decode_step: each row's new token compressed at its own position and
+    attended together with the prefix before it. The new records equal the
+    oracle's, the outputs and scores equal the oracle's attention over the
+    resulting cache, and they equal the separate calls (sq_compress_kv of one
+    token, then sq_attn_decode) on a second cache. Covers the two-launch
+    tcgen05 step (head_dim 128 and 256) and the separate-launch path (head_dim 32)."""
+    from gpu_helpers import compare_compressed
+    w = make_workload(name, batch=batch, tokens=ctx)
+    cfg = w.cfg
+    g = cfg["n_q"] // cfg["n_kv"]
+    nkv = min(heads, cfg["n_kv"])
+    nq, d = nkv * g, cfg["d"]
+    ck = calibrate_oracle(w.k_cal[:nkv], cfg["bits_k"], True)
+    cv = calibrate_oracle(w.v_cal[:nkv], cfg["bits_v"], False)
+    rk, rv = records_to_device(ck), records_to_device(cv)
+    cap = ctx + 32
+    caches = []
+    for _ in range(2):
+        kc = sq.alloc_cache(batch, nkv, cap, ck[0].words, True)
+        vc = sq.alloc_cache(batch, nkv, cap, cv[0].words, False)
+        sq.sq_compress_kv(rk, rv, w.k[:, :nkv, :ctx - 1].contiguous().cuda(), w.v[:, :nkv, :ctx - 1].contiguous().cuda(),
+                          batch, nkv, d, ctx - 1, None, kc, vc)
+        caches.append((kc, vc))
+    pos_l = [ctx - 1 - (37 * b) % 61 for b in range(batch)]
+    pos = torch.tensor(pos_l, dtype=torch.int32, device="cuda")
+    k_new = w.k[:, :nkv, ctx - 1:].contiguous().cuda()
+    v_new = w.v[:, :nkv, ctx - 1:].contiguous().cuda()
+    q = w.q[:, :nq].contiguous().cuda()
+    max_ctx = ctx
+    ws = torch.empty(sq.sq_attn_workspace(batch, nq, nkv, d, max_ctx), dtype=torch.uint8, device="cuda")
+    outs, scs = [], []
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    (kc, vc), (kc2, vc2) = caches
+    out = torch.empty(batch, nq, d, device="cuda")
+    sc = torch.full((batch, nq, max_ctx), float("nan"), device="cuda")
+    sq.sq_decode_step(rk, rv, kc, vc, k_new, v_new, q, pos, batch, nq, nkv, d, max_ctx, 0.0, out, sc, ws, flags)
+    out2 = torch.empty_like(out)
+    sc2 = torch.full_like(sc, float("nan"))
+    sq.sq_compress_kv(rk, rv, k_new, v_new, batch, nkv, d, 1, pos, kc2, vc2, flags)
+    sq.sq_attn_decode(rk, rv, kc2, vc2, pos + 1, batch, nq, nkv, d, max_ctx, q, 0.0, out2, sc2, ws, flags)
+    torch.cuda.synchronize()
+    assert flags.item() == 0
+    assert np.array_equal(kc.words_u32(), kc2.words_u32()) and np.array_equal(vc.words_u32(), vc2.words_u32())
+    kw, vw = kc.words_u32(), vc.words_u32()
+    for b, p in enumerate(pos_l):
+        for h in range(nkv):
+            compare_compressed(kw[b, h, p:p + 1], kc.norm[b, h, p:p + 1].cpu().numpy(),
+                               kc.rnorm[b, h, p:p + 1].cpu().numpy(), k_new[b, h].double().cpu().numpy(), ck[h])
+            compare_compressed(vw[b, h, p:p + 1], vc.norm[b, h, p:p + 1].cpu().numpy(), None,
+                               v_new[b, h].double().cpu().numpy(), cv[h])
+    lens = [p + 1 for p in pos_l]
+    ref_out, ref_sc = oattn.attn_decode(q.double().cpu().numpy(), kw, kc.norm.cpu().numpy(), kc.rnorm.cpu().numpy(),
+                                        vw, vc.norm.cpu().numpy(), ck, cv, lens, 1.0 / math.sqrt(d))
+    o, s = out.cpu().numpy(), sc.cpu().numpy()
+    _assert_close(o, s, ref_out, ref_sc, lens)
+    np.testing.assert_allclose(o, out2.cpu().numpy(), rtol=1e-5, atol=1e-6)

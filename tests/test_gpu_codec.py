@@ -29,7 +29,7 @@ from compressed_attention_head_b200 import sq  # noqa: E402
 def _case(name, batch=2, tokens=333, heads=None, bits_k=None, bits_v=None, qjl=True, normalize=True):
     w = make_workload(name, batch=batch, tokens=tokens)
     cfg = w.cfg
-    nh = heads or cfg["n_kv"]
+    nh = min(heads, cfg["n_kv"]) if heads else cfg["n_kv"]
     bk = cfg["bits_k"] if bits_k is None else bits_k
     bv = cfg["bits_v"] if bits_v is None else bits_v
     ck = calibrate_oracle(w.k_cal[:nh], bk, True, qjl=qjl, normalize=normalize)
