@@ -1,5 +1,6 @@
 // libsq host entry points: argument checks, per-device table upload, launches.
 // The public contract (arguments, layouts, ownership, errors) is in include/sq.h.
+#include <cstdio>
 #include <mutex>
 
 #include "sq_common.cuh"
@@ -46,7 +47,13 @@ bool supported_d(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 bool valid_dtype(int t) { return t == SQ_F32 || t == SQ_F16 || t == SQ_BF16; }
 
-sq_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA; }
+// The name of the last CUDA error a call of this thread ran into (for sq_last_error).
+thread_local char g_last_err[160] = "none";
+sq_status cuda_ok(cudaError_t e) {
+  if (e == cudaSuccess) return SQ_OK;
+  snprintf(g_last_err, sizeof(g_last_err), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return SQ_ERR_CUDA;
+}
 
 // Cell tables of the tensor-core compress for widths 4..8 (see tc_compress.cuh)
 // from the float32 positive thresholds T_1 < ... < T_n of each width; false if
@@ -84,8 +91,9 @@ bool build_cell_tables(const double* th, float4* q, uint8_t* cell, tcc::QuantCon
 }
 
 // Dynamic shared memory the tcgen05 decode kernel may take: 227 KB per block
-// minus its static width-3 table (8 KB).
-constexpr int kTdSmemLimit = 232448 - 8192;
+// minus its static shared memory (the 8 KB width-3 table, a flag, and the
+// padding that aligns the dynamic part to 1 KB), with 1 KB to spare.
+constexpr int kTdSmemLimit = 232448 - 9216 - 1024;
 
 // Uploads the Lloyd-Max tables to the current device once.
 sq_status ensure_init(int* dev_out = nullptr) {
@@ -150,7 +158,7 @@ sq_status ensure_init(int* dev_out = nullptr) {
     SQ_SP_ATTR(float); SQ_SP_ATTR(__half); SQ_SP_ATTR(__nv_bfloat16);
 #undef SQ_SP_ATTR
   }
-  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
   int sms = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   g_sms[dev] = sms > 0 ? sms : 148;
@@ -307,7 +315,7 @@ sq_status launch_compress_tc(const void* recs, const void* x, int batch, int n_h
   P.n_tiles = (int64_t)batch * n_heads * P.tiles_per_row;
   int64_t grid = P.n_tiles < g_sms[dev] ? P.n_tiles : g_sms[dev];
   tcc::k_compress_tc<<<(unsigned)grid, tcc::NUM_THREADS, tcc::SMEM_BYTES, st>>>(map, P, g_kq);
-  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
   // Heads with more than tcc::MSIG QJL dimensions: the reference kernel, one
   // block per (batch, head); every other block returns at once.
   dim3 g2(1, n_heads, batch);
@@ -354,6 +362,8 @@ using namespace sq;
 extern "C" {
 
 int sq_abi_version(void) { return SQ_ABI_VERSION; }
+
+const char* sq_last_error(void) { return g_last_err; }
 
 const char* sq_status_str(sq_status s) {
   switch (s) {
@@ -428,14 +438,14 @@ sq_status sq_calibrate(const sq_calib_params* p, const void* x, sq_dtype dtype, 
     case SQ_F16: k_second_moment<__half><<<g1, b1, 0, st>>>((const __half*)x, d, n_tokens, stride_head, stride_tok, cov); break;
     default: k_second_moment<__nv_bfloat16><<<g1, b1, 0, st>>>((const __nv_bfloat16*)x, d, n_tokens, stride_head, stride_tok, cov); break;
   }
-  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
   if (p->rotation == 1) {
     k_random_basis<<<p->n_heads, 256, 0, st>>>(cov, vt, d, p->seed, calib_out, d_status);
   } else {
     size_t jsm = d <= 128 ? (size_t)8 * d * d : 0;
     k_jacobi<<<p->n_heads, 256, jsm, st>>>(cov, vt, d, p->max_sweeps, p->tol, calib_out, d_status);
   }
-  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
   FinalizeArgs fa{B, p->is_key, p->qjl, p->normalize, p->d_eff_override, p->max_bits, p->seed, p->avg_bits,
                   p->cumvar, p->rotation};
   k_finalize<<<p->n_heads, 256, 0, st>>>(calib_out, d, fa, d_status);
@@ -691,7 +701,7 @@ sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* 
     dim3 gp(n_kv_heads, (unsigned)((batch + prow - 1) / prow));
     k_attn_prepare<TQ><<<gp, 256, prep_smem(d), st>>>(rk, (const TQ*)q, sh, sc, w, d_flags);
   }
-  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
   // ---- launch 2: partials (the tcgen05 kernel merges the splits itself)
   dim3 gpart(sh.splits, n_kv_heads, batch);
   size_t smem = attn_partial_smem(d, sh.group, kc->words, vc->words);
@@ -732,7 +742,7 @@ sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* 
     k_attn_partial<8><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags);
   else
     k_attn_partial<16><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags);
-  if (cudaGetLastError() != cudaSuccess) return SQ_ERR_CUDA;
+  if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
   // ---- launch 3: combine
   dim3 gc(n_kv_heads, batch);
   k_attn_combine<<<gc, 256, combine_scratch_floats(d, sh.splits) * 4, st>>>(rv, sh, w, out, (int)out_dtype);

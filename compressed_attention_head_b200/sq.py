@@ -26,7 +26,8 @@ DTYPE_CODE = {torch.float32: SQ_F32, torch.float16: SQ_F16, torch.bfloat16: SQ_B
 
 class SqError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what}: {sq_status_str(status)} ({status})")
+        detail = f" [{lib().sq_last_error().decode()}]" if status == SQ_ERR_CUDA else ""
+        super().__init__(f"{what}: {sq_status_str(status)} ({status}){detail}")
         self.status = status
 
 
@@ -49,6 +50,7 @@ _P = ctypes.c_void_p
 _SIGNATURES = {
     "sq_abi_version": (ctypes.c_int, []),
     "sq_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+    "sq_last_error": (ctypes.c_char_p, []),
     "sq_calib_bytes": (ctypes.c_size_t, [ctypes.c_int]),
     "sq_record_words": (ctypes.c_int, [ctypes.POINTER(sq_calib_params)]),
     "sq_codebook": (ctypes.c_int, [ctypes.c_int, _P, _P, _P]),

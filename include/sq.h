@@ -197,6 +197,10 @@ size_t sq_calib_bytes(int d);
 /* ABI version (SQ_ABI_VERSION). */
 int sq_abi_version(void);
 
+/* Name and description of the last CUDA error a call of the calling thread
+ * returned SQ_ERR_CUDA for ("none" before any). Static per thread; never NULL. */
+const char* sq_last_error(void);
+
 /* Static string naming a status. Never NULL. */
 const char* sq_status_str(sq_status s);
 
