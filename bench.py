@@ -130,6 +130,7 @@ def rep_divisor(n: int, want: int) -> int:
 KERNEL_SOURCES = {
     "k_compress_tc": ["tc_compress.cuh", "sm100.cuh", "sq_common.cuh"],
     "k_attn_partial_tc": ["fast_attn.cuh", "attention.cuh", "sq_common.cuh"],
+    "k_decode_tc": ["tc_decode.cuh", "attention.cuh", "sm100.cuh", "sq_common.cuh"],
 }
 
 
@@ -587,19 +588,35 @@ def measure_decode(cfg, args, world, dev):
 
     def step(ev):
         if ev: ev[0].record()
-        sq.sq_compress_kv(rk, rv, k_new, v_new, B, H, d, 1, posT, kc, vc, flags)
-        if ev: ev[1].record()
-        sq.sq_attn_decode(rk, rv, kc, vc, lens, B, HQ, H, d, max_ctx, q, 0.0, out, None, aws, flags)
+        if args.separate:
+            sq.sq_compress_kv(rk, rv, k_new, v_new, B, H, d, 1, posT, kc, vc, flags)
+            if ev: ev[1].record()
+            sq.sq_attn_decode(rk, rv, kc, vc, lens, B, HQ, H, d, max_ctx, q, 0.0, out, None, aws, flags)
+        else:
+            # the fused step: appends + query preparation in one launch, partials with the
+            # last-block combine in the other (two launches on the tcgen05 path)
+            sq.sq_decode_step(rk, rv, kc, vc, k_new, v_new, q, posT, B, HQ, H, d, max_ctx, 0.0, out, None, aws, flags)
+            if ev: ev[1].record()
         if ev: ev[2].record()
 
     eager, marks = _time_loop(step, args.steps, args.warmup, world, dev, 3)
     graph = None if args.no_graph else _time_graph(step, args.steps, args.warmup, world, dev)
-    app_ms, att_ms = _mean_ms(marks, 0, 1), _mean_ms(marks, 1, 2)
     rec_k, rec_v = record_bytes(words_k, qjl), record_bytes(words_v, False)
     attn_bytes = B * H * (T + 1) * (rec_k + rec_v)
+    td = args.attn_path == 0 and cfg["d"] in (64, 128, 256) and cfg["n_q"] // cfg["n_kv"] <= 16
+    if args.separate:
+        app_ms, att_ms = _mean_ms(marks, 0, 1), _mean_ms(marks, 1, 2)
+        launches = 2 + (2 if td else 3)
+        kernel = "sq_attn_decode (prepare + partials" + (" merging their splits)" if td else " + combine)")
+    else:
+        # one call: its two launches are timed together (the step's whole time)
+        app_ms, att_ms = 0.0, _mean_ms(marks, 0, 1)
+        launches = 2 if td else 5
+        kernel = ("sq_decode_step (append + prepare launch, partials launch merging their splits)" if td
+                  else "sq_decode_step (appends, prepare, partials, combine)")
     res = dict(cfg=cfg, step_s=graph or eager, eager_s=eager, graph_s=graph, calib_ms=calib_ms, n_bad=n_bad,
                calib_heads=2 * nkv, app_ms=app_ms, att_ms=att_ms, attn_bytes=attn_bytes, rec_k=rec_k,
-               rec_v=rec_v, tokens=step_tokens(cfg), launches=2 + 3, flags=flags, base_rows=b0,
+               rec_v=rec_v, tokens=step_tokens(cfg), launches=launches, kernel=kernel, flags=flags, base_rows=b0,
                cache_bytes=sum(t.numel() * t.element_size() for t in (kc.codes, kc.norm, vc.codes, vc.norm)
                                + ((kc.rnorm,) if kc.rnorm is not None else ())))
     if not args.no_e2e:
@@ -610,8 +627,12 @@ def measure_decode(cfg, args, world, dev):
             k_new.copy_(hkn, non_blocking=True)
             v_new.copy_(hvn, non_blocking=True)
             q.copy_(hq, non_blocking=True)
-            sq.sq_compress_kv(rk, rv, k_new, v_new, B, H, d, 1, posT, kc, vc, flags)
-            sq.sq_attn_decode(rk, rv, kc, vc, lens, B, HQ, H, d, max_ctx, q, 0.0, out, None, aws, flags)
+            if args.separate:
+                sq.sq_compress_kv(rk, rv, k_new, v_new, B, H, d, 1, posT, kc, vc, flags)
+                sq.sq_attn_decode(rk, rv, kc, vc, lens, B, HQ, H, d, max_ctx, q, 0.0, out, None, aws, flags)
+            else:
+                sq.sq_decode_step(rk, rv, kc, vc, k_new, v_new, q, posT, B, HQ, H, d, max_ctx, 0.0, out, None, aws,
+                                  flags)
             hout.copy_(out, non_blocking=True)
 
         t_e2e, _ = _time_loop(e2e_step, args.steps, args.warmup, world, dev, 1)
@@ -655,7 +676,8 @@ def run_gpu(args, rank, world, local_rank):
     flag_val = int(main["flags"].item()) | (int(comp["flags"].item()) if comp else 0)
     value = main["tokens"] * world / main["step_s"]
     B, T = cfg["batch"], cfg["ctx"]
-    att = _roofline("sq_attn_decode (prepare + partials + combine)", "k_attn_partial_tc", main["attn_bytes"],
+    att = _roofline(main.get("kernel", "sq_attn_decode (prepare + partials + combine)"),
+                    "k_decode_tc" if args.attn_path == 0 else "k_attn_partial_tc", main["attn_bytes"],
                     main["att_ms"], B * cfg["layers"] * cfg["n_kv"] * (T + 1), peak, peak_kind)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -732,6 +754,8 @@ def main():
                     help="headline (Gemma-shaped decode + Llama-shaped prompt compress) or a workload name")
     ap.add_argument("--bits", type=float, default=None, help="bits per coordinate for K and V (Gemma sweep)")
     ap.add_argument("--no-qjl", action="store_true")
+    ap.add_argument("--separate", action="store_true",
+                    help="decode step as separate calls (compress one token, then attention) instead of sq_decode_step")
     ap.add_argument("--attn-path", type=int, default=0,
                     help="attention partial kernel: 0 tcgen05 (default), 1 SIMT, 2 mma.sync (comparison runs)")
     ap.add_argument("--base-rows", type=int, default=2, help="distinct batch rows of a decode cache")

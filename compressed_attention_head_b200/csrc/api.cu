@@ -649,21 +649,37 @@ bool attn_args_ok(const void* calib_k, const void* calib_v, const sq_cache* kc, 
 // d_lens[b] and attended (len_offset 1). The tcgen05 path takes two launches
 // (append + prepare in one; partials with the last-block combine); the
 // others take prepare, partials and combine (and the appends before them).
+// Query positions per kernel row of a causal prefill with qg query heads per
+// KV head: as many as fit 16 MMA columns.
+int prefill_cols(int qg) { return qg >= 16 ? 1 : 16 / qg; }
+
 template <typename TQ>
 sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
                       const int32_t* d_lens, int len_offset, int batch, int n_q_heads, int n_kv_heads, int d,
                       int64_t max_ctx, const void* q, float scale, void* out, sq_dtype out_dtype, float* scores_out,
-                      void* ws, uint32_t* d_flags, cudaStream_t st, const void* k_new, const void* v_new, int dev) {
-  const int group = n_q_heads / n_kv_heads;
+                      void* ws, uint32_t* d_flags, cudaStream_t st, const void* k_new, const void* v_new, int dev,
+                      int n_qtok = 0) {
+  // causal prefill when n_qtok > 0: kernel rows (batch row, block of positions), columns (position, head)
+  const int qg = n_q_heads / n_kv_heads;
+  const bool causal = n_qtok > 0;
+  const int pcols = causal ? prefill_cols(qg) : 1;
+  const int ncb = causal ? (n_qtok + pcols - 1) / pcols : 1;
+  const int group = qg * pcols;
+  const int rows = batch * ncb;
   const int nrec = td_nrec(d, kc->words, vc->words);
   const bool use_td = g_attn_path == 0 && (d == 64 || d == 128 || d == 256) && group <= 16 && nrec > 0;
   AttnShape sh;
-  sh.batch = batch;
-  sh.n_q = n_q_heads;
+  sh.batch = rows;
+  sh.n_q = n_kv_heads * group;
   sh.n_kv = n_kv_heads;
   sh.group = group;
   sh.d = d;
-  sh.splits = use_td ? attn_splits_td(batch, n_kv_heads, d, max_ctx) : attn_splits(batch, n_kv_heads, d, max_ctx);
+  sh.causal = causal ? 1 : 0;
+  sh.pcols = pcols;
+  sh.ncb = ncb;
+  sh.qg = qg;
+  sh.n_qtok = n_qtok;
+  sh.splits = use_td ? attn_splits_td(rows, n_kv_heads, d, max_ctx) : attn_splits(rows, n_kv_heads, d, max_ctx);
   sh.max_ctx = max_ctx;
   sh.len_offset = len_offset;
   int64_t per = (max_ctx + sh.splits - 1) / sh.splits;
@@ -675,7 +691,7 @@ sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* 
   const uint8_t* rv = (const uint8_t*)calib_v;
   CacheArgs ka = cache_args(kc), va = cache_args(vc);
   const int prow = prep_rows(group);
-  const unsigned n_prep = (unsigned)(n_kv_heads * ((batch + prow - 1) / prow));
+  const unsigned n_prep = (unsigned)(n_kv_heads * ((rows + prow - 1) / prow));
   // ---- launch 1: prepare (with the appends of a decode step)
   if (k_new && use_td) {
     const int nv = append_nv(batch);
@@ -698,15 +714,16 @@ sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* 
       if (s == SQ_OK) s = launch_compress<TQ>(calib_v, v_new, batch, n_kv_heads, d, 1, d_lens, vc, d_flags, st);
       if (s != SQ_OK) return s;
     }
-    dim3 gp(n_kv_heads, (unsigned)((batch + prow - 1) / prow));
+    dim3 gp(n_kv_heads, (unsigned)((rows + prow - 1) / prow));
     k_attn_prepare<TQ><<<gp, 256, prep_smem(d), st>>>(rk, (const TQ*)q, sh, sc, w, d_flags);
   }
   if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
   // ---- launch 2: partials (the tcgen05 kernel merges the splits itself)
-  dim3 gpart(sh.splits, n_kv_heads, batch);
+  if (rows > 65535) return SQ_ERR_ARG;
+  dim3 gpart(sh.splits, n_kv_heads, rows);
   size_t smem = attn_partial_smem(d, sh.group, kc->words, vc->words);
-  const bool fast = g_attn_path != 1 && sh.group <= 8 && (d == 64 || d == 128 || d == 256) && kc->words <= d / 8 &&
-                    vc->words <= d / 8;
+  const bool fast = !causal && g_attn_path != 1 && sh.group <= 8 && (d == 64 || d == 128 || d == 256) &&
+                    kc->words <= d / 8 && vc->words <= d / 8;
   if (use_td) {
     const int MGv = sh.group <= 2 ? 2 : (sh.group <= 4 ? 4 : (sh.group <= 8 ? 8 : 16));
 #define SQ_TD_LAUNCH(DD, MG)                                                                                  \
@@ -744,7 +761,7 @@ sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* 
     k_attn_partial<16><<<gpart, 128, smem, st>>>(rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags);
   if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
   // ---- launch 3: combine
-  dim3 gc(n_kv_heads, batch);
+  dim3 gc(n_kv_heads, rows);
   k_attn_combine<<<gc, 256, combine_scratch_floats(d, sh.splits) * 4, st>>>(rv, sh, w, out, (int)out_dtype);
   (void)dev;
   return cuda_ok(cudaGetLastError());
@@ -754,18 +771,20 @@ sq_status attn_dispatch(const void* calib_k, const void* calib_v, const sq_cache
                         const int32_t* d_lens, int len_offset, int batch, int n_q_heads, int n_kv_heads, int d,
                         int64_t max_ctx, const void* q, sq_dtype dtype, float scale, void* out, sq_dtype out_dtype,
                         float* scores_out, void* ws, uint32_t* d_flags, cudaStream_t st, const void* k_new,
-                        const void* v_new, int dev) {
+                        const void* v_new, int dev, int n_qtok = 0) {
   switch (dtype) {
     case SQ_F32:
       return attn_launch<float>(calib_k, calib_v, kc, vc, d_lens, len_offset, batch, n_q_heads, n_kv_heads, d,
-                                max_ctx, q, scale, out, out_dtype, scores_out, ws, d_flags, st, k_new, v_new, dev);
+                                max_ctx, q, scale, out, out_dtype, scores_out, ws, d_flags, st, k_new, v_new, dev,
+                                n_qtok);
     case SQ_F16:
       return attn_launch<__half>(calib_k, calib_v, kc, vc, d_lens, len_offset, batch, n_q_heads, n_kv_heads, d,
-                                 max_ctx, q, scale, out, out_dtype, scores_out, ws, d_flags, st, k_new, v_new, dev);
+                                 max_ctx, q, scale, out, out_dtype, scores_out, ws, d_flags, st, k_new, v_new, dev,
+                                 n_qtok);
     default:
       return attn_launch<__nv_bfloat16>(calib_k, calib_v, kc, vc, d_lens, len_offset, batch, n_q_heads, n_kv_heads,
                                         d, max_ctx, q, scale, out, out_dtype, scores_out, ws, d_flags, st, k_new,
-                                        v_new, dev);
+                                        v_new, dev, n_qtok);
   }
 }
 
@@ -805,6 +824,38 @@ sq_status sq_decode_step(const void* calib_k, const void* calib_v, const sq_cach
   if (s != SQ_OK) return s;
   return attn_dispatch(calib_k, calib_v, kc, vc, d_pos, 1, batch, n_q_heads, n_kv_heads, d, max_ctx, q, dtype, scale,
                        out, out_dtype, scores_out, ws, d_flags, (cudaStream_t)stream, k_new, v_new, dev);
+}
+
+size_t sq_attn_prefill_workspace(int batch, int n_q_heads, int n_kv_heads, int d, int64_t n_qtok, int64_t max_ctx) {
+  if (batch < 1 || n_q_heads < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads || !supported_d(d) || n_qtok < 1 ||
+      max_ctx < 1)
+    return 0;
+  const int qg = n_q_heads / n_kv_heads;
+  const int pcols = prefill_cols(qg);
+  const int64_t rows = (int64_t)batch * ((n_qtok + pcols - 1) / pcols);
+  if (rows > 65535) return 0;
+  const int s1 = attn_splits((int)rows, n_kv_heads, d, max_ctx);
+  const int s2 = attn_splits_td((int)rows, n_kv_heads, d, max_ctx);
+  return attn_ws_bytes((int)rows, n_kv_heads * qg * pcols, n_kv_heads, d, s1 > s2 ? s1 : s2);
+}
+
+sq_status sq_attn_prefill(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
+                          const int32_t* d_start, int batch, int n_q_heads, int n_kv_heads, int d, int64_t n_qtok,
+                          int64_t max_ctx, const void* q, sq_dtype q_dtype, float scale, void* out, sq_dtype out_dtype,
+                          void* ws, size_t ws_bytes, uint32_t* d_flags, sq_stream stream) {
+  if (!supported_d(d) || !valid_dtype(q_dtype) || !valid_dtype(out_dtype)) return SQ_ERR_UNSUPPORTED;
+  if (n_qtok < 1 || n_qtok > 0x7fffffff || max_ctx < n_qtok ||
+      !attn_args_ok(calib_k, calib_v, kc, vc, d_start, batch, n_q_heads, n_kv_heads, q, out, nullptr, ws))
+    return SQ_ERR_ARG;
+  const size_t need = sq_attn_prefill_workspace(batch, n_q_heads, n_kv_heads, d, n_qtok, max_ctx);
+  if (need == 0) return SQ_ERR_ARG;
+  if (ws_bytes < need) return SQ_ERR_WORKSPACE;
+  int dev = 0;
+  sq_status s = ensure_init(&dev);
+  if (s != SQ_OK) return s;
+  return attn_dispatch(calib_k, calib_v, kc, vc, d_start, 0, batch, n_q_heads, n_kv_heads, d, max_ctx, q, q_dtype,
+                       scale, out, out_dtype, nullptr, ws, d_flags, (cudaStream_t)stream, nullptr, nullptr, dev,
+                       (int)n_qtok);
 }
 
 // ---------------------------------------------------------------------------

@@ -20,11 +20,37 @@ namespace sq {
 constexpr int kAttnTile = 128;     // tokens per tile of the partial kernel
 constexpr int kAttnMaxG = 16;      // query heads per KV head
 
+// Shape of one attention call as the kernels see it. Decode: one query per
+// (batch row, query head); the kernels' "rows" are batch rows and their
+// "columns" the G query heads of a KV head. Prefill (causal): the query tokens
+// of a row are cut into blocks of pcols positions, and a kernel row is
+// (batch row, block) while its columns are (position in the block, query
+// head): group = pcols * qg columns per KV head (at most 16).
 struct AttnShape {
-  int batch, n_q, n_kv, group, d, splits;
+  int batch, n_q, n_kv, group, d, splits;   // kernel rows, kernel columns in all, KV heads, columns per KV head
   int64_t max_ctx, chunk;
-  int len_offset;     // attended length = seq_lens[b] + len_offset (1 when seq_lens holds the new token's position)
+  int len_offset;     // decode: attended length = seq_lens[b] + len_offset (1 when seq_lens holds the new token's position)
+  int causal;         // prefill: seq_lens[b] is the position of row b's first query token
+  int pcols;          // prefill: query positions per block (1 for decode)
+  int ncb;            // prefill: blocks per batch row (1 for decode)
+  int qg;             // query heads per KV head (= group for decode)
+  int n_qtok;         // prefill: query tokens per batch row
 };
+
+// Cache row of kernel row r (batch row).
+__host__ __device__ __forceinline__ int attn_cache_row(const AttnShape& s, int r) { return s.causal ? r / s.ncb : r; }
+// Query element (kernel row r, KV head g, column c, coordinate 0) of q:
+// decode [batch][n_q][d], prefill [batch][n_kv qg][n_qtok][d].
+__host__ __device__ __forceinline__ size_t attn_q_index(const AttnShape& s, int r, int g, int c) {
+  if (!s.causal) return ((size_t)r * s.n_q + (size_t)g * s.group + c) * s.d;
+  const int b = r / s.ncb, t = (r % s.ncb) * s.pcols + c / s.qg, hh = c % s.qg;
+  return (((size_t)b * s.n_kv * s.qg + (size_t)g * s.qg + hh) * s.n_qtok + t) * s.d;
+}
+// Whether column c of kernel row r is a query at all (the last block of a
+// prefill row may be partial).
+__host__ __device__ __forceinline__ bool attn_col_live(const AttnShape& s, int r, int c) {
+  return !s.causal || ((r % s.ncb) * s.pcols + c / s.qg) < s.n_qtok;
+}
 
 // Workspace layout (floats): w[batch][n_q][d], u[batch][n_q][d],
 // acc[batch][n_q][splits][d], ml[batch][n_q][splits][2], then one uint32
@@ -39,9 +65,20 @@ __device__ __forceinline__ uint32_t* attn_counters(float* ws, const AttnShape& s
   return (uint32_t*)(ws + attn_ws_floats(s.batch, s.n_q, s.d, s.splits));
 }
 
-// Attended length of row b (the new token included when len_offset is 1).
-__device__ __forceinline__ int64_t attn_len(const int32_t* seq_lens, const AttnShape& s, int b) {
-  return (int64_t)seq_lens[b] + s.len_offset;
+// Attended length of kernel row r: decode, seq_lens[r] (+ 1 with the new
+// token); prefill, the last query position of the row's block + 1.
+__device__ __forceinline__ int64_t attn_len(const int32_t* seq_lens, const AttnShape& s, int r) {
+  if (!s.causal) return (int64_t)seq_lens[r] + s.len_offset;
+  const int b = r / s.ncb, cb = r % s.ncb;
+  const int last = min((cb + 1) * s.pcols, s.n_qtok);      // exclusive
+  return (int64_t)seq_lens[b] + last;
+}
+// Causal bound of column c of kernel row r: keys at positions <= this are
+// attended (no bound for decode).
+__device__ __forceinline__ int64_t attn_col_pos(const int32_t* seq_lens, const AttnShape& s, int r, int c) {
+  if (!s.causal) return INT64_MAX;
+  const int b = r / s.ncb, cb = r % s.ncb;
+  return (int64_t)seq_lens[b] + cb * s.pcols + c / s.qg;
 }
 
 // ---------------------------------------------------------------------------
@@ -74,7 +111,7 @@ __device__ void prepare_body(const uint8_t* __restrict__ recs_k, const TQ* __res
   for (int e = tid; e < nv * d; e += nth) {
     const int v = e / d, j = e % d;
     const int r = v / G, hh = v % G;
-    qs[e] = to_float<TQ>(q[((size_t)(b0 + r) * s.n_q + (size_t)g * G + hh) * d + j]);
+    qs[e] = attn_col_live(s, b0 + r, hh) ? to_float<TQ>(q[attn_q_index(s, b0 + r, g, hh) + j]) : 0.0f;
   }
   __syncthreads();
   const float* V = rec.V_f();
@@ -219,7 +256,7 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
   for (int hh = 0; hh < MAXG; ++hh) oacc[hh][0] = oacc[hh][1] = 0.0f;
   __syncthreads();
 
-  const size_t row = (size_t)b * s.n_kv + g;
+  const size_t row = (size_t)attn_cache_row(s, b) * s.n_kv + g;
   const uint32_t* kcodes = kc.codes + row * kc.cap * wk;
   const uint32_t* vcodes = vc.codes + row * vc.cap * wv;
   for (int64_t t0 = t_lo; t0 < t_hi; t0 += kAttnTile) {
@@ -270,9 +307,10 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
         }
       }
       for (int hh = 0; hh < G; ++hh) {
-        float sv = tid < nt ? kn[tid] * a[hh] : -INFINITY;
+        const bool vis = tid < nt && t0 + tid <= attn_col_pos(seq_lens, s, b, hh);
+        float sv = vis ? kn[tid] * a[hh] : -INFINITY;
         sc[hh * kAttnTile + tid] = sv;
-        if (scores_out && tid < nt) scores_out[((size_t)b * s.n_q + g * G + hh) * s.max_ctx + t0 + tid] = sv;
+        if (scores_out && vis) scores_out[((size_t)b * s.n_q + g * G + hh) * s.max_ctx + t0 + tid] = sv;
       }
     }
     __syncthreads();
@@ -290,7 +328,8 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
     }
     __syncthreads();
     for (int hh = 0; hh < G; ++hh) {
-      float pv = tid < nt ? __expf(sc[hh * kAttnTile + tid] - mrun[hh]) : 0.0f;
+      const float svv = sc[hh * kAttnTile + tid];
+      float pv = (tid < nt && svv != -INFINITY) ? __expf(svv - mrun[hh]) : 0.0f;
       float ps = warp_sum(pv);
       sc[hh * kAttnTile + tid] = pv * (tid < nt ? vn[tid] : 0.0f);
       if ((tid & 31) == 0) red[hh * 4 + (tid >> 5)] = ps;
@@ -417,7 +456,7 @@ __device__ void combine_one(const uint8_t* __restrict__ recs_v, const AttnShape&
         }
       }
       o = warp_sum(o);
-      if (lane == 0) store_out(out, out_dt, (qh0 + hh) * d + j, o);
+      if (lane == 0 && attn_col_live(s, b, hh)) store_out(out, out_dt, attn_q_index(s, b, g, hh) + j, o);
     }
   }
 }

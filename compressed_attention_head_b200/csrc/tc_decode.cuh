@@ -422,12 +422,14 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
 
   // ---- per-group state
   float mref[MG], lpart[MG];
+  int cpos[MG];        // causal bound of each column (prefill; no bound for decode)
 #pragma unroll
   for (int h = 0; h < MG; ++h) {
     mref[h] = -INFINITY;
     lpart[h] = 0.0f;
+    cpos[h] = (h < G && attn_col_live(s, b, h)) ? (int)min(attn_col_pos(seq_lens, s, b, h), (int64_t)INT32_MAX) : -1;
   }
-  const size_t rowi = (size_t)b * s.n_kv + g;
+  const size_t rowi = (size_t)attn_cache_row(s, b) * s.n_kv + g;
   const uint32_t* kcodes = kc.codes + rowi * (size_t)kc.cap * wk;
   const uint32_t* vcodes = vc.codes + rowi * (size_t)vc.cap * wv;
   const float* knorm = kc.norm + rowi * kc.cap;
@@ -579,7 +581,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
       sm100::tmem_ld16(tmem_base + t_lanes + gcol + (uint32_t)col_s, raw);
 #pragma unroll
       for (int h = 0; h < MG; ++h) {
-        const bool vh = valid && h < G;
+        const bool vh = valid && h < G && (int)(t0 + tok) <= cpos[h];
         const float v = kn * inv_wsc * raw[h];
         sv[h] = vh ? v : -INFINITY;
         if (scores_out && vh) scores_out[(qbase + h) * s.max_ctx + t0 + tok] = v;

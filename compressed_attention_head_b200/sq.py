@@ -80,6 +80,11 @@ _SIGNATURES = {
                                       ctypes.c_int, _P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int64, ctypes.c_float, _P, ctypes.c_int, _P, _P, ctypes.c_size_t, _P,
                                       _P]),
+    "sq_attn_prefill_workspace": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_int64, ctypes.c_int64]),
+    "sq_attn_prefill": (ctypes.c_int, [_P, _P, ctypes.POINTER(sq_cache), ctypes.POINTER(sq_cache), _P, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, _P,
+                                       ctypes.c_int, ctypes.c_float, _P, ctypes.c_int, _P, ctypes.c_size_t, _P, _P]),
     "sq_attn_decode_noalloc": (ctypes.c_int, [_P, _P, ctypes.POINTER(sq_cache), ctypes.POINTER(sq_cache), _P,
                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_int64, _P, ctypes.c_int, ctypes.c_float, _P, ctypes.c_int,
@@ -281,6 +286,20 @@ def sq_attn_decode(calib_k, calib_v, kc, vc, seq_lens, batch, n_q_heads, n_kv_he
                                 DTYPE_CODE[q.dtype], float(scale), _ptr(out), DTYPE_CODE[out.dtype],
                                 _ptr(scores_out), _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0,
                                 _ptr(flags), _stream(stream)), "sq_attn_decode")
+
+
+def sq_attn_prefill_workspace(batch, n_q_heads, n_kv_heads, d, n_qtok, max_ctx) -> int:
+    return lib().sq_attn_prefill_workspace(batch, n_q_heads, n_kv_heads, d, n_qtok, max_ctx)
+
+
+def sq_attn_prefill(calib_k, calib_v, kc, vc, start, batch, n_q_heads, n_kv_heads, d, n_qtok, max_ctx, q, scale, out,
+                    ws, flags=None, stream=None):
+    """Causal attention of q [batch, n_q, n_qtok, d] at positions start[b] + t (see sq.h)."""
+    kcs, vcs = kc.struct(), vc.struct()
+    _check(lib().sq_attn_prefill(_ptr(calib_k), _ptr(calib_v), ctypes.byref(kcs), ctypes.byref(vcs), _ptr(start),
+                                 batch, n_q_heads, n_kv_heads, d, n_qtok, max_ctx, _ptr(q), DTYPE_CODE[q.dtype],
+                                 float(scale), _ptr(out), DTYPE_CODE[out.dtype], _ptr(ws),
+                                 ws.numel() * ws.element_size(), _ptr(flags), _stream(stream)), "sq_attn_prefill")
 
 
 def sq_decode_step(calib_k, calib_v, kc, vc, k_new, v_new, q, pos, batch, n_q_heads, n_kv_heads, d, max_ctx, scale,

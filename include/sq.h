@@ -418,6 +418,31 @@ sq_status sq_decode_step(const void* calib_k, const void* calib_v, const sq_cach
                          sq_dtype out_dtype, float* scores_out, void* ws, size_t ws_bytes, uint32_t* d_flags,
                          sq_stream stream);
 
+/* Workspace bytes sq_attn_prefill needs for this shape (0 if unsupported). */
+size_t sq_attn_prefill_workspace(int batch, int n_q_heads, int n_kv_heads, int d, int64_t n_qtok, int64_t max_ctx);
+
+/*
+ * Causal attention of a chunk of query tokens over the packed cache (prefill or
+ * chunked prefill; the README's "Key Findings" 3 measures the method over
+ * sequence lengths 512-2048, whose prompts pass through attention before
+ * decoding). Query token t of batch row b sits at position d_start[b] + t and
+ * attends to the cache positions 0 .. d_start[b] + t, with the same scores,
+ * softmax and output as sq_attn_decode gives a single query over that prefix.
+ * The cache must already hold those positions (compress the chunk first).
+ *  q       device, q_dtype [batch][n_q_heads][n_qtok][d].
+ *  out     device, out_dtype [batch][n_q_heads][n_qtok][d].
+ *  d_start device int32[batch]; d_start[b] + n_qtok <= max_ctx and <= cap.
+ *  ws      device workspace of at least sq_attn_prefill_workspace() bytes.
+ * The query positions of a row are taken in blocks of floor(16 / G) (G = query
+ * heads per KV head), whose G x block columns share each decoded key and value
+ * tile in the 16-column MMAs; the causal mask is applied per column.
+ * Returns SQ_ERR_ARG when batch x blocks exceeds 65535.
+ */
+sq_status sq_attn_prefill(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
+                          const int32_t* d_start, int batch, int n_q_heads, int n_kv_heads, int d, int64_t n_qtok,
+                          int64_t max_ctx, const void* q, sq_dtype q_dtype, float scale, void* out, sq_dtype out_dtype,
+                          void* ws, size_t ws_bytes, uint32_t* d_flags, sq_stream stream);
+
 /*
  * sq_attn_decode without a workspace argument, for callers that cannot
  * allocate device memory where they run decode attention: a serving loop whose

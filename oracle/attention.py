@@ -89,6 +89,35 @@ def attn_decode(q, k_words, k_norm, k_rnorm, v_words, v_norm, cals_k, cals_v,
     return out, scores
 
 
+def attn_prefill(q, k_words, k_norm, k_rnorm, v_words, v_norm, cals_k, cals_v, starts, scale: float | None = None):
+    """Causal attention of a chunk of queries over the packed cache (prefill).
+
+    q [B, n_q, T, d]; query t of row b sits at position starts[b] + t and
+    attends to the packed tokens 0 .. starts[b] + t of its KV head, exactly as
+    one decode query over that prefix (``attend_one``). Returns out [B, n_q, T, d].
+    Reading taken: the pages measure the method over sequence lengths 512-2048
+    (SpectralQuant README, "Key Findings" 3) without stating how prompts pass
+    through attention; causal attention over the compressed cache is the plain
+    reading.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    bsz, n_q, t_len, d = q.shape
+    n_kv = len(cals_k)
+    group = n_q // n_kv
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    out = np.zeros((bsz, n_q, t_len, d))
+    for b in range(bsz):
+        for h in range(n_q):
+            g = h // group
+            for t in range(t_len):
+                n = int(starts[b]) + t + 1
+                rnorm = k_rnorm[b, g, :n] if k_rnorm is not None else np.zeros(n)
+                out[b, h, t], _ = attend_one(q[b, h, t], k_words[b, g, :n], k_norm[b, g, :n], rnorm,
+                                             v_words[b, g, :n], v_norm[b, g, :n], cals_k[g], cals_v[g], scale)
+    return out
+
+
 def dense_attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray, scale: float):
     """Softmax attention of one query over explicit keys [L, d] and values [L, d]."""
     s = scale * (np.asarray(keys, np.float64) @ np.asarray(q, np.float64))

@@ -286,3 +286,46 @@ def test_decode_step_appends_then_attends(name, batch, ctx, heads):
     o, s = out.cpu().numpy(), sc.cpu().numpy()
     _assert_close(o, s, ref_out, ref_sc, lens)
     np.testing.assert_allclose(o, out2.cpu().numpy(), rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("name,batch,prefix,chunk,heads", [
+    ("llama8b", 2, 300, 37, 1),          # G = 4: blocks of 4 positions, a partial last block
+    ("qwen14b", 1, 129, 31, 1),          # G = 5: blocks of 3 positions (15 columns)
+    ("gemma9b_sweep", 2, 100, 19, 1),    # G = 2, head_dim 256: blocks of 8 positions
+    ("qwen1_5b_long", 1, 600, 40, 1),    # G = 6: blocks of 2 positions, several splits
+    ("tiny", 2, 60, 21, 2),              # head_dim 32: the SIMT partials
+])
+def test_prefill_attention_matches_the_oracle(name, batch, prefix, chunk, heads):
+    """sq_attn_prefill: each query token of a chunk at position start[b] + t
+    attends causally to the packed cache 0 .. start[b] + t (ragged starts per
+    row); every (row, head, token) output against the oracle."""
+    w = make_workload(name, batch=batch, tokens=prefix + chunk)
+    cfg = w.cfg
+    g = cfg["n_q"] // cfg["n_kv"]
+    nkv = min(heads, cfg["n_kv"])
+    nq, d = nkv * g, cfg["d"]
+    ck = calibrate_oracle(w.k_cal[:nkv], cfg["bits_k"], True)
+    cv = calibrate_oracle(w.v_cal[:nkv], cfg["bits_v"], False)
+    rk, rv = records_to_device(ck), records_to_device(cv)
+    T = prefix + chunk
+    kc = sq.alloc_cache(batch, nkv, T, ck[0].words, True)
+    vc = sq.alloc_cache(batch, nkv, T, cv[0].words, False)
+    sq.sq_compress_kv(rk, rv, w.k[:, :nkv].contiguous().cuda(), w.v[:, :nkv].contiguous().cuda(), batch, nkv, d, T,
+                      None, kc, vc)
+    gen = torch.Generator().manual_seed(5)
+    qs = w.q[:, :nq, None, :].float() * (1.0 + 0.3 * torch.randn(batch, nq, chunk, 1, generator=gen))
+    qs = qs.to(w.q.dtype).contiguous().cuda()
+    starts_l = [prefix - 13 * b for b in range(batch)]
+    starts = torch.tensor(starts_l, dtype=torch.int32, device="cuda")
+    ws = torch.empty(sq.sq_attn_prefill_workspace(batch, nq, nkv, d, chunk, T), dtype=torch.uint8, device="cuda")
+    out = torch.full((batch, nq, chunk, d), float("nan"), device="cuda")
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sq.sq_attn_prefill(rk, rv, kc, vc, starts, batch, nq, nkv, d, chunk, T, qs, 0.0, out, ws, flags)
+    torch.cuda.synchronize()
+    assert flags.item() == 0
+    ref = oattn.attn_prefill(qs.double().cpu().numpy(), kc.words_u32(), kc.norm.cpu().numpy(),
+                             kc.rnorm.cpu().numpy(), vc.words_u32(), vc.norm.cpu().numpy(), ck, cv, starts_l,
+                             1.0 / math.sqrt(d))
+    got = out.cpu().numpy()
+    err = rel_l2_rows(got.reshape(-1, d), ref.reshape(-1, d))
+    assert np.max(err) <= TOL_OUT, np.max(err)

@@ -82,3 +82,38 @@ def test_dense_attention_matches_library_softmax_attention():
             torch.from_numpy(vals)[None, None], scale=scale)[0, 0, 0].numpy()
         assert np.allclose(o, ref, rtol=1e-12, atol=1e-12)
         assert np.allclose(s, scale * keys @ q, rtol=1e-13, atol=1e-13)
+
+
+def test_prefill_equals_causal_dense_attention_on_decompressed_vectors():
+    """The prefill oracle against PyTorch's causal scaled_dot_product_attention
+    (float64) over the decompressed keys (with their QJL term) and values: a
+    chunk of 9 queries at positions 23 .. 31 of a 32-token cache, G = 2."""
+    g = 2
+    q, kw, kn, kr, vw, vn, ck, cv = _build(g=g, tokens=32)
+    rng = np.random.default_rng(3)
+    t_len, start = 9, 23
+    qs = rng.standard_normal((1, q.shape[1], t_len, q.shape[2])) * 0.5
+    scale = 1 / math.sqrt(q.shape[2])
+    out = attention.attn_prefill(qs, kw, kn, kr, vw, vn, ck, cv, [start], scale)
+    for h in range(qs.shape[1]):
+        kv = h // g
+        keys = codec.decompress(kw[0, kv], kn[0, kv], kr[0, kv], ck[kv], apply_qjl=True)
+        vals = codec.decompress(vw[0, kv], vn[0, kv], None, cv[kv], apply_qjl=False)
+        # query t sees keys 0 .. start + t: a boolean mask over the 32 keys
+        mask = np.arange(32)[None, :] <= (start + np.arange(t_len))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(qs[0, h])[None, None], torch.from_numpy(keys)[None, None],
+            torch.from_numpy(vals)[None, None], attn_mask=torch.from_numpy(mask)[None, None], scale=scale)[0, 0]
+        assert np.allclose(out[0, h], ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_prefill_last_query_is_a_decode_query():
+    """The last query of a chunk ending at the cache's end attends to the whole
+    cache: it equals attn_decode of the same query at that length."""
+    q, kw, kn, kr, vw, vn, ck, cv = _build(g=1, tokens=20)
+    qs = np.repeat(q[:, :, None, :], 4, axis=2)
+    out = attention.attn_prefill(qs, kw, kn, kr, vw, vn, ck, cv, [16], None)
+    dec, _ = attention.attn_decode(q, kw, kn, kr, vw, vn, ck, cv, [20], None)
+    assert np.allclose(out[0, :, 3], dec[0], rtol=1e-13, atol=1e-14)
+    dec16, _ = attention.attn_decode(q, kw, kn, kr, vw, vn, ck, cv, [17], None)
+    assert np.allclose(out[0, :, 0], dec16[0], rtol=1e-13, atol=1e-14)
