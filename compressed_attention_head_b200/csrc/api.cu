@@ -122,6 +122,13 @@ sq_status ensure_init(int* dev_out = nullptr) {
   if (cudaMemcpyToSymbol(c_th64, th, sizeof(th)) != cudaSuccess) return SQ_ERR_CUDA;
   if (cudaMemcpyToSymbol(c_lv32, lv32, sizeof(lv32)) != cudaSuccess) return SQ_ERR_CUDA;
   if (cudaMemcpyToSymbol(c_D, dist, sizeof(dist)) != cudaSuccess) return SQ_ERR_CUDA;
+  {
+    static uint8_t img[td::kImgBytes];
+    static uint32_t p3r[64 * 32];
+    td::build_tables_host(lv, img, p3r);
+    if (cudaMemcpyToSymbol(td::g_img, img, sizeof(img)) != cudaSuccess) return SQ_ERR_CUDA;
+    if (cudaMemcpyToSymbol(td::g_p3r, p3r, sizeof(p3r)) != cudaSuccess) return SQ_ERR_CUDA;
+  }
   // Kernels that take more than 48 KB of dynamic shared memory.
   const int big = 200 * 1024;
   cudaFuncSetAttribute(k_jacobi, cudaFuncAttributeMaxDynamicSharedMemorySize, big);

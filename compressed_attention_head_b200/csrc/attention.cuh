@@ -432,31 +432,43 @@ __device__ void combine_one(const uint8_t* __restrict__ recs_v, const AttnShape&
     a[hh * d + i] = ok ? v * s_inv_l[hh] * sig[i] : 0.0f;
   }
   __syncthreads();
-  // o_h = V_V a_h: warp w takes rows w, w + nwarp, ...; lane reads 16-byte pieces
+  // o_h = V_V a_h: warp w takes rows w, w + nwarp, ... in batches of RB rows
+  // whose loads (16-byte pieces, lane-strided) are all in flight together
   const float4* V4 = (const float4*)rv.V_f();
   const int q4 = d / 4;
-  for (int j = warp; j < d; j += nwarp) {
-    float4 vv[2];
+  constexpr int RB = 8;
+  for (int j0 = warp; j0 < d; j0 += nwarp * RB) {
+    float4 vv[RB][2];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int col = lane + 32 * c;
-      vv[c] = (ok && col < q4) ? V4[(size_t)j * q4 + col] : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    for (int hh = 0; hh < G; ++hh) {
-      float o = 0.0f;
+    for (int r = 0; r < RB; ++r) {
+      const int j = j0 + nwarp * r;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const int col = lane + 32 * c;
-        if (col < q4) {
-          const float4 av = *(const float4*)&a[hh * d + 4 * col];
-          o = fmaf(vv[c].x, av.x, o);
-          o = fmaf(vv[c].y, av.y, o);
-          o = fmaf(vv[c].z, av.z, o);
-          o = fmaf(vv[c].w, av.w, o);
-        }
+        vv[r][c] = (ok && j < d && col < q4) ? __ldg(V4 + (size_t)j * q4 + col) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      o = warp_sum(o);
-      if (lane == 0 && attn_col_live(s, b, hh)) store_out(out, out_dt, attn_q_index(s, b, g, hh) + j, o);
+    }
+    for (int hh = 0; hh < G; ++hh) {
+      float4 av[2];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int col = lane + 32 * c;
+        av[c] = col < q4 ? *(const float4*)&a[hh * d + 4 * col] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        const int j = j0 + nwarp * r;
+        float o = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          o = fmaf(vv[r][c].x, av[c].x, o);
+          o = fmaf(vv[r][c].y, av[c].y, o);
+          o = fmaf(vv[r][c].z, av[c].z, o);
+          o = fmaf(vv[r][c].w, av[c].w, o);
+        }
+        o = warp_sum(o);
+        if (lane == 0 && j < d && attn_col_live(s, b, hh)) store_out(out, out_dt, attn_q_index(s, b, g, hh) + j, o);
+      }
     }
   }
 }

@@ -83,6 +83,43 @@ struct Plan {
 };
 static_assert(kLevelsTotal * 2 <= 1024 && kLevelsTotal * 4 <= 2048, "level tables");
 
+// The level tables every block of the kernel starts from, built once per
+// device from the Lloyd-Max levels (td_build_tables) and copied into shared
+// memory by one bulk copy per block: kImgBytes is the span of the plan from P1
+// to CH (width-1 and width-2 pair tables, a zero guard, fp16 levels, a zero
+// guard, fp16 hi | lo levels); g_p3r is the lane-replicated width-3 table.
+constexpr int kImgBytes = 16 + 64 + 16 + 1024 + 16 + 2048;
+__device__ __align__(128) uint8_t g_img[kImgBytes];
+__device__ __align__(128) uint32_t g_p3r[64 * 32];
+
+// Host side of the tables above, from the levels lv (lv_off layout, float64):
+// the same values the kernel's decode steps expect (pairs of fp16 levels of
+// the float32 levels; fp16 hi and lo parts of the float64 levels).
+inline uint16_t h16_bits(__half h) {
+  const __half_raw r = h;
+  return r.x;
+}
+inline uint32_t pair_h2_host(float lo, float hi) {
+  return (uint32_t)h16_bits(__float2half_rn(lo)) | ((uint32_t)h16_bits(__float2half_rn(hi)) << 16);
+}
+inline void build_tables_host(const double* lv, uint8_t* img, uint32_t* p3r) {
+  for (int i = 0; i < kImgBytes; ++i) img[i] = 0;
+  uint32_t* p1 = (uint32_t*)img;
+  uint32_t* p2 = (uint32_t*)(img + 16);
+  uint16_t* l16 = (uint16_t*)(img + 16 + 64 + 16);
+  uint32_t* hl = (uint32_t*)(img + 16 + 64 + 16 + 1024 + 16);
+  auto f = [&](int b, int k) { return (float)lv[lv_off(b) + k]; };
+  for (int t = 0; t < 4; ++t) p1[t] = pair_h2_host(f(1, t & 1), f(1, t >> 1));
+  for (int t = 0; t < 16; ++t) p2[t] = pair_h2_host(f(2, t & 3), f(2, t >> 2));
+  for (int e = 0; e < 64 * 32; ++e) p3r[e] = pair_h2_host(f(3, (e >> 5) & 7), f(3, e >> 8));
+  for (int e = 0; e < kLevelsTotal; ++e) {
+    const __half hi = __double2half(lv[e]);
+    const __half lo = __double2half(lv[e] - (double)__half2float(hi));
+    l16[e] = h16_bits(hi);
+    hl[e] = (uint32_t)h16_bits(hi) | ((uint32_t)h16_bits(lo) << 16);
+  }
+}
+
 // Bytes of one group's region: V^T tile, P tile, nrec record buffers.
 template <int D>
 __host__ __device__ constexpr size_t group_bytes(int wk, int wv, int nrec) {
@@ -321,28 +358,54 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   const int col_s = gstride - NW - C::OCOLS;     // scores, then O^T, at the end of the group's columns
   const int col_o = gstride - C::OCOLS;
 
+  // ---- records of the block's cache row: the issuer of group gi copies tile
+  // kk of the group (tokens t0 .. t0 + 127) into its record buffer bf
+  const size_t rowi = (size_t)attn_cache_row(s, b) * s.n_kv + g;
+  const uint32_t* kcodes = kc.codes + rowi * (size_t)kc.cap * wk;
+  const uint32_t* vcodes = vc.codes + rowi * (size_t)vc.cap * wv;
+  const float* knorm = kc.norm + rowi * kc.cap;
+  const float* krho = kc.rnorm ? kc.rnorm + rowi * kc.cap : nullptr;
+  const float* vnorm = vc.norm + rowi * vc.cap;
+  const size_t rec_buf = (((size_t)(wk + wv) * TILE * 4 + 3 * TILE * 4 + 1023) & ~(size_t)1023);
+  uint64_t* bars = (uint64_t*)(sm + PL::BAR);
+  auto issue_records = [&](int gi, int kk, int bf) {
+    const int64_t t0 = t_lo + (int64_t)(gi + kk * ngr) * TILE;
+    const int64_t blk0 = t0 >> 5;
+    const int nb = (int)min((int64_t)4, (kc.cap - t0) >> 5);    // whole 32-token blocks inside the cache
+    uint8_t* rb = sm + PL::GRP + (size_t)gi * group_bytes<D>(wk, wv, nrec) + C::VT_BYTES + C::P_BYTES +
+                  (size_t)bf * rec_buf;
+    uint64_t* bar = bars + 5 * gi + bf;
+    const uint32_t kbytes = (uint32_t)(nb * wk * 128), vbytes = (uint32_t)(nb * wv * 128), nbytes = nb * 128;
+    const uint32_t total = kbytes + vbytes + nbytes * (krho ? 3u : 2u);
+    sm100::mbar_expect_tx(bar, total);
+    sm100::bulk_load(rb, kcodes + blk0 * wk * 32, kbytes, bar);
+    sm100::bulk_load(rb + (size_t)wk * TILE * 4, vcodes + blk0 * wv * 32, vbytes, bar);
+    uint8_t* nr = rb + (size_t)(wk + wv) * TILE * 4;
+    sm100::bulk_load(nr, knorm + t0, nbytes, bar);
+    sm100::bulk_load(nr + 2 * TILE * 4, vnorm + t0, nbytes, bar);
+    if (krho) sm100::bulk_load(nr + TILE * 4, krho + t0, nbytes, bar);
+  };
+
   // ---- block tables (as in the mma.sync kernel, plus the score B operand)
-  uint32_t* tP1 = (uint32_t*)(sm + PL::P1);
-  uint32_t* tP2 = (uint32_t*)(sm + PL::P2);
-  uint32_t* tP3 = s_p3r;
-  __half* tL16 = (__half*)(sm + PL::L16);
-  uint32_t* tHL = (uint32_t*)(sm + PL::HL);
   uint32_t* tCH = (uint32_t*)(sm + PL::CH);
   uint32_t* tCD = (uint32_t*)(sm + PL::CD);
-  uint64_t* bars = (uint64_t*)(sm + PL::BAR);
   uint32_t* misc = (uint32_t*)(sm + PL::MISC);    // [0] TMEM base, [1] abort, [2] max |weight| (float bits)
-  if (tid < 4) tP1[tid] = pack_h2(c_lv32[lv_off(1) + (tid & 1)], c_lv32[lv_off(1) + (tid >> 1)]);
-  if (tid < 16) tP2[tid] = pack_h2(c_lv32[lv_off(2) + (tid & 3)], c_lv32[lv_off(2) + (tid >> 2)]);
-  for (int e = tid; e < 64 * 32; e += C::NTH) {
-    const int f = e >> 5;
-    tP3[e] = pack_h2(c_lv32[lv_off(3) + (f & 7)], c_lv32[lv_off(3) + (f >> 3)]);
-  }
-  for (int e = tid; e < kLevelsTotal; e += C::NTH) {
-    const double lv = c_lv64[e];
-    const __half hi = __double2half(lv);
-    const __half lo = __double2half(lv - (double)__half2float(hi));
-    tL16[e] = hi;
-    tHL[e] = (uint32_t)__half_as_ushort(hi) | ((uint32_t)__half_as_ushort(lo) << 16);
+  uint64_t* b_setup = (uint64_t*)(misc + 4);       // level tables copied in
+  if (tid == 0) {
+    misc[1] = 0u;
+    misc[2] = 0u;
+    for (int k = 0; k < 5 * C::NG; ++k) sm100::mbar_init(&bars[k], 1);
+    sm100::mbar_init(b_setup, 1);
+    sm100::fence_mbar_init();
+    // the level tables, and the first record tiles of every group, start
+    // arriving while the block builds its other tables and the query operand
+    sm100::mbar_expect_tx(b_setup, (uint32_t)(kImgBytes + 64 * 32 * 4));
+    sm100::bulk_load(sm + PL::P1, g_img, (uint32_t)kImgBytes, b_setup);
+    sm100::bulk_load(s_p3r, g_p3r, 64u * 32u * 4u, b_setup);
+    for (int gi = 0; gi < ngr; ++gi) {
+      const int ntk = gi < ntile ? (ntile - gi + ngr - 1) / ngr : 0;
+      for (int kk = 0; kk < nrec && kk < ntk; ++kk) issue_records(gi, kk, kk);
+    }
   }
   if (tid < 2 * NCH && ok) {
     const Rec r = tid < NCH ? rk : rv;
@@ -359,16 +422,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     const int i = e < D ? e : e - D;
     tCD[e] = ok ? coord_desc(r.bits()[i], r.offsets()[i]) : 0u;
   }
-  if (tid < 4) {
-    ((uint32_t*)(sm + PL::L16))[-1 - tid] = 0u;
-    ((uint32_t*)(sm + PL::HL))[-1 - tid] = 0u;
-  }
-  if (tid == 0) {
-    misc[1] = 0u;
-    misc[2] = 0u;
-    for (int k = 0; k < 5 * C::NG; ++k) sm100::mbar_init(&bars[k], 1);
-    sm100::fence_mbar_init();
-  }
+  __syncwarp();
   if (warp == 0) {
     sm100::tmem_alloc(&misc[0], 512);
     sm100::tmem_relinquish();
@@ -392,9 +446,10 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   {
     uint8_t* Wb = sm + Tab::W;
     const int nks = NCH + 2 + nqs;
+    static_assert(NW == 16, "W operand index arithmetic");
     for (int e = tid; e < NW * 16 * nks; e += C::NTH) {
-      const int n = e / (16 * nks), kk = e % (16 * nks);
-      const int st = kk >> 4, j = kk & 15;
+      // e = (st NW + n) 16 + j: k-step st, head n, k j within the step (coalesced over j)
+      const int st = e >> 8, n = (e >> 4) & 15, j = e & 15, kk = 16 * st + j;
       float v = 0.0f;
       bool lo = false;
       if (n < G) {
@@ -429,13 +484,6 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     lpart[h] = 0.0f;
     cpos[h] = (h < G && attn_col_live(s, b, h)) ? (int)min(attn_col_pos(seq_lens, s, b, h), (int64_t)INT32_MAX) : -1;
   }
-  const size_t rowi = (size_t)attn_cache_row(s, b) * s.n_kv + g;
-  const uint32_t* kcodes = kc.codes + rowi * (size_t)kc.cap * wk;
-  const uint32_t* vcodes = vc.codes + rowi * (size_t)vc.cap * wv;
-  const float* knorm = kc.norm + rowi * kc.cap;
-  const float* krho = kc.rnorm ? kc.rnorm + rowi * kc.cap : nullptr;
-  const float* vnorm = vc.norm + rowi * vc.cap;
-  const size_t rec_buf = (((size_t)(wk + wv) * TILE * 4 + 3 * TILE * 4 + 1023) & ~(size_t)1023);
   uint8_t* gr = sm + PL::GRP + (size_t)grp * group_bytes<D>(wk, wv, nrec);
   uint8_t* sVt = gr;
   uint8_t* sP = gr + C::VT_BYTES;
@@ -464,33 +512,13 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   const uint32_t p_lane = sm100::smem_u32(sP) + (uint32_t)((st_kc >> 3) * (NW * 128) + st_row * 128 +
                                                           (((st_kc & 7) ^ st_row) << 4));
   uint32_t* err = flags;
+  // operand descriptors at the starts of the score B operand, the V^T tile and the P tile
+  const uint64_t w_desc = sm100::sw128_desc(sm100::smem_u32(sm + Tab::W));
+  const uint64_t vt_desc = sm100::sw128_desc(sm100::smem_u32(sVt));
+  const uint64_t p_desc = sm100::sw128_desc(sm100::smem_u32(sP));
 
-  // bulk copies of tile kk's records into buffer bf (issuer only)
-  auto issue_records = [&](int kk, int bf) {
-    const int64_t t0 = t_lo + (int64_t)(grp + kk * ngr) * TILE;
-    const int64_t blk0 = t0 >> 5;
-    const int nb = (int)min((int64_t)4, (kc.cap - t0) >> 5);    // whole 32-token blocks inside the cache
-    uint8_t* rb = sRec + (size_t)bf * rec_buf;
-    const uint32_t kbytes = (uint32_t)(nb * wk * 128), vbytes = (uint32_t)(nb * wv * 128), nbytes = nb * 128;
-    const uint32_t total = kbytes + vbytes + nbytes * (krho ? 3u : 2u);
-    sm100::mbar_expect_tx(&b_rec[bf], total);
-    sm100::bulk_load(rb, kcodes + blk0 * wk * 32, kbytes, &b_rec[bf]);
-    sm100::bulk_load(rb + (size_t)wk * TILE * 4, vcodes + blk0 * wv * 32, vbytes, &b_rec[bf]);
-    uint8_t* nr = rb + (size_t)(wk + wv) * TILE * 4;
-    sm100::bulk_load(nr, knorm + t0, nbytes, &b_rec[bf]);
-    sm100::bulk_load(nr + 2 * TILE * 4, vnorm + t0, nbytes, &b_rec[bf]);
-    if (krho) sm100::bulk_load(nr + TILE * 4, krho + t0, nbytes, &b_rec[bf]);
-  };
-
-  int n_issued = 0;   // tiles whose records the issuer requested (a prefix)
-  if (issuer && ntg > 0) {
-    issue_records(0, 0);
-    n_issued = 1;
-    if (nrec > 1 && ntg > 1) {
-      issue_records(1, 1);
-      n_issued = 2;
-    }
-  }
+  if (!sm100::mbar_wait(b_setup, 0u, err)) *abort_flag = 1;   // level tables in shared memory
+  int n_issued = min(ntg, nrec);   // tiles whose records were requested (a prefix; the first by thread 0)
   const float LOG2E = 1.4426950408889634f;
   for (int kk = 0; kk < ntg; ++kk) {
     const int bf = kk % nrec;
@@ -547,13 +575,17 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
       sm100::tc_fence_after();
       const uint32_t ak = tmem_base + gcol;
       const uint32_t dS = tmem_base + gcol + (uint32_t)col_s;
-      const uint32_t wb = sm100::smem_u32(sm + Tab::W);
       const int nks = NCH + 2 + nqs;
+      // A columns of k-step st: c0 hi for 0 and 1, c0 lo for 2, chunk st - 2
+      // (block st - 1) after; B: k-step st of W (four 32-byte steps per
+      // 2048-byte atom). Descriptors advance in the start-address field
+      // (16-byte units, no carry out of it).
+      uint32_t a_col = ak;
+      uint64_t bd = w_desc;
       for (int st = 0; st < nks; ++st) {
-        // A columns of k-step st: c0 hi for 0 and 1, c0 lo for 2, chunk st - 2 (block st - 1) after
-        const int ablk = st < 2 ? 0 : st - 1;
-        const uint64_t bd = sm100::sw128_desc(wb + (uint32_t)((st >> 2) * (NW * 128) + (st & 3) * 32));
-        sm100::mma_f16_ts(dS, ak + (uint32_t)(8 * ablk), bd, idesc, st > 0 ? 1u : 0u);
+        sm100::mma_f16_ts(dS, a_col, bd, idesc, st > 0 ? 1u : 0u);
+        a_col += st > 0 ? 8u : 0u;
+        bd += (st & 3) == 3 ? (uint64_t)((NW * 128 - 96) >> 4) : 2u;
       }
       sm100::mma_commit(b_s);
     }
@@ -595,7 +627,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     sm100::named_bar(1 + grp, 128);
     // the records of this tile are consumed: the next tile for this buffer may load
     if (issuer && live && kk + nrec < ntg) {
-      issue_records(kk + nrec, bf);
+      issue_records(grp, kk + nrec, bf);
       n_issued = kk + nrec + 1;
     }
     const bool raise = (votes[0] | votes[1] | votes[2] | votes[3]) != 0u;
@@ -662,14 +694,12 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     sm100::named_bar(1 + grp, 128);
     if (issuer && live) {
       sm100::tc_fence_after();
-      const uint32_t vt = sm100::smem_u32(sVt), pp = sm100::smem_u32(sP);
 #pragma unroll
       for (int ks = 0; ks < TILE / 16; ++ks) {
-        const uint64_t bd = sm100::sw128_desc(pp + (uint32_t)((ks >> 2) * (NW * 128) + (ks & 3) * 32));
+        const uint64_t bd = p_desc + (uint64_t)(((ks >> 2) * (NW * 128) + (ks & 3) * 32) >> 4);
 #pragma unroll
         for (int mh = 0; mh < C::MH; ++mh) {
-          const uint64_t ad =
-              sm100::sw128_desc(vt + (uint32_t)((ks >> 2) * (D * 128) + mh * (128 * 128) + (ks & 3) * 32));
+          const uint64_t ad = vt_desc + (uint64_t)(((ks >> 2) * (D * 128) + mh * (128 * 128) + (ks & 3) * 32) >> 4);
           sm100::mma_f16(tmem_base + gcol + (uint32_t)(col_o + 16 * mh), ad, bd, idesc,
                          (kk > 0 || ks > 0) ? 1u : 0u);
         }
@@ -766,6 +796,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   // every copy and MMA a group's issuer started has completed before the block
   // frees its tensor memory and exits (on the normal path they have; after a
   // timed-out wait some may still run): bounded waits
+  if (tid == 0) sm100::mbar_wait(b_setup, 0u, nullptr);
   if (issuer) {
     for (int kk = max(0, n_issued - nrec); kk < n_issued; ++kk)
       sm100::mbar_wait(&b_rec[kk % nrec], (uint32_t)((kk / nrec) & 1), nullptr);
