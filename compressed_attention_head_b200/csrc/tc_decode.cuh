@@ -45,12 +45,18 @@ namespace td {
 constexpr int TILE = 128;          // tokens per tile (4 warps x 32)
 constexpr int NW = 16;             // N of every MMA: query heads, padded
 constexpr float kMarginLog2 = 2.0f;   // reference max raised when a score exceeds it by > 2 (log2 units)
+constexpr unsigned kPollSleepNs = 256;   // idle poll interval of the MMA-issuing thread
 
 template <int D>
 struct Cfg {
   static constexpr int NCH = D / 16;                          // 16-coordinate chunks
-  static constexpr int NG = D == 64 ? 4 : (D == 128 ? 3 : 2);  // warp groups
-  static constexpr int NTH = NG * 128;
+  static constexpr int NG = D == 64 ? 4 : (D == 128 ? 3 : 2);  // warp groups decoding tiles
+  // head_dim 256: a warp of its own issues the MMAs of both groups (35 per
+  // tile; issued from a decode warp they held its group back). With three
+  // or four groups the SM's issue slots are the limit and a decode warp of
+  // each group issues its MMAs.
+  static constexpr bool MW = D == 256;
+  static constexpr int NTH = NG * 128 + (MW ? 32 : 0);
   static constexpr int MH = D > 128 ? 2 : 1;                  // 128-row halves of V^T / O^T
   static constexpr int OCOLS = 16 * MH;                       // TMEM columns of O^T
   static constexpr int AK0 = 8 * (NCH + 1);                   // key operand columns without QJL blocks
@@ -75,8 +81,8 @@ struct Plan {
   static constexpr int HL = L16 + 1024 + 16;           // u32 [kLevelsTotal]: fp16 hi | fp16 lo << 16
   static constexpr int CH = HL + 2048;                 // u32 [2][16]: chunk descriptors K, V
   static constexpr int CD = CH + 128;                  // u32 [2][D]: coordinate descriptors K, V
-  static constexpr int BAR = CD + 8 * D;               // u64 [NG][5]: records full x2, scores, PV done, drain
-  static constexpr int MISC = BAR + 8 * 5 * 4;         // u32 [16]: TMEM base, abort, wmax
+  static constexpr int BAR = CD + 8 * D;               // u64 [NG][6]: records x2, scores, PV done, keys in, P in
+  static constexpr int MISC = BAR + 8 * 6 * 4;         // u32 [16]: TMEM base, abort, wmax; u64 setup, drain
   static constexpr int GS = MISC + 64;                 // per group: votes [4], maxima [4][16], l [4][16], mref [16], misc
   static constexpr int GS_BYTES = 16 + 256 + 256 + 64 + 64;
   static constexpr int GRP = (GS + Cfg<D>::NG * GS_BYTES + 1023) & ~1023;   // group regions (1024-aligned)
@@ -374,7 +380,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     const int nb = (int)min((int64_t)4, (kc.cap - t0) >> 5);    // whole 32-token blocks inside the cache
     uint8_t* rb = sm + PL::GRP + (size_t)gi * group_bytes<D>(wk, wv, nrec) + C::VT_BYTES + C::P_BYTES +
                   (size_t)bf * rec_buf;
-    uint64_t* bar = bars + 5 * gi + bf;
+    uint64_t* bar = bars + 6 * gi + bf;
     const uint32_t kbytes = (uint32_t)(nb * wk * 128), vbytes = (uint32_t)(nb * wv * 128), nbytes = nb * 128;
     const uint32_t total = kbytes + vbytes + nbytes * (krho ? 3u : 2u);
     sm100::mbar_expect_tx(bar, total);
@@ -391,11 +397,16 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   uint32_t* tCD = (uint32_t*)(sm + PL::CD);
   uint32_t* misc = (uint32_t*)(sm + PL::MISC);    // [0] TMEM base, [1] abort, [2] max |weight| (float bits)
   uint64_t* b_setup = (uint64_t*)(misc + 4);       // level tables copied in
+  uint64_t* b_drain = (uint64_t*)(misc + 6);       // every MMA of the block done (before the free)
   if (tid == 0) {
     misc[1] = 0u;
     misc[2] = 0u;
-    for (int k = 0; k < 5 * C::NG; ++k) sm100::mbar_init(&bars[k], 1);
+    // per group: records x2, scores, PV (one arrival: copy or commit); keys
+    // and P stored (one arrival per thread of the group) with the MMA warp,
+    // else the group's drain (one commit)
+    for (int k = 0; k < 6 * C::NG; ++k) sm100::mbar_init(&bars[k], (k % 6 >= 4 && C::MW) ? 128u : 1u);
     sm100::mbar_init(b_setup, 1);
+    sm100::mbar_init(b_drain, 1);
     sm100::fence_mbar_init();
     // the level tables, and the first record tiles of every group, start
     // arriving while the block builds its other tables and the query operand
@@ -489,11 +500,14 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   uint8_t* sP = gr + C::VT_BYTES;
   uint8_t* sRec = sP + C::P_BYTES;
   uint8_t* gs = sm + PL::GS + grp * PL::GS_BYTES;          // votes [4] (u32), maxima [4][16] (int), l [4][16], mref [16]
-  uint64_t* b_rec = bars + 5 * grp;                          // [0], [1]: records of buffer 0 / 1
-  uint64_t* b_s = bars + 5 * grp + 2;                        // scores ready
-  uint64_t* b_pv = bars + 5 * grp + 3;                       // PV of the group's last tile done
-  uint64_t* b_drain = bars + 5 * grp + 4;                    // every MMA of the group done (before the free)
-  const bool issuer = q == 0 && lane == 0;
+  uint64_t* b_rec = bars + 6 * grp;                          // [0], [1]: records of buffer 0 / 1
+  uint64_t* b_s = bars + 6 * grp + 2;                        // scores ready
+  uint64_t* b_pv = bars + 6 * grp + 3;                       // PV of the group's last tile done
+  uint64_t* b_kf = bars + 6 * grp + 4;                       // the tile's keys are in tensor memory (MW)
+  uint64_t* b_pf = bars + 6 * grp + 5;                       // the tile's V^T and P are in shared memory (MW)
+  uint64_t* b_gdrain = bars + 6 * grp + 4;                   // the group's MMAs done (without MW)
+  const bool mma_warp = warp == 4 * C::NG;
+  const bool issuer = q == 0 && lane == 0 && !mma_warp;     // the group's record copies
   const bool active = grp < ngr;
   const int ntg = active && grp < ntile ? (ntile - grp + ngr - 1) / ngr : 0;   // tiles of this group
   const uint32_t gcol = (uint32_t)(grp * gstride);
@@ -512,14 +526,100 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   const uint32_t p_lane = sm100::smem_u32(sP) + (uint32_t)((st_kc >> 3) * (NW * 128) + st_row * 128 +
                                                           (((st_kc & 7) ^ st_row) << 4));
   uint32_t* err = flags;
-  // operand descriptors at the starts of the score B operand, the V^T tile and the P tile
+  // descriptor of the score B operand (k-step 0)
   const uint64_t w_desc = sm100::sw128_desc(sm100::smem_u32(sm + Tab::W));
-  const uint64_t vt_desc = sm100::sw128_desc(sm100::smem_u32(sVt));
-  const uint64_t p_desc = sm100::sw128_desc(sm100::smem_u32(sP));
 
   if (!sm100::mbar_wait(b_setup, 0u, err)) *abort_flag = 1;   // level tables in shared memory
   int n_issued = min(ntg, nrec);   // tiles whose records were requested (a prefix; the first by thread 0)
   const float LOG2E = 1.4426950408889634f;
+  // The MMAs of a tile of group gi. Scores: A = the keys in tensor memory
+  // (k-step st reads c0 hi for st = 0 and 1, c0 lo for 2, chunk st - 2 =
+  // column block st - 1 after), B = W (four 32-byte k-steps per 2048-byte
+  // atom). PV: O^T += V^T P. Descriptors advance in their start-address
+  // field (16-byte units, no carry out of it).
+  const int nks = NCH + 2 + nqs;
+  auto issue_scores = [&](int gi) {
+    const uint32_t gc = tmem_base + (uint32_t)(gi * gstride);
+    uint32_t a_col = gc;
+    uint64_t bd = w_desc;
+    for (int st = 0; st < nks; ++st) {
+      sm100::mma_f16_ts(gc + (uint32_t)col_s, a_col, bd, idesc, st > 0 ? 1u : 0u);
+      a_col += st > 0 ? 8u : 0u;
+      bd += (st & 3) == 3 ? (uint64_t)((NW * 128 - 96) >> 4) : 2u;
+    }
+    sm100::mma_commit(bars + 6 * gi + 2);
+  };
+  auto issue_pv = [&](int gi, int kt) {
+    const uint32_t gc = tmem_base + (uint32_t)(gi * gstride);
+    const uint32_t vt = sm100::smem_u32(sm + PL::GRP + (size_t)gi * group_bytes<D>(wk, wv, nrec));
+    const uint64_t vd = sm100::sw128_desc(vt), pd = sm100::sw128_desc(vt + (uint32_t)C::VT_BYTES);
+#pragma unroll
+    for (int ks = 0; ks < TILE / 16; ++ks) {
+      const uint64_t bd = pd + (uint64_t)(((ks >> 2) * (NW * 128) + (ks & 3) * 32) >> 4);
+#pragma unroll
+      for (int mh = 0; mh < C::MH; ++mh) {
+        const uint64_t ad = vd + (uint64_t)(((ks >> 2) * (D * 128) + mh * (128 * 128) + (ks & 3) * 32) >> 4);
+        sm100::mma_f16(gc + (uint32_t)(col_o + 16 * mh), ad, bd, idesc, (kt > 0 || ks > 0) ? 1u : 0u);
+      }
+    }
+    sm100::mma_commit(bars + 6 * gi + 3);
+  };
+  // ---- the MMA warp (MW): one thread issues every group's MMAs as their
+  // operands arrive (a tile's score MMAs once its keys are in tensor memory,
+  // its PV MMAs once V^T and P are in shared memory), polling the groups'
+  // barriers in turn; it gives up after kTimeoutNs without progress
+  if constexpr (C::MW) {
+    if (mma_warp) {
+      if (lane == 0) {
+        int ev[C::NG], ntk[C::NG];
+        int remaining = 0;
+#pragma unroll
+        for (int gi = 0; gi < C::NG; ++gi) {
+          ev[gi] = 0;
+          ntk[gi] = (gi < ngr && gi < ntile) ? (ntile - gi + ngr - 1) / ngr : 0;
+          remaining += 2 * ntk[gi];
+        }
+        uint32_t idle = 0;
+        uint64_t t_idle = 0;
+        while (remaining > 0 && *abort_flag == 0) {
+          bool progress = false;
+#pragma unroll
+          for (int gi = 0; gi < C::NG; ++gi) {
+            if (ev[gi] >= 2 * ntk[gi]) continue;
+            const int kt = ev[gi] >> 1;
+            uint64_t* gb = bars + 6 * gi;
+            if ((ev[gi] & 1) == 0) {
+              if (!sm100::mbar_test(gb + 4, (uint32_t)(kt & 1))) continue;
+              sm100::tc_fence_after();
+              issue_scores(gi);
+            } else {
+              if (!sm100::mbar_test(gb + 5, (uint32_t)(kt & 1))) continue;
+              sm100::tc_fence_after();
+              issue_pv(gi, kt);
+            }
+            ++ev[gi];
+            --remaining;
+            progress = true;
+          }
+          if (progress) {
+            idle = 0;
+            continue;
+          }
+          // nothing ready: sleep, so that the polling takes no issue slots from
+          // the decode warps (the operands of a tile take microseconds to arrive)
+          if (idle++ == 0) {
+            t_idle = sm100::global_ns();
+          } else if ((idle & 15u) == 0u && sm100::global_ns() - t_idle > sm100::kTimeoutNs) {
+            *abort_flag = 1;
+            if (err) atomicOr(err, SQ_FLAG_TIMEOUT);
+            break;
+          }
+          __nanosleep(kPollSleepNs);
+        }
+      }
+      __syncwarp();
+    }
+  }
   for (int kk = 0; kk < ntg; ++kk) {
     const int bf = kk % nrec;
     const int64_t t0 = t_lo + (int64_t)(grp + kk * ngr) * TILE;
@@ -570,24 +670,14 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     }
     sm100::tmem_wait_st();
     sm100::tc_fence_before();
-    sm100::named_bar(1 + grp, 128);
-    if (issuer && live) {
-      sm100::tc_fence_after();
-      const uint32_t ak = tmem_base + gcol;
-      const uint32_t dS = tmem_base + gcol + (uint32_t)col_s;
-      const int nks = NCH + 2 + nqs;
-      // A columns of k-step st: c0 hi for 0 and 1, c0 lo for 2, chunk st - 2
-      // (block st - 1) after; B: k-step st of W (four 32-byte steps per
-      // 2048-byte atom). Descriptors advance in the start-address field
-      // (16-byte units, no carry out of it).
-      uint32_t a_col = ak;
-      uint64_t bd = w_desc;
-      for (int st = 0; st < nks; ++st) {
-        sm100::mma_f16_ts(dS, a_col, bd, idesc, st > 0 ? 1u : 0u);
-        a_col += st > 0 ? 8u : 0u;
-        bd += (st & 3) == 3 ? (uint64_t)((NW * 128 - 96) >> 4) : 2u;
+    if constexpr (C::MW) {
+      sm100::mbar_arrive(b_kf);
+    } else {
+      sm100::named_bar(1 + grp, 128);
+      if (issuer && live) {
+        sm100::tc_fence_after();
+        issue_scores(grp);
       }
-      sm100::mma_commit(b_s);
     }
     // ---- values -> V^T tile (the previous tile's PV must be done with it)
     if (live && kk > 0) live = sm100::mbar_wait(b_pv, (uint32_t)((kk - 1) & 1), err);
@@ -691,20 +781,14 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     }
     sm100::fence_async_smem();
     sm100::tc_fence_before();
-    sm100::named_bar(1 + grp, 128);
-    if (issuer && live) {
-      sm100::tc_fence_after();
-#pragma unroll
-      for (int ks = 0; ks < TILE / 16; ++ks) {
-        const uint64_t bd = p_desc + (uint64_t)(((ks >> 2) * (NW * 128) + (ks & 3) * 32) >> 4);
-#pragma unroll
-        for (int mh = 0; mh < C::MH; ++mh) {
-          const uint64_t ad = vt_desc + (uint64_t)(((ks >> 2) * (D * 128) + mh * (128 * 128) + (ks & 3) * 32) >> 4);
-          sm100::mma_f16(tmem_base + gcol + (uint32_t)(col_o + 16 * mh), ad, bd, idesc,
-                         (kk > 0 || ks > 0) ? 1u : 0u);
-        }
+    if constexpr (C::MW) {
+      sm100::mbar_arrive(b_pf);
+    } else {
+      sm100::named_bar(1 + grp, 128);
+      if (issuer && live) {
+        sm100::tc_fence_after();
+        issue_pv(grp, kk);
       }
-      sm100::mma_commit(b_pv);
     }
   }
   // ---- the group's sums and accumulator
@@ -720,9 +804,9 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
 #pragma unroll
   for (int h = 0; h < MG; ++h) {
     const float v = warp_sum(lpart[h]);
-    if (lane == 0) lsum[q * 16 + h] = v;
+    if (lane == 0 && !mma_warp) lsum[q * 16 + h] = v;
   }
-  if (q == 0 && lane == 0) {
+  if (issuer) {
 #pragma unroll
     for (int h = 0; h < MG; ++h) gref[h] = mref[h];
   }
@@ -800,8 +884,15 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   if (issuer) {
     for (int kk = max(0, n_issued - nrec); kk < n_issued; ++kk)
       sm100::mbar_wait(&b_rec[kk % nrec], (uint32_t)((kk / nrec) & 1), nullptr);
-    sm100::mma_commit(b_drain);
-    if (!sm100::mbar_wait(b_drain, 0u, err)) *abort_flag = 1;
+  }
+  if constexpr (C::MW) {
+    if (mma_warp && lane == 0) {
+      sm100::mma_commit(b_drain);
+      if (!sm100::mbar_wait(b_drain, 0u, err)) *abort_flag = 1;
+    }
+  } else if (issuer) {
+    sm100::mma_commit(b_gdrain);
+    if (!sm100::mbar_wait(b_gdrain, 0u, err)) *abort_flag = 1;
   }
   sm100::tc_fence_before();
   __syncthreads();
