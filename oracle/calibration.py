@@ -60,6 +60,7 @@ FLAG_QJL = 2
 FLAG_NORMALIZE = 4
 FLAG_RANDOM_ROTATION = 8
 FLAG_CUMVAR = 16
+FLAG_FITTED = 32               # per-regime codebooks fitted to the calibration data (fitted.py)
 ROTATION_SALT = 0x524F54       # seed salt of the random-rotation stream ("ROT")
 
 
@@ -189,6 +190,8 @@ class HeadCalib:
     S: np.ndarray         # [m, m] QJL projection
     bits: np.ndarray      # [d] int
     offsets: np.ndarray   # [d] int
+    fit_lv: np.ndarray | None = None   # [2, 510] fitted levels (signal, noise regime) or None
+    fit_th: np.ndarray | None = None   # [2, 502] fitted thresholds or None
 
     @property
     def is_key(self) -> bool:
@@ -201,6 +204,19 @@ class HeadCalib:
     @property
     def normalize(self) -> bool:
         return bool(self.flags & FLAG_NORMALIZE)
+
+    @property
+    def fitted(self) -> bool:
+        return bool(self.flags & FLAG_FITTED)
+
+    def codebook(self, i: int):
+        """(levels, thresholds) that code coordinate i (its width b_i >= 1)."""
+        b = int(self.bits[i])
+        if self.fitted:
+            from . import fitted
+            return fitted.codebook_of(self.fit_lv, self.fit_th, fitted.regime_of(i, self.d_eff), b)
+        levels, thr, _ = codebook.lloyd_max(b)
+        return levels, thr
 
 
 def budget(d: int, avg_bits: float) -> int:
@@ -239,12 +255,34 @@ def finalize(lam: np.ndarray, vec: np.ndarray, *, avg_bits: float, is_key: bool,
         offsets=bit_offsets(bits))
 
 
-def calibrate(x: np.ndarray, *, rotation: str = "spectral", **kw) -> HeadCalib:
+def fit_codebooks(cal: HeadCalib, x: np.ndarray, iters: int | None = None) -> HeadCalib:
+    """``cal`` with per-regime codebooks fitted to its calibration vectors
+    ``x`` [N, d] (the z the compressor would quantize; see fitted.py)."""
+    from . import codec, fitted
+    it = fitted.FIT_ITERS if iters is None else iters
+    _, y = codec.rotate(x, cal)
+    z = codec.scaled(y, cal)
+    lv, th = fitted.fit_tables(z, cal.bits, cal.d_eff, it)
+    cal.fit_lv, cal.fit_th = lv, th
+    cal.flags |= FLAG_FITTED
+    return cal
+
+
+def calibrate(x: np.ndarray, *, rotation: str = "spectral", codebooks: str = "gaussian",
+              fit_iters: int | None = None, **kw) -> HeadCalib:
     """Calibrate one head from its calibration vectors ``x`` [N, d]; ``rotation``
-    is "spectral" (the calibrated eigenbasis) or "random" (the A/B baseline)."""
+    is "spectral" (the calibrated eigenbasis) or "random" (the A/B baseline);
+    ``codebooks`` is "gaussian" (the shared Lloyd-Max tables) or "fitted"
+    (per-regime tables fitted to ``x``)."""
     c = second_moment(x)
     if rotation == "random":
         lam, vec = random_basis(c, kw.get("seed", 42), kw.get("stream", 0))
-        return finalize(lam, vec, random_rotation=True, **kw)
-    lam, vec = eigenbasis(c)
-    return finalize(lam, vec, **kw)
+        cal = finalize(lam, vec, random_rotation=True, **kw)
+    else:
+        lam, vec = eigenbasis(c)
+        cal = finalize(lam, vec, **kw)
+    if codebooks == "fitted":
+        cal = fit_codebooks(cal, x, fit_iters)
+    elif codebooks != "gaussian":
+        raise ValueError(f"unknown codebooks {codebooks!r}")
+    return cal

@@ -18,6 +18,8 @@ The steps, per vector x of one head with calibration ``cal``:
   2. y = V^T u: coordinates in the calibrated eigenbasis.
   3. z_i = y_i / sigma_i (0 where sigma_i = 0); code_i = number of the b_i-bit
      thresholds strictly below z_i; c_hat_i = level of code_i (0 if b_i = 0).
+     The b-bit codebook is the Gaussian Lloyd-Max one, or, for a calibration
+     with fitted codebooks, the one of coordinate i's regime (fitted.py).
   4. Keys with QJL, signal dims i < m: r = y[:m] - sigma[:m] * c_hat[:m],
      rho = ||r||, sign bit j = 1 if (S r)_j >= 0 else 0.
   5. Pack (reading taken; the pages fix no layout): one record of B bits per
@@ -68,7 +70,11 @@ def quantize(z: np.ndarray, cal: HeadCalib) -> np.ndarray:
     codes = np.zeros(z.shape, dtype=np.int64)
     for i in range(cal.d):
         if cal.bits[i] > 0:
-            codes[:, i] = codebook.quantize(z[:, i], int(cal.bits[i]))
+            if cal.fitted:
+                _, thr = cal.codebook(i)
+                codes[:, i] = (z[:, i][:, None] > thr[None, :]).sum(axis=1)
+            else:
+                codes[:, i] = codebook.quantize(z[:, i], int(cal.bits[i]))
     return codes
 
 
@@ -76,7 +82,11 @@ def levels(codes: np.ndarray, cal: HeadCalib) -> np.ndarray:
     """Reconstruction levels c_hat [T, d] of the codes."""
     out = np.zeros(codes.shape)
     for i in range(cal.d):
-        out[:, i] = codebook.dequantize(codes[:, i], int(cal.bits[i]))
+        if cal.fitted and cal.bits[i] > 0:
+            lv, _ = cal.codebook(i)
+            out[:, i] = lv[np.asarray(codes[:, i], dtype=np.int64)]
+        else:
+            out[:, i] = codebook.dequantize(codes[:, i], int(cal.bits[i]))
     return out
 
 
@@ -178,7 +188,7 @@ def exemptions(out: dict, cal: HeadCalib):
         b = int(cal.bits[i])
         if b == 0:
             continue
-        _, thr, _ = codebook.lloyd_max(b)
+        _, thr = cal.codebook(i)
         dist = np.abs(z[:, i:i + 1] - thr[None, :])
         code_ex[:, i] = np.any(dist <= EXEMPT_REL * np.maximum(1.0, np.abs(thr))[None, :], axis=1)
     m = cal.m
