@@ -164,6 +164,13 @@ sq_status ensure_init(int* dev_out = nullptr) {
   cudaFuncSetAttribute(k_step_prep<T, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, ps)
     SQ_SP_ATTR(float); SQ_SP_ATTR(__half); SQ_SP_ATTR(__nv_bfloat16);
 #undef SQ_SP_ATTR
+#define SQ_AP_ATTR(T)                                                                                          \
+  cudaFuncSetAttribute(k_append<T, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)append_smem(1));     \
+  cudaFuncSetAttribute(k_append<T, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)append_smem(2));     \
+  cudaFuncSetAttribute(k_append<T, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)append_smem(4));     \
+  cudaFuncSetAttribute(k_append<T, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)append_smem(8))
+    SQ_AP_ATTR(float); SQ_AP_ATTR(__half); SQ_AP_ATTR(__nv_bfloat16);
+#undef SQ_AP_ATTR
   }
   if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
   int sms = 0;
@@ -413,9 +420,10 @@ sq_status sq_set_option(int option, int value) {
 }
 
 size_t sq_calibrate_workspace(const sq_calib_params* p, int64_t n_tokens) {
-  (void)n_tokens;
-  if (!p || !supported_d(p->d) || p->n_heads < 1) return 0;
-  return (size_t)p->n_heads * 16u * (size_t)p->d * (size_t)p->d;
+  if (!p || !supported_d(p->d) || p->n_heads < 1 || n_tokens < 0) return 0;
+  size_t b = (size_t)p->n_heads * 16u * (size_t)p->d * (size_t)p->d;
+  if (p->codebooks == 1) b += (size_t)p->n_heads * (size_t)n_tokens * (size_t)p->d * 8u;   // z of the fit
+  return b;
 }
 
 sq_status sq_calibrate(const sq_calib_params* p, const void* x, sq_dtype dtype, int64_t n_tokens,
@@ -431,7 +439,9 @@ sq_status sq_calibrate(const sq_calib_params* p, const void* x, sq_dtype dtype, 
       stride_head < 0 || !x || !calib_out || ((uintptr_t)calib_out & 255u) || !ws || !aligned16(ws) ||
       (p->is_key != 0 && p->is_key != 1) || (p->qjl != 0 && p->qjl != 1) ||
       (p->normalize != 0 && p->normalize != 1) || (d_status && !aligned16(d_status)) || (B + 31) / 32 > kMaxWords ||
-      (p->rotation != 0 && p->rotation != 1) || !(p->cumvar >= 0.0 && p->cumvar <= 1.0))
+      (p->rotation != 0 && p->rotation != 1) || !(p->cumvar >= 0.0 && p->cumvar <= 1.0) ||
+      (p->codebooks != 0 && p->codebooks != 1) || p->fit_iters < 0 || p->fit_iters > 100000 ||
+      (p->codebooks == 1 && (p->n_heads > 65535 || (n_tokens + 7) / 8 > 0x7fffffff)))
     return SQ_ERR_ARG;
   if (ws_bytes < sq_calibrate_workspace(p, n_tokens)) return SQ_ERR_WORKSPACE;
   sq_status s = ensure_init();
@@ -454,8 +464,21 @@ sq_status sq_calibrate(const sq_calib_params* p, const void* x, sq_dtype dtype, 
   }
   if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
   FinalizeArgs fa{B, p->is_key, p->qjl, p->normalize, p->d_eff_override, p->max_bits, p->seed, p->avg_bits,
-                  p->cumvar, p->rotation};
+                  p->cumvar, p->rotation, p->codebooks};
   k_finalize<<<p->n_heads, 256, 0, st>>>(calib_out, d, fa, d_status);
+  if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
+  if (p->codebooks == 1) {
+    double* z = vt + (size_t)p->n_heads * d * d;
+    dim3 gz((unsigned)((n_tokens + 7) / 8), (unsigned)p->n_heads);
+    switch (dtype) {
+      case SQ_F32: k_fit_z<float><<<gz, 256, 0, st>>>((const float*)x, d, n_tokens, stride_head, stride_tok, calib_out, z); break;
+      case SQ_F16: k_fit_z<__half><<<gz, 256, 0, st>>>((const __half*)x, d, n_tokens, stride_head, stride_tok, calib_out, z); break;
+      default: k_fit_z<__nv_bfloat16><<<gz, 256, 0, st>>>((const __nv_bfloat16*)x, d, n_tokens, stride_head, stride_tok, calib_out, z); break;
+    }
+    if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
+    const int iters = p->fit_iters > 0 ? p->fit_iters : kFitIters;
+    k_fit_lloyd<<<dim3((unsigned)p->n_heads, 2, SQ_MAX_BITS), 256, 0, st>>>(z, d, n_tokens, calib_out, iters);
+  }
   return cuda_ok(cudaGetLastError());
 }
 

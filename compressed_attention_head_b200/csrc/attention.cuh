@@ -90,7 +90,7 @@ __device__ __forceinline__ int64_t attn_col_pos(const int32_t* seq_lens, const A
 // ---------------------------------------------------------------------------
 constexpr int kPrepVecs = 32;    // query vectors per prepare block
 __host__ __device__ inline int prep_rows(int G) { return G >= kPrepVecs ? 1 : kPrepVecs / G; }
-__host__ __device__ inline size_t prep_smem(int d) { return (size_t)2 * kPrepVecs * d * 4; }
+__host__ __device__ constexpr size_t prep_smem(int d) { return (size_t)2 * kPrepVecs * d * 4; }
 
 template <typename TQ>
 __device__ void prepare_body(const uint8_t* __restrict__ recs_k, const TQ* __restrict__ q, const AttnShape& s,
@@ -173,8 +173,8 @@ __global__ void __launch_bounds__(256) k_attn_prepare(const uint8_t* __restrict_
 __host__ __device__ inline size_t attn_partial_smem(int d, int G, int wk, int wv) {
   return (size_t)4 * G * d            // w
          + (size_t)4 * G * d          // u (m <= d)
-         + (size_t)4 * kLevelsTotal   // levels
-         + (size_t)4 * 4 * d          // bits/offsets of K and V
+         + (size_t)4 * 4 * kLevelsTotal   // levels of K and V, two regimes each
+         + (size_t)4 * 6 * d          // bits / offsets / level bases of K and V
          + (size_t)4 * d              // sigma_V (unused here, reserved)
          + (size_t)4 * kAttnTile * (wk + 1) + (size_t)4 * kAttnTile * (wv + 1)
          + (size_t)4 * 3 * kAttnTile  // k norm, rho, v norm
@@ -224,11 +224,13 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
   unsigned char* p = sm;
   float* w = (float*)p;        p += (size_t)4 * G * d;
   float* u = (float*)p;        p += (size_t)4 * G * d;
-  float* lv = (float*)p;       p += (size_t)4 * kLevelsTotal;
+  float* lv = (float*)p;       p += (size_t)4 * 4 * kLevelsTotal;   // K regime 0, 1; V regime 0, 1
   int* kb = (int*)p;           p += (size_t)4 * d;
   int* ko = (int*)p;           p += (size_t)4 * d;
   int* vb = (int*)p;           p += (size_t)4 * d;
   int* vo = (int*)p;           p += (size_t)4 * d;
+  int* kl = (int*)p;           p += (size_t)4 * d;   // level-table base of each key coordinate
+  int* vl = (int*)p;           p += (size_t)4 * d;
   p += (size_t)4 * d;
   uint32_t* kw = (uint32_t*)p; p += (size_t)4 * kAttnTile * (wk + 1);
   uint32_t* vw = (uint32_t*)p; p += (size_t)4 * kAttnTile * (wv + 1);
@@ -244,11 +246,20 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
   const size_t qbase = ((size_t)b * s.n_q + (size_t)g * G);
   for (int e = tid; e < G * d; e += blockDim.x) w[e] = wq[qbase * d + e];
   for (int e = tid; e < G * m; e += blockDim.x) u[e] = uq[(qbase + e / m) * d + e % m];
-  for (int e = tid; e < kLevelsTotal; e += blockDim.x) lv[e] = c_lv32[e];
+  // codebooks: each record's fitted per-regime tables (flag kFlagFitted), else
+  // the shared Gaussian Lloyd-Max tables
+  for (int e = tid; e < 4 * kLevelsTotal; e += blockDim.x) {
+    const Rec& r = e < 2 * kLevelsTotal ? rk : rv;
+    const int f = e % (2 * kLevelsTotal);
+    lv[e] = (ok && (r.hdr()->flags & kFlagFitted)) ? (float)r.fit_lv()[f] : c_lv32[f % kLevelsTotal];
+  }
   if (ok)
     for (int i = tid; i < d; i += blockDim.x) {
       kb[i] = rk.bits()[i]; ko[i] = rk.offsets()[i];
       vb[i] = rv.bits()[i]; vo[i] = rv.offsets()[i];
+      const bool kfit = (hk->flags & kFlagFitted) != 0u, vfit = (hv->flags & kFlagFitted) != 0u;
+      kl[i] = ((kfit && i >= hk->d_eff) ? kLevelsTotal : 0) + lv_off(kb[i]);
+      vl[i] = 2 * kLevelsTotal + ((vfit && i >= hv->d_eff) ? kLevelsTotal : 0) + lv_off(vb[i]);
     }
   for (int hh = tid; hh < G; hh += blockDim.x) { mrun[hh] = -INFINITY; lrun[hh] = 0.0f; }
   float oacc[MAXG][2];
@@ -286,7 +297,7 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
         for (int i = 0; i < d; ++i) {
           int bw = kb[i];
           if (bw == 0) continue;
-          float lvv = lv[lv_off(bw) + (int)field(rw, ko[i], bw)];
+          float lvv = lv[kl[i] + (int)field(rw, ko[i], bw)];
 #pragma unroll
           for (int hh = 0; hh < MAXG; ++hh)
             if (hh < G) a[hh] = fmaf(w[hh * d + i], lvv, a[hh]);
@@ -348,8 +359,9 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
       int bw = vb[i];
       if (bw == 0) continue;
       int o = vo[i];
+      const int lb = vl[i];
       for (int t = 0; t < nt; ++t) {
-        float lvv = lv[lv_off(bw) + (int)field(vw + t * (wv + 1), o, bw)];
+        float lvv = lv[lb + (int)field(vw + t * (wv + 1), o, bw)];
 #pragma unroll
         for (int hh = 0; hh < MAXG; ++hh)
           if (hh < G) oacc[hh][c2] = fmaf(sc[hh * kAttnTile + t], lvv, oacc[hh][c2]);

@@ -211,6 +211,7 @@ struct FinalizeArgs {
   double avg_bits;
   double cumvar;      // 0: participation-ratio d_eff; (0, 1]: cumulative-variance d_eff
   int rotation;       // 1: the basis is the random rotation (record flag only)
+  int fitted;         // 1: per-regime codebooks fitted afterwards (k_fit_z, k_fit_lloyd)
 };
 
 // Writes one derived part (float copies) of a record whose canonical part is complete.
@@ -323,6 +324,10 @@ __global__ void __launch_bounds__(256) k_finalize(void* __restrict__ recs, int d
   const uint64_t s0 = mix64(a.seed ^ mix64((uint64_t)h + 1ull));
   double* S = rec.S();
   for (int e = tid; e < d * d; e += nth) if (e >= m * m) S[e] = 0.0;
+  // fitted-codebook section: the Gaussian tables in both regimes (the start of
+  // the fit, and the tables of widths no coordinate uses) or zeros
+  for (int e = tid; e < 2 * kLevelsTotal; e += nth) rec.fit_lv()[e] = a.fitted ? c_lv64[e % kLevelsTotal] : 0.0;
+  for (int e = tid; e < 2 * kThreshTotal; e += nth) rec.fit_th()[e] = a.fitted ? c_th64[e % kThreshTotal] : 0.0;
   for (int pidx = tid; 2 * pidx < m * m; pidx += nth) {
     uint64_t r1 = sm64_at(s0, 2ull * pidx), r2 = sm64_at(s0, 2ull * pidx + 1ull);
     double u1 = (double)((r1 >> 11) + 1ull) * 0x1.0p-53;
@@ -344,7 +349,8 @@ __global__ void __launch_bounds__(256) k_finalize(void* __restrict__ recs, int d
     hd->code_bits = s_code_bits;
     hd->words = (a.total_bits + 31) / 32;
     hd->flags = (a.is_key ? kFlagKey : 0u) | (m > 0 ? kFlagQjl : 0u) | (a.normalize ? kFlagNormalize : 0u) |
-                (a.rotation ? kFlagRandomRotation : 0u) | (a.cumvar > 0.0 ? kFlagCumvar : 0u);
+                (a.rotation ? kFlagRandomRotation : 0u) | (a.cumvar > 0.0 ? kFlagCumvar : 0u) |
+                (a.fitted ? kFlagFitted : 0u);
     hd->stream = h;
     hd->max_bits = a.max_bits;
     hd->seed = a.seed;
@@ -456,6 +462,139 @@ __global__ void __launch_bounds__(256) k_random_basis(const double* __restrict__
 }
 
 // ---------------------------------------------------------------------------
+// Fitted per-regime codebooks (SpectralQuant README, "Repository Structure":
+// nonuniform_quantization.py, Lloyd-Max with per-regime codebooks; the
+// conftest fixture gaussian_data_1d: a Lloyd-Max quantizer fitted to samples).
+// Regime 0 holds the coordinates i < d_eff, regime 1 the rest; each width a
+// regime uses gets a codebook fitted by Lloyd's algorithm to the pooled
+// scaled coordinates z of the calibration vectors over the regime's
+// coordinates of that width, from the Gaussian Lloyd-Max codebook, for a
+// fixed number of iterations: thresholds at the midpoints of neighbouring
+// levels, each sample coded as the compressor codes it (the number of
+// thresholds strictly below), each level moved to the mean of its samples, a
+// level without samples kept.
+// ---------------------------------------------------------------------------
+
+constexpr int kFitIters = 30;   // Lloyd iterations of the fit unless the caller sets another count
+
+// z[h][t][i] = (V^T u_t)_i / sigma_i, u = x / ||x|| (normalized records) or x;
+// 0 where sigma_i = 0 or ||x|| = 0. Grid (token groups of 8, heads), 256
+// threads: warp w takes one token, lane i coordinates i, i + 32, ...
+template <typename T>
+__global__ void __launch_bounds__(256) k_fit_z(const T* __restrict__ x, int d, int64_t n_tok, int64_t stride_head,
+                                               int64_t stride_tok, const void* __restrict__ recs,
+                                               double* __restrict__ z) {
+  __shared__ double xs[8][kMaxD];
+  const int h = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * 8 + warp;
+  Rec rec = rec_at(recs, d, h);
+  const RecHeader* hd = rec.hdr();
+  if (t >= n_tok || !(hd->flags & kFlagFitted) || hd->derived_valid == 0u) return;
+  const T* xt = x + (size_t)h * stride_head + (size_t)t * stride_tok;
+  double ss = 0.0;
+  for (int j = lane; j < d; j += 32) {
+    const double v = (double)to_float<T>(xt[j]);
+    xs[warp][j] = v;
+    ss += v * v;
+  }
+  ss = warp_sum(ss);
+  __syncwarp();
+  const bool normalize = (hd->flags & kFlagNormalize) != 0u;
+  const double nrm = normalize ? sqrt(ss) : 1.0;
+  const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
+  const double* V = rec.V();
+  const double* sig = rec.sigma();
+  double* zt = z + ((size_t)h * n_tok + t) * d;
+  for (int i = lane; i < d; i += 32) {
+    double y = 0.0;
+    for (int j = 0; j < d; ++j) y = fma(V[(size_t)j * d + i], xs[warp][j], y);
+    y *= inv;
+    zt[i] = sig[i] > 0.0 ? y / sig[i] : 0.0;
+  }
+}
+
+// One codebook per block: grid (heads, 2 regimes, widths 1..SQ_MAX_BITS),
+// 256 threads. Widths up to 3 sum in registers (per thread, then per warp);
+// wider ones in shared memory.
+__global__ void __launch_bounds__(256) k_fit_lloyd(const double* __restrict__ z, int d, int64_t n_tok,
+                                                   void* __restrict__ recs, int iters) {
+  __shared__ int cols[kMaxD];
+  __shared__ int s_nc;
+  __shared__ double lvl[256], thr[255], sums[256];
+  __shared__ unsigned long long cnts[256];
+  const int h = blockIdx.x, r = blockIdx.y, b = blockIdx.z + 1, tid = threadIdx.x, lane = tid & 31;
+  Rec rec = rec_at(recs, d, h);
+  const RecHeader* hd = rec.hdr();
+  if (!(hd->flags & kFlagFitted) || hd->derived_valid == 0u) return;
+  const int nl = 1 << b;
+  if (tid == 0) {
+    int nc = 0;
+    for (int i = 0; i < d; ++i)
+      if ((int)rec.bits()[i] == b && ((i >= hd->d_eff) ? 1 : 0) == r) cols[nc++] = i;
+    s_nc = nc;
+  }
+  double* lv_out = rec.fit_lv() + r * kLevelsTotal + lv_off(b);
+  double* th_out = rec.fit_th() + r * kThreshTotal + th_off(b);
+  for (int k = tid; k < nl; k += 256) lvl[k] = lv_out[k];
+  __syncthreads();
+  const int nc = s_nc;
+  if (nc == 0) return;
+  // samples (t, c): token t, coordinate cols[c]; thread tid starts at the
+  // tid-th and steps by 256 (st_t tokens and st_c columns, with carry)
+  const int st_t = 256 / nc, st_c = 256 % nc;
+  const double* zh = z + (size_t)h * n_tok * d;
+  for (int it = 0; it < iters; ++it) {
+    for (int k = tid; k + 1 < nl; k += 256) thr[k] = 0.5 * (lvl[k] + lvl[k + 1]);
+    for (int k = tid; k < nl; k += 256) { sums[k] = 0.0; cnts[k] = 0ull; }
+    __syncthreads();
+    if (b <= 3) {
+      double ps[8];
+      unsigned pc[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) { ps[k] = 0.0; pc[k] = 0u; }
+      for (int64_t t = tid / nc, c = tid % nc; t < n_tok;) {
+        const double zv = zh[(size_t)t * d + cols[c]];
+        const int code = code_of(zv, thr, b);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (k == code) { ps[k] += zv; pc[k] += 1u; }
+        c += st_c;
+        t += st_t;
+        if (c >= nc) { c -= nc; ++t; }
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k >= nl) break;
+        const double sv = warp_sum(ps[k]);
+        unsigned cv = pc[k];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cv += __shfl_xor_sync(0xffffffffu, cv, o);
+        if (lane == 0) {
+          atomicAdd(&sums[k], sv);
+          atomicAdd(&cnts[k], (unsigned long long)cv);
+        }
+      }
+    } else {
+      for (int64_t t = tid / nc, c = tid % nc; t < n_tok;) {
+        const double zv = zh[(size_t)t * d + cols[c]];
+        const int code = code_of(zv, thr, b);
+        atomicAdd(&sums[code], zv);
+        atomicAdd(&cnts[code], 1ull);
+        c += st_c;
+        t += st_t;
+        if (c >= nc) { c -= nc; ++t; }
+      }
+    }
+    __syncthreads();
+    for (int k = tid; k < nl; k += 256)
+      if (cnts[k] > 0ull) lvl[k] = sums[k] / (double)cnts[k];
+    __syncthreads();
+  }
+  for (int k = tid; k < nl; k += 256) lv_out[k] = lvl[k];
+  for (int k = tid; k + 1 < nl; k += 256) th_out[k] = 0.5 * (lvl[k] + lvl[k + 1]);
+}
+
+// ---------------------------------------------------------------------------
 // Import: validate canonical parts written elsewhere and build derived parts.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_import(void* __restrict__ recs, int d, int* __restrict__ status) {
@@ -475,6 +614,19 @@ __global__ void __launch_bounds__(256) k_import(void* __restrict__ recs, int d, 
         o += b;
       }
       ok = ok && (o == hd->code_bits);
+    }
+    if (ok && (hd->flags & kFlagFitted)) {
+      // fitted codebooks: finite, and strictly increasing levels for every
+      // width a coordinate of the regime uses
+      for (int i = 0; i < d && ok; ++i) {
+        const int b = rec.bits()[i];
+        if (b == 0) continue;
+        const int r = (i >= hd->d_eff) ? 1 : 0;
+        const double* l = rec.fit_lv() + r * kLevelsTotal + lv_off(b);
+        const double* t = rec.fit_th() + r * kThreshTotal + th_off(b);
+        for (int k = 0; k < (1 << b) && ok; ++k) ok = isfinite(l[k]) && (k == 0 || l[k] > l[k - 1]);
+        for (int k = 0; k + 1 < (1 << b) && ok; ++k) ok = isfinite(t[k]) && t[k] >= l[k] && t[k] <= l[k + 1];
+      }
     }
     s_ok = ok;
     hd->derived_valid = 0u;

@@ -17,10 +17,28 @@ namespace sq {
 
 constexpr int kCodecWarps = 4;
 
+// The codebooks that code a record's coordinates, staged into shared memory as
+// th[2][kThreshTotal] and lv[2][kLevelsTotal]: the record's per-regime tables
+// fitted to its calibration data (flag kFlagFitted; SpectralQuant README,
+// "Repository Structure": Lloyd-Max with per-regime codebooks), or the shared
+// Gaussian Lloyd-Max tables in both halves.
+__device__ inline void stage_codebooks(const Rec& rec, double* th, double* lv, int tid, int nth) {
+  const bool fit = (rec.hdr()->flags & kFlagFitted) != 0;
+  const double* ft = rec.fit_th();
+  const double* fl = rec.fit_lv();
+  for (int e = tid; e < 2 * kThreshTotal; e += nth) th[e] = fit ? ft[e] : c_th64[e % kThreshTotal];
+  for (int e = tid; e < 2 * kLevelsTotal; e += nth) lv[e] = fit ? fl[e] : c_lv64[e % kLevelsTotal];
+}
+// Regime of coordinate i: 1 (noise) for i >= d_eff in a record with fitted
+// codebooks, else 0 (the signal regime, or the shared tables).
+__device__ __forceinline__ int regime_of(const RecHeader* h, int i) {
+  return ((h->flags & kFlagFitted) != 0u && i >= h->d_eff) ? 1 : 0;
+}
+
 // Shared-memory bytes of k_compress_ref / k_decompress_ref for head_dim d.
 __host__ __device__ inline size_t codec_ref_smem(int d) {
   size_t v = d <= 128 ? (size_t)8 * d * (d + 1) : 0;             // V (padded rows) in float64
-  return v + (size_t)8 * (kThreshTotal + kLevelsTotal)             // tables
+  return v + (size_t)16 * (kThreshTotal + kLevelsTotal)            // tables (two regimes)
          + (size_t)8 * d * 2                                      // sigma, 1/sigma
          + (size_t)4 * d * 2                                      // bits, offsets
          + (size_t)kCodecWarps * (8 * d + 4 * kMaxWords + 8 * d);        // per warp: x row, words, residual
@@ -39,9 +57,10 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   Rec rec = rec_at(recs, d, h);
   const RecHeader* hd = rec.hdr();
-  if (min_m > 0) {   // second pass after another kernel: only heads with m >= min_m, no flags
+  if (min_m > 0) {   // second pass after another kernel: heads with m >= min_m or fitted codebooks, no flags
     const int64_t sp0 = start_pos ? (int64_t)start_pos[b] : 0;
-    if (!record_ok(hd, d) || hd->words != c.words || hd->m < min_m || c.rnorm == nullptr || sp0 < 0 ||
+    const bool take = hd->m >= min_m || (hd->flags & kFlagFitted) != 0u;
+    if (!record_ok(hd, d) || hd->words != c.words || !take || (hd->m > 0 && c.rnorm == nullptr) || sp0 < 0 ||
         sp0 + n_tok > c.cap)
       return;
   }
@@ -58,8 +77,8 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
   const int ld = d + 1;
   unsigned char* p = sm;
   double* Vs = (double*)p;            p += vsm ? (size_t)8 * d * ld : 0;
-  double* th = (double*)p;            p += 8 * kThreshTotal;
-  double* lv = (double*)p;            p += 8 * kLevelsTotal;
+  double* th = (double*)p;            p += 16 * kThreshTotal;
+  double* lv = (double*)p;            p += 16 * kLevelsTotal;
   double* sig = (double*)p;           p += 8 * d;
   double* isig = (double*)p;          p += 8 * d;
   int* bits = (int*)p;                p += 4 * d;
@@ -71,8 +90,7 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
   const double* Vg = rec.V();
   if (vsm)
     for (int e = threadIdx.x; e < d * d; e += blockDim.x) Vs[(e / d) * ld + e % d] = Vg[e];
-  for (int e = threadIdx.x; e < kThreshTotal; e += blockDim.x) th[e] = c_th64[e];
-  for (int e = threadIdx.x; e < kLevelsTotal; e += blockDim.x) lv[e] = c_lv64[e];
+  stage_codebooks(rec, th, lv, threadIdx.x, blockDim.x);
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
     double s = rec.sigma()[i];
     sig[i] = s;
@@ -110,13 +128,14 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
       y *= inv;
       int bw = bits[i];
       int code = 0;
+      const int rg = regime_of(hd, i);
       if (bw > 0) {
-        code = code_of(y * isig[i], th + th_off(bw), bw);
+        code = code_of(y * isig[i], th + rg * kThreshTotal + th_off(bw), bw);
         int o = offs[i], wi = o >> 5, sh = o & 31;
         atomicOr(&wb[wi], (uint32_t)code << sh);
         if (sh + bw > 32) atomicOr(&wb[wi + 1], (uint32_t)code >> (32 - sh));
       }
-      if (i < m) rs[i] = y - sig[i] * (bw > 0 ? lv[lv_off(bw) + code] : 0.0);
+      if (i < m) rs[i] = y - sig[i] * (bw > 0 ? lv[rg * kLevelsTotal + lv_off(bw) + code] : 0.0);
     }
     __syncwarp();
     float rho = 0.0f;
@@ -161,7 +180,7 @@ inline int append_nv(int64_t nvec) { return nvec <= 1 ? 1 : (nvec <= 2 ? 2 : (nv
 
 // Shared-memory bytes of append_body<T, NV>.
 __host__ __device__ constexpr size_t append_smem(int nv) {
-  return (size_t)nv * kMaxD * 8 + (size_t)nv * 256 * 8 + (size_t)kThreshTotal * 8 + (size_t)kLevelsTotal * 8 +
+  return (size_t)nv * kMaxD * 8 + (size_t)nv * 256 * 8 + (size_t)kThreshTotal * 16 + (size_t)kLevelsTotal * 16 +
          (size_t)nv * kMaxWords * 4 + (size_t)nv * 8 + (size_t)nv * 4 + 64;
 }
 
@@ -175,8 +194,8 @@ __device__ void append_body(const uint8_t* __restrict__ recs, const T* __restric
   double (*xs)[kMaxD] = (double (*)[kMaxD])sm;                            // input, then the signal residual
   double (*ys)[256] = (double (*)[256])(sm + (size_t)NV * kMaxD * 8);    // partial sums of V^T x
   double* th = (double*)(sm + (size_t)NV * kMaxD * 8 + (size_t)NV * 256 * 8);
-  double* lv = th + kThreshTotal;
-  uint32_t (*wb)[kMaxWords] = (uint32_t (*)[kMaxWords])(lv + kLevelsTotal);
+  double* lv = th + 2 * kThreshTotal;
+  uint32_t (*wb)[kMaxWords] = (uint32_t (*)[kMaxWords])(lv + 2 * kLevelsTotal);
   double* s_inv = (double*)(wb + NV);
   int* s_ok = (int*)(s_inv + NV);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -205,8 +224,7 @@ __device__ void append_body(const uint8_t* __restrict__ recs, const T* __restric
   double vv[UB];
 #pragma unroll
   for (int u = 0; u < UB; ++u) vv[u] = j_beg + u < j_end ? V[(size_t)(j_beg + u) * d + i_col] : 0.0;
-  for (int e = tid; e < kThreshTotal; e += 256) th[e] = c_th64[e];
-  for (int e = tid; e < kLevelsTotal; e += 256) lv[e] = c_lv64[e];
+  stage_codebooks(rec, th, lv, tid, 256);
   for (int e = tid; e < NV * kMaxWords; e += 256) wb[e / kMaxWords][e % kMaxWords] = 0u;
   // inputs (vectors past the end, or of rows over capacity, are zeros and not stored)
   if (tid < NV) {
@@ -282,14 +300,15 @@ __device__ void append_body(const uint8_t* __restrict__ recs, const T* __restric
     y *= s_inv[v];
     const int bw = bits[i];
     const double s = sig[i];
+    const int rg = regime_of(hd, i);
     int code = 0;
     if (bw > 0) {
-      code = code_of(s > 0.0 ? y * (1.0 / s) : 0.0, th + th_off(bw), bw);
+      code = code_of(s > 0.0 ? y * (1.0 / s) : 0.0, th + rg * kThreshTotal + th_off(bw), bw);
       const int o = offs[i], wi = o >> 5, sh = o & 31;
       atomicOr(&wb[v][wi], (uint32_t)code << sh);
       if (sh + bw > 32) atomicOr(&wb[v][wi + 1], (uint32_t)code >> (32 - sh));
     }
-    if (i < m) xs[v][i] = y - s * (bw > 0 ? lv[lv_off(bw) + code] : 0.0);
+    if (i < m) xs[v][i] = y - s * (bw > 0 ? lv[rg * kLevelsTotal + lv_off(bw) + code] : 0.0);
   }
   __syncthreads();
   // rho and the QJL sign bits: warp v
@@ -359,8 +378,8 @@ __global__ void __launch_bounds__(128) k_decompress_ref(const uint8_t* __restric
   const int ld = d + 1;
   unsigned char* p = sm;
   double* Vs = (double*)p;            p += vsm ? (size_t)8 * d * ld : 0;
-  p += 8 * kThreshTotal;
-  double* lv = (double*)p;            p += 8 * kLevelsTotal;
+  double* th = (double*)p;            p += 16 * kThreshTotal;
+  double* lv = (double*)p;            p += 16 * kLevelsTotal;
   double* sig = (double*)p;           p += 8 * d;
   p += 8 * d;
   int* bits = (int*)p;                p += 4 * d;
@@ -371,7 +390,7 @@ __global__ void __launch_bounds__(128) k_decompress_ref(const uint8_t* __restric
   const double* Vg = rec.V();
   if (vsm)
     for (int e = threadIdx.x; e < d * d; e += blockDim.x) Vs[(e / d) * ld + e % d] = Vg[e];
-  for (int e = threadIdx.x; e < kLevelsTotal; e += blockDim.x) lv[e] = c_lv64[e];
+  stage_codebooks(rec, th, lv, threadIdx.x, blockDim.x);
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
     sig[i] = rec.sigma()[i];
     bits[i] = rec.bits()[i];
@@ -392,7 +411,7 @@ __global__ void __launch_bounds__(128) k_decompress_ref(const uint8_t* __restric
     __syncwarp();
     for (int i = lane; i < d; i += 32) {
       int bw = bits[i];
-      ws[i] = bw > 0 ? sig[i] * lv[lv_off(bw) + (int)field(wb, offs[i], bw)] : 0.0;
+      ws[i] = bw > 0 ? sig[i] * lv[regime_of(hd, i) * kLevelsTotal + lv_off(bw) + (int)field(wb, offs[i], bw)] : 0.0;
     }
     __syncwarp();
     if (qjl) {

@@ -14,6 +14,8 @@
 
 namespace sq {
 
+static_assert(append_smem(8) <= prep_smem(kMaxD), "the fused step's shared memory holds every append role");
+
 // Blocks [0, n_app): keys of head i % n_kv, rows of group i / n_kv; [n_app,
 // 2 n_app): the same for values; then one prepare block per (KV head, row
 // group of prep_rows(G)). 256 threads; shared memory max(append_smem(NV),

@@ -16,10 +16,11 @@
 namespace sq {
 
 constexpr uint32_t kMagic = 0x31435153u;
-constexpr uint32_t kVersion = 1u;
+constexpr uint32_t kVersion = 2u;
 constexpr int kHeader = 128;
 constexpr int kMaxD = 256;
-constexpr uint32_t kFlagKey = 1u, kFlagQjl = 2u, kFlagNormalize = 4u, kFlagRandomRotation = 8u, kFlagCumvar = 16u;
+constexpr uint32_t kFlagKey = 1u, kFlagQjl = 2u, kFlagNormalize = 4u, kFlagRandomRotation = 8u, kFlagCumvar = 16u,
+                   kFlagFitted = 32u;
 constexpr int kMaxWords = 64;   // B <= 8 bits x 256 coordinates
 
 // Packed-cache layout: the records of 32 consecutive tokens of one (batch,
@@ -51,10 +52,14 @@ __host__ __device__ constexpr int th_off(int b) { return (1 << b) - 1 - b; }
 constexpr int kLevelsTotal = lv_off(SQ_MAX_BITS + 1);      // 510
 constexpr int kThreshTotal = th_off(SQ_MAX_BITS + 1);      // 502
 
-// Host-side record geometry (must match sq.h).
-__host__ __device__ inline size_t canon_bytes(int d) {
+// Host-side record geometry (must match sq.h). The canonical part ends with
+// the fitted-codebook section: levels [2][kLevelsTotal] and thresholds
+// [2][kThreshTotal] in float64 (regime 0: coordinates below d_eff, 1: the rest).
+constexpr size_t kFitBytes = 8u * 2u * ((size_t)kLevelsTotal + (size_t)kThreshTotal);
+__host__ __device__ inline size_t fit_off(int d) {
   return (size_t)kHeader + 21u * (size_t)d + 16u * (size_t)d * (size_t)d;
 }
+__host__ __device__ inline size_t canon_bytes(int d) { return fit_off(d) + kFitBytes; }
 __host__ __device__ inline size_t derived_off(int d) { return (canon_bytes(d) + 255u) & ~(size_t)255u; }
 // Derived part: float32 copies used by the kernels,
 //   sigma_f[d], inv_sigma_f[d], pad to 256 B, V_f[d*d] (same layout as V), S_f[d*d],
@@ -95,6 +100,8 @@ struct Rec {
   __host__ __device__ double* S() const { return (double*)(base + kHeader + 16 * d + 8 * d * d); }
   __host__ __device__ uint8_t* bits() const { return base + kHeader + 16 * d + 16 * d * d; }
   __host__ __device__ int32_t* offsets() const { return (int32_t*)(base + kHeader + 17 * d + 16 * d * d); }
+  __host__ __device__ double* fit_lv() const { return (double*)(base + fit_off(d)); }
+  __host__ __device__ double* fit_th() const { return (double*)(base + fit_off(d)) + 2 * kLevelsTotal; }
   __host__ __device__ uint8_t* derived() const { return base + derived_off(d); }
   __host__ __device__ float* sigma_f() const { return (float*)derived(); }
   __host__ __device__ float* inv_sigma_f() const { return (float*)derived() + d; }

@@ -612,6 +612,8 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
     Rec rec = rec_at(P.recs, D, h);
     const RecHeader* hd = rec.hdr();
     const bool rec_ok = record_ok(hd, D) && hd->words == P.c.words && (hd->m == 0 || P.c.rnorm != nullptr);
+    // records with fitted codebooks are left to the reference kernel's second pass
+    const bool fitted = (hd->flags & kFlagFitted) != 0u;
     const int64_t sp = P.start_pos ? (int64_t)P.start_pos[bidx] : 0;
     const bool cap_ok = sp >= 0 && sp + P.n_tok <= P.c.cap;
     if (threadIdx.x == 0 && err) {
@@ -619,7 +621,7 @@ k_compress_tc(const __grid_constant__ CUtensorMap tmap, Params P, const __grid_c
       else if (!cap_ok) atomicOr(err, SQ_FLAG_CAPACITY);
     }
     const int m = rec_ok ? hd->m : 0;
-    if (!rec_ok || !cap_ok || m > MSIG) {   // m > MSIG: the reference kernel takes this head
+    if (!rec_ok || !cap_ok || m > MSIG || fitted) {   // m > MSIG, fitted: the reference kernel takes this head
       s0 = s1;
       continue;
     }

@@ -338,8 +338,9 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   float* uq = ws + (size_t)s.batch * s.n_q * D;
   float* acc_out = uq + (size_t)s.batch * s.n_q * D;
   float* ml_out = acc_out + (size_t)s.batch * s.n_q * s.splits * D;
+  // (records with fitted codebooks are served by the SIMT kernel: refused here)
   const bool ok = record_ok(hk, D) && record_ok(hv, D) && hk->words == kc.words && hv->words == vc.words &&
-                  (hk->m == 0 || kc.rnorm != nullptr);
+                  (hk->m == 0 || kc.rnorm != nullptr) && ((hk->flags | hv->flags) & kFlagFitted) == 0u;
   int64_t L = attn_len(seq_lens, s, b);
   if (L < 0 || L > s.max_ctx || L > kc.cap) {
     if (tid == 0 && split == 0 && g == 0 && flags) atomicOr(flags, SQ_FLAG_SEQLEN);

@@ -36,7 +36,7 @@ class sq_calib_params(ctypes.Structure):
                 ("is_key", ctypes.c_int), ("qjl", ctypes.c_int), ("normalize", ctypes.c_int),
                 ("d_eff_override", ctypes.c_int), ("max_bits", ctypes.c_int), ("seed", ctypes.c_uint64),
                 ("max_sweeps", ctypes.c_int), ("tol", ctypes.c_double), ("rotation", ctypes.c_int),
-                ("cumvar", ctypes.c_double)]
+                ("cumvar", ctypes.c_double), ("codebooks", ctypes.c_int), ("fit_iters", ctypes.c_int)]
 
 
 class sq_cache(ctypes.Structure):
@@ -139,12 +139,15 @@ def sq_calib_bytes(d: int) -> int:
 
 
 def calib_params(d, n_heads, avg_bits, is_key, qjl=True, normalize=True, d_eff_override=0, max_bits=8,
-                 seed=42, max_sweeps=30, tol=1e-13, rotation=0, cumvar=0.0) -> sq_calib_params:
+                 seed=42, max_sweeps=30, tol=1e-13, rotation=0, cumvar=0.0, codebooks=0,
+                 fit_iters=0) -> sq_calib_params:
     """rotation: 0 calibrated eigenbasis, 1 random rotation (A/B baseline);
-    cumvar: 0 participation-ratio d_eff, else the cumulative-variance fraction."""
+    cumvar: 0 participation-ratio d_eff, else the cumulative-variance fraction;
+    codebooks: 0 shared Gaussian Lloyd-Max, 1 per-regime codebooks fitted to the
+    calibration vectors (fit_iters Lloyd iterations, 0 = the library's 30)."""
     return sq_calib_params(d, n_heads, float(avg_bits), int(bool(is_key)), int(bool(qjl)), int(bool(normalize)),
                            int(d_eff_override), int(max_bits), int(seed) & ((1 << 64) - 1), int(max_sweeps),
-                           float(tol), int(rotation), float(cumvar))
+                           float(tol), int(rotation), float(cumvar), int(codebooks), int(fit_iters))
 
 
 def sq_record_words(params: sq_calib_params) -> int:

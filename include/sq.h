@@ -76,7 +76,9 @@ typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2 } sq_dtype;
 #define SQ_FLAG_TIMEOUT 0x80000000u
 
 #define SQ_MAX_BITS 8         /* largest code width of one coordinate                     */
-#define SQ_ABI_VERSION 2   /* 2: word-interleaved 32-token blocks in sq_cache.codes */
+#define SQ_ABI_VERSION 3   /* 2: word-interleaved 32-token blocks in sq_cache.codes;
+                              3: records of version 2 (fitted-codebook section),
+                                 sq_calib_params.codebooks and .fit_iters */
 
 /*
  * Calibration parameters (host struct).
@@ -107,6 +109,23 @@ typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2 } sq_dtype;
  *                 smallest k >= 1 whose top-k lambda hold at least this fraction
  *                 of the trace (the README's results/deff_sweep/ compares
  *                 "participation ratio vs cumvar").
+ *  codebooks      0: every coordinate is coded with the shared unit-Gaussian
+ *                 Lloyd-Max codebook of its width; 1: per-regime codebooks
+ *                 fitted to the calibration vectors (README "Repository
+ *                 Structure": nonuniform_quantization.py, "Lloyd-Max with
+ *                 per-regime codebooks"). Regime 0 is the coordinates i < d_eff,
+ *                 regime 1 the rest; for each width a regime uses, Lloyd's
+ *                 algorithm runs from the Gaussian codebook on the pooled scaled
+ *                 coordinates z = (V^T u)_i / sigma_i of the calibration vectors
+ *                 over the regime's coordinates of that width: thresholds at the
+ *                 midpoints of neighbouring levels, each sample coded as the
+ *                 compressor codes it, each level moved to the mean of its
+ *                 samples (a level without samples kept). Records with fitted
+ *                 codebooks are compressed by the float64 reference kernels and
+ *                 attended by the SIMT kernel (SQ_OPT_ATTN_PATH 1): the tensor-
+ *                 core attention kernels refuse them with SQ_FLAG_RECORD.
+ *  fit_iters      Lloyd iterations of the fit (0: 30). The sums of a fit are
+ *                 accumulated with atomics, in an order that varies between runs.
  */
 typedef struct {
   int d;
@@ -122,6 +141,8 @@ typedef struct {
   double tol;
   int rotation;
   double cumvar;
+  int codebooks;
+  int fit_iters;
 } sq_calib_params;
 
 /*
@@ -165,7 +186,7 @@ typedef struct {
  *
  *  offset               type  field
  *  0                    u32   magic 0x31435153 ("SQC1")
- *  4                    u32   version 1
+ *  4                    u32   version 2
  *  8                    i32   d
  *  12                   i32   d_eff (participation ratio (sum l)^2 / sum l^2, rounded half to even)
  *  16                   i32   m (QJL sign dimensions, 0 without QJL)
@@ -173,7 +194,7 @@ typedef struct {
  *  24                   i32   code_bits = sum of b_i = B - m
  *  28                   i32   words = ceil(B / 32)
  *  32                   u32   flags: 1 key, 2 QJL, 4 normalized, 8 random rotation,
- *                             16 cumulative-variance d_eff
+ *                             16 cumulative-variance d_eff, 32 fitted codebooks
  *  36                   i32   eigensolver sweeps used
  *  40                   i32   stream (head index of the QJL Gaussian stream)
  *  44                   i32   max_bits
@@ -190,6 +211,11 @@ typedef struct {
  *  128 + 16d + 8d^2     f64   S[d*d]: the m x m QJL matrix, row-major, in the first m*m slots
  *  128 + 16d + 16d^2    u8    bits[d]: code width b_i (greedy water-filling)
  *  128 + 17d + 16d^2    i32   offset[d]: bit position of coordinate i's code
+ *  128 + 21d + 16d^2    f64   fitted levels [2][510]: regime r (0: i < d_eff, 1: the rest),
+ *                             width b at r * 510 + 2^b - 2, 2^b ascending levels;
+ *                             zero unless flag 32
+ *  8288 + 21d + 16d^2   f64   fitted thresholds [2][502]: width b at r * 502 + 2^b - 1 - b,
+ *                             2^b - 1 ascending thresholds (midpoints of the levels)
  *  then, from the next 256-byte boundary: the library's derived part (private).
  */
 size_t sq_calib_bytes(int d);
@@ -274,7 +300,9 @@ sq_status sq_calibrate(const sq_calib_params* p, const void* x, sq_dtype dtype, 
 /*
  * Imports n_heads records whose canonical part was written elsewhere (saved
  * records, or another implementation): checks each header (magic, version,
- * d, bit counts, offsets) and builds the library's derived part. The record
+ * d, bit counts, offsets; with fitted codebooks, finite tables whose levels
+ * increase and whose thresholds lie between them for every width in use) and
+ * builds the library's derived part. The record
  * holds what the README's "Overview" calls the one-time calibration (the
  * calibrated eigenbasis, d_eff and kappa of calibration.py, the water-filled
  * widths); importing lets a calibration computed once be reused.

@@ -41,7 +41,7 @@ def test_exports_every_declared_symbol(libsq):
 
 
 def test_status_strings_and_version(libsq):
-    assert sq.sq_abi_version() == 2
+    assert sq.sq_abi_version() == 3
     for s in range(8):
         assert sq.sq_status_str(s) and "unknown" not in sq.sq_status_str(s)
     assert "unknown" in sq.sq_status_str(99)
