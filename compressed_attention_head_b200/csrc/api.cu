@@ -1,5 +1,6 @@
 // libsq host entry points: argument checks, per-device table upload, launches.
 // The public contract (arguments, layouts, ownership, errors) is in include/sq.h.
+#include <algorithm>
 #include <cstdio>
 #include <mutex>
 
@@ -220,28 +221,36 @@ int device_sms() {
   return sms;
 }
 
-// tcgen05 decode kernel: record buffers per group that fit (2, else 1), or 0
-// when even one does not (records wider than the kernel's shared memory holds).
-int td_nrec(int d, int wk, int wv) {
-  for (int nrec = 2; nrec >= 1; --nrec) {
-    const size_t need = d == 64 ? td::smem_bytes<64>(wk, wv, nrec)
-                                : (d == 128 ? td::smem_bytes<128>(wk, wv, nrec) : td::smem_bytes<256>(wk, wv, nrec));
-    if (need <= (size_t)kTdSmemLimit) return nrec;
-  }
-  return 0;
-}
+// tcgen05 decode kernel: the warp groups whose regions fit in shared memory
+// (as many as the kernel has, else fewer) and the record buffers per group
+// (2, else 1); ng = 0 when not even one group with one buffer fits.
 int td_groups(int d) { return d == 64 ? td::Cfg<64>::NG : (d == 128 ? td::Cfg<128>::NG : td::Cfg<256>::NG); }
+size_t td_smem(int d, int wk, int wv, int nrec, int ng) {
+  return d == 64 ? td::smem_bytes<64>(wk, wv, nrec, ng)
+                 : (d == 128 ? td::smem_bytes<128>(wk, wv, nrec, ng) : td::smem_bytes<256>(wk, wv, nrec, ng));
+}
+void td_config(int d, int wk, int wv, int* nrec_out, int* ng_out) {
+  *nrec_out = 0;
+  *ng_out = 0;
+  for (int ng = td_groups(d); ng >= 1; --ng)
+    for (int nrec = 2; nrec >= 1; --nrec)
+      if (td_smem(d, wk, wv, nrec, ng) <= (size_t)kTdSmemLimit) {
+        *nrec_out = nrec;
+        *ng_out = ng;
+        return;
+      }
+}
 
 // Splits of the context for the tcgen05 kernel: one block per SM, whose NG
 // warp groups take its 128-token tiles in turn. With equal blocks in
 // ceil(blocks / SMs) waves, the cost of S splits is waves(S) x (1 + tiles per
 // group), the 1 standing for the block's setup (tables, query operand, merge);
 // the cheapest S wins (the smaller on ties).
-int attn_splits_td(int batch, int n_kv, int d, int64_t max_ctx) {
+int attn_splits_td(int batch, int n_kv, int64_t max_ctx, int ngroups) {
   const int64_t units = (int64_t)batch * n_kv;
   const int64_t slots = (int64_t)device_sms();
   const int64_t ctx = max_ctx > 0 ? max_ctx : 1;
-  const int64_t ng = td_groups(d);
+  const int64_t ng = ngroups > 0 ? ngroups : 1;
   int best = 1;
   int64_t best_cost = INT64_MAX;
   for (int64_t S = 1; S <= 256; ++S) {
@@ -654,9 +663,9 @@ sq_status sq_decompress_kv(const void* calib, const sq_cache* cache, int d, int6
 size_t sq_attn_workspace(int batch, int n_q_heads, int n_kv_heads, int d, int64_t max_ctx) {
   if (batch < 1 || n_q_heads < 1 || n_kv_heads < 1 || !supported_d(d) || max_ctx < 0) return 0;
   // enough for whichever partial kernel the call picks (that depends on the records)
-  const int s1 = attn_splits(batch, n_kv_heads, d, max_ctx);
-  const int s2 = attn_splits_td(batch, n_kv_heads, d, max_ctx);
-  return attn_ws_bytes(batch, n_q_heads, n_kv_heads, d, s1 > s2 ? s1 : s2);
+  int s = attn_splits(batch, n_kv_heads, d, max_ctx);
+  for (int ng = 1; ng <= td_groups(d); ++ng) s = std::max(s, attn_splits_td(batch, n_kv_heads, max_ctx, ng));
+  return attn_ws_bytes(batch, n_q_heads, n_kv_heads, d, s);
 }
 
 }  // extern "C"
@@ -696,7 +705,8 @@ sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* 
   const int ncb = causal ? (n_qtok + pcols - 1) / pcols : 1;
   const int group = qg * pcols;
   const int rows = batch * ncb;
-  const int nrec = td_nrec(d, kc->words, vc->words);
+  int nrec = 0, ngs = 0;
+  td_config(d, kc->words, vc->words, &nrec, &ngs);
   const bool use_td = g_attn_path == 0 && (d == 64 || d == 128 || d == 256) && group <= 16 && nrec > 0;
   AttnShape sh;
   sh.batch = rows;
@@ -709,7 +719,7 @@ sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* 
   sh.ncb = ncb;
   sh.qg = qg;
   sh.n_qtok = n_qtok;
-  sh.splits = use_td ? attn_splits_td(rows, n_kv_heads, d, max_ctx) : attn_splits(rows, n_kv_heads, d, max_ctx);
+  sh.splits = use_td ? attn_splits_td(rows, n_kv_heads, max_ctx, ngs) : attn_splits(rows, n_kv_heads, d, max_ctx);
   sh.max_ctx = max_ctx;
   sh.len_offset = len_offset;
   int64_t per = (max_ctx + sh.splits - 1) / sh.splits;
@@ -757,8 +767,8 @@ sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* 
   if (use_td) {
     const int MGv = sh.group <= 2 ? 2 : (sh.group <= 4 ? 4 : (sh.group <= 8 ? 8 : 16));
 #define SQ_TD_LAUNCH(DD, MG)                                                                                  \
-  td::k_decode_tc<DD, MG><<<gpart, td::Cfg<DD>::NTH, td::smem_bytes<DD>(kc->words, vc->words, nrec), st>>>( \
-      rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags, nrec, out, (int)out_dtype)
+  td::k_decode_tc<DD, MG><<<gpart, td::Cfg<DD>::NTH, td::smem_bytes<DD>(kc->words, vc->words, nrec, ngs), st>>>( \
+      rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags, nrec, ngs, out, (int)out_dtype)
 #define SQ_TD_G(DD)                                                                                       \
   if (MGv == 2) SQ_TD_LAUNCH(DD, 2); else if (MGv == 4) SQ_TD_LAUNCH(DD, 4); else if (MGv == 8) SQ_TD_LAUNCH(DD, 8); \
   else SQ_TD_LAUNCH(DD, 16)
@@ -864,9 +874,9 @@ size_t sq_attn_prefill_workspace(int batch, int n_q_heads, int n_kv_heads, int d
   const int pcols = prefill_cols(qg);
   const int64_t rows = (int64_t)batch * ((n_qtok + pcols - 1) / pcols);
   if (rows > 65535) return 0;
-  const int s1 = attn_splits((int)rows, n_kv_heads, d, max_ctx);
-  const int s2 = attn_splits_td((int)rows, n_kv_heads, d, max_ctx);
-  return attn_ws_bytes((int)rows, n_kv_heads * qg * pcols, n_kv_heads, d, s1 > s2 ? s1 : s2);
+  int s = attn_splits((int)rows, n_kv_heads, d, max_ctx);
+  for (int ng = 1; ng <= td_groups(d); ++ng) s = std::max(s, attn_splits_td((int)rows, n_kv_heads, max_ctx, ng));
+  return attn_ws_bytes((int)rows, n_kv_heads * qg * pcols, n_kv_heads, d, s);
 }
 
 sq_status sq_attn_prefill(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,

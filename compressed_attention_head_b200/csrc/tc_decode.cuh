@@ -45,22 +45,23 @@ namespace td {
 constexpr int TILE = 128;          // tokens per tile (4 warps x 32)
 constexpr int NW = 16;             // N of every MMA: query heads, padded
 constexpr float kMarginLog2 = 2.0f;   // reference max raised when a score exceeds it by > 2 (log2 units)
-constexpr unsigned kPollSleepNs = 256;   // idle poll interval of the MMA-issuing thread
 
 template <int D>
 struct Cfg {
   static constexpr int NCH = D / 16;                          // 16-coordinate chunks
-  static constexpr int NG = D == 64 ? 4 : (D == 128 ? 3 : 2);  // warp groups decoding tiles
-  // head_dim 256: a warp of its own issues the MMAs of both groups (35 per
-  // tile; issued from a decode warp they held its group back). With three
-  // or four groups the SM's issue slots are the limit and a decode warp of
-  // each group issues its MMAs.
-  static constexpr bool MW = D == 256;
-  static constexpr int NTH = NG * 128 + (MW ? 32 : 0);
-  static constexpr int MH = D > 128 ? 2 : 1;                  // 128-row halves of V^T / O^T
+  // head_dim 256 decodes a tile's keys and values in two halves of 128
+  // coordinates each (the key operand in tensor memory and the V^T tile hold
+  // one half at a time), so that three warp groups fit the SM's 512 TMEM
+  // columns and its shared memory
+  static constexpr bool SPL = D == 256;
+  static constexpr int KCH = SPL ? NCH / 2 : NCH;             // key chunks of the first (or only) part
+  static constexpr int NG = D == 64 ? 4 : 3;                  // warp groups decoding tiles
+  static constexpr int NTH = NG * 128;
+  static constexpr int MH = D > 128 ? 2 : 1;                  // 128-row halves of O^T
   static constexpr int OCOLS = 16 * MH;                       // TMEM columns of O^T
-  static constexpr int AK0 = 8 * (NCH + 1);                   // key operand columns without QJL blocks
-  static constexpr int VT_BYTES = D * TILE * 2;               // K-major V^T tile
+  static constexpr int AK0 = 8 * (KCH + 1);                   // key operand columns of the first part, no QJL
+  static constexpr int VTR = SPL ? 128 : D;                   // coordinate rows of the V^T tile
+  static constexpr int VT_BYTES = VTR * TILE * 2;             // K-major V^T tile
   static constexpr int P_BYTES = NW * TILE * 2;               // K-major P tile
   static constexpr int NKS_MAX = NCH + 2 + NCH;               // score k-steps with m <= D
   static constexpr int W_BYTES = ((NKS_MAX + 3) / 4) * 2048;  // score B operand
@@ -81,8 +82,10 @@ struct Plan {
   static constexpr int HL = L16 + 1024 + 16;           // u32 [kLevelsTotal]: fp16 hi | fp16 lo << 16
   static constexpr int CH = HL + 2048;                 // u32 [2][16]: chunk descriptors K, V
   static constexpr int CD = CH + 128;                  // u32 [2][D]: coordinate descriptors K, V
-  static constexpr int BAR = CD + 8 * D;               // u64 [NG][6]: records x2, scores, PV done, keys in, P in
-  static constexpr int MISC = BAR + 8 * 6 * 4;         // u32 [16]: TMEM base, abort, wmax; u64 setup, drain
+  // u64 [NG][8]: records x2, scores, PV done, drain, spare, first key part
+  // consumed, PV of the first V^T half done
+  static constexpr int BAR = CD + 8 * D;
+  static constexpr int MISC = BAR + 8 * 8 * 4;         // u32 [16]: TMEM base, abort, wmax; u64 setup
   static constexpr int GS = MISC + 64;                 // per group: votes [4], maxima [4][16], l [4][16], mref [16], misc
   static constexpr int GS_BYTES = 16 + 256 + 256 + 64 + 64;
   static constexpr int GRP = (GS + Cfg<D>::NG * GS_BYTES + 1023) & ~1023;   // group regions (1024-aligned)
@@ -133,8 +136,8 @@ __host__ __device__ constexpr size_t group_bytes(int wk, int wv, int nrec) {
          (size_t)nrec * (((size_t)(wk + wv) * TILE * 4 + 3 * TILE * 4 + 1023) & ~(size_t)1023);
 }
 template <int D>
-__host__ __device__ constexpr size_t smem_bytes(int wk, int wv, int nrec) {
-  return (size_t)Plan<D>::GRP + (size_t)Cfg<D>::NG * group_bytes<D>(wk, wv, nrec) + 1024;   // + alignment slack
+__host__ __device__ constexpr size_t smem_bytes(int wk, int wv, int nrec, int ng) {
+  return (size_t)Plan<D>::GRP + (size_t)ng * group_bytes<D>(wk, wv, nrec) + 1024;   // + alignment slack
 }
 
 constexpr uint32_t kMixedChunk = 0xFFu;
@@ -244,19 +247,20 @@ struct ValSink {
   }
 };
 
-// Decodes chunks c0 .. NCH-1 of one side into the sink (keys: column block
-// c + 1, values: chunk c); two neighbouring chunks of one width in one step.
+// Decodes chunks c0 .. c1-1 of one side into the sink (keys: column block
+// c + 1 - shift, values: chunk c - shift of the V^T tile); two neighbouring
+// chunks of one width in one step.
 template <int D, bool KEYS, typename Sink>
 __device__ __forceinline__ void decode_side(const uint32_t* rec, const uint32_t* chd, const uint32_t* cd, int c0,
-                                            int lane, const uint8_t* sm, int p1off, const uint8_t* p3r, uint32_t lb3,
-                                            const unsigned short* l16m1, const Sink& sink) {
-  constexpr int NCH = D / 16;
+                                            int c1, int shift, int lane, const uint8_t* sm, int p1off,
+                                            const uint8_t* p3r, uint32_t lb3, const unsigned short* l16m1,
+                                            const Sink& sink) {
 #pragma unroll 1
-  for (int c = c0; c < NCH;) {
+  for (int c = c0; c < c1;) {
     const uint32_t cw = chd[c];
     const int o = (int)(cw >> 8);
     const uint32_t w = cw & 0xFFu;
-    const bool pair = c + 1 < NCH && w >= 1u && w <= 8u && (chd[c + 1] & 0xFFu) == w;
+    const bool pair = c + 1 < c1 && w >= 1u && w <= 8u && (chd[c + 1] & 0xFFu) == w;
     uint32_t h[16];
     if (pair) {
       switch (w) {
@@ -269,8 +273,8 @@ __device__ __forceinline__ void decode_side(const uint32_t* rec, const uint32_t*
         case 7: decode_chunk<7, 2>(rec, o, lane, sm, p1off, p3r, lb3, h); break;
         default: decode_chunk<8, 2>(rec, o, lane, sm, p1off, p3r, lb3, h); break;
       }
-      sink.put(KEYS ? 8 * (c + 1) : c, h);
-      sink.put(KEYS ? 8 * (c + 2) : c + 1, h + 8);
+      sink.put(KEYS ? 8 * (c + 1 - shift) : c - shift, h);
+      sink.put(KEYS ? 8 * (c + 2 - shift) : c + 1 - shift, h + 8);
       c += 2;
       continue;
     }
@@ -289,7 +293,7 @@ __device__ __forceinline__ void decode_side(const uint32_t* rec, const uint32_t*
       case 8: decode_chunk<8, 1>(rec, o, lane, sm, p1off, p3r, lb3, h); break;
       default: decode_mixed(rec + lane, cd + 16 * c, l16m1, h); break;
     }
-    sink.put(KEYS ? 8 * (c + 1) : c, h);
+    sink.put(KEYS ? 8 * (c + 1 - shift) : c - shift, h);
     ++c;
   }
 }
@@ -319,7 +323,8 @@ template <int D, int MG>
 __global__ void __launch_bounds__(Cfg<D>::NTH, 1)
 k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs_v, CacheArgs kc, CacheArgs vc,
             const int32_t* __restrict__ seq_lens, AttnShape s, float* __restrict__ ws,
-            float* __restrict__ scores_out, uint32_t* __restrict__ flags, int nrec, void* out, int out_dt) {
+            float* __restrict__ scores_out, uint32_t* __restrict__ flags, int nrec, int ngs, void* out,
+            int out_dt) {
   using C = Cfg<D>;
   using PL = Plan<D>;
   constexpr int NCH = C::NCH;
@@ -357,11 +362,12 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   const int m = ok ? hk->m : 0;
   const int nqs = (m + 15) >> 4;
   const int wk = kc.words, wv = vc.words, kcb = ok ? hk->code_bits : 0;
-  // TMEM columns per group: key operand, scores, O^T; as many groups as fit in 512
-  const int ak_cols = C::AK0 + 8 * nqs;
+  // TMEM columns per group: key operand (split: the larger part), scores, O^T;
+  // as many groups as fit in 512 columns and (ngs) in shared memory
+  const int ak_cols = C::SPL ? max(C::AK0, 8 * (C::KCH + nqs)) : C::AK0 + 8 * nqs;
   const int need = ak_cols + NW + C::OCOLS;
   const int gstride = need <= 128 ? 128 : (need <= 256 ? 256 : 512);
-  const int ngr = min(C::NG, 512 / gstride);
+  const int ngr = min(min(C::NG, 512 / gstride), ngs);
   const int col_s = gstride - NW - C::OCOLS;     // scores, then O^T, at the end of the group's columns
   const int col_o = gstride - C::OCOLS;
 
@@ -381,7 +387,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     const int nb = (int)min((int64_t)4, (kc.cap - t0) >> 5);    // whole 32-token blocks inside the cache
     uint8_t* rb = sm + PL::GRP + (size_t)gi * group_bytes<D>(wk, wv, nrec) + C::VT_BYTES + C::P_BYTES +
                   (size_t)bf * rec_buf;
-    uint64_t* bar = bars + 6 * gi + bf;
+    uint64_t* bar = bars + 8 * gi + bf;
     const uint32_t kbytes = (uint32_t)(nb * wk * 128), vbytes = (uint32_t)(nb * wv * 128), nbytes = nb * 128;
     const uint32_t total = kbytes + vbytes + nbytes * (krho ? 3u : 2u);
     sm100::mbar_expect_tx(bar, total);
@@ -398,16 +404,13 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   uint32_t* tCD = (uint32_t*)(sm + PL::CD);
   uint32_t* misc = (uint32_t*)(sm + PL::MISC);    // [0] TMEM base, [1] abort, [2] max |weight| (float bits)
   uint64_t* b_setup = (uint64_t*)(misc + 4);       // level tables copied in
-  uint64_t* b_drain = (uint64_t*)(misc + 6);       // every MMA of the block done (before the free)
   if (tid == 0) {
     misc[1] = 0u;
     misc[2] = 0u;
-    // per group: records x2, scores, PV (one arrival: copy or commit); keys
-    // and P stored (one arrival per thread of the group) with the MMA warp,
-    // else the group's drain (one commit)
-    for (int k = 0; k < 6 * C::NG; ++k) sm100::mbar_init(&bars[k], (k % 6 >= 4 && C::MW) ? 128u : 1u);
+    // per group: records x2, scores, PV, drain, spare, first key part
+    // consumed, first PV half (one arrival each: an expect-tx or a commit)
+    for (int k = 0; k < 8 * C::NG; ++k) sm100::mbar_init(&bars[k], 1u);
     sm100::mbar_init(b_setup, 1);
-    sm100::mbar_init(b_drain, 1);
     sm100::fence_mbar_init();
     // the level tables, and the first record tiles of every group, start
     // arriving while the block builds its other tables and the query operand
@@ -501,14 +504,13 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   uint8_t* sP = gr + C::VT_BYTES;
   uint8_t* sRec = sP + C::P_BYTES;
   uint8_t* gs = sm + PL::GS + grp * PL::GS_BYTES;          // votes [4] (u32), maxima [4][16] (int), l [4][16], mref [16]
-  uint64_t* b_rec = bars + 6 * grp;                          // [0], [1]: records of buffer 0 / 1
-  uint64_t* b_s = bars + 6 * grp + 2;                        // scores ready
-  uint64_t* b_pv = bars + 6 * grp + 3;                       // PV of the group's last tile done
-  uint64_t* b_kf = bars + 6 * grp + 4;                       // the tile's keys are in tensor memory (MW)
-  uint64_t* b_pf = bars + 6 * grp + 5;                       // the tile's V^T and P are in shared memory (MW)
-  uint64_t* b_gdrain = bars + 6 * grp + 4;                   // the group's MMAs done (without MW)
-  const bool mma_warp = warp == 4 * C::NG;
-  const bool issuer = q == 0 && lane == 0 && !mma_warp;     // the group's record copies
+  uint64_t* b_rec = bars + 8 * grp;                          // [0], [1]: records of buffer 0 / 1
+  uint64_t* b_s = bars + 8 * grp + 2;                        // scores ready
+  uint64_t* b_pv = bars + 8 * grp + 3;                       // PV of the group's last tile done
+  uint64_t* b_gdrain = bars + 8 * grp + 4;                   // the group's MMAs done (before the free)
+  uint64_t* b_ka = bars + 8 * grp + 6;                       // split: the first key part's MMAs done
+  uint64_t* b_pv1 = bars + 8 * grp + 7;                      // split: the first V^T half's PV done
+  const bool issuer = q == 0 && lane == 0;                   // the group's copies and MMAs
   const bool active = grp < ngr;
   const int ntg = active && grp < ntile ? (ntile - grp + ngr - 1) / ngr : 0;   // tiles of this group
   const uint32_t gcol = (uint32_t)(grp * gstride);
@@ -522,7 +524,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   const int st_i = lane >> 3, st_c = lane & 7;
   const int st_row = 2 * st_i + (st_c & 1);
   const int st_kc = 4 * q + (st_c >> 1);
-  const uint32_t vt_lane = sm100::smem_u32(sVt) + (uint32_t)((st_kc >> 3) * (D * 128) + st_row * 128 +
+  const uint32_t vt_lane = sm100::smem_u32(sVt) + (uint32_t)((st_kc >> 3) * (C::VTR * 128) + st_row * 128 +
                                                             (((st_kc & 7) ^ st_row) << 4));
   const uint32_t p_lane = sm100::smem_u32(sP) + (uint32_t)((st_kc >> 3) * (NW * 128) + st_row * 128 +
                                                           (((st_kc & 7) ^ st_row) << 4));
@@ -533,94 +535,60 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   if (!sm100::mbar_wait(b_setup, 0u, err)) *abort_flag = 1;   // level tables in shared memory
   int n_issued = min(ntg, nrec);   // tiles whose records were requested (a prefix; the first by thread 0)
   const float LOG2E = 1.4426950408889634f;
-  // The MMAs of a tile of group gi. Scores: A = the keys in tensor memory
-  // (k-step st reads c0 hi for st = 0 and 1, c0 lo for 2, chunk st - 2 =
-  // column block st - 1 after), B = W (four 32-byte k-steps per 2048-byte
-  // atom). PV: O^T += V^T P. Descriptors advance in their start-address
-  // field (16-byte units, no carry out of it).
+  // The MMAs of a tile of group gi. Scores, k-steps [s0, s1): A = the keys in
+  // tensor memory (k-step st reads c0 hi for st = 0 and 1, c0 lo for 2, chunk
+  // st - 2 = column block st - 1 after; the second key part of a split tile
+  // sits sub columns lower), B = W (four 32-byte k-steps per 2048-byte atom).
+  // PV: O^T += V^T P over the V^T tile (split: the coordinate half h).
+  // Descriptors advance in their start-address field (16-byte units, no carry
+  // out of it).
   const int nks = NCH + 2 + nqs;
-  auto issue_scores = [&](int gi) {
-    const uint32_t gc = tmem_base + (uint32_t)(gi * gstride);
-    uint32_t a_col = gc;
-    uint64_t bd = w_desc;
-    for (int st = 0; st < nks; ++st) {
-      sm100::mma_f16_ts(gc + (uint32_t)col_s, a_col, bd, idesc, st > 0 ? 1u : 0u);
+  auto issue_scores = [&](int s0, int s1, int sub, uint64_t* bar) {
+    const uint32_t d_s = tmem_base + gcol + (uint32_t)col_s;
+    uint32_t a_col = tmem_base + gcol + (uint32_t)((s0 < 2 ? 0 : 8 * (s0 - 1)) - sub);
+    uint64_t bd = w_desc + (uint64_t)(((s0 >> 2) * (NW * 128) + (s0 & 3) * 32) >> 4);
+    for (int st = s0; st < s1; ++st) {
+      sm100::mma_f16_ts(d_s, a_col, bd, idesc, st > 0 ? 1u : 0u);
       a_col += st > 0 ? 8u : 0u;
       bd += (st & 3) == 3 ? (uint64_t)((NW * 128 - 96) >> 4) : 2u;
     }
-    sm100::mma_commit(bars + 6 * gi + 2);
+    sm100::mma_commit(bar);
   };
-  auto issue_pv = [&](int gi, int kt) {
-    const uint32_t gc = tmem_base + (uint32_t)(gi * gstride);
-    const uint32_t vt = sm100::smem_u32(sm + PL::GRP + (size_t)gi * group_bytes<D>(wk, wv, nrec));
-    const uint64_t vd = sm100::sw128_desc(vt), pd = sm100::sw128_desc(vt + (uint32_t)C::VT_BYTES);
+  const uint64_t vt_desc = sm100::sw128_desc(sm100::smem_u32(sVt));
+  const uint64_t p_desc = sm100::sw128_desc(sm100::smem_u32(sP));
+  auto issue_pv = [&](int kt, int h, uint64_t* bar) {
 #pragma unroll
     for (int ks = 0; ks < TILE / 16; ++ks) {
-      const uint64_t bd = pd + (uint64_t)(((ks >> 2) * (NW * 128) + (ks & 3) * 32) >> 4);
+      const uint64_t bd = p_desc + (uint64_t)(((ks >> 2) * (NW * 128) + (ks & 3) * 32) >> 4);
 #pragma unroll
-      for (int mh = 0; mh < C::MH; ++mh) {
-        const uint64_t ad = vd + (uint64_t)(((ks >> 2) * (D * 128) + mh * (128 * 128) + (ks & 3) * 32) >> 4);
-        sm100::mma_f16(gc + (uint32_t)(col_o + 16 * mh), ad, bd, idesc, (kt > 0 || ks > 0) ? 1u : 0u);
+      for (int mh = 0; mh < (C::SPL ? 1 : C::MH); ++mh) {
+        const uint64_t ad =
+            vt_desc + (uint64_t)(((ks >> 2) * (C::VTR * 128) + mh * (128 * 128) + (ks & 3) * 32) >> 4);
+        sm100::mma_f16(tmem_base + gcol + (uint32_t)(col_o + 16 * (mh + h)), ad, bd, idesc,
+                       (kt > 0 || ks > 0) ? 1u : 0u);
       }
     }
-    sm100::mma_commit(bars + 6 * gi + 3);
+    sm100::mma_commit(bar);
   };
-  // ---- the MMA warp (MW): one thread issues every group's MMAs as their
-  // operands arrive (a tile's score MMAs once its keys are in tensor memory,
-  // its PV MMAs once V^T and P are in shared memory), polling the groups'
-  // barriers in turn; it gives up after kTimeoutNs without progress
-  if constexpr (C::MW) {
-    if (mma_warp) {
-      if (lane == 0) {
-        int ev[C::NG], ntk[C::NG];
-        int remaining = 0;
+  // The QJL sign blocks of the lane's token into key-operand columns col ..:
+  // bit 2k -> sign of the low half, bit 2k + 1 -> sign of the high half (1 = +rho)
+  auto store_qjl = [&](int col, bool valid, const float* nrm, int tok, const uint32_t* recK) {
+    if (m == 0) return;
+    const float rho = valid ? nrm[TILE + tok] : 0.0f;
+    const uint32_t rp = pack_h2(rho, rho);
+    for (int j = 0; j < nqs; ++j) {
+      uint32_t pc = 0u;
+      pieces<1>(recK, kcb + 16 * j, lane, &pc);
+      uint32_t qh[8];
 #pragma unroll
-        for (int gi = 0; gi < C::NG; ++gi) {
-          ev[gi] = 0;
-          ntk[gi] = (gi < ngr && gi < ntile) ? (ntile - gi + ngr - 1) / ngr : 0;
-          remaining += 2 * ntk[gi];
-        }
-        uint32_t idle = 0;
-        uint64_t t_idle = 0;
-        while (remaining > 0 && *abort_flag == 0) {
-          bool progress = false;
-#pragma unroll
-          for (int gi = 0; gi < C::NG; ++gi) {
-            if (ev[gi] >= 2 * ntk[gi]) continue;
-            const int kt = ev[gi] >> 1;
-            uint64_t* gb = bars + 6 * gi;
-            if ((ev[gi] & 1) == 0) {
-              if (!sm100::mbar_test(gb + 4, (uint32_t)(kt & 1))) continue;
-              sm100::tc_fence_after();
-              issue_scores(gi);
-            } else {
-              if (!sm100::mbar_test(gb + 5, (uint32_t)(kt & 1))) continue;
-              sm100::tc_fence_after();
-              issue_pv(gi, kt);
-            }
-            ++ev[gi];
-            --remaining;
-            progress = true;
-          }
-          if (progress) {
-            idle = 0;
-            continue;
-          }
-          // nothing ready: sleep, so that the polling takes no issue slots from
-          // the decode warps (the operands of a tile take microseconds to arrive)
-          if (idle++ == 0) {
-            t_idle = sm100::global_ns();
-          } else if ((idle & 15u) == 0u && sm100::global_ns() - t_idle > sm100::kTimeoutNs) {
-            *abort_flag = 1;
-            if (err) atomicOr(err, SQ_FLAG_TIMEOUT);
-            break;
-          }
-          __nanosleep(kPollSleepNs);
-        }
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t bits2 = (pc >> (2 * k)) & 3u;
+        const uint32_t neg = ((~bits2 & 1u) << 15) | ((~bits2 & 2u) << 30);
+        qh[k] = rp ^ neg;
       }
-      __syncwarp();
+      sm100::tmem_st8(tmem_base + t_lanes + gcol + (uint32_t)(col + 8 * j), qh);
     }
-  }
+  };
   for (int kk = 0; kk < ntg; ++kk) {
     const int bf = kk % nrec;
     const int64_t t0 = t_lo + (int64_t)(grp + kk * ngr) * TILE;
@@ -650,47 +618,45 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
         sm100::tmem_st8(ks.taddr, hh);
         sm100::tmem_st8(ks.taddr + 8, ll);
       }
-      decode_side<D, true>(recK, tCH, tCD, 1, lane, sm, PL::P1, p3r, lb3, l16m1, ks);
-      if (m > 0) {
-        const float rho = valid ? nrm[TILE + tok] : 0.0f;
-        const uint32_t rp = pack_h2(rho, rho);
-        for (int j = 0; j < nqs; ++j) {
-          uint32_t pc = 0u;
-          pieces<1>(recK, kcb + 16 * j, lane, &pc);
-          uint32_t qh[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            // bit 2k -> sign of the low half, bit 2k + 1 -> sign of the high half (1 = +rho)
-            const uint32_t bits2 = (pc >> (2 * k)) & 3u;
-            const uint32_t neg = ((~bits2 & 1u) << 15) | ((~bits2 & 2u) << 30);
-            qh[k] = rp ^ neg;
-          }
-          sm100::tmem_st8(ks.taddr + (uint32_t)(8 * (NCH + 1 + j)), qh);
-        }
-      }
+      decode_side<D, true>(recK, tCH, tCD, 1, C::KCH, 0, lane, sm, PL::P1, p3r, lb3, l16m1, ks);
+      if (!C::SPL) store_qjl(8 * (NCH + 1), valid, nrm, tok, recK);
     }
     sm100::tmem_wait_st();
     sm100::tc_fence_before();
-    if constexpr (C::MW) {
-      sm100::mbar_arrive(b_kf);
-    } else {
-      sm100::named_bar(1 + grp, 128);
-      if (issuer && live) {
-        sm100::tc_fence_after();
-        issue_scores(grp);
-      }
+    sm100::named_bar(1 + grp, 128);
+    if (issuer && live) {
+      sm100::tc_fence_after();
+      issue_scores(0, C::SPL ? C::KCH + 2 : nks, 0, C::SPL ? b_ka : b_s);
     }
     // ---- values -> V^T tile (the previous tile's PV must be done with it)
     if (live && kk > 0) live = sm100::mbar_wait(b_pv, (uint32_t)((kk - 1) & 1), err);
     if (!live) *abort_flag = 1;
-    if (live) {
-      const ValSink vsnk{vt_lane};
-      decode_side<D, false>(recV, tCH + 16, tCD + D, 0, lane, sm, PL::P1, p3r, lb3, l16m1, vsnk);
-    }
+    const ValSink vsnk{vt_lane};
+    if (live) decode_side<D, false>(recV, tCH + 16, tCD + D, 0, C::KCH, 0, lane, sm, PL::P1, p3r, lb3, l16m1, vsnk);
     const float kn = valid ? nrm[tok] : 0.0f;
     const float vn = valid ? nrm[2 * TILE + tok] : 0.0f;
     sm100::fence_async_smem();
-    // the record buffer is consumed once all four warps pass the vote barrier below
+    if constexpr (C::SPL) {
+      // ---- keys, second part: chunks KCH .. NCH-1 and the QJL blocks, into
+      // the columns of the first part once its MMAs have read them
+      if (live) live = sm100::mbar_wait(b_ka, (uint32_t)(kk & 1), err);
+      if (!live) *abort_flag = 1;
+      sm100::tc_fence_after();
+      if (live) {
+        const KeySink ks{tmem_base + t_lanes + gcol};
+        decode_side<D, true>(recK, tCH, tCD, C::KCH, NCH, C::KCH + 1, lane, sm, PL::P1, p3r, lb3, l16m1, ks);
+        store_qjl(8 * C::KCH, valid, nrm, tok, recK);
+      }
+      sm100::tmem_wait_st();
+      sm100::tc_fence_before();
+      sm100::named_bar(1 + grp, 128);
+      if (issuer && live) {
+        sm100::tc_fence_after();
+        issue_scores(C::KCH + 2, nks, 8 * (C::KCH + 1), b_s);
+      }
+    }
+    // the record buffer is consumed once all four warps pass the vote barrier
+    // below (split: the barrier after the second V^T half)
     // ---- scores -> softmax
     float sv[MG];
 #pragma unroll
@@ -717,7 +683,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     if (lane == 0) votes[q] = wv_any;
     sm100::named_bar(1 + grp, 128);
     // the records of this tile are consumed: the next tile for this buffer may load
-    if (issuer && live && kk + nrec < ntg) {
+    if (!C::SPL && issuer && live && kk + nrec < ntg) {
       issue_records(grp, kk + nrec, bf);
       n_issued = kk + nrec + 1;
     }
@@ -782,13 +748,28 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     }
     sm100::fence_async_smem();
     sm100::tc_fence_before();
-    if constexpr (C::MW) {
-      sm100::mbar_arrive(b_pf);
-    } else {
+    sm100::named_bar(1 + grp, 128);
+    if (issuer && live) {
+      sm100::tc_fence_after();
+      issue_pv(kk, 0, C::SPL ? b_pv1 : b_pv);
+    }
+    if constexpr (C::SPL) {
+      // ---- values, second half: coordinates 128 .. 255 into the V^T tile once
+      // the first half's PV has read it
+      if (live) live = sm100::mbar_wait(b_pv1, (uint32_t)(kk & 1), err);
+      if (!live) *abort_flag = 1;
+      if (live) decode_side<D, false>(recV, tCH + 16, tCD + D, C::KCH, NCH, C::KCH, lane, sm, PL::P1, p3r, lb3,
+                                      l16m1, vsnk);
+      sm100::fence_async_smem();
+      sm100::tc_fence_before();
       sm100::named_bar(1 + grp, 128);
       if (issuer && live) {
         sm100::tc_fence_after();
-        issue_pv(grp, kk);
+        issue_pv(kk, 1, b_pv);
+        if (kk + nrec < ntg) {   // the records of this tile are consumed
+          issue_records(grp, kk + nrec, bf);
+          n_issued = kk + nrec + 1;
+        }
       }
     }
   }
@@ -805,7 +786,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
 #pragma unroll
   for (int h = 0; h < MG; ++h) {
     const float v = warp_sum(lpart[h]);
-    if (lane == 0 && !mma_warp) lsum[q * 16 + h] = v;
+    if (lane == 0) lsum[q * 16 + h] = v;
   }
   if (issuer) {
 #pragma unroll
@@ -886,12 +867,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     for (int kk = max(0, n_issued - nrec); kk < n_issued; ++kk)
       sm100::mbar_wait(&b_rec[kk % nrec], (uint32_t)((kk / nrec) & 1), nullptr);
   }
-  if constexpr (C::MW) {
-    if (mma_warp && lane == 0) {
-      sm100::mma_commit(b_drain);
-      if (!sm100::mbar_wait(b_drain, 0u, err)) *abort_flag = 1;
-    }
-  } else if (issuer) {
+  if (issuer) {
     sm100::mma_commit(b_gdrain);
     if (!sm100::mbar_wait(b_gdrain, 0u, err)) *abort_flag = 1;
   }

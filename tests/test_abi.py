@@ -141,10 +141,11 @@ def _splits_mma(batch, n_kv, d, ctx):
     return min(_valid(ctx), key=lambda S: (cost(S), S))
 
 
-def _splits_td(batch, n_kv, d, ctx):
-    """tcgen05 partials: one block per SM (148) whose NG warp groups (4 / 3 / 2
-    for d 64 / 128 / 256) take the tiles; cost waves x (1 + tiles per group)."""
-    ng = 4 if d <= 64 else (3 if d <= 128 else 2)
+def _splits_td(batch, n_kv, d, ctx, ng=None):
+    """tcgen05 partials: one block per SM (148) whose ng warp groups (at most 4
+    for d 64, 3 for d 128 and 256; fewer when the records' buffers do not fit)
+    take the tiles; cost waves x (1 + tiles per group)."""
+    ng = ng or (4 if d <= 64 else 3)
     units = batch * n_kv
 
     def cost(S):
@@ -155,15 +156,18 @@ def _splits_td(batch, n_kv, d, ctx):
 def test_attention_split_count(libsq):
     """The context split counts behind sq_attn_workspace: every split holds
     tokens (spans of whole 128-token tiles), each partial kernel's count
-    minimises its documented wave cost, and the workspace holds the larger of
-    the two (the kernel a call takes depends on its records)."""
+    minimises its documented wave cost, and the workspace holds the largest
+    count over the partial kernels and the tcgen05 kernel's group counts (which
+    kernel and how many groups a call takes depends on its records)."""
     L = sq.lib()
     for (batch, n_kv, g, d, ctx) in [(1, 256, 4, 128, 2049), (4, 384, 5, 128, 8193), (16, 56, 6, 128, 32769),
                                      (1, 2, 1, 64, 600), (2, 3, 2, 128, 1), (3, 7, 1, 128, 100000),
                                      (1, 1, 1, 128, 300000), (64, 336, 2, 256, 4097)]:
         s = _splits_from_workspace(L, batch, n_kv * g, n_kv, d, ctx)
         assert 1 <= s <= 256
-        assert s == max(_splits_mma(batch, n_kv, d, ctx), _splits_td(batch, n_kv, d, ctx)), (batch, n_kv, d, ctx)
+        ngmax = 4 if d <= 64 else 3
+        want = max([_splits_mma(batch, n_kv, d, ctx)] + [_splits_td(batch, n_kv, d, ctx, ng) for ng in range(1, ngmax + 1)])
+        assert s == want, (batch, n_kv, d, ctx)
     # the decode shapes of the benchmark (split counts of the tcgen05 kernel)
     assert _splits_td(4, 384, 128, 8193) == 2
     assert _splits_td(16, 56, 128, 32769) >= 1
