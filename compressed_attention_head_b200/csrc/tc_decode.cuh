@@ -82,10 +82,10 @@ struct Plan {
   static constexpr int HL = L16 + 1024 + 16;           // u32 [kLevelsTotal]: fp16 hi | fp16 lo << 16
   static constexpr int CH = HL + 2048;                 // u32 [2][16]: chunk descriptors K, V
   static constexpr int CD = CH + 128;                  // u32 [2][D]: coordinate descriptors K, V
-  // u64 [NG][8]: records x2, scores, PV done, drain, spare, first key part
-  // consumed, PV of the first V^T half done
+  // u64 [NG][10]: key records x2, scores, PV done, drain, spare, first key
+  // part consumed, PV of the first V^T half done, value records x2
   static constexpr int BAR = CD + 8 * D;
-  static constexpr int MISC = BAR + 8 * 8 * 4;         // u32 [16]: TMEM base, abort, wmax; u64 setup
+  static constexpr int MISC = BAR + 8 * 10 * 4;        // u32 [16]: TMEM base, abort, wmax; u64 setup
   static constexpr int GS = MISC + 64;                 // per group: votes [4], maxima [4][16], l [4][16], mref [16], misc
   static constexpr int GS_BYTES = 16 + 256 + 256 + 64 + 64;
   static constexpr int GRP = (GS + Cfg<D>::NG * GS_BYTES + 1023) & ~1023;   // group regions (1024-aligned)
@@ -381,22 +381,31 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   const float* vnorm = vc.norm + rowi * vc.cap;
   const size_t rec_buf = (((size_t)(wk + wv) * TILE * 4 + 3 * TILE * 4 + 1023) & ~(size_t)1023);
   uint64_t* bars = (uint64_t*)(sm + PL::BAR);
-  auto issue_records = [&](int gi, int kk, int bf) {
+  // parts: 1 = the key words, norms and rho (barrier 10 gi + bf), 2 = the
+  // value words and norms (barrier 10 gi + 8 + bf; without the split, the
+  // key barrier too: both parts are consumed and requested together)
+  auto issue_records = [&](int gi, int kk, int bf, int parts) {
     const int64_t t0 = t_lo + (int64_t)(gi + kk * ngr) * TILE;
     const int64_t blk0 = t0 >> 5;
     const int nb = (int)min((int64_t)4, (kc.cap - t0) >> 5);    // whole 32-token blocks inside the cache
     uint8_t* rb = sm + PL::GRP + (size_t)gi * group_bytes<D>(wk, wv, nrec) + C::VT_BYTES + C::P_BYTES +
                   (size_t)bf * rec_buf;
-    uint64_t* bar = bars + 8 * gi + bf;
-    const uint32_t kbytes = (uint32_t)(nb * wk * 128), vbytes = (uint32_t)(nb * wv * 128), nbytes = nb * 128;
-    const uint32_t total = kbytes + vbytes + nbytes * (krho ? 3u : 2u);
-    sm100::mbar_expect_tx(bar, total);
-    sm100::bulk_load(rb, kcodes + blk0 * wk * 32, kbytes, bar);
-    sm100::bulk_load(rb + (size_t)wk * TILE * 4, vcodes + blk0 * wv * 32, vbytes, bar);
     uint8_t* nr = rb + (size_t)(wk + wv) * TILE * 4;
-    sm100::bulk_load(nr, knorm + t0, nbytes, bar);
-    sm100::bulk_load(nr + 2 * TILE * 4, vnorm + t0, nbytes, bar);
-    if (krho) sm100::bulk_load(nr + TILE * 4, krho + t0, nbytes, bar);
+    const uint32_t nbytes = nb * 128;
+    const uint32_t kbytes = (uint32_t)(nb * wk * 128), vbytes = (uint32_t)(nb * wv * 128);
+    if (parts & 1) {
+      uint64_t* bar = bars + 10 * gi + bf;
+      sm100::mbar_expect_tx(bar, kbytes + nbytes * (krho ? 2u : 1u) + (C::SPL ? 0u : vbytes + nbytes));
+      sm100::bulk_load(rb, kcodes + blk0 * wk * 32, kbytes, bar);
+      sm100::bulk_load(nr, knorm + t0, nbytes, bar);
+      if (krho) sm100::bulk_load(nr + TILE * 4, krho + t0, nbytes, bar);
+    }
+    if (parts & 2) {
+      uint64_t* bar = bars + 10 * gi + (C::SPL ? 8 : 0) + bf;
+      if (C::SPL) sm100::mbar_expect_tx(bar, vbytes + nbytes);
+      sm100::bulk_load(rb + (size_t)wk * TILE * 4, vcodes + blk0 * wv * 32, vbytes, bar);
+      sm100::bulk_load(nr + 2 * TILE * 4, vnorm + t0, nbytes, bar);
+    }
   };
 
   // ---- block tables (as in the mma.sync kernel, plus the score B operand)
@@ -407,9 +416,10 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   if (tid == 0) {
     misc[1] = 0u;
     misc[2] = 0u;
-    // per group: records x2, scores, PV, drain, spare, first key part
-    // consumed, first PV half (one arrival each: an expect-tx or a commit)
-    for (int k = 0; k < 8 * C::NG; ++k) sm100::mbar_init(&bars[k], 1u);
+    // per group: key records x2, scores, PV, drain, spare, first key part
+    // consumed, first PV half, value records x2 (one arrival each: an
+    // expect-tx or a commit)
+    for (int k = 0; k < 10 * C::NG; ++k) sm100::mbar_init(&bars[k], 1u);
     sm100::mbar_init(b_setup, 1);
     sm100::fence_mbar_init();
     // the level tables, and the first record tiles of every group, start
@@ -419,7 +429,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     sm100::bulk_load(s_p3r, g_p3r, 64u * 32u * 4u, b_setup);
     for (int gi = 0; gi < ngr; ++gi) {
       const int ntk = gi < ntile ? (ntile - gi + ngr - 1) / ngr : 0;
-      for (int kk = 0; kk < nrec && kk < ntk; ++kk) issue_records(gi, kk, kk);
+      for (int kk = 0; kk < nrec && kk < ntk; ++kk) issue_records(gi, kk, kk, 3);
     }
   }
   if (tid < 2 * NCH && ok) {
@@ -504,12 +514,13 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   uint8_t* sP = gr + C::VT_BYTES;
   uint8_t* sRec = sP + C::P_BYTES;
   uint8_t* gs = sm + PL::GS + grp * PL::GS_BYTES;          // votes [4] (u32), maxima [4][16] (int), l [4][16], mref [16]
-  uint64_t* b_rec = bars + 8 * grp;                          // [0], [1]: records of buffer 0 / 1
-  uint64_t* b_s = bars + 8 * grp + 2;                        // scores ready
-  uint64_t* b_pv = bars + 8 * grp + 3;                       // PV of the group's last tile done
-  uint64_t* b_gdrain = bars + 8 * grp + 4;                   // the group's MMAs done (before the free)
-  uint64_t* b_ka = bars + 8 * grp + 6;                       // split: the first key part's MMAs done
-  uint64_t* b_pv1 = bars + 8 * grp + 7;                      // split: the first V^T half's PV done
+  uint64_t* b_rec = bars + 10 * grp;                         // [0], [1]: key records of buffer 0 / 1
+  uint64_t* b_recv = bars + 10 * grp + 8;                    // [0], [1]: value records of buffer 0 / 1
+  uint64_t* b_s = bars + 10 * grp + 2;                       // scores ready
+  uint64_t* b_pv = bars + 10 * grp + 3;                      // PV of the group's last tile done
+  uint64_t* b_gdrain = bars + 10 * grp + 4;                  // the group's MMAs done (before the free)
+  uint64_t* b_ka = bars + 10 * grp + 6;                      // split: the first key part's MMAs done
+  uint64_t* b_pv1 = bars + 10 * grp + 7;                     // split: the first V^T half's PV done
   const bool issuer = q == 0 && lane == 0;                   // the group's copies and MMAs
   const bool active = grp < ngr;
   const int ntg = active && grp < ntile ? (ntile - grp + ngr - 1) / ngr : 0;   // tiles of this group
@@ -533,7 +544,8 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   const uint64_t w_desc = sm100::sw128_desc(sm100::smem_u32(sm + Tab::W));
 
   if (!sm100::mbar_wait(b_setup, 0u, err)) *abort_flag = 1;   // level tables in shared memory
-  int n_issued = min(ntg, nrec);   // tiles whose records were requested (a prefix; the first by thread 0)
+  // tiles whose key / value records were requested (prefixes; the first by thread 0)
+  int n_issued = min(ntg, nrec), n_issued_v = min(ntg, nrec);
   const float LOG2E = 1.4426950408889634f;
   // The MMAs of a tile of group gi. Scores, k-steps [s0, s1): A = the keys in
   // tensor memory (k-step st reads c0 hi for st = 0 and 1, c0 lo for 2, chunk
@@ -630,6 +642,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     }
     // ---- values -> V^T tile (the previous tile's PV must be done with it)
     if (live && kk > 0) live = sm100::mbar_wait(b_pv, (uint32_t)((kk - 1) & 1), err);
+    if (C::SPL && live) live = sm100::mbar_wait(&b_recv[bf], (uint32_t)((kk / nrec) & 1), err);
     if (!live) *abort_flag = 1;
     const ValSink vsnk{vt_lane};
     if (live) decode_side<D, false>(recV, tCH + 16, tCD + D, 0, C::KCH, 0, lane, sm, PL::P1, p3r, lb3, l16m1, vsnk);
@@ -653,6 +666,10 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
       if (issuer && live) {
         sm100::tc_fence_after();
         issue_scores(C::KCH + 2, nks, 8 * (C::KCH + 1), b_s);
+        if (kk + nrec < ntg) {   // the key records of this tile are consumed
+          issue_records(grp, kk + nrec, bf, 1);
+          n_issued = kk + nrec + 1;
+        }
       }
     }
     // the record buffer is consumed once all four warps pass the vote barrier
@@ -684,8 +701,8 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     sm100::named_bar(1 + grp, 128);
     // the records of this tile are consumed: the next tile for this buffer may load
     if (!C::SPL && issuer && live && kk + nrec < ntg) {
-      issue_records(grp, kk + nrec, bf);
-      n_issued = kk + nrec + 1;
+      issue_records(grp, kk + nrec, bf, 3);
+      n_issued = n_issued_v = kk + nrec + 1;
     }
     const bool raise = (votes[0] | votes[1] | votes[2] | votes[3]) != 0u;
     if (raise) {
@@ -766,9 +783,9 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
       if (issuer && live) {
         sm100::tc_fence_after();
         issue_pv(kk, 1, b_pv);
-        if (kk + nrec < ntg) {   // the records of this tile are consumed
-          issue_records(grp, kk + nrec, bf);
-          n_issued = kk + nrec + 1;
+        if (kk + nrec < ntg) {   // the value records of this tile are consumed
+          issue_records(grp, kk + nrec, bf, 2);
+          n_issued_v = kk + nrec + 1;
         }
       }
     }
@@ -866,6 +883,9 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   if (issuer) {
     for (int kk = max(0, n_issued - nrec); kk < n_issued; ++kk)
       sm100::mbar_wait(&b_rec[kk % nrec], (uint32_t)((kk / nrec) & 1), nullptr);
+    if (C::SPL)
+      for (int kk = max(0, n_issued_v - nrec); kk < n_issued_v; ++kk)
+        sm100::mbar_wait(&b_recv[kk % nrec], (uint32_t)((kk / nrec) & 1), nullptr);
   }
   if (issuer) {
     sm100::mma_commit(b_gdrain);
