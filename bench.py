@@ -146,15 +146,16 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str, tokens_per_launch: int):
+def profiled_traffic(kernel: str, algorithmic_bytes: float):
     """DRAM bytes per launch of `kernel` from profiles/traffic.json (written from an ncu
-    capture of the same sources), scaled to this launch's tokens; None if stale or absent."""
+    capture of the same sources), scaled by this launch's algorithmic bytes over the
+    captured launch's (DRAM traffic grows with the records read); None if stale or absent."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             ent = json.load(f)["kernels"][kernel]
         if ent["source_hash"] != kernel_source_hash(kernel):
             return None
-        return ent["dram_bytes"] * tokens_per_launch / ent["tokens"]
+        return ent["dram_bytes"] * algorithmic_bytes / ent["algorithmic_bytes"]
     except Exception:
         return None
 
@@ -645,7 +646,7 @@ def measure_decode(cfg, args, world, dev):
 def _roofline(kernel, ncu_name, nbytes, ms, tokens, peak, peak_kind):
     achieved = nbytes / (ms / 1e3) / 1e9
     return {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
-            "unit": "GB/s", "frac": achieved / peak, "traffic": profiled_traffic(ncu_name, tokens),
+            "unit": "GB/s", "frac": achieved / peak, "traffic": profiled_traffic(ncu_name, nbytes),
             "bytes_per_launch": nbytes, "launch_ms": ms}
 
 

@@ -908,6 +908,25 @@ sq_status sq_attn_prefill(const void* calib_k, const void* calib_v, const sq_cac
 // this entry point: its scratch is a fixed array in the library's own device
 // memory (every GPU that loads libsq keeps it until the process exits).
 // ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace sq {
+// A bounded wait that runs out: one thread waits on an mbarrier that nothing
+// arrives on, through the same helper (sm100::mbar_wait) every tensor-core
+// kernel waits with, here with a short limit; it gives up, sets the timeout
+// flag and returns.
+__global__ void k_wait_selftest(uint64_t limit_ns, uint32_t* flags) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1u);
+    sm100::fence_mbar_init();
+    (void)sm100::mbar_wait(&bar, 0u, flags, limit_ns);
+  }
+}
+}  // namespace sq
+
+extern "C" {
+
 constexpr size_t kStaticScratchBytes = SQ_ATTN_NOALLOC_MAX_BYTES;
 static __device__ __align__(256) unsigned char g_attn_scratch[kStaticScratchBytes];
 static void* g_attn_scratch_addr[128];     // device address of the array, per device
@@ -935,6 +954,14 @@ sq_status sq_attn_decode_noalloc(const void* calib_k, const void* calib_v, const
   return sq_attn_decode(calib_k, calib_v, kc, vc, d_seq_lens, batch, n_q_heads, n_kv_heads, d, max_ctx, q, q_dtype,
                         scale, out, out_dtype, scores_out, g_attn_scratch_addr[dev], kStaticScratchBytes, d_flags,
                         stream);
+}
+
+sq_status sq_wait_selftest(uint32_t limit_us, uint32_t* d_flags, sq_stream stream) {
+  if (limit_us < 1 || limit_us > 2000000u || !d_flags || !aligned16(d_flags)) return SQ_ERR_ARG;
+  sq_status s = ensure_init();
+  if (s != SQ_OK) return s;
+  k_wait_selftest<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_us * 1000ull, d_flags);
+  return cuda_ok(cudaGetLastError());
 }
 
 }  // extern "C"

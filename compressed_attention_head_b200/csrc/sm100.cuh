@@ -56,13 +56,15 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 // Bounded wait for the phase with the given parity: false (and bit 31 of *err
-// set) once kTimeoutNs has passed without the phase completing.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+// set) once limit_ns (kTimeoutNs unless a self-test asks for less) has passed
+// without the phase completing.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                          uint64_t limit_ns = kTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0 && global_ns() - t0 > kTimeoutNs) {
+    if ((i & 63u) == 0 && global_ns() - t0 > limit_ns) {
       if (err) atomicOr(err, 0x80000000u);
       return false;
     }

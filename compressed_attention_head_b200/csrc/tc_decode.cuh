@@ -55,7 +55,7 @@ struct Cfg {
   // columns and its shared memory
   static constexpr bool SPL = D == 256;
   static constexpr int KCH = SPL ? NCH / 2 : NCH;             // key chunks of the first (or only) part
-  static constexpr int NG = D == 64 ? 4 : 3;                  // warp groups decoding tiles
+  static constexpr int NG = D == 256 ? 3 : 4;                 // warp groups decoding tiles
   static constexpr int NTH = NG * 128;
   static constexpr int MH = D > 128 ? 2 : 1;                  // 128-row halves of O^T
   static constexpr int OCOLS = 16 * MH;                       // TMEM columns of O^T
@@ -382,8 +382,10 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   const size_t rec_buf = (((size_t)(wk + wv) * TILE * 4 + 3 * TILE * 4 + 1023) & ~(size_t)1023);
   uint64_t* bars = (uint64_t*)(sm + PL::BAR);
   // parts: 1 = the key words, norms and rho (barrier 10 gi + bf), 2 = the
-  // value words and norms (barrier 10 gi + 8 + bf; without the split, the
-  // key barrier too: both parts are consumed and requested together)
+  // value words and norms (barrier 10 gi + 8 + bf). Without the split both
+  // parts are requested together after the vote barrier, on the key barrier
+  // (measured: requesting the key part right after the key barrier, or
+  // waiting on two barriers, cost 3-4 % at head_dim 128).
   auto issue_records = [&](int gi, int kk, int bf, int parts) {
     const int64_t t0 = t_lo + (int64_t)(gi + kk * ngr) * TILE;
     const int64_t blk0 = t0 >> 5;
@@ -633,6 +635,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
       decode_side<D, true>(recK, tCH, tCD, 1, C::KCH, 0, lane, sm, PL::P1, p3r, lb3, l16m1, ks);
       if (!C::SPL) store_qjl(8 * (NCH + 1), valid, nrm, tok, recK);
     }
+    const float kn = valid ? nrm[tok] : 0.0f;
     sm100::tmem_wait_st();
     sm100::tc_fence_before();
     sm100::named_bar(1 + grp, 128);
@@ -646,7 +649,6 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     if (!live) *abort_flag = 1;
     const ValSink vsnk{vt_lane};
     if (live) decode_side<D, false>(recV, tCH + 16, tCD + D, 0, C::KCH, 0, lane, sm, PL::P1, p3r, lb3, l16m1, vsnk);
-    const float kn = valid ? nrm[tok] : 0.0f;
     const float vn = valid ? nrm[2 * TILE + tok] : 0.0f;
     sm100::fence_async_smem();
     if constexpr (C::SPL) {
@@ -672,8 +674,8 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
         }
       }
     }
-    // the record buffer is consumed once all four warps pass the vote barrier
-    // below (split: the barrier after the second V^T half)
+    // the records are consumed once all four warps pass the vote barrier
+    // below (split: the value records after the second V^T half)
     // ---- scores -> softmax
     float sv[MG];
 #pragma unroll
@@ -699,8 +701,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     const uint32_t wv_any = __any_sync(0xffffffffu, over) ? 1u : 0u;
     if (lane == 0) votes[q] = wv_any;
     sm100::named_bar(1 + grp, 128);
-    // the records of this tile are consumed: the next tile for this buffer may load
-    if (!C::SPL && issuer && live && kk + nrec < ntg) {
+    if (!C::SPL && issuer && live && kk + nrec < ntg) {   // the records of this tile are consumed
       issue_records(grp, kk + nrec, bf, 3);
       n_issued = n_issued_v = kk + nrec + 1;
     }

@@ -89,6 +89,7 @@ _SIGNATURES = {
                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_int64, _P, ctypes.c_int, ctypes.c_float, _P, ctypes.c_int,
                                               _P, _P, _P]),
+    "sq_wait_selftest": (ctypes.c_int, [ctypes.c_uint32, _P, _P]),
 }
 
 SQ_ATTN_NOALLOC_MAX_BYTES = 8 << 20
@@ -325,3 +326,10 @@ def sq_attn_decode_noalloc(calib_k, calib_v, kc, vc, seq_lens, batch, n_q_heads,
                                         _ptr(seq_lens), batch, n_q_heads, n_kv_heads, d, max_ctx, _ptr(q),
                                         DTYPE_CODE[q.dtype], float(scale), _ptr(out), DTYPE_CODE[out.dtype],
                                         _ptr(scores_out), _ptr(flags), _stream(stream)), "sq_attn_decode_noalloc")
+
+
+def sq_wait_selftest(limit_us, flags, stream=None):
+    """One GPU thread waits on an mbarrier nothing arrives on for limit_us
+    microseconds with the library's bounded-wait helper, then sets
+    SQ_FLAG_TIMEOUT in flags (see sq.h)."""
+    _check(lib().sq_wait_selftest(int(limit_us), _ptr(flags), _stream(stream)), "sq_wait_selftest")

@@ -500,6 +500,18 @@ sq_status sq_attn_decode_noalloc(const void* calib_k, const void* calib_v, const
                                  float scale, void* out, sq_dtype out_dtype, float* scores_out,
                                  uint32_t* d_flags, sq_stream stream);
 
+/*
+ * Self-test of the bounded waits (no fault, no hang): one GPU thread waits on
+ * an mbarrier that nothing arrives on, through the same helper every
+ * tensor-core kernel of the library waits with, but with a limit of limit_us
+ * microseconds (1 .. 2 000 000; the kernels use 2 s); it then gives up, ORs
+ * SQ_FLAG_TIMEOUT into *d_flags and returns, leaving the context usable. For
+ * tests of the timeout path.
+ *  d_flags  device uint32, 16-byte aligned.
+ * Returns SQ_ERR_ARG for a limit out of range or a missing / misaligned word.
+ */
+sq_status sq_wait_selftest(uint32_t limit_us, uint32_t* d_flags, sq_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
