@@ -623,18 +623,51 @@ def measure_decode(cfg, args, world, dev):
     if not args.no_e2e:
         hkn, hvn, hq = k_new.cpu().pin_memory(), v_new.cpu().pin_memory(), q.cpu().pin_memory()
         hout = torch.empty_like(out, device="cpu").pin_memory()
+        # The step in chunks of batch rows: the inputs of chunk i + 1 are copied in
+        # (pinned host -> device, a copy stream) while chunk i computes, and the
+        # outputs of chunk i are copied out while chunk i + 1 computes.
+        nch = args.e2e_chunks if (not args.separate and args.e2e_chunks > 1 and B % args.e2e_chunks == 0) else 1
+        rows = B // nch
+        c_in, c_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(nch)]
+        ev_done = [torch.cuda.Event() for _ in range(nch)]
+        ev_out = torch.cuda.Event()
+
+        def sub(cache, r0, r1):
+            return sq.PackedCache(cache.codes[r0:r1], cache.norm[r0:r1],
+                                  cache.rnorm[r0:r1] if cache.rnorm is not None else None, r1 - r0, cache.n_heads,
+                                  cache.cap, cache.words)
+
+        parts = [(i * rows, (i + 1) * rows, sub(kc, i * rows, (i + 1) * rows), sub(vc, i * rows, (i + 1) * rows))
+                 for i in range(nch)]
 
         def e2e_step(ev):
-            k_new.copy_(hkn, non_blocking=True)
-            v_new.copy_(hvn, non_blocking=True)
-            q.copy_(hq, non_blocking=True)
             if args.separate:
+                k_new.copy_(hkn, non_blocking=True)
+                v_new.copy_(hvn, non_blocking=True)
+                q.copy_(hq, non_blocking=True)
                 sq.sq_compress_kv(rk, rv, k_new, v_new, B, H, d, 1, posT, kc, vc, flags)
                 sq.sq_attn_decode(rk, rv, kc, vc, lens, B, HQ, H, d, max_ctx, q, 0.0, out, None, aws, flags)
-            else:
-                sq.sq_decode_step(rk, rv, kc, vc, k_new, v_new, q, posT, B, HQ, H, d, max_ctx, 0.0, out, None, aws,
-                                  flags)
-            hout.copy_(out, non_blocking=True)
+                hout.copy_(out, non_blocking=True)
+                return
+            cur = torch.cuda.current_stream()
+            c_in.wait_stream(cur)
+            for i, (r0, r1, kci, vci) in enumerate(parts):
+                with torch.cuda.stream(c_in):
+                    k_new[r0:r1].copy_(hkn[r0:r1], non_blocking=True)
+                    v_new[r0:r1].copy_(hvn[r0:r1], non_blocking=True)
+                    q[r0:r1].copy_(hq[r0:r1], non_blocking=True)
+                    ev_in[i].record(c_in)
+            for i, (r0, r1, kci, vci) in enumerate(parts):
+                cur.wait_event(ev_in[i])
+                sq.sq_decode_step(rk, rv, kci, vci, k_new[r0:r1], v_new[r0:r1], q[r0:r1], posT[r0:r1], r1 - r0, HQ, H,
+                                  d, max_ctx, 0.0, out[r0:r1], None, aws, flags)
+                ev_done[i].record(cur)
+                with torch.cuda.stream(c_out):
+                    c_out.wait_event(ev_done[i])
+                    hout[r0:r1].copy_(out[r0:r1], non_blocking=True)
+            ev_out.record(c_out)
+            cur.wait_event(ev_out)
 
         t_e2e, _ = _time_loop(e2e_step, args.steps, args.warmup, world, dev, 1)
         res["e2e"] = {"value": B * world / t_e2e, "unit": "tokens/s",
@@ -761,6 +794,8 @@ def main():
                     help="attention partial kernel: 0 tcgen05 (default), 1 SIMT, 2 mma.sync (comparison runs)")
     ap.add_argument("--base-rows", type=int, default=2, help="distinct batch rows of a decode cache")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=4,
+                    help="batch-row chunks of the end-to-end decode step (copies overlap compute)")
     ap.add_argument("--no-graph", action="store_true", help="time the eager launches only")
     ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling captures only)")
     ap.add_argument("--no-cpu", action="store_true")
