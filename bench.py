@@ -545,6 +545,29 @@ def measure_prefill(cfg, args, world, dev):
         h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hkn, hvn, hq))
         res["e2e"] = {"value": step_tokens(cfg) * world / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                       "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+    if not args.no_prefill_attn:
+        # causal attention of the whole prompt over its packed cache (every query
+        # position of every head attends to the positions up to its own): queries
+        # drawn like the keys of their KV head, scaled to the decode queries' norm
+        del wl["k_new"], wl["v_new"]
+        G = HQ // H
+        kq = wl["k"].repeat_interleave(G, dim=1)
+        scale_q = (wl["q"].float().norm(dim=-1).mean() / wl["k"][:, :, :64].float().norm(dim=-1).mean()).item()
+        qp = (kq.float() * scale_q).to(wl["k"].dtype).contiguous()
+        del kq
+        outp = torch.empty(B, HQ, T, d, dtype=torch.float16, device=dev)
+        pws = torch.empty(sq.sq_attn_prefill_workspace(B, HQ, H, d, T, max_ctx), dtype=torch.uint8, device=dev)
+
+        def pf_step(ev):
+            sq.sq_attn_prefill(rk, rv, kc, vc, pos0, B, HQ, H, d, T, max_ctx, qp, 0.0, outp, pws, flags)
+
+        t_pf, _ = _time_loop(pf_step, max(2, args.steps // 4), 3, world, dev, 1)
+        res["prefill_attn"] = {
+            "workload": f"causal attention of the {T}-token prompt over its packed cache: {B} x {HQ} query heads "
+                        f"({cfg['layers']} layers x {cfg['n_q']}) x {T} positions, fp16 queries and outputs",
+            "ms": 1e3 * t_pf, "query_tokens_per_s": B * T * world / t_pf,
+            "query_head_positions_per_s": B * HQ * T * world / t_pf, "launches": 2}
+        del qp, outp, pws
     return res
 
 
@@ -748,6 +771,7 @@ def run_gpu(args, rank, world, local_rank):
             "step_ms": 1e3 * comp["step_s"], "step_tokens_per_s": comp["tokens"] * world / comp["step_s"],
             "attention_ms": comp["att_ms"], "append_ms": comp["app_ms"],
             "e2e": comp.get("e2e"), "gpu_launches_per_step": comp["launches"],
+            "prefill_attention": comp.get("prefill_attn"),
         }
     line["cpu_baseline"] = None
     if world == 1 and not args.no_cpu:
@@ -771,6 +795,8 @@ def run_gpu(args, rank, world, local_rank):
                    "compress_GBps": (main["comp_k"] + main["comp_v"]) / ((main["ck_ms"] + main["cv_ms"]) / 1e3)
                    / 1e9})
     line["breakdown"] = bd
+    if main.get("prefill_attn"):
+        line["prefill_attention"] = main["prefill_attn"]
     line["calibration"] = {"ms": main["calib_ms"], "heads": main["calib_heads"],
                            "tokens_per_head": cfg["n_cal"], "status_nonzero": main["n_bad"]}
     line["device_flags"] = flag_val
@@ -799,6 +825,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="time the eager launches only")
     ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling captures only)")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-prefill-attn", action="store_true", help="skip the prefill-attention line of the compress workload")
     ap.add_argument("--cpu-tokens", type=int, default=32768)
     ap.add_argument("--cpu-ctx", type=int, default=8192)
     ap.add_argument("--cpu-pairs", type=int, default=96)

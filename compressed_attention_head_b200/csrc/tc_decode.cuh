@@ -29,10 +29,15 @@
 //    sit along K in the order k(t) = 8 (t mod 4) + t / 4 within a warp, which
 //    is the order stmatrix .trans produces from lane = token registers; V^T
 //    and P share it, so the contraction over tokens is unchanged.
+//  * head_dim 256: a tile's keys and values are decoded in halves of 128
+//    coordinates; the key operand and the V^T tile hold one half at a time
+//    (the score MMAs of the first key half, and the PV of the first value
+//    half, finish before the second half overwrites them), which lets three
+//    groups fit the 512 TMEM columns and the shared memory.
 //  * One elected thread per group issues that group's bulk copies and MMAs;
 //    mbarriers (bounded waits) and named barriers order the rest. The groups'
-//    partials are merged at the end and written in the layout k_attn_combine
-//    reads.
+//    partials are merged at the end; the last block of a (row, KV head) to
+//    finish merges the splits and rotates the output back.
 #pragma once
 
 #include "attention.cuh"
