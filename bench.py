@@ -544,7 +544,7 @@ def measure_prefill(cfg, args, world, dev):
         t_e2e, _ = _time_loop(e2e_step, args.steps, args.warmup, world, dev, 1)
         h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hkn, hvn, hq))
         res["e2e"] = {"value": step_tokens(cfg) * world / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                      "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+                      "d2h_bytes_per_step": hout.numel() * hout.element_size(), "chunks": nch}
     if not args.no_prefill_attn:
         # causal attention of the whole prompt over its packed cache (every query
         # position of every head attends to the positions up to its own): queries
@@ -648,8 +648,11 @@ def measure_decode(cfg, args, world, dev):
         hout = torch.empty_like(out, device="cpu").pin_memory()
         # The step in chunks of batch rows: the inputs of chunk i + 1 are copied in
         # (pinned host -> device, a copy stream) while chunk i computes, and the
-        # outputs of chunk i are copied out while chunk i + 1 computes.
-        nch = args.e2e_chunks if (not args.separate and args.e2e_chunks > 1 and B % args.e2e_chunks == 0) else 1
+        # outputs of chunk i are copied out while chunk i + 1 computes. Each chunk
+        # pays a split setup and combine of its own: worth it only for long copies.
+        copy_bytes = sum(t.numel() * t.element_size() for t in (hkn, hvn, hq, hout))
+        want = args.e2e_chunks or (4 if copy_bytes >= (16 << 20) else 1)
+        nch = want if (not args.separate and want > 1 and B % want == 0) else 1
         rows = B // nch
         c_in, c_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
         ev_in = [torch.cuda.Event() for _ in range(nch)]
@@ -663,6 +666,12 @@ def measure_decode(cfg, args, world, dev):
 
         parts = [(i * rows, (i + 1) * rows, sub(kc, i * rows, (i + 1) * rows), sub(vc, i * rows, (i + 1) * rows))
                  for i in range(nch)]
+        # the library wants 16-byte aligned position arrays: one buffer per chunk
+        pos_parts = [posT[r0:r1].clone() for r0, r1, _, _ in parts]
+        # fewer rows per call can take more context splits per row: size the
+        # workspace for the chunk too
+        ws_e2e = max(aws.numel(), sq.sq_attn_workspace(rows, HQ, H, d, max_ctx))
+        aws_e2e = aws if ws_e2e == aws.numel() else torch.empty(ws_e2e, dtype=torch.uint8, device=dev)
 
         def e2e_step(ev):
             if args.separate:
@@ -683,8 +692,8 @@ def measure_decode(cfg, args, world, dev):
                     ev_in[i].record(c_in)
             for i, (r0, r1, kci, vci) in enumerate(parts):
                 cur.wait_event(ev_in[i])
-                sq.sq_decode_step(rk, rv, kci, vci, k_new[r0:r1], v_new[r0:r1], q[r0:r1], posT[r0:r1], r1 - r0, HQ, H,
-                                  d, max_ctx, 0.0, out[r0:r1], None, aws, flags)
+                sq.sq_decode_step(rk, rv, kci, vci, k_new[r0:r1], v_new[r0:r1], q[r0:r1], pos_parts[i], r1 - r0,
+                                  HQ, H, d, max_ctx, 0.0, out[r0:r1], None, aws_e2e, flags)
                 ev_done[i].record(cur)
                 with torch.cuda.stream(c_out):
                     c_out.wait_event(ev_done[i])
@@ -695,7 +704,7 @@ def measure_decode(cfg, args, world, dev):
         t_e2e, _ = _time_loop(e2e_step, args.steps, args.warmup, world, dev, 1)
         res["e2e"] = {"value": B * world / t_e2e, "unit": "tokens/s",
                       "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hkn, hvn, hq)),
-                      "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+                      "d2h_bytes_per_step": hout.numel() * hout.element_size(), "chunks": nch}
     return res
 
 
@@ -820,12 +829,14 @@ def main():
                     help="attention partial kernel: 0 tcgen05 (default), 1 SIMT, 2 mma.sync (comparison runs)")
     ap.add_argument("--base-rows", type=int, default=2, help="distinct batch rows of a decode cache")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-chunks", type=int, default=4,
-                    help="batch-row chunks of the end-to-end decode step (copies overlap compute)")
+    ap.add_argument("--e2e-chunks", type=int, default=0,
+                    help="batch-row chunks of the end-to-end decode step (copies overlap compute); "
+                         "0: four when the step copies at least 16 MB, else one")
     ap.add_argument("--no-graph", action="store_true", help="time the eager launches only")
     ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling captures only)")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--no-prefill-attn", action="store_true", help="skip the prefill-attention line of the compress workload")
+    ap.add_argument("--no-prefill-attn", action="store_true",
+                    help="skip the prefill-attention line of the compress workload")
     ap.add_argument("--cpu-tokens", type=int, default=32768)
     ap.add_argument("--cpu-ctx", type=int, default=8192)
     ap.add_argument("--cpu-pairs", type=int, default=96)
