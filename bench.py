@@ -544,7 +544,7 @@ def measure_prefill(cfg, args, world, dev):
         t_e2e, _ = _time_loop(e2e_step, args.steps, args.warmup, world, dev, 1)
         h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hkn, hvn, hq))
         res["e2e"] = {"value": step_tokens(cfg) * world / t_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                      "d2h_bytes_per_step": hout.numel() * hout.element_size(), "chunks": nch}
+                      "d2h_bytes_per_step": hout.numel() * hout.element_size()}
     if not args.no_prefill_attn:
         # causal attention of the whole prompt over its packed cache (every query
         # position of every head attends to the positions up to its own): queries
