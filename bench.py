@@ -594,6 +594,28 @@ def measure_decode(cfg, args, world, dev):
     flags = torch.zeros(1, dtype=torch.int32, device=dev)
     sq.sq_compress_kv(rk0, rv0, w.k, w.v, b0, nkv, d, T, None, k1, v1, flags)
     torch.cuda.synchronize()
+    comp = None
+    if not args.no_cache_compress:
+        # the prompt compress of this shape (one layer's heads, the base rows),
+        # keys and values timed apart; it rewrites the same records. Its inputs
+        # may fit in L2: a 256 MB write before each step evicts them.
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+        def comp_step(ev):
+            flush.fill_(1)
+            if ev: ev[0].record()
+            sq.sq_compress_kv(rk0, None, w.k, None, b0, nkv, d, T, None, k1, None, flags)
+            if ev: ev[1].record()
+            sq.sq_compress_kv(None, rv0, None, w.v, b0, nkv, d, T, None, None, v1, flags)
+            if ev: ev[2].record()
+
+        _, cmarks = _time_loop(comp_step, max(2, args.steps // 4), 3, world, dev, 3)
+        n_vec, esz = b0 * nkv * T, w.k.element_size()
+        comp = dict(n=n_vec, rows=b0, k_ms=_mean_ms(cmarks, 0, 1), v_ms=_mean_ms(cmarks, 1, 2),
+                    k_bytes=n_vec * (d * esz + record_bytes(words_k, qjl)),
+                    v_bytes=n_vec * (d * esz + record_bytes(words_v, False)),
+                    tensor_core=w.k.dtype == torch.float16 and d == 128 and T >= 64)
+        del flush
     del w
     rb = B // b0
 
@@ -641,6 +663,7 @@ def measure_decode(cfg, args, world, dev):
     res = dict(cfg=cfg, step_s=graph or eager, eager_s=eager, graph_s=graph, calib_ms=calib_ms, n_bad=n_bad,
                calib_heads=2 * nkv, app_ms=app_ms, att_ms=att_ms, attn_bytes=attn_bytes, rec_k=rec_k,
                rec_v=rec_v, tokens=step_tokens(cfg), launches=launches, kernel=kernel, flags=flags, base_rows=b0,
+               cache_compress=comp,
                cache_bytes=sum(t.numel() * t.element_size() for t in (kc.codes, kc.norm, vc.codes, vc.norm)
                                + ((kc.rnorm,) if kc.rnorm is not None else ())))
     if not args.no_e2e:
@@ -756,6 +779,21 @@ def run_gpu(args, rank, world, local_rank):
     }
     if cfg["mode"] == "decode":
         line["roofline"] = att
+        cm = main.get("cache_compress")
+        if cm:
+            kname = ("tcc::k_compress_tc" if cm["tensor_core"] else
+                     "blk::k_compress_blk (float64, block-tiled)" if cfg["d"] in (64, 128, 256) and T >= 16 else
+                     "k_compress_ref (float64, one warp per vector)")
+            line["compress_decode_shape"] = {
+                "workload": f"prompt compress of {cm['rows']} batch rows x {cfg['n_kv']} KV heads x {T} tokens "
+                            f"(one layer), {cfg['dtype']}, head_dim {cfg['d']}",
+                "kernel": kname, "l2": "flushed before each step (256 MB write, outside the timed launches)",
+                "compress_k_ms": cm["k_ms"], "compress_v_ms": cm["v_ms"],
+                "compress_tokens_per_s": cm["n"] * world / ((cm["k_ms"] + cm["v_ms"]) / 1e3),
+                "roofline": _roofline(kname + " (mean of the K and V launches)",
+                                      "k_compress_tc" if cm["tensor_core"] else "k_compress_blk",
+                                      (cm["k_bytes"] + cm["v_bytes"]) / 2, (cm["k_ms"] + cm["v_ms"]) / 2, cm["n"],
+                                      peak, peak_kind)}
         line["config"]["cache"] = (f"packed records of layer 0's {cfg['n_kv']} KV heads for {main['base_rows']} "
                                    f"batch rows, compressed from synthetic draws and repeated over the "
                                    f"{cfg['layers']} layers and {B} rows ({main['cache_bytes'] / 1e9:.1f} GB "
@@ -835,6 +873,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="time the eager launches only")
     ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling captures only)")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-cache-compress", action="store_true",
+                    help="skip the prompt-compress line of a decode workload")
     ap.add_argument("--no-prefill-attn", action="store_true",
                     help="skip the prefill-attention line of the compress workload")
     ap.add_argument("--cpu-tokens", type=int, default=32768)

@@ -16,8 +16,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsq.so")
 SOURCES = ["api.cu", "codebook.cpp"]
-HEADERS = ["sq_common.cuh", "sm100.cuh", "calibrate.cuh", "codec.cuh", "attention.cuh", "tc_compress.cuh", "fast_attn.cuh",
-           "tc_decode.cuh", "decode_step.cuh"]
+HEADERS = ["sq_common.cuh", "sm100.cuh", "calibrate.cuh", "codec.cuh", "blk_compress.cuh", "attention.cuh",
+           "tc_compress.cuh", "fast_attn.cuh", "tc_decode.cuh", "decode_step.cuh"]
 
 NVCC_FLAGS = [
     "-std=c++17", "-O3", "-lineinfo",

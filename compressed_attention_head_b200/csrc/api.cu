@@ -23,6 +23,7 @@ __device__ uint8_t c_tccell[560];      // tcc cell tables: positive thresholds b
 #include "attention.cuh"
 #include "calibrate.cuh"
 #include "codec.cuh"
+#include "blk_compress.cuh"
 #include "fast_attn.cuh"
 #include "tc_compress.cuh"
 #include "tc_decode.cuh"
@@ -143,6 +144,12 @@ sq_status ensure_init(int* dev_out = nullptr) {
   cudaFuncSetAttribute(k_attn_partial<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   cudaFuncSetAttribute(k_attn_partial<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   cudaFuncSetAttribute(tcc::k_compress_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, tcc::SMEM_BYTES);
+#define SQ_BLK_ATTR(T)                                                                                        \
+  cudaFuncSetAttribute(blk::k_compress_blk<T, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, blk::Geo<64>::SMEM);  \
+  cudaFuncSetAttribute(blk::k_compress_blk<T, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, blk::Geo<128>::SMEM); \
+  cudaFuncSetAttribute(blk::k_compress_blk<T, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, blk::Geo<256>::SMEM)
+  SQ_BLK_ATTR(float); SQ_BLK_ATTR(__half); SQ_BLK_ATTR(__nv_bfloat16);
+#undef SQ_BLK_ATTR
   cudaFuncSetAttribute(fa::k_attn_partial_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::smem_bytes<64>());
   cudaFuncSetAttribute(fa::k_attn_partial_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::smem_bytes<128>());
   cudaFuncSetAttribute(fa::k_attn_partial_tc<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::smem_bytes<256>());
@@ -348,6 +355,20 @@ sq_status launch_compress_tc(const void* recs, const void* x, int batch, int n_h
   return cuda_ok(cudaGetLastError());
 }
 
+// Prompts of the shapes the tensor-core kernel does not take: the block-tiled
+// float64 kernel (same bits as k_compress_ref).
+template <typename T, int D>
+sq_status launch_compress_blk(const void* recs, const void* x, int batch, int n_heads, int64_t n_tok,
+                              const int32_t* sp, const sq_cache* c, uint32_t* flags, cudaStream_t st) {
+  using G = blk::Geo<D>;
+  const int64_t gx = (n_tok + G::NT - 1) / G::NT;
+  if (gx > 0x7fffffff) return SQ_ERR_ARG;
+  dim3 grid((unsigned)gx, n_heads, batch);
+  blk::k_compress_blk<T, D><<<grid, blk::kThreads, G::SMEM, st>>>((const uint8_t*)recs, (const T*)x, n_heads, n_tok,
+                                                                   sp, cache_args(c), flags);
+  return cuda_ok(cudaGetLastError());
+}
+
 template <typename T>
 sq_status launch_compress(const void* recs, const void* x, int batch, int n_heads, int d, int64_t n_tok,
                           const int32_t* sp, const sq_cache* c, uint32_t* flags, cudaStream_t st) {
@@ -367,6 +388,11 @@ sq_status launch_compress(const void* recs, const void* x, int batch, int n_head
       default: k_append<T, 8><<<grid, 256, append_smem(8), st>>>(r8, xt, batch, n_heads, d, n_tok, sp, ca, flags); break;
     }
     return cuda_ok(cudaGetLastError());
+  }
+  if (!g_force_ref) {
+    if (d == 64) return launch_compress_blk<T, 64>(recs, x, batch, n_heads, n_tok, sp, c, flags, st);
+    if (d == 128) return launch_compress_blk<T, 128>(recs, x, batch, n_heads, n_tok, sp, c, flags, st);
+    if (d == 256) return launch_compress_blk<T, 256>(recs, x, batch, n_heads, n_tok, sp, c, flags, st);
   }
   const int tpb = n_tok >= 1024 ? 256 : 64;
   const int64_t gx = (n_tok + tpb - 1) / tpb;

@@ -35,6 +35,69 @@ __device__ __forceinline__ int regime_of(const RecHeader* h, int i) {
   return ((h->flags & kFlagFitted) != 0u && i >= h->d_eff) ? 1 : 0;
 }
 
+// The per-vector steps after the rotation, shared by the compress kernels
+// that take one warp per vector at that stage: the staged tables of the
+// vector's head, and the warp's word buffer and QJL residual.
+struct VecEnc {
+  const RecHeader* hd;
+  const double* th;      // [2][kThreshTotal]
+  const double* lv;      // [2][kLevelsTotal]
+  const double* sig;
+  const double* isig;
+  const int* bits;
+  const int* offs;
+  uint32_t* wb;          // the record's words (zeroed before the first coordinate)
+  double* rs;            // residual of the signal coordinates (keys with QJL)
+  int m;
+};
+// Coordinate i with rotated, normalised value y: its code into the words
+// (shared-memory atomics: neighbouring lanes share words) and, below m, the
+// residual y - sigma_i * level.
+__device__ __forceinline__ void encode_coord(const VecEnc& e, int i, double y) {
+  const int bw = e.bits[i];
+  int code = 0;
+  const int rg = regime_of(e.hd, i);
+  if (bw > 0) {
+    code = code_of(y * e.isig[i], e.th + rg * kThreshTotal + th_off(bw), bw);
+    const int o = e.offs[i], wi = o >> 5, sh = o & 31;
+    atomicOr(&e.wb[wi], (uint32_t)code << sh);
+    if (sh + bw > 32) atomicOr(&e.wb[wi + 1], (uint32_t)code >> (32 - sh));
+  }
+  if (i < e.m) e.rs[i] = y - e.sig[i] * (bw > 0 ? e.lv[rg * kLevelsTotal + lv_off(bw) + code] : 0.0);
+}
+// After every coordinate of the vector (the warp synchronised): rho and the
+// QJL signs (bit cbits + j is set when (S r)_j >= 0), then the words, ||x||
+// and rho into slot pos of cache row `row`.
+__device__ __forceinline__ void finish_vector(const VecEnc& e, const double* S, int cbits, int W, const CacheArgs& c,
+                                              size_t row, int64_t pos, double nrm, int lane) {
+  const int m = e.m;
+  float rho = 0.0f;
+  if (m > 0) {
+    double r2 = 0.0;
+    for (int k = lane; k < m; k += 32) r2 += e.rs[k] * e.rs[k];
+    r2 = warp_sum(r2);
+    rho = (float)sqrt(r2);
+    for (int j = 0; j < m; ++j) {
+      double pj = 0.0;
+      for (int k = lane; k < m; k += 32) pj = fma(S[j * m + k], e.rs[k], pj);
+      pj = warp_sum(pj);
+      if (lane == 0 && pj >= 0.0) {
+        const int o = cbits + j;
+        atomicOr(&e.wb[o >> 5], 1u << (o & 31));
+      }
+    }
+  }
+  __syncwarp();
+  const size_t slot = row * c.cap + pos;
+  const size_t r0 = rec_word0(row, c.cap, W, pos);
+  for (int w = lane; w < W; w += 32) c.codes[r0 + (size_t)w * 32] = e.wb[w];
+  if (lane == 0) {
+    c.norm[slot] = (float)nrm;
+    if (c.rnorm) c.rnorm[slot] = rho;
+  }
+  __syncwarp();
+}
+
 // Shared-memory bytes of k_compress_ref / k_decompress_ref for head_dim d.
 __host__ __device__ inline size_t codec_ref_smem(int d) {
   size_t v = d <= 128 ? (size_t)8 * d * (d + 1) : 0;             // V (padded rows) in float64
@@ -105,6 +168,7 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
   const int64_t t_begin = (int64_t)blockIdx.x * tok_per_block;
   const int64_t t_end = min(n_tok, t_begin + tok_per_block);
   const size_t row = ((size_t)b * n_heads + h);
+  const VecEnc enc{hd, th, lv, sig, isig, bits, offs, wb, rs, m};
   for (int64_t t = t_begin + warp; t < t_end; t += kCodecWarps) {
     const T* xt = x + (row * n_tok + t) * d;
     double ss = 0.0;
@@ -126,43 +190,10 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
         for (int j = 0; j < d; ++j) y = fma(Vg[(size_t)j * d + i], xs[j], y);
       }
       y *= inv;
-      int bw = bits[i];
-      int code = 0;
-      const int rg = regime_of(hd, i);
-      if (bw > 0) {
-        code = code_of(y * isig[i], th + rg * kThreshTotal + th_off(bw), bw);
-        int o = offs[i], wi = o >> 5, sh = o & 31;
-        atomicOr(&wb[wi], (uint32_t)code << sh);
-        if (sh + bw > 32) atomicOr(&wb[wi + 1], (uint32_t)code >> (32 - sh));
-      }
-      if (i < m) rs[i] = y - sig[i] * (bw > 0 ? lv[rg * kLevelsTotal + lv_off(bw) + code] : 0.0);
+      encode_coord(enc, i, y);
     }
     __syncwarp();
-    float rho = 0.0f;
-    if (m > 0) {
-      double r2 = 0.0;
-      for (int k = lane; k < m; k += 32) r2 += rs[k] * rs[k];
-      r2 = warp_sum(r2);
-      rho = (float)sqrt(r2);
-      for (int j = 0; j < m; ++j) {
-        double pj = 0.0;
-        for (int k = lane; k < m; k += 32) pj = fma(S[j * m + k], rs[k], pj);
-        pj = warp_sum(pj);
-        if (lane == 0 && pj >= 0.0) {
-          int o = cbits + j;
-          atomicOr(&wb[o >> 5], 1u << (o & 31));
-        }
-      }
-    }
-    __syncwarp();
-    const size_t slot = row * c.cap + sp + t;
-    const size_t r0 = rec_word0(row, c.cap, W, sp + t);
-    for (int w = lane; w < W; w += 32) c.codes[r0 + (size_t)w * 32] = wb[w];
-    if (lane == 0) {
-      c.norm[slot] = (float)nrm;
-      if (c.rnorm) c.rnorm[slot] = rho;
-    }
-    __syncwarp();
+    finish_vector(enc, S, cbits, W, c, row, sp + t, nrm, lane);
   }
 }
 

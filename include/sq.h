@@ -252,8 +252,10 @@ sq_status sq_init(void);
 /*
  * Process-wide options (host-only; no GPU work).
  *  SQ_OPT_COMPRESS_PATH: 0 = automatic (tensor-core kernel for fp16 head_dim-128
- *  prompts of >= 64 tokens, float64 reference kernel otherwise), 1 = always the
- *  float64 reference kernel. Both produce identical codes (see sq_compress_kv).
+ *  prompts of >= 64 tokens; for other prompts of >= 16 tokens at head_dim 64,
+ *  128 or 256 a block-tiled float64 kernel; the float64 one-warp-per-vector
+ *  reference kernel otherwise), 1 = always the reference kernel. All produce
+ *  identical codes (see sq_compress_kv).
  *  SQ_OPT_ATTN_PATH: 0 = automatic (the tcgen05 partials for head_dim 64/128/256
  *  and up to 16 query heads per KV head whose records fit its shared memory;
  *  SIMT partials otherwise), 1 = always the SIMT partials, 2 = the mma.sync

@@ -197,6 +197,38 @@ def test_tensor_core_path_matches_oracle_and_reference_kernel(name, tokens):
     assert torch.allclose(kc.rnorm, kr.rnorm, rtol=1e-6, atol=0)
 
 
+@pytest.mark.parametrize("cfg,tokens,batch,dtype", [
+    ("gemma9b_sweep", 77, 2, None),                          # bf16, head_dim 256: a ragged last block of 32
+    ("gemma9b_sweep", 4096, 1, None),                        # the decode-cache prompt of one row
+    ("qwen14b", 40, 2, None),                                # fp16 head_dim 128 under one 64-token tile
+    ("llama8b", 150, 2, torch.float32),                      # f32 head_dim 128
+    (dict(CONFIGS["llama8b"], d=64), 300, 2, None),          # fp16 head_dim 64: a ragged last block of 128
+    (dict(CONFIGS["llama8b"], d=64, dtype="bf16"), 16, 1, None),   # the shortest prompt it takes
+])
+def test_block_kernel_matches_reference_kernel(cfg, tokens, batch, dtype):
+    """The block-tiled float64 compress (every prompt of >= 16 tokens that the
+    tensor-core kernel does not take) sums each rotated coordinate in the same
+    order as the one-warp-per-vector reference kernel, and ||x|| with the same
+    lane-strided sum: records, norms and QJL norms identical bit for bit, and
+    parity with the oracle."""
+    w, ck, cv, k, v, nh = _case(cfg, batch=batch, tokens=tokens, heads=2)
+    if dtype is not None:
+        k, v = k.to(dtype), v.to(dtype)
+    try:
+        sq.sq_set_option(sq.SQ_OPT_COMPRESS_PATH, 0)
+        _, _, kc, vc = _compress(ck, cv, k, v)
+        sq.sq_set_option(sq.SQ_OPT_COMPRESS_PATH, 1)
+        _, _, kr, vr = _compress(ck, cv, k, v)
+    finally:
+        sq.sq_set_option(sq.SQ_OPT_COMPRESS_PATH, 0)
+    for a, b in ((kc, kr), (vc, vr)):
+        assert torch.equal(a.codes, b.codes)
+        assert torch.equal(a.norm, b.norm)
+    assert torch.equal(kc.rnorm, kr.rnorm)
+    ex = _check_side(kc, ck, k) + _check_side(vc, cv, v)
+    assert ex < 1e-3 * (k.numel() + v.numel())
+
+
 def test_full_size_prefill_in_bench_launch_configuration():
     """Llama-shaped prompt: all 32 layers x 8 KV heads (2048 tokens) compressed in one
     call, as the benchmark times it; sampled (head, token) records against the oracle."""
