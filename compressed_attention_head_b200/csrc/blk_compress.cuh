@@ -10,17 +10,20 @@
 // of it from L2. Here one block of 256 threads takes NT = 8192 / D tokens of
 // one head:
 //
-//  * the tokens are staged once, float64 and transposed (coordinate-major),
-//    together with ||x|| of each (the same lane-strided sum and warp
-//    reduction as k_compress_ref);
-//  * V streams through shared memory in chunks of 16 rows (cp.async,
+//  * the tokens are staged once, float64 and transposed (coordinate-major,
+//    token pairs XOR-swizzled), together with ||x|| of each (the same
+//    lane-strided sum and warp reduction as k_compress_ref);
+//  * V streams through shared memory in chunks of 8 rows (cp.async,
 //    double-buffered), each chunk used by all NT tokens;
 //  * each thread accumulates a 4-token x 8-coordinate tile of Y = X V in
 //    registers (a warp covers 16 tokens x 64 coordinates, so that every
 //    shared-memory load of the inner loop is one wavefront);
 //  * Y goes back to shared memory, and one warp per vector forms the codes,
 //    the QJL signs and the record words with the per-vector steps of
-//    k_compress_ref.
+//    k_compress_ref;
+//  * 110 KB of shared memory and at most 128 registers per thread, so that
+//    two blocks share an SM and one block's staging and per-vector steps
+//    overlap the other's multiply-adds.
 //
 // Every y_i is the same chain of fused multiply-adds over j = 0 .. d-1 as in
 // k_compress_ref, scaled by the same 1/||x||, so the two kernels write the
@@ -32,22 +35,30 @@
 namespace sq {
 namespace blk {
 
-constexpr int kThreads = 256;   // 8 warps
-constexpr int kChunk = 16;      // rows of V per shared-memory stage
+constexpr int kThreads = 256;   // 8 warps; two blocks per SM
+constexpr int kChunk = 8;       // rows of V per shared-memory stage
 
 template <int D>
 struct Geo {
   static constexpr int NT = 8192 / D;        // tokens per block
-  static constexpr int LDX = NT + 2;         // row length (doubles) of the transposed token tile
-  static constexpr int LDY = D + 2;          // row length of the Y tile (same storage)
-  static constexpr int XY_BYTES = 8 * (D * LDX > NT * LDY ? D * LDX : NT * LDY);
+  static constexpr int XY_BYTES = 8 * D * NT;   // token tile [D][NT], later Y [NT][D] (64 KB)
   static constexpr int VB_BYTES = 8 * kChunk * D;   // one V stage
   static constexpr int WARPS_C = D / 64;     // warps along the coordinates
   static constexpr int WARPS_T = NT / 16;    // warps along the tokens
   static_assert(WARPS_C * WARPS_T == kThreads / 32, "eight warp tiles per block");
-  static constexpr int SMEM = XY_BYTES + 2 * VB_BYTES + 16 * kThreshTotal + 16 * kLevelsTotal + 16 * D + 8 * D +
-                              8 * NT + 4 * kMaxWords * (kThreads / 32) + 8 * D * (kThreads / 32);
+  // after the product the two V stages hold each warp's QJL residual and words
+  static_assert(8 * D * (kThreads / 32) + 4 * kMaxWords * (kThreads / 32) <= 2 * VB_BYTES, "scratch fits");
+  static constexpr int SMEM = XY_BYTES + 2 * VB_BYTES + 8 * kThreshTotal + 8 * kLevelsTotal + 16 * D + 8 * D + 8 * NT;
+  static_assert(SMEM <= 113 * 1024, "two blocks per SM");
 };
+
+// Column of token tt in row j of the token tile: XOR-swizzled by pairs (a
+// token pair stays adjacent), so that the coordinate-major stores of one
+// token's row spread over the banks.
+template <int D>
+__device__ __forceinline__ int xcol(int j, int tt) {
+  return tt ^ ((2 * j) & (Geo<D>::NT - 1));
+}
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
@@ -61,7 +72,7 @@ __device__ __forceinline__ void cp_async_wait() {
 
 // grid (token blocks of NT, heads, batch), kThreads threads, Geo<D>::SMEM bytes.
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 k_compress_blk(const uint8_t* __restrict__ recs, const T* __restrict__ x, int n_heads, int64_t n_tok,
                const int32_t* __restrict__ start_pos, CacheArgs c, uint32_t* __restrict__ flags) {
   using G = Geo<D>;
@@ -79,18 +90,16 @@ k_compress_blk(const uint8_t* __restrict__ recs, const T* __restrict__ x, int n_
     if (tid == 0 && blockIdx.x == 0 && flags) atomicOr(flags, SQ_FLAG_CAPACITY);
     return;
   }
-  double* XY = (double*)sm;                                  // tokens [D][LDX], later Y [NT][LDY]
-  double* VB = (double*)(sm + G::XY_BYTES);                  // two stages of kChunk rows of V
+  double* XY = (double*)sm;
+  double* VB = (double*)(sm + G::XY_BYTES);
   unsigned char* p = sm + G::XY_BYTES + 2 * G::VB_BYTES;
-  double* th = (double*)p;       p += 16 * kThreshTotal;
-  double* lv = (double*)p;       p += 16 * kLevelsTotal;
+  double* th = (double*)p;       p += 8 * kThreshTotal;   // regime 0 (the only one without fitted tables)
+  double* lv = (double*)p;       p += 8 * kLevelsTotal;
   double* sig = (double*)p;      p += 8 * D;
   double* isig = (double*)p;     p += 8 * D;
   int* bits = (int*)p;           p += 4 * D;
   int* offs = (int*)p;           p += 4 * D;
-  double* nrm_s = (double*)p;    p += 8 * G::NT;
-  uint32_t* wb = (uint32_t*)p + warp * kMaxWords;   p += 4 * kMaxWords * (kThreads / 32);
-  double* rs = (double*)p + warp * D;
+  double* nrm_s = (double*)p;
 
   const double* Vg = rec.V();
   auto load_chunk = [&](int q) {
@@ -100,7 +109,13 @@ k_compress_blk(const uint8_t* __restrict__ recs, const T* __restrict__ x, int n_
     cp_async_commit();
   };
   load_chunk(0);
-  stage_codebooks(rec, th, lv, tid, kThreads);
+  const bool fitted = (hd->flags & kFlagFitted) != 0u;
+  {
+    const double* ft = rec.fit_th();
+    const double* fl = rec.fit_lv();
+    for (int e = tid; e < kThreshTotal; e += kThreads) th[e] = fitted ? ft[e] : c_th64[e];
+    for (int e = tid; e < kLevelsTotal; e += kThreads) lv[e] = fitted ? fl[e] : c_lv64[e];
+  }
   for (int i = tid; i < D; i += kThreads) {
     const double s = rec.sigma()[i];
     sig[i] = s;
@@ -119,11 +134,11 @@ k_compress_blk(const uint8_t* __restrict__ recs, const T* __restrict__ x, int n_
       const T* xt = x + (row * n_tok + t) * D;
       for (int j = lane; j < D; j += 32) {
         double v = (double)to_float<T>(xt[j]);
-        XY[j * G::LDX + tt] = v;
+        XY[j * G::NT + xcol<D>(j, tt)] = v;
         ss += v * v;
       }
     } else {
-      for (int j = lane; j < D; j += 32) XY[j * G::LDX + tt] = 0.0;
+      for (int j = lane; j < D; j += 32) XY[j * G::NT + xcol<D>(j, tt)] = 0.0;
     }
     ss = warp_sum(ss);
     if (lane == 0) nrm_s[tt] = normalize ? sqrt(ss) : 1.0;
@@ -150,11 +165,12 @@ k_compress_blk(const uint8_t* __restrict__ recs, const T* __restrict__ x, int n_
     }
     __syncthreads();
     const double* vq = VB + (q & 1) * kChunk * D;
-#pragma unroll 4
+#pragma unroll
     for (int kk = 0; kk < kChunk; ++kk) {
-      const double* xr = XY + (q * kChunk + kk) * G::LDX;
-      const double2 x01 = *(const double2*)(xr + tb);
-      const double2 x89 = *(const double2*)(xr + tb + 8);
+      const int j = q * kChunk + kk;
+      const double* xr = XY + j * G::NT;
+      const double2 x01 = *(const double2*)(xr + xcol<D>(j, tb));
+      const double2 x89 = *(const double2*)(xr + xcol<D>(j, tb + 8));
       const double xa[4] = {x01.x, x01.y, x89.x, x89.y};
       double2 v[4];
 #pragma unroll
@@ -174,13 +190,17 @@ k_compress_blk(const uint8_t* __restrict__ recs, const T* __restrict__ x, int n_
     const int t = tb + (a & 1) + 8 * (a >> 1);
 #pragma unroll
     for (int s = 0; s < 4; ++s)
-      *(double2*)(XY + t * G::LDY + cb + 16 * s) = make_double2(acc[a][2 * s], acc[a][2 * s + 1]);
+      *(double2*)(XY + t * D + cb + 16 * s) = make_double2(acc[a][2 * s], acc[a][2 * s + 1]);
   }
   __syncthreads();
 
-  // codes, QJL signs and words: warp per vector
+  // codes, QJL signs and words: warp per vector (residual and words in the V stages)
+  double* rs = VB + warp * D;
+  uint32_t* wb = (uint32_t*)(VB + (kThreads / 32) * D) + warp * kMaxWords;
   const int W = hd->words, cbits = hd->code_bits;
-  const VecEnc enc{hd, th, lv, sig, isig, bits, offs, wb, rs, (int)hd->m};
+  const double* th1 = fitted ? rec.fit_th() + kThreshTotal : th;
+  const double* lv1 = fitted ? rec.fit_lv() + kLevelsTotal : lv;
+  const VecEnc enc{hd, {th, th1}, {lv, lv1}, sig, isig, bits, offs, wb, rs, (int)hd->m};
   const double* S = rec.S();
   for (int tt = warp; tt < G::NT; tt += kThreads / 32) {
     const int64_t t = t0 + tt;
@@ -190,7 +210,7 @@ k_compress_blk(const uint8_t* __restrict__ recs, const T* __restrict__ x, int n_
     const double nrm = nrm_s[tt];
     const double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
     for (int i = lane; i < D; i += 32) {
-      double y = XY[tt * G::LDY + i];
+      double y = XY[tt * D + i];
       y *= inv;
       encode_coord(enc, i, y);
     }

@@ -40,8 +40,8 @@ __device__ __forceinline__ int regime_of(const RecHeader* h, int i) {
 // vector's head, and the warp's word buffer and QJL residual.
 struct VecEnc {
   const RecHeader* hd;
-  const double* th;      // [2][kThreshTotal]
-  const double* lv;      // [2][kLevelsTotal]
+  const double* th[2];   // thresholds of each regime ([kThreshTotal] each)
+  const double* lv[2];   // levels of each regime ([kLevelsTotal] each)
   const double* sig;
   const double* isig;
   const int* bits;
@@ -58,12 +58,12 @@ __device__ __forceinline__ void encode_coord(const VecEnc& e, int i, double y) {
   int code = 0;
   const int rg = regime_of(e.hd, i);
   if (bw > 0) {
-    code = code_of(y * e.isig[i], e.th + rg * kThreshTotal + th_off(bw), bw);
+    code = code_of(y * e.isig[i], (rg ? e.th[1] : e.th[0]) + th_off(bw), bw);
     const int o = e.offs[i], wi = o >> 5, sh = o & 31;
     atomicOr(&e.wb[wi], (uint32_t)code << sh);
     if (sh + bw > 32) atomicOr(&e.wb[wi + 1], (uint32_t)code >> (32 - sh));
   }
-  if (i < e.m) e.rs[i] = y - e.sig[i] * (bw > 0 ? e.lv[rg * kLevelsTotal + lv_off(bw) + code] : 0.0);
+  if (i < e.m) e.rs[i] = y - e.sig[i] * (bw > 0 ? (rg ? e.lv[1] : e.lv[0])[lv_off(bw) + code] : 0.0);
 }
 // After every coordinate of the vector (the warp synchronised): rho and the
 // QJL signs (bit cbits + j is set when (S r)_j >= 0), then the words, ||x||
@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(128) k_compress_ref(const uint8_t* __restrict_
   const int64_t t_begin = (int64_t)blockIdx.x * tok_per_block;
   const int64_t t_end = min(n_tok, t_begin + tok_per_block);
   const size_t row = ((size_t)b * n_heads + h);
-  const VecEnc enc{hd, th, lv, sig, isig, bits, offs, wb, rs, m};
+  const VecEnc enc{hd, {th, th + kThreshTotal}, {lv, lv + kLevelsTotal}, sig, isig, bits, offs, wb, rs, m};
   for (int64_t t = t_begin + warp; t < t_end; t += kCodecWarps) {
     const T* xt = x + (row * n_tok + t) * d;
     double ss = 0.0;
