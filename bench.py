@@ -131,6 +131,7 @@ KERNEL_SOURCES = {
     "k_compress_tc": ["tc_compress.cuh", "sm100.cuh", "sq_common.cuh"],
     "k_attn_partial_tc": ["fast_attn.cuh", "attention.cuh", "sq_common.cuh"],
     "k_decode_tc": ["tc_decode.cuh", "attention.cuh", "sm100.cuh", "sq_common.cuh"],
+    "k_compress_blk": ["blk_compress.cuh", "codec.cuh", "sq_common.cuh"],
 }
 
 

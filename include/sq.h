@@ -121,9 +121,10 @@ typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2 } sq_dtype;
  *                 midpoints of neighbouring levels, each sample coded as the
  *                 compressor codes it, each level moved to the mean of its
  *                 samples (a level without samples kept). Records with fitted
- *                 codebooks are compressed by the float64 reference kernels and
- *                 attended by the SIMT kernel (SQ_OPT_ATTN_PATH 1): the tensor-
- *                 core attention kernels refuse them with SQ_FLAG_RECORD.
+ *                 codebooks are compressed by the float64 kernels (block-tiled
+ *                 or reference; the tensor-core compress leaves them to these)
+ *                 and attended by the SIMT kernel (SQ_OPT_ATTN_PATH 1): the
+ *                 tensor-core attention kernels refuse them with SQ_FLAG_RECORD.
  *  fit_iters      Lloyd iterations of the fit (0: 30). The sums of a fit are
  *                 accumulated with atomics, in an order that varies between runs.
  */
