@@ -80,8 +80,8 @@ struct Tab {
 };
 template <int D>
 struct Plan {
-  static constexpr int P1 = Tab::W + Cfg<D>::W_BYTES;  // u32 [4]: width-1 pairs
-  static constexpr int P2 = P1 + 16;                   // u32 [16]: width-2 pairs
+  static constexpr int P1 = Tab::W + Cfg<D>::W_BYTES;  // uint2 [16]: width-1 quads
+  static constexpr int P2 = P1 + 128;                  // u32 [16]: width-2 pairs
   // 16 zero bytes precede L16 and HL: entry -1 reads as 0 (width-0 coordinates)
   static constexpr int L16 = P2 + 64 + 16;             // half [kLevelsTotal]
   static constexpr int HL = L16 + 1024 + 16;           // u32 [kLevelsTotal]: fp16 hi | fp16 lo << 16
@@ -100,9 +100,9 @@ static_assert(kLevelsTotal * 2 <= 1024 && kLevelsTotal * 4 <= 2048, "level table
 // The level tables every block of the kernel starts from, built once per
 // device from the Lloyd-Max levels (td_build_tables) and copied into shared
 // memory by one bulk copy per block: kImgBytes is the span of the plan from P1
-// to CH (width-1 and width-2 pair tables, a zero guard, fp16 levels, a zero
-// guard, fp16 hi | lo levels); g_p3r is the lane-replicated width-3 table.
-constexpr int kImgBytes = 16 + 64 + 16 + 1024 + 16 + 2048;
+// to CH (width-1 quad and width-2 pair tables, a zero guard, fp16 levels, a
+// zero guard, fp16 hi | lo levels); g_p3r is the lane-replicated width-3 table.
+constexpr int kImgBytes = 128 + 64 + 16 + 1024 + 16 + 2048;
 __device__ __align__(128) uint8_t g_img[kImgBytes];
 __device__ __align__(128) uint32_t g_p3r[64 * 32];
 
@@ -119,11 +119,14 @@ inline uint32_t pair_h2_host(float lo, float hi) {
 inline void build_tables_host(const double* lv, uint8_t* img, uint32_t* p3r) {
   for (int i = 0; i < kImgBytes; ++i) img[i] = 0;
   uint32_t* p1 = (uint32_t*)img;
-  uint32_t* p2 = (uint32_t*)(img + 16);
-  uint16_t* l16 = (uint16_t*)(img + 16 + 64 + 16);
-  uint32_t* hl = (uint32_t*)(img + 16 + 64 + 16 + 1024 + 16);
+  uint32_t* p2 = (uint32_t*)(img + 128);
+  uint16_t* l16 = (uint16_t*)(img + 128 + 64 + 16);
+  uint32_t* hl = (uint32_t*)(img + 128 + 64 + 16 + 1024 + 16);
   auto f = [&](int b, int k) { return (float)lv[lv_off(b) + k]; };
-  for (int t = 0; t < 4; ++t) p1[t] = pair_h2_host(f(1, t & 1), f(1, t >> 1));
+  for (int t = 0; t < 16; ++t) {   // four 1-bit codes: two fp16 level pairs
+    p1[2 * t] = pair_h2_host(f(1, t & 1), f(1, (t >> 1) & 1));
+    p1[2 * t + 1] = pair_h2_host(f(1, (t >> 2) & 1), f(1, t >> 3));
+  }
   for (int t = 0; t < 16; ++t) p2[t] = pair_h2_host(f(2, t & 3), f(2, t >> 2));
   for (int e = 0; e < 64 * 32; ++e) p3r[e] = pair_h2_host(f(3, (e >> 5) & 7), f(3, e >> 8));
   for (int e = 0; e < kLevelsTotal; ++e) {
@@ -188,19 +191,23 @@ __device__ __forceinline__ void decode_chunk(const uint32_t* rec, int o, int lan
   constexpr int NP = (16 * NC * B + 31) / 32;
   uint32_t p[NP];
   pieces<NP>(rec, o, lane, p);
-  if (B == 1) {
-    const uint32_t* t = (const uint32_t*)(sm + p1off);
+  if (B == 1) {   // four coordinates per lookup
+    const uint2* t = (const uint2*)(sm + p1off);
 #pragma unroll
-    for (int k = 0; k < 8 * NC; ++k) h[k] = t[fld(p, 2, 2 * k)];
+    for (int k = 0; k < 4 * NC; ++k) {
+      const uint2 e = t[fld(p, 4, 4 * k)];
+      h[2 * k] = e.x;
+      h[2 * k + 1] = e.y;
+    }
   } else if (B == 2) {
-    const uint32_t* t = (const uint32_t*)(sm + p1off + 16);
+    const uint32_t* t = (const uint32_t*)(sm + p1off + 128);
 #pragma unroll
     for (int k = 0; k < 8 * NC; ++k) h[k] = t[fld(p, 4, 4 * k)];
   } else if (B == 3) {
 #pragma unroll
     for (int k = 0; k < 8 * NC; ++k) h[k] = *(const uint32_t*)(p3r + fld6x128(p, 6 * k, lb3));
   } else {
-    const unsigned short* t = (const unsigned short*)(sm + p1off + 16 + 64 + 16) + lv_off(B);
+    const unsigned short* t = (const unsigned short*)(sm + p1off + 128 + 64 + 16) + lv_off(B);
 #pragma unroll
     for (int k = 0; k < 8 * NC; ++k) {
       const uint32_t a = t[fld(p, B, B * (2 * k))];
