@@ -285,6 +285,8 @@ def test_append_groups_of_vectors(name, batch, ntok):
     ("llama8b", 2, 333, 3, 1, torch.float16),        # tensor-core path, one head per piece
     ("qwen14b", 3, 200, 4, 3, torch.float16),        # pieces of 3 heads and a ragged last piece
     ("tiny", 2, 100, 4, 2, torch.float32),           # float64 reference path, head_dim 32
+    ("gemma9b_sweep", 2, 100, 2, 1, torch.bfloat16), # block-tiled float64 path, head_dim 256
+    ("llama8b", 2, 150, 2, 2, torch.float32),        # block-tiled float64 path, f32 inputs
 ])
 def test_host_input_compress_matches_device_input(name, batch, tokens, heads, slab_heads, dtype):
     """sq_compress_kv_host (pinned host inputs, copies overlapped through a
