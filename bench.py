@@ -567,7 +567,7 @@ def measure_prefill(cfg, args, world, dev):
             "workload": f"causal attention of the {T}-token prompt over its packed cache: {B} x {HQ} query heads "
                         f"({cfg['layers']} layers x {cfg['n_q']}) x {T} positions, fp16 queries and outputs",
             "ms": 1e3 * t_pf, "query_tokens_per_s": B * T * world / t_pf,
-            "query_head_positions_per_s": B * HQ * T * world / t_pf, "launches": 2}
+            "query_head_positions_per_s": B * HQ * T * world / t_pf, "launches": 3}
         del qp, outp, pws
     return res
 
@@ -641,7 +641,8 @@ def measure_decode(cfg, args, world, dev):
             sq.sq_attn_decode(rk, rv, kc, vc, lens, B, HQ, H, d, max_ctx, q, 0.0, out, None, aws, flags)
         else:
             # the fused step: appends + query preparation in one launch, partials with the
-            # last-block combine in the other (two launches on the tcgen05 path)
+            # last-block merge in the next, the rotation back in the last (three on the
+            # tcgen05 path)
             sq.sq_decode_step(rk, rv, kc, vc, k_new, v_new, q, posT, B, HQ, H, d, max_ctx, 0.0, out, None, aws, flags)
             if ev: ev[1].record()
         if ev: ev[2].record()
@@ -653,14 +654,14 @@ def measure_decode(cfg, args, world, dev):
     td = args.attn_path == 0 and cfg["d"] in (64, 128, 256) and cfg["n_q"] // cfg["n_kv"] <= 16
     if args.separate:
         app_ms, att_ms = _mean_ms(marks, 0, 1), _mean_ms(marks, 1, 2)
-        launches = 2 + (2 if td else 3)
-        kernel = "sq_attn_decode (prepare + partials" + (" merging their splits)" if td else " + combine)")
+        launches = 2 + 3
+        kernel = "sq_attn_decode (prepare + partials" + (" merging their splits + rotation)" if td else " + combine)")
     else:
-        # one call: its two launches are timed together (the step's whole time)
+        # one call: its launches are timed together (the step's whole time)
         app_ms, att_ms = 0.0, _mean_ms(marks, 0, 1)
-        launches = 2 if td else 5
-        kernel = ("sq_decode_step (append + prepare launch, partials launch merging their splits)" if td
-                  else "sq_decode_step (appends, prepare, partials, combine)")
+        launches = 3 if td else 5
+        kernel = ("sq_decode_step (append + prepare launch, partials launch merging their splits, rotation "
+                  "launch)" if td else "sq_decode_step (appends, prepare, partials, combine)")
     res = dict(cfg=cfg, step_s=graph or eager, eager_s=eager, graph_s=graph, calib_ms=calib_ms, n_bad=n_bad,
                calib_heads=2 * nkv, app_ms=app_ms, att_ms=att_ms, attn_bytes=attn_bytes, rec_k=rec_k,
                rec_v=rec_v, tokens=step_tokens(cfg), launches=launches, kernel=kernel, flags=flags, base_rows=b0,

@@ -711,9 +711,10 @@ bool attn_args_ok(const void* calib_k, const void* calib_v, const sq_cache* kc, 
 
 // Every launch of one decode-attention call. With k_new / v_new (a decode
 // step) the new token of each row is first compressed into the caches at
-// d_lens[b] and attended (len_offset 1). The tcgen05 path takes two launches
-// (append + prepare in one; partials with the last-block combine); the
-// others take prepare, partials and combine (and the appends before them).
+// d_lens[b] and attended (len_offset 1). The tcgen05 path takes three
+// launches (append + prepare in one; partials with the last-block merge; the
+// rotation back batched over the rows of each KV head); the others take
+// prepare, partials and combine (and the appends before them).
 // Query positions per kernel row of a causal prefill with qg query heads per
 // KV head: as many as fit 16 MMA columns.
 int prefill_cols(int qg) { return qg >= 16 ? 1 : 16 / qg; }
@@ -803,6 +804,13 @@ sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* 
     else { SQ_TD_G(256); }
 #undef SQ_TD_G
 #undef SQ_TD_LAUNCH
+    if (cuda_ok(cudaGetLastError()) != SQ_OK) return SQ_ERR_CUDA;
+    // ---- launch 3: the rotation back (o = V_V a), batched over the rows of each KV head
+    const int64_t nvec = (int64_t)rows * sh.group;
+    dim3 gr(n_kv_heads, (unsigned)std::min<int64_t>(65535, (nvec + 31) / 32));
+    if (d == 64) k_rotate_out<64><<<gr, 256, 0, st>>>(rv, sh, w, out, (int)out_dtype);
+    else if (d == 128) k_rotate_out<128><<<gr, 256, 0, st>>>(rv, sh, w, out, (int)out_dtype);
+    else k_rotate_out<256><<<gr, 256, 0, st>>>(rv, sh, w, out, (int)out_dtype);
     return cuda_ok(cudaGetLastError());
   }
   if (fast) {

@@ -54,7 +54,7 @@ __host__ __device__ __forceinline__ bool attn_col_live(const AttnShape& s, int r
 
 // Workspace layout (floats): w[batch][n_q][d], u[batch][n_q][d],
 // acc[batch][n_q][splits][d], ml[batch][n_q][splits][2], then one uint32
-// arrival counter per (batch, KV head) for the last-block combine.
+// arrival counter per (batch, KV head) for the last-block merge.
 __host__ __device__ inline size_t attn_ws_floats(int batch, int n_q, int d, int splits) {
   return (size_t)batch * n_q * (2 * (size_t)d + (size_t)splits * (d + 2));
 }
@@ -98,7 +98,7 @@ __device__ void prepare_body(const uint8_t* __restrict__ recs_k, const TQ* __res
                              float* smem, int tid, int nth) {
   const int d = s.d, G = s.group;
   const int nb = min(prep_rows(G), s.batch - b0);
-  if (tid < nb) attn_counters(ws, s)[(size_t)(b0 + tid) * s.n_kv + g] = 0u;   // for the last-block combine
+  if (tid < nb) attn_counters(ws, s)[(size_t)(b0 + tid) * s.n_kv + g] = 0u;   // for the last-block merge
   Rec rec = rec_at(recs_k, d, g);
   const RecHeader* hd = rec.hdr();
   if (!record_ok(hd, d)) {
@@ -385,10 +385,11 @@ __global__ void __launch_bounds__(128) k_attn_partial(const uint8_t* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// Combine of one (batch, KV head): merges the splits of its G query heads and
-// rotates back with V_V, which is read once for all of them:
-// a_h,i = sigma_V,i * sum_s e^(m_s - M) acc_s,i / sum_s e^(m_s - M) l_s;  o_h = V_V a_h.
-// scr: [16][d] floats (a), [16][splits] floats (split weights), [16] (1 / l).
+// Combine of one (batch, KV head): merge the splits of its G query heads,
+// a_h,i = sigma_V,i * sum_s e^(m_s - M) acc_s,i / sum_s e^(m_s - M) l_s, and
+// rotate back, o_h = V_V a_h (combine_one: both in one block, V_V read once
+// for the G heads; merge_one + k_rotate_out: the rotation batched over the
+// rows of each KV head, V_V read once per 32 column vectors).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void store_out(void* out, int dt, size_t idx, float v) {
   if (dt == SQ_F32) ((float*)out)[idx] = v;
@@ -396,18 +397,19 @@ __device__ __forceinline__ void store_out(void* out, int dt, size_t idx, float v
   else ((__nv_bfloat16*)out)[idx] = __float2bfloat16_rn(v);
 }
 
-__device__ void combine_one(const uint8_t* __restrict__ recs_v, const AttnShape& s, const float* ws, void* out,
-                            int out_dt, int g, int b, float* scr, int tid, int nth) {
+// The splits of KV head g in kernel row b merged: for each column hh < G,
+// a_h = sigma ⊙ (sum_k w_k acc_k) / l with w_k = exp(m_k - max m), into
+// dst[hh * d + i] (zero when the record is invalid). scr: 16 * (splits + 1)
+// floats of shared memory; the caller synchronises before reading dst.
+__device__ void merge_splits(const Rec& rv, bool ok, const AttnShape& s, const float* ws, int g, int b, float* dst,
+                             float* scr, int tid, int nth) {
   const int d = s.d, G = s.group;
   const int lane = tid & 31, warp = tid >> 5, nwarp = nth >> 5;
-  Rec rv = rec_at(recs_v, d, g);
-  float* a = scr;                       // [16][d]
-  float* sw = scr + 16 * d;             // [16][splits]
+  float* sw = scr;                      // [16][splits]
   float* s_inv_l = sw + 16 * s.splits;  // [16]
   const float* acc = ws + (size_t)s.batch * s.n_q * d * 2;
   const float* ml = acc + (size_t)s.batch * s.n_q * s.splits * d;
   const size_t qh0 = (size_t)b * s.n_q + (size_t)g * G;
-  const bool ok = record_ok(rv.hdr(), d);
   const float* sig = rv.sigma_f();
   for (int hh = warp; hh < G; hh += nwarp) {
     const float* mlh = ml + (qh0 + hh) * s.splits * 2;
@@ -441,8 +443,30 @@ __device__ void combine_one(const uint8_t* __restrict__ recs_v, const AttnShape&
       v = fmaf(swh[k + 3], a3, v);
     }
     for (; k < s.splits; ++k) v = fmaf(swh[k], __ldcg(ah + (size_t)k * d), v);
-    a[hh * d + i] = ok ? v * s_inv_l[hh] * sig[i] : 0.0f;
+    dst[hh * d + i] = ok ? v * s_inv_l[hh] * sig[i] : 0.0f;
   }
+}
+
+// The merged column vectors of (b, g) over their query operands w[b][h] in
+// the workspace (every block of (b, g) has read them by now): the rotation
+// back, o = V_V a, runs for all rows of a KV head at once in k_rotate_out.
+__device__ void merge_one(const uint8_t* __restrict__ recs_v, const AttnShape& s, float* ws, int g, int b,
+                          float* scr, int tid, int nth) {
+  const Rec rv = rec_at(recs_v, s.d, g);
+  const bool ok = record_ok(rv.hdr(), s.d);
+  merge_splits(rv, ok, s, ws, g, b, ws + ((size_t)b * s.n_q + (size_t)g * s.group) * s.d, scr, tid, nth);
+}
+
+// Merge and rotate back in one block per (b, g). scr: [16][d] floats (a),
+// [16][splits] (split weights), [16] (1 / l).
+__device__ void combine_one(const uint8_t* __restrict__ recs_v, const AttnShape& s, const float* ws, void* out,
+                            int out_dt, int g, int b, float* scr, int tid, int nth) {
+  const int d = s.d, G = s.group;
+  const int lane = tid & 31, warp = tid >> 5, nwarp = nth >> 5;
+  const Rec rv = rec_at(recs_v, d, g);
+  const bool ok = record_ok(rv.hdr(), d);
+  float* a = scr;                       // [16][d]
+  merge_splits(rv, ok, s, ws, g, b, a, scr + 16 * d, tid, nth);
   __syncthreads();
   // o_h = V_V a_h: warp w takes rows w, w + nwarp, ... in batches of RB rows
   // whose loads (16-byte pieces, lane-strided) are all in flight together
@@ -491,6 +515,74 @@ __global__ void __launch_bounds__(256, 2) k_attn_combine(const uint8_t* __restri
                                                       const float* __restrict__ ws, void* out, int out_dt) {
   extern __shared__ __align__(16) float cscr[];
   combine_one(recs_v, s, ws, out, out_dt, blockIdx.x, blockIdx.y, cscr, threadIdx.x, blockDim.x);
+}
+
+// The rotation back for the kernels that leave merged column vectors in the
+// workspace (merge_one): o = V_V a for every column vector of KV head g, as a
+// small product per block, O[32 vectors x D] = A V_V^T, so that V_V is read once
+// per 32 vectors instead of once per (row, KV head). grid (n_kv, tiles of 32 of
+// the rows x columns vectors, striding when there are more than gridDim.y
+// tiles), 256 threads; each thread 4 vectors x D/32 outputs, float32.
+template <int D>
+__global__ void __launch_bounds__(256) k_rotate_out(const uint8_t* __restrict__ recs_v, AttnShape s,
+                                                   const float* __restrict__ ws, void* out, int out_dt) {
+  constexpr int RT = 32, KC = 32, OJ = D / 32;
+  __shared__ float As[KC][RT + 1];   // chunk of the vectors, coordinate-major
+  __shared__ float Vs[KC][D + 1];    // chunk of V_V^T: Vs[i][j] = V_V[j][i0 + i]
+  const int g = blockIdx.x, tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
+  const Rec rv = rec_at(recs_v, D, g);
+  const bool ok = record_ok(rv.hdr(), D);
+  const float* V = rv.V_f();
+  const int nvec = s.batch * s.group;
+  for (int v0 = blockIdx.y * RT; v0 < nvec; v0 += gridDim.y * RT) {
+    float acc[4][OJ];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int u = 0; u < OJ; ++u) acc[a][u] = 0.0f;
+    if (ok) {
+      for (int i0 = 0; i0 < D; i0 += KC) {
+        // vectors: element (v, i0 + ii) of vector v0 + v (rows b, columns hh of head g)
+        for (int e = tid; e < RT * KC; e += 256) {
+          const int v = e / KC, ii = e % KC, vg = v0 + v;
+          float x = 0.0f;
+          if (vg < nvec) {
+            const int b = vg / s.group, hh = vg % s.group;
+            x = ws[((size_t)b * s.n_q + (size_t)g * s.group + hh) * D + i0 + ii];
+          }
+          As[ii][v] = x;
+        }
+        for (int e = tid; e < D * KC; e += 256) {
+          const int j = e / KC, ii = e % KC;
+          Vs[ii][j] = __ldg(V + (size_t)j * D + i0 + ii);
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int ii = 0; ii < KC; ++ii) {
+          float av[4];
+#pragma unroll
+          for (int a = 0; a < 4; ++a) av[a] = As[ii][ty * 4 + a];
+#pragma unroll
+          for (int u = 0; u < OJ; ++u) {
+            const float vv = Vs[ii][tx + 32 * u];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) acc[a][u] = fmaf(vv, av[a], acc[a][u]);
+          }
+        }
+        __syncthreads();
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int vg = v0 + ty * 4 + a;
+      if (vg >= nvec) continue;
+      const int b = vg / s.group, hh = vg % s.group;
+      if (!attn_col_live(s, b, hh)) continue;
+      const size_t base = attn_q_index(s, b, g, hh);
+#pragma unroll
+      for (int u = 0; u < OJ; ++u) store_out(out, out_dt, base + tx + 32 * u, acc[a][u]);
+    }
+  }
 }
 
 // Shared-memory floats combine_one needs.

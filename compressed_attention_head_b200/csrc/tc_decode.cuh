@@ -37,7 +37,8 @@
 //  * One elected thread per group issues that group's bulk copies and MMAs;
 //    mbarriers (bounded waits) and named barriers order the rest. The groups'
 //    partials are merged at the end; the last block of a (row, KV head) to
-//    finish merges the splits and rotates the output back.
+//    finish merges the splits, and k_rotate_out (a launch of its own, batched
+//    over the rows of each KV head) rotates the outputs back.
 #pragma once
 
 #include "attention.cuh"
@@ -932,7 +933,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   if (tid == 0 && *abort_flag && err) atomicOr(err, SQ_FLAG_TIMEOUT);
   if (s_last) {
     __threadfence();
-    combine_one(recs_v, s, ws, out, out_dt, g, b, (float*)sm, tid, C::NTH);
+    merge_one(recs_v, s, ws, g, b, (float*)sm, tid, C::NTH);
   }
 }
 

@@ -438,10 +438,11 @@ sq_status sq_attn_decode(const void* calib_k, const void* calib_v, const sq_cach
  *  Other arguments, workspace (sq_attn_workspace of the same shape), results
  *  and flags as sq_compress_kv and sq_attn_decode; max_ctx >= 1.
  * On the tcgen05 path (head_dim 64/128/256, up to 16 query heads per KV head)
- * the step is two launches: the appends share one with the query preparation,
- * and the attention partials merge their splits themselves (the last block of
- * each (row, KV head) to finish combines them); otherwise the step runs the
- * appends, prepare, partials and combine as separate launches.
+ * the step is three launches: the appends share one with the query
+ * preparation, the attention partials merge their splits themselves (the last
+ * block of each (row, KV head) to finish), and one launch rotates every output
+ * back (o = V_V a, batched over the rows of each KV head); otherwise the step
+ * runs the appends, prepare, partials and combine as separate launches.
  */
 sq_status sq_decode_step(const void* calib_k, const void* calib_v, const sq_cache* kc, const sq_cache* vc,
                          const void* k_new, const void* v_new, const void* q, sq_dtype dtype, const int32_t* d_pos,
