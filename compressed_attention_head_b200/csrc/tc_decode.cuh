@@ -881,6 +881,21 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
       }
     }
     const size_t base = (qbase + h) * s.splits + split;
+    if (s.splits == 1) {
+      // the only block of (b, g): its merged vector a = sigma ⊙ acc / l goes
+      // straight over the column's query operand row (what merge_one writes)
+      const float inv_l = lt > 0.0f ? 1.0f / lt : 0.0f;
+      const bool okv = record_ok(hv, D);
+      const float* sigv = rv.sigma_f();
+      for (int i = tid; i < D; i += C::NTH) {
+        float v = 0.0f;
+#pragma unroll
+        for (int k = 0; k < C::NG; ++k)
+          if (fw[k] != 0.0f) v += fw[k] * mrg[((size_t)k * 16 + h) * D + i];
+        wq[(qbase + h) * D + i] = okv ? v * inv_l * sigv[i] : 0.0f;
+      }
+      continue;
+    }
     for (int i = tid; i < D; i += C::NTH) {
       float v = 0.0f;
 #pragma unroll
@@ -931,7 +946,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     sm100::tmem_dealloc(tmem_base, 512);
   }
   if (tid == 0 && *abort_flag && err) atomicOr(err, SQ_FLAG_TIMEOUT);
-  if (s_last) {
+  if (s_last && s.splits > 1) {
     __threadfence();
     merge_one(recs_v, s, ws, g, b, (float*)sm, tid, C::NTH);
   }
