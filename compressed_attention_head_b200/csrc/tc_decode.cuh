@@ -482,14 +482,26 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
     sm100::tmem_alloc(&misc[0], 512);
     sm100::tmem_relinquish();
   }
-  // max |weight| over the G heads (w, and u on its first m entries) -> one
-  // power-of-two scale for the fp16 operand
+  // the G heads' weights w (and u on its first m entries) read once into the
+  // first group's V^T tile (free until the tiles start), with their max |.|
+  // -> one power-of-two scale for the fp16 operand
   const size_t qbase = (size_t)b * s.n_q + (size_t)g * G;
+  float* wst = (float*)(sm + PL::GRP);            // [G][D] w, then [G][m] u
+  float* ust = wst + G * D;
+  static_assert(16 * 2 * D * 4 <= C::VT_BYTES, "weight staging fits the V^T tile");
   __syncthreads();
   {
     float mx = 0.0f;
-    for (int e = tid; e < G * D; e += C::NTH) mx = fmaxf(mx, fabsf(wq[qbase * D + e]));
-    for (int e = tid; e < G * m; e += C::NTH) mx = fmaxf(mx, fabsf(uq[(qbase + e / m) * D + e % m]));
+    for (int e = tid; e < G * D; e += C::NTH) {
+      const float x = wq[qbase * D + e];
+      wst[e] = x;
+      mx = fmaxf(mx, fabsf(x));
+    }
+    for (int e = tid; e < G * m; e += C::NTH) {
+      const float x = uq[(qbase + e / m) * D + e % m];
+      ust[e] = x;
+      mx = fmaxf(mx, fabsf(x));
+    }
     mx = warp_max(mx);
     if (lane == 0) atomicMax(&misc[2], __float_as_uint(mx));
   }
@@ -509,13 +521,13 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
       bool lo = false;
       if (n < G) {
         if (st < 3) {
-          v = wq[(qbase + n) * D + j] * wsc;
+          v = wst[n * D + j] * wsc;
           lo = st == 1;
         } else if (st < NCH + 2) {
-          v = wq[(qbase + n) * D + 16 * (st - 2) + j] * wsc;
+          v = wst[n * D + 16 * (st - 2) + j] * wsc;
         } else {
           const int jj = 16 * (st - NCH - 2) + j;
-          v = jj < m ? uq[(qbase + n) * D + jj] * wsc : 0.0f;
+          v = jj < m ? ust[n * m + jj] * wsc : 0.0f;
         }
       }
       __half h = __float2half_rn(v);
@@ -912,7 +924,7 @@ k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs
   // publishes its partials, then counts itself; the counter was cleared by
   // the prepare step of this call)
   __shared__ int s_last;
-  __threadfence();
+  if (s.splits > 1) __threadfence();
   __syncthreads();
   if (tid == 0) {
     int last = 1;
