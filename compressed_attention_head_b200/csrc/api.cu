@@ -795,7 +795,7 @@ sq_status attn_launch(const void* calib_k, const void* calib_v, const sq_cache* 
     const int MGv = sh.group <= 2 ? 2 : (sh.group <= 4 ? 4 : (sh.group <= 8 ? 8 : 16));
 #define SQ_TD_LAUNCH(DD, MG)                                                                                  \
   td::k_decode_tc<DD, MG><<<gpart, td::Cfg<DD>::NTH, td::smem_bytes<DD>(kc->words, vc->words, nrec, ngs), st>>>( \
-      rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags, nrec, ngs, out, (int)out_dtype)
+      rk, rv, ka, va, d_lens, sh, w, scores_out, d_flags, nrec, ngs)
 #define SQ_TD_G(DD)                                                                                       \
   if (MGv == 2) SQ_TD_LAUNCH(DD, 2); else if (MGv == 4) SQ_TD_LAUNCH(DD, 4); else if (MGv == 8) SQ_TD_LAUNCH(DD, 8); \
   else SQ_TD_LAUNCH(DD, 16)

@@ -351,8 +351,7 @@ template <int D, int MG>
 __global__ void __launch_bounds__(Cfg<D>::NTH, 1)
 k_decode_tc(const uint8_t* __restrict__ recs_k, const uint8_t* __restrict__ recs_v, CacheArgs kc, CacheArgs vc,
             const int32_t* __restrict__ seq_lens, AttnShape s, float* __restrict__ ws,
-            float* __restrict__ scores_out, uint32_t* __restrict__ flags, int nrec, int ngs, void* out,
-            int out_dt) {
+            float* __restrict__ scores_out, uint32_t* __restrict__ flags, int nrec, int ngs) {
   using C = Cfg<D>;
   using PL = Plan<D>;
   constexpr int NCH = C::NCH;
